@@ -1,0 +1,147 @@
+/*
+ * lf.h -- C ABI of liblf.so: Longformer banded + global self-attention on
+ * NVIDIA B200 (sm_100a).
+ *
+ * "FTL" below is the page "FasterTransformer Longformer 推理加速实践：
+ * PyTorch 集成、输入约束与端到端性能解析"; each entry point cites the
+ * section of that page defining the operation it performs.
+ *
+ * Conventions for every entry point:
+ *   - Tensor arguments are DEVICE pointers to caller-owned, dense, row-major
+ *     memory on the current CUDA device, unless marked "host".  The library
+ *     never frees or retains them after the call's work has finished.
+ *   - Device pointers must be 16-byte aligned (LF_ERR_MISALIGNED otherwise).
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and is asynchronous unless the description says otherwise.
+ *   - Host-side validation happens before anything is launched; a non-zero
+ *     return means nothing was enqueued (except LF_ERR_CUDA, which reports a
+ *     failed launch).
+ *   - Errors that depend on mask CONTENTS are found on the device.  Kernels
+ *     record the first such error in a per-device status word, read (and
+ *     optionally cleared) by lf_device_status().
+ *   - Outputs must not alias inputs.
+ *   - head_dim is fixed at 64 (FTL §使用前提：四条硬性约束, item 2): there is no
+ *     head-dim argument.
+ */
+#ifndef LF_H_
+#define LF_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st* lf_stream_t;
+
+typedef enum {
+    LF_OK = 0,
+    LF_ERR_NULL = 1,                 /* a required pointer is NULL */
+    LF_ERR_BAD_DIM = 2,              /* B, H, L or w <= 0 */
+    LF_ERR_L_NOT_MULTIPLE_OF_W = 3,  /* FTL §使用前提 item 1: L % w != 0 */
+    LF_ERR_L_LT_2W = 4,              /* FTL §使用前提 item 1: L < 2w */
+    LF_ERR_G_GT_W = 5,               /* FTL §使用前提 item 3: global tokens > w */
+    LF_ERR_GLOBAL_NOT_PREFIX = 6,    /* FTL §使用前提 item 4: globals not at 0..g-1 */
+    LF_ERR_DTYPE = 7,                /* unsupported dtype value */
+    LF_ERR_MISALIGNED = 8,           /* a device pointer is not 16-byte aligned */
+    LF_ERR_CUDA = 9,                 /* a CUDA runtime call or launch failed */
+    LF_ERR_DEVICE_TIMEOUT = 10,      /* a bounded device-side wait expired */
+    LF_ERR_UNSUPPORTED_DEVICE = 11,  /* current device is not compute capability 10.0 */
+    LF_ERR_WORKSPACE = 12,           /* workspace pointer/size too small */
+    LF_ERR_TOO_LARGE = 13            /* a size exceeds the documented maximum */
+} lf_status;
+
+typedef enum { LF_F32 = 0, LF_F16 = 1, LF_BF16 = 2 } lf_dtype;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* lf_status_string(int status);
+
+/* Library ABI version (major * 100 + minor). */
+int lf_version(void);
+
+/*
+ * lf_device_status -- synchronise `stream`, then return the first
+ * content-dependent error recorded by this library's kernels on the current
+ * device since the last reset (LF_OK if none).  reset != 0 clears the word.
+ * Errors recorded: LF_ERR_G_GT_W, LF_ERR_GLOBAL_NOT_PREFIX,
+ * LF_ERR_DEVICE_TIMEOUT.
+ */
+lf_status lf_device_status(lf_stream_t stream, int reset);
+
+/*
+ * lf_init_global_idx -- global-token index partition.
+ * FTL §Longformer Encoder 计算流程 / 预处理 (invokeInitLongformerIdx): for each
+ * sample b, positions j with global_mask[b,j] == 0.0f are "global".
+ *
+ *   global_mask       [B, L] float32, device.  0.0 = global token, any other
+ *                     value (the page uses -10000.0) = not global.
+ *   global_idx        [B, L] int32, device, written: the global positions in
+ *                     ascending order, followed by the other positions in
+ *                     descending order (the order of a stable flagged
+ *                     partition that writes rejected items from the back).
+ *   global_token_nums [B] int32, device, written: g_b = number of globals.
+ *   max_global_out    HOST int*, may be NULL.  If non-NULL the call
+ *                     synchronises `stream`, writes max_b g_b there and
+ *                     returns the content check below directly; the device
+ *                     status word is cleared before the launch in that mode.
+ *
+ * Content check (FTL §使用前提 items 3 and 4): every g_b <= w and the globals
+ * of each sample are exactly positions 0..g_b-1; otherwise
+ * LF_ERR_G_GT_W / LF_ERR_GLOBAL_NOT_PREFIX (device status word, or the
+ * return value in synchronous mode).  Outputs are written in full either way.
+ * Shape checks: B, L, w > 0, L % w == 0, L >= 2w (FTL §使用前提 item 1).
+ */
+lf_status lf_init_global_idx(const float* global_mask, int B, int L, int w,
+                             int32_t* global_idx, int32_t* global_token_nums,
+                             int* max_global_out, lf_stream_t stream);
+
+/*
+ * lf_attention_forward -- Longformer self-attention of one layer.
+ * FTL §Longformer Encoder 计算流程 / 每个 Transformer 层, steps 3-5
+ * (LongformerAttentionLayer::forward, longformerMHASoftmax and
+ * TransposeMultiHeadToSingle), fused into one kernel.
+ *
+ *   q, k, v, qg, kg, vg  [B, H, L, 64] of `dtype`, device (the layout after
+ *                        AddBiasTransposeToMultiHead, step 2).  qg is read
+ *                        only at rows i < g_b.
+ *   local_mask           [B, L] float32: 1.0 = token, 0.0 = padding.
+ *   global_mask          [B, L] float32: 0.0 = global, -10000.0 = not.
+ *   out                  [B, L, H*64] of `dtype`, device, written in full.
+ *
+ * With lb[j] = fmaf(local_mask[b,j], 10000, -10000), s = 1/8 and
+ * g_b = number of leading 0.0 entries of global_mask[b]:
+ *   row i with lb[i] != 0                -> out row = 0;
+ *   row i <  g_b (global row)            -> softmax_j(s*qg_i.kg_j + lb[j]) over
+ *                                           all j, values vg;
+ *   row i >= g_b (local row)             -> softmax over the set
+ *                                           {|i-j| <= w} U {0..g_b-1} (each key
+ *                                           once) of s*q_i.k_j + lb[j], values v.
+ * dtype: LF_F32 (CUDA-core FMA path), LF_F16 or LF_BF16 (tensor-core path,
+ * fp32 accumulation and softmax, output rounded to nearest even).
+ * Shape checks as lf_init_global_idx.  Content: a sample with g_b > w records
+ * LF_ERR_G_GT_W and gets an all-zero output; a 0.0 entry of global_mask after
+ * position g_b records LF_ERR_GLOBAL_NOT_PREFIX (output computed with g_b).
+ * Scratch: the call uses a library-owned per-device scratch buffer, allocated
+ * (cudaMalloc) on the first call on a device and regrown when a call needs
+ * more; make that first call before any stream capture.  Calls that overlap
+ * on the GPU (different streams) share the scratch and must not overlap.
+ */
+lf_status lf_attention_forward(const void* q, const void* k, const void* v,
+                               const void* qg, const void* kg, const void* vg,
+                               const float* local_mask, const float* global_mask,
+                               int B, int H, int L, int w, lf_dtype dtype,
+                               lf_stream_t stream, void* out);
+
+/* Bytes of scratch lf_attention_forward needs for this shape (0 if none). */
+size_t lf_attention_scratch_bytes(int B, int H, int L, int w, lf_dtype dtype);
+
+/* Free the library-owned scratch of the current device (synchronises it). */
+lf_status lf_release_scratch(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LF_H_ */

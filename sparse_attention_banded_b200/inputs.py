@@ -1,0 +1,123 @@
+"""Seeded synthetic inputs for the Longformer attention workloads.
+
+This module only draws random numbers and lays out masks; it holds none of
+the attention arithmetic.  Both the tests (for the oracle and the CUDA path)
+and the benchmark take their inputs from here.
+
+Workloads (all head_dim 64; values ~ N(0, 1) * 0.5 rounded to the dtype):
+  1  fp32  B=1 H=2  L=512   w=64  g=8 prefix globals, no padding
+  2  fp16  B=1 H=16 L=4096  w=256 g=64, last 300 positions padded
+  3  bf16  B=4 H=16 L=4096  w=256 per-sample g ~ U{1..128}, padding tail
+           ~ U{0..1024}, drawn in the order g_0, pad_0, g_1, pad_1, ...
+  4  fp16  B=1 H=12 L=16384 w=256 g=32, no padding
+  5  fp16  one encoder layer: B=1 L=4096 hidden 1024 (16 x 64) FFN 4096,
+           w=256 g=64; x ~ N(0,1), weights ~ N(0, 0.02), biases 0,
+           LayerNorm gamma 1 beta 0.
+Mask conventions follow the FasterTransformer Longformer page's input list:
+local_mask 1.0 = token / 0.0 = padding; global_mask 0.0 = global /
+-10000.0 = not global.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass, field
+from typing import List
+
+import torch
+
+TORCH_DTYPES = {"f32": torch.float32, "f16": torch.float16, "bf16": torch.bfloat16}
+NAMES = ("q", "k", "v", "qg", "kg", "vg")
+
+
+@dataclass
+class Workload:
+    cid: int
+    name: str
+    dtype: str
+    B: int
+    H: int
+    L: int
+    w: int
+    g: List[int] = field(default_factory=list)
+    pad: List[int] = field(default_factory=list)
+    seed: int = 0
+
+
+def workload(cid: int) -> Workload:
+    if cid == 1:
+        return Workload(1, "fp32 B1 H2 L512 w64 g8", "f32", 1, 2, 512, 64, [8], [0], 1001)
+    if cid == 2:
+        return Workload(2, "fp16 Longformer-large B1 H16 L4096 w256 g64 pad300", "f16",
+                        1, 16, 4096, 256, [64], [300], 1002)
+    if cid == 3:
+        gen = torch.Generator().manual_seed(1003)
+        g, pad = [], []
+        for _ in range(4):
+            g.append(int(torch.randint(1, 129, (1,), generator=gen)))
+            pad.append(int(torch.randint(0, 1025, (1,), generator=gen)))
+        return Workload(3, "bf16 batched B4 H16 L4096 w256 g~U[1,128] pad~U[0,1024]", "bf16",
+                        4, 16, 4096, 256, g, pad, 1003)
+    if cid == 4:
+        return Workload(4, "fp16 long document B1 H12 L16384 w256 g32", "f16",
+                        1, 12, 16384, 256, [32], [0], 1004)
+    if cid == 5:
+        return Workload(5, "fp16 encoder layer B1 L4096 hidden1024 H16 w256 g64 ffn4096", "f16",
+                        1, 16, 4096, 256, [64], [0], 1005)
+    raise ValueError("unknown workload %r" % cid)
+
+
+def masks(B: int, L: int, g: List[int], pad: List[int]):
+    """local_mask / global_mask [B, L] float32 for prefix globals g[b] and a
+    padding tail of pad[b] positions."""
+    local = torch.ones(B, L, dtype=torch.float32)
+    glob = torch.full((B, L), -10000.0, dtype=torch.float32)
+    for b in range(B):
+        if pad[b] > 0:
+            local[b, L - pad[b]:] = 0.0
+        glob[b, :g[b]] = 0.0
+    return local, glob
+
+
+def attention_inputs(B: int, H: int, L: int, dtype: str, seed: int, scale: float = 0.5,
+                     device: str = "cpu"):
+    """q, k, v, qg, kg, vg: [B, H, L, 64] ~ N(0,1)*scale, rounded to dtype."""
+    gen = torch.Generator().manual_seed(seed)
+    out = {}
+    for n in NAMES:
+        t = torch.randn(B, H, L, 64, generator=gen, dtype=torch.float32) * scale
+        out[n] = t.to(TORCH_DTYPES[dtype]).to(device)
+    return out
+
+
+def workload_inputs(cid: int, device: str = "cpu"):
+    """(Workload, tensors dict, local_mask, global_mask) for workload cid."""
+    wl = workload(cid)
+    t = attention_inputs(wl.B, wl.H, wl.L, wl.dtype, wl.seed, device=device)
+    lm, gm = masks(wl.B, wl.L, wl.g, wl.pad)
+    return wl, t, lm.to(device), gm.to(device)
+
+
+def layer_inputs(cid: int = 5, hidden: int = 1024, ffn: int = 4096, device: str = "cpu"):
+    """Encoder-layer input x [B, L, hidden] and weights (y = x @ W + b, W
+    stored [in, out]; q k v kg vg weights contiguous as [5, hidden, hidden])."""
+    wl = workload(cid)
+    dt = TORCH_DTYPES[wl.dtype]
+    gen = torch.Generator().manual_seed(wl.seed)
+    x = torch.randn(wl.B, wl.L, hidden, generator=gen)
+    w = {}
+    mats = [("W_q", (hidden, hidden)), ("W_k", (hidden, hidden)), ("W_v", (hidden, hidden)),
+            ("W_kg", (hidden, hidden)), ("W_vg", (hidden, hidden)), ("W_qg", (hidden, hidden)),
+            ("W_o", (hidden, hidden)), ("W_1", (hidden, ffn)), ("W_2", (ffn, hidden))]
+    for n, shp in mats:
+        w[n] = torch.randn(*shp, generator=gen) * 0.02
+    weights = {
+        "W_qkv_kgvg": torch.stack([w["W_q"], w["W_k"], w["W_v"], w["W_kg"], w["W_vg"]]).to(dt),
+        "b_qkv_kgvg": torch.zeros(5, hidden).to(dt),
+        "W_qg": w["W_qg"].to(dt), "b_qg": torch.zeros(hidden).to(dt),
+        "W_o": w["W_o"].to(dt), "b_o": torch.zeros(hidden).to(dt),
+        "ln1_gamma": torch.ones(hidden), "ln1_beta": torch.zeros(hidden),
+        "W_1": w["W_1"].to(dt), "b_1": torch.zeros(ffn).to(dt),
+        "W_2": w["W_2"].to(dt), "b_2": torch.zeros(hidden).to(dt),
+        "ln2_gamma": torch.ones(hidden), "ln2_beta": torch.zeros(hidden),
+    }
+    lm, gm = masks(wl.B, wl.L, wl.g, wl.pad)
+    return wl, x.to(dt).to(device), {k: v.to(device) for k, v in weights.items()}, lm.to(device), gm.to(device)
