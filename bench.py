@@ -1,0 +1,368 @@
+#!/usr/bin/env python
+"""Benchmark of the Longformer banded + global attention hot path on B200.
+
+One step = one pass of the whole path over one batch of the fp16
+Longformer-large workload (B=1, H=16, L=4096, w=256, 64 prefix globals, last
+300 positions padded): the global-index partition kernel, then the fused
+attention kernel.  Inputs are synthetic and seeded.  The workload's HBM
+footprint (~50 MB) fits in L2, so L2 is flushed (a 2 x L2 write) before
+every timed step, outside the step's event pair.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+Under torchrun each rank runs its own replica of the workload (weak scaling,
+no collective on the data path); timings are the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from sparse_attention_banded_b200 import inputs, metrics  # noqa: E402
+
+METRIC = "Longformer attention tokens/s & TFLOP/s (fp16 L=4096 w=256) and % tensor peak"
+WORKLOAD_ID = 2
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=50)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clock and throttle reasons while running."""
+    FIELDS = ("pci.bus_id,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.path = None
+        try:
+            props = torch.cuda.get_device_properties(device_index)
+            self.bus = "%08X:%02X:%02X.0" % (props.pci_domain_id, props.pci_bus_id, props.pci_device_id)
+        except Exception:
+            self.bus = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(["nvidia-smi", "--query-gpu=" + self.FIELDS, "--format=csv,noheader",
+                                          "-lms", "100", "-f", self.path],
+                                         stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                if self.bus and parts[0].upper()[-len(self.bus):] != self.bus and \
+                        not parts[0].upper().endswith(self.bus[4:]):
+                    continue
+                rows.append(parts)
+        os.remove(self.path)
+        if not rows:
+            return None
+        sm = [float(re.sub(r"[^0-9.]", "", r[1]) or 0) for r in rows]
+        mx = [float(re.sub(r"[^0-9.]", "", r[2]) or 0) for r in rows]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[k] for r in rows for k in range(4) if r[5 + k].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ---------------------------------------------------------------- our arm
+
+def traffic_from_profile(kernel_src_hash: str):
+    """DRAM bytes per attention launch from the committed ncu summary, or
+    None if the summary was taken on a different kernel source."""
+    path = os.path.join(ROOT, "profiles", "attention_tc_workload2.md")
+    if not os.path.exists(path):
+        return None
+    txt = open(path).read()
+    m = re.search(r"kernel_source_sha256:\s*([0-9a-f]+)", txt)
+    t = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", txt)
+    if not m or not t or m.group(1) != kernel_src_hash:
+        return None
+    return float(t.group(1))
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for name in ("lf_attn_tc.cu", "sm100.cuh"):
+        with open(os.path.join(ROOT, "sparse_attention_banded_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def cpu_baseline(wl, t, lm, gm, budget_s=10.0):
+    import numpy as np
+    import oracle
+    arrs = [t[n].double().numpy() for n in inputs.NAMES]
+    lmn, gmn = lm.numpy(), gm.numpy()
+    passes, t0 = 0, time.perf_counter()
+    while True:
+        oracle.attention(*arrs, lmn, gmn, wl.w)
+        passes += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    el = time.perf_counter() - t0
+    return {"value": wl.B * wl.L * passes / el, "unit": "tokens/s", "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": "%d full pass(es) of the workload (%d query rows each), float64 C oracle" %
+                      (passes, wl.B * wl.H * wl.L)}
+
+
+def run_ours(args):
+    from sparse_attention_banded_b200 import lf
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    wl, t_cpu, lm_cpu, gm_cpu = inputs.workload_inputs(WORKLOAD_ID)
+    t = {n: t_cpu[n].to(dev) for n in inputs.NAMES}
+    lm, gm = lm_cpu.to(dev), gm_cpu.to(dev)
+    out = torch.empty(wl.B, wl.L, wl.H * 64, dtype=t["q"].dtype, device=dev)
+    gidx = torch.empty(wl.B, wl.L, dtype=torch.int32, device=dev)
+    gnum = torch.empty(wl.B, dtype=torch.int32, device=dev)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = torch.empty(max(2 * l2, 256 << 20) // 4, dtype=torch.float32, device=dev)
+    args_in = [t[n] for n in inputs.NAMES]
+
+    def step(ev_a=None):
+        lf.lf_init_global_idx(gm, wl.w, gidx, gnum, sync=False)
+        if ev_a is not None:
+            ev_a.record()
+        lf.lf_attention_forward(*args_in, lm, gm, wl.w, out=out)
+
+    lf.lf_device_status(reset=True)
+    for _ in range(max(args.warmup, 3)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    st = lf.lf_device_status(reset=True)
+    if st != 0:
+        raise RuntimeError("device status after warm-up: %s" % lf.status_string(st))
+
+    K = args.steps
+    ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ev_a = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    sampler = ClockSampler(local)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.3)  # let the sampler attach before the timed region
+    for k in range(K):
+        flush.zero_()
+        ev_s[k].record()
+        step(ev_a[k])
+        ev_e[k].record()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    clocks = sampler.stop()
+    step_ms = [ev_s[k].elapsed_time(ev_e[k]) for k in range(K)]
+    attn_ms = [ev_a[k].elapsed_time(ev_e[k]) for k in range(K)]
+    total_ms = sum(step_ms)
+    attn_avg_ms = sum(attn_ms) / K
+    if world > 1:
+        x = torch.tensor([total_ms, attn_avg_ms], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(x, op=torch.distributed.ReduceOp.MAX)
+        total_ms, attn_avg_ms = x.tolist()
+
+    # end to end through the public call: pinned host inputs -> device ->
+    # partition + attention -> output back to pinned host memory
+    E = max(1, args.e2e_steps)
+    h_in = [x.cpu().pin_memory() for x in args_in] + [lm_cpu.pin_memory(), gm_cpu.pin_memory()]
+    d_in = [torch.empty_like(x, device=dev) for x in h_in]
+    h_out = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    h2d = sum(x.numel() * x.element_size() for x in h_in)
+    d2h = h_out.numel() * h_out.element_size()
+
+    def e2e_step():
+        for h, d in zip(h_in, d_in):
+            d.copy_(h, non_blocking=True)
+        lf.lf_init_global_idx(d_in[7], wl.w, gidx, gnum, sync=False)
+        lf.lf_attention_forward(*d_in[:6], d_in[6], d_in[7], wl.w, out=out)
+        h_out.copy_(out, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(E):
+        e2e_step()
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / E
+    if world > 1:
+        x = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(x, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = x.item()
+    st = lf.lf_device_status(reset=True)
+    if st != 0:
+        raise RuntimeError("device status after timing: %s" % lf.status_string(st))
+
+    pk, pk_kind = peaks()
+    F = metrics.flops(wl.B, wl.H, wl.L, wl.w, wl.g, wl.pad)
+    By = metrics.algorithmic_bytes(wl.B, wl.H, wl.L, wl.w, wl.g, wl.dtype)
+    t_attn = attn_avg_ms * 1e-3
+    tokens = wl.B * wl.L
+    value = world * tokens * K / (total_ms * 1e-3)
+    res = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": total_ms / K,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f16",
+        "data": "synthetic (seeded N(0,1)*0.5 inputs of the workload's shape)",
+        "config": {"workload": wl.name, "B": wl.B, "H": wl.H, "L": wl.L, "w": wl.w, "g": wl.g,
+                   "pad": wl.pad, "head_dim": 64, "l2": "flushed before every timed step (2 x L2 write)",
+                   "parallelism": "replica per GPU (weak)" if world > 1 else "single GPU"},
+        "tflops": F / (total_ms * 1e-3 / K) / 1e12,
+        "attention_kernel": {
+            "avg_us": attn_avg_ms * 1e3,
+            "tflops": F / t_attn / 1e12,
+            "tensor_peak_frac": F / t_attn / 1e12 / pk["bf16_tflops"],
+            "tensor_peak_tflops": pk["bf16_tflops"],
+            "note": "fp16 and bf16 dense tensor rates are equal; peak = measured bf16 burst (%s)" % pk_kind,
+        },
+        "roofline": {
+            "bound": "hbm",
+            "achieved": By / t_attn / 1e9,
+            "peak": pk["hbm_gbs"],
+            "unit": "GB/s",
+            "frac": By / t_attn / 1e9 / pk["hbm_gbs"],
+            "traffic": traffic_from_profile(kernel_source_hash()),
+            "peak_kind": pk_kind,
+            "algorithmic_bytes_per_launch": By,
+            "flops_per_launch": F,
+        },
+        "e2e": {"value": world * tokens / (e2e_ms * 1e-3), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": 2 * K,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline(wl, t_cpu, lm_cpu, gm_cpu)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(res))
+
+
+# ---------------------------------------------------------------- reference arm (the oracle)
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    import numpy as np
+    import oracle
+    wl, t_cpu, lm_cpu, gm_cpu = inputs.workload_inputs(WORKLOAD_ID)
+    arrs = [t_cpu[n].double().numpy() for n in inputs.NAMES]
+    lmn, gmn = lm_cpu.numpy(), gm_cpu.numpy()
+    H = wl.H
+
+    def rows_for(pos0, npos):
+        pos = (np.arange(npos) + pos0) % wl.L
+        return np.array([[0, h, p] for p in pos for h in range(H)], dtype=np.int32)
+
+    # calibrate: size each step so the whole run takes about a minute
+    t0 = time.perf_counter()
+    oracle.attention_rows(*arrs, lmn, gmn, wl.w, rows_for(0, 64))
+    per_pos = (time.perf_counter() - t0) / 64
+    K, W = args.steps, args.warmup
+    npos = int(max(1, min(wl.L, 60.0 / max(1, K + W) / per_pos)))
+    for k in range(W):
+        oracle.attention_rows(*arrs, lmn, gmn, wl.w, rows_for(k * npos, npos))
+    t0 = time.perf_counter()
+    for k in range(K):
+        oracle.attention_rows(*arrs, lmn, gmn, wl.w, rows_for((W + k) * npos, npos))
+    el = time.perf_counter() - t0
+    value = npos * K / el
+    res = {
+        "impl": "reference",
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": W,
+        "ms_per_step": el * 1e3 / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic (seeded N(0,1)*0.5 inputs of the workload's shape)",
+        "config": {"workload": wl.name, "B": wl.B, "H": wl.H, "L": wl.L, "w": wl.w, "g": wl.g,
+                   "pad": wl.pad, "head_dim": 64},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+                         "sample": "%d positions x %d heads per step (float64 C oracle)" % (npos, H)},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(res))
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

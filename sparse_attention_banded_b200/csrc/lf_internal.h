@@ -1,0 +1,60 @@
+// Internal declarations shared by the liblf.so translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "lf.h"
+
+namespace lf {
+
+// Device status word: holds LF_STATUS_CLEAR or (sample << 8) | code, and is
+// only ever lowered with atomicMin, so the word keeps the error of the
+// lowest-numbered failing sample (lowest code within a sample).
+constexpr int LF_STATUS_CLEAR = 0x7fffffff;
+
+__device__ __forceinline__ void record_status(int* word, int sample, int code) {
+    atomicMin(word, (sample << 8) | code);
+}
+
+struct DeviceCtx {
+    bool init = false;
+    int ordinal = -1;
+    int sm_count = 0;
+    int cc_major = 0, cc_minor = 0;
+    int* status = nullptr;  // device word, see LF_STATUS_CLEAR
+    void* scratch = nullptr;
+    size_t scratch_bytes = 0;
+};
+
+// Current device's context (initialised on first use; NULL + status on error).
+DeviceCtx* current_device(lf_status* st);
+// Make sure the current device's library scratch holds `bytes` (grows by
+// cudaMalloc; the new region is zeroed).
+lf_status ensure_scratch(DeviceCtx* dev, size_t bytes);
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+lf_status check_shape(int B, int H, int L, int w);
+
+// ---- launchers (return LF_OK or LF_ERR_CUDA) ----
+lf_status launch_global_idx(const float* global_mask, int B, int L, int w, int32_t* global_idx,
+                            int32_t* global_token_nums, int* status, cudaStream_t stream);
+
+lf_status launch_attention_simt_f32(const float* q, const float* k, const float* v, const float* qg,
+                                    const float* kg, const float* vg, const float* local_mask,
+                                    const float* global_mask, int B, int H, int L, int w,
+                                    float scale, float* out, int* status, cudaStream_t stream);
+
+// Tensor-core path (fp16 / bf16).  `scratch` must hold
+// attention_tc_scratch_bytes(B, H, L, w) bytes whose counter region is zero
+// on entry (the kernel leaves it zero).
+size_t attention_tc_scratch_bytes(int B, int H, int L, int w);
+lf_status launch_attention_tc(const void* q, const void* k, const void* v, const void* qg,
+                              const void* kg, const void* vg, const float* local_mask,
+                              const float* global_mask, int B, int H, int L, int w, float scale,
+                              lf_dtype dtype, void* out, void* scratch, int* status,
+                              int sm_count, cudaStream_t stream);
+
+}  // namespace lf

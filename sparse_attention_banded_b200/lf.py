@@ -1,0 +1,128 @@
+"""ctypes binding of liblf.so (argument marshalling only).
+
+Each function mirrors the C entry point of the same name in ``include/lf.h``:
+it takes torch CUDA tensors, passes their device pointers, sizes and the
+current CUDA stream to the library, and raises :class:`LFError` on a non-zero
+status.  All computation happens in the library's CUDA kernels; if the
+library is missing this module raises instead of falling back to anything.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "liblf.so")
+HEADER = os.path.join(os.path.dirname(_HERE), "include", "lf.h")
+
+LF_F32, LF_F16, LF_BF16 = 0, 1, 2
+DTYPE_CODE = {torch.float32: LF_F32, torch.float16: LF_F16, torch.bfloat16: LF_BF16}
+
+_lib = None
+
+
+class LFError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__("%s: %s" % (where, status_string(status)))
+
+
+def lib():
+    """Load liblf.so once (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError("liblf.so is not built; run `python -m sparse_attention_banded_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i, st = ctypes.c_void_p, ctypes.c_int, ctypes.c_int
+        L.lf_status_string.argtypes = [i]
+        L.lf_status_string.restype = ctypes.c_char_p
+        L.lf_version.restype = i
+        L.lf_device_status.argtypes = [vp, i]
+        L.lf_device_status.restype = st
+        L.lf_init_global_idx.argtypes = [vp, i, i, i, vp, vp, ctypes.POINTER(ctypes.c_int), vp]
+        L.lf_init_global_idx.restype = st
+        L.lf_attention_forward.argtypes = [vp] * 8 + [i, i, i, i, i, vp, vp]
+        L.lf_attention_forward.restype = st
+        L.lf_attention_scratch_bytes.argtypes = [i, i, i, i, i]
+        L.lf_attention_scratch_bytes.restype = ctypes.c_size_t
+        L.lf_release_scratch.restype = st
+        _lib = L
+    return _lib
+
+
+def declared_functions():
+    """Names of the functions include/lf.h declares."""
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[\w\*\s]+?\b(lf_\w+)\s*\(", text, re.M)))
+
+
+def status_string(status: int) -> str:
+    return lib().lf_status_string(int(status)).decode()
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("expected a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError("expected a contiguous tensor")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _check(status, where):
+    if status != 0:
+        raise LFError(status, where)
+
+
+def lf_device_status(reset: bool = False, stream=None) -> int:
+    """Synchronise and return the device status word (see lf.h)."""
+    return lib().lf_device_status(_stream(stream), 1 if reset else 0)
+
+
+def lf_init_global_idx(global_mask, w: int, global_idx=None, global_token_nums=None, sync: bool = True,
+                       stream=None):
+    """Global-token partition.  Returns (global_idx, global_token_nums,
+    max_g); max_g is None when sync is False (then content errors go to the
+    device status word)."""
+    B, L = global_mask.shape
+    if global_idx is None:
+        global_idx = torch.empty(B, L, dtype=torch.int32, device=global_mask.device)
+    if global_token_nums is None:
+        global_token_nums = torch.empty(B, dtype=torch.int32, device=global_mask.device)
+    mx = ctypes.c_int(-1)
+    st = lib().lf_init_global_idx(_ptr(global_mask), B, L, w, _ptr(global_idx), _ptr(global_token_nums),
+                                  ctypes.byref(mx) if sync else None, _stream(stream))
+    _check(st, "lf_init_global_idx")
+    return global_idx, global_token_nums, (mx.value if sync else None)
+
+
+def lf_attention_forward(q, k, v, qg, kg, vg, local_mask, global_mask, w: int, out=None, stream=None):
+    """Longformer attention; q..vg [B, H, L, 64], masks [B, L] float32.
+    Returns out [B, L, H*64] in the input dtype."""
+    B, H, L, _ = q.shape
+    if out is None:
+        out = torch.empty(B, L, H * 64, dtype=q.dtype, device=q.device)
+    code = DTYPE_CODE.get(q.dtype, 99)
+    st = lib().lf_attention_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(qg), _ptr(kg), _ptr(vg),
+                                    _ptr(local_mask), _ptr(global_mask), B, H, L, w, code,
+                                    _stream(stream), _ptr(out))
+    _check(st, "lf_attention_forward")
+    return out
+
+
+def lf_attention_scratch_bytes(B: int, H: int, L: int, w: int, dtype) -> int:
+    return lib().lf_attention_scratch_bytes(B, H, L, w, DTYPE_CODE[dtype])
+
+
+def lf_release_scratch():
+    _check(lib().lf_release_scratch(), "lf_release_scratch")
