@@ -4,29 +4,43 @@
 // 实践"), §Longformer Encoder 计算流程 / 每个 Transformer 层 steps 3-5, runs
 // this layer as window GEMMs over head/middle/tail segments, a separate
 // masked-softmax kernel and a transpose kernel.  Here it is ONE persistent
-// kernel per call:
+// kernel per call.
 //
-//   work item "band"   (b, h, 128-query tile t): the tile's key blocks are the
-//       128-key blocks overlapping rows' windows |i - j| <= w, plus the blocks
-//       holding global keys 0..g_b-1 that some row of the tile sees outside its
-//       window.  Every key block is visited once, with the mask
-//       allowed(i, j) = j < g_b || |i - j| <= w, so a global key inside the
-//       window is counted once.
-//   work item "global" (b, h, row tile rt, key split s): rows i < g_b attend
-//       to all keys through qg/kg/vg; the keys are split into chunks of
-//       kChunkBlocks blocks, each item leaves (m, l, O) partials in scratch and
-//       the last item of a (b, h, rt) to finish merges them (log-sum-exp) and
-//       writes the rows.
+// Work items (taken from a global atomic counter; band pairs first, then the
+// smaller global pairs, so that the last items handed out are short):
+//   global pair (b, h, row tile rt, splits 2s and 2s+1): rows i < g_b attend
+//       to every key through qg/kg/vg.  Keys are cut into chunks of
+//       kChunkBlocks 128-key blocks; each split leaves (m, l, O) partials in
+//       scratch and the warp that finishes the last split of its 32 rows
+//       merges them (log-sum-exp) and writes the rows.
+//   band pair (b, h, tiles 2p and 2p+1 of 128 query rows): each tile visits
+//       the 128-key blocks that meet its rows' windows |i - j| <= w and the
+//       blocks of global keys 0..g_b-1 seen outside the window, with the mask
+//       allowed(i, j) = j < g_b || |i - j| <= w, so a global key inside a
+//       window counts once.  The two tiles share every K/V block they both
+//       need (loaded once).
 //
-// Per CTA: warp 0 issues TMA loads (Q tile double-buffered, K/V blocks in a
-// kStages ring), warp 1 issues tcgen05.mma (S = Q K^T into TMEM, double
-// buffered; O_blk = P V into TMEM, double buffered), warps 2-5 (one thread per
-// query row) read S from TMEM, apply scale, padding bias and mask, run the
-// online softmax, write P (fp16/bf16) to shared memory in the 128B-swizzled
-// K-major layout the MMA reads, and accumulate O in registers.  All waits are
-// bounded; on expiry the CTA records LF_ERR_DEVICE_TIMEOUT and winds down.
+// Roles (384 threads = 3 warpgroups): warp 2 fetches items and publishes
+// their plans through a ring; warp 0 issues TMA loads (Q of both tiles, K/V
+// blocks into a kStages ring); warp 1 issues tcgen05.mma; warp 3 only hands
+// its registers over; warpgroups 1 and 2
+// are the softmax warpgroups of tile A and tile B (one thread per query row).
+// Registers are rebalanced with setmaxnreg: launched at 168 per thread,
+// warpgroup 0 drops to 64 and the softmax warpgroups rise to 216
+// (4*32*64 + 8*32*216 = 63488 <= 384*168 = 64512).  Per tile X and key block:
+//   S_X = Q_X K^T           (TMEM, fp32)
+//   softmax warps: read S_X, scale, padding bias, mask, row max; rescale the
+//   TMEM accumulator O_X only when the running max grows by more than 8 (in
+//   log2 units, so P <= 2^8); P = exp2(x - m) written back into TMEM over S_X
+//   as fp16/bf16 pairs
+//   O_X += P_X V            (tcgen05.mma with A from TMEM)
+// The MMA warp alternates the two tiles, so one tile's MMAs run while the
+// other tile's softmax runs.  All waits are bounded; on expiry the CTA
+// records LF_ERR_DEVICE_TIMEOUT and winds down.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
+
+#include <stdlib.h>
 
 #include <mutex>
 
@@ -38,83 +52,141 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kBM = 128;           // query rows per tile
-constexpr int kBN = 128;           // keys per block
-constexpr int kHD = 64;            // head dim
-constexpr int kStages = 3;         // K/V ring depth
-constexpr int kChunkBlocks = 4;    // key blocks per global-row split
-constexpr int kThreads = 192;      // 6 warps
-constexpr int kSoftmaxWarp0 = 2;
+constexpr int kBM = 128;          // query rows per tile
+constexpr int kBN = 128;          // keys per block
+constexpr int kHD = 64;           // head dim
+constexpr int kStages = 4;        // K/V ring depth
+constexpr int kChunkBlocks = 4;   // key blocks per global-row split
+constexpr int kRing = 4;          // item-id ring depth
+constexpr int kWarps = 12;
+constexpr int kThreads = kWarps * 32;
+constexpr int kSoftmaxWarp0 = 4;
+constexpr uint32_t kRegsProducer = 64;
+constexpr uint32_t kRegsSoftmax = 216;
+static_assert(4 * 32 * kRegsProducer + 8 * 32 * kRegsSoftmax <= kThreads * 168, "register split");
+constexpr int kItemConsumers = 1 + 1 + 8;  // TMA warp + MMA warp + 8 softmax warps
 constexpr uint32_t kTileBytes = kBM * kHD * 2;  // 16 KB
-constexpr uint32_t kPBytes = kBM * kBN * 2;     // 32 KB
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kRescaleThreshold = 8.0f;
 
 // Shared memory map (offsets from a 1024-byte aligned base).
-constexpr uint32_t kOffQ = 0;                                // 2 x 16 KB
-constexpr uint32_t kOffK = kOffQ + 2 * kTileBytes;           // kStages x 16 KB
-constexpr uint32_t kOffV = kOffK + kStages * kTileBytes;     // kStages x 16 KB
-constexpr uint32_t kOffP = kOffV + kStages * kTileBytes;     // 2 x 32 KB
-constexpr uint32_t kOffBias = kOffP + 2 * kPBytes;           // 4 warps x 2 x 128 floats
-constexpr uint32_t kOffBar = kOffBias + 4 * 2 * kBN * 4;
-constexpr uint32_t kNumBars = 2 + 2 + 2 * kStages + 2 + 2 + 2 + 2 + 1;
+constexpr uint32_t kOffQ = 0;                                 // [2 parity][2 tile] x 16 KB
+constexpr uint32_t kOffK = kOffQ + 4 * kTileBytes;            // kStages x 16 KB
+constexpr uint32_t kOffV = kOffK + kStages * kTileBytes;      // kStages x 16 KB
+constexpr uint32_t kOffBias = kOffV + kStages * kTileBytes;   // 8 warps x 128 floats
+constexpr uint32_t kOffPlans = kOffBias + 8 * kBN * 4;        // kRing plans
+constexpr uint32_t kOffBar = kOffPlans + kRing * 128;
+constexpr uint32_t kNumBars = 2 + 2 + 2 * kStages + 2 * 4 + 2 * kRing + 2;
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
 constexpr uint32_t kSmemBytes = kOffMisc + 64 + 1024;  // + alignment slack
 
-// TMEM columns: S[0..1] at 0 / 128, PV[0..1] at 256 / 320.
+// TMEM columns: S_A [0,128), S_B [128,256), O_A [256,320), O_B [320,384).
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kTmemS = 0;
-constexpr uint32_t kTmemPV = 256;
+constexpr uint32_t kTmemO = 256;
 
 struct Params {
     int B, H, L, w;
-    int NKB;       // key blocks per head
-    int NT;        // query tiles per head
-    int RT;        // global row tiles per head (ceil(w / 128))
-    int NS;        // key splits per global row tile
-    int n_glob;    // number of global items (they come first)
+    int NKB;     // key blocks per head
+    int NT;      // query tiles per head
+    int RT;      // global row tiles per head (ceil(w / 128))
+    int NS;      // key splits per global row tile
+    int NSP;     // split pairs per global row tile
+    int NTP;     // tile pairs per head
+    int n_band;  // band pair items (they come first; global pairs follow)
     int n_items;
-    float scale_log2;
+    float scale_log2;  // scale * log2(e)
+    float inv_scale;   // 1 / scale: the padding bias in raw score units
     const float* local_mask;
     const float* global_mask;
     void* out;
-    float* part_o;    // [B*H*RT*NS][128][64]
-    float* part_ml;   // [B*H*RT*NS][128][2]
-    int* counters;    // [B*H*RT][4]: one per 32-row group of a global row tile
+    float* part_o;   // [B*H*RT*NS][128][64]
+    float* part_ml;  // [B*H*RT*NS][128][2]
+    int* counters;   // [B*H*RT][4]: per 32-row group of a global row tile
+    int* sched;      // [0] next item, [1] finished CTAs
     int* status;
+    int* trace;      // diagnostic builds only: [CTA][16 roles][state, item, a, b]
 };
+
+// Diagnostic builds (-DLF_TRACE=1) record, per CTA and role, the wait site
+// each role is at into host-mapped memory, readable while the kernel runs.
+#ifndef LF_TRACE
+#define LF_TRACE 0
+#endif
+#ifndef LF_TRACE_STATES
+#define LF_TRACE_STATES 1
+#endif
+#if LF_TRACE
+#if LF_TRACE_STATES
+#define TRACE(role, state, item, a, b)                                                 \
+    do {                                                                               \
+        if (p.trace) {                                                                 \
+            volatile int* t_ = p.trace + ((blockIdx.x * 16 + (role)) * 4);             \
+            t_[1] = (int)(item);                                                       \
+            t_[2] = (int)(a);                                                          \
+            t_[3] = (int)(b);                                                          \
+            __threadfence_system();                                                    \
+            t_[0] = (state);                                                           \
+        }                                                                              \
+    } while (0)
+#else
+#define TRACE(role, state, item, a, b) \
+    do {                               \
+    } while (0)
+#endif
+// Cycle accounting per role: TIMED(k, stmt) adds the clock64() cycles of
+// stmt to slot k; TDUMP(role) writes the 16 slots after the state words.
+#define TIMED(k, stmt)                    \
+    do {                                  \
+        const long long t0_ = clock64();  \
+        stmt;                             \
+        tacc[k] += clock64() - t0_;       \
+    } while (0)
+#define TDECL long long tacc[16] = {0}; const long long tstart_ = clock64()
+#define TDUMP(role)                                                                               \
+    do {                                                                                          \
+        if (p.trace) {                                                                            \
+            tacc[15] = clock64() - tstart_;                                                       \
+            volatile int* d_ = p.trace + gridDim.x * 16 * 4 + (blockIdx.x * 16 + (role)) * 16;    \
+            for (int k_ = 0; k_ < 16; ++k_) d_[k_] = (int)tacc[k_];                               \
+        }                                                                                         \
+    } while (0)
+#else
+#define TRACE(role, state, item, a, b) \
+    do {                               \
+    } while (0)
+#define TIMED(k, stmt) \
+    do {               \
+        stmt;          \
+    } while (0)
+#define TDECL \
+    do {      \
+    } while (0)
+#define TDUMP(role) \
+    do {            \
+    } while (0)
+#endif
 
 struct Maps {
     CUtensorMap q, k, v, qg, kg, vg;
 };
 
-struct Item {
-    int global;   // 1 = global-row item
-    int b, h, bh;
-    int tile;     // t (band) or rt (global)
-    int split;
-    int r0;       // first query row
+struct Tile {
+    int present;         // has key blocks
+    int r0;              // first query row
+    int split;           // global: key split
+    int glob_hi, lo, hi; // band: blocks [0, glob_hi) U [lo, hi]; global: [lo, hi]
 };
 
-__device__ __forceinline__ Item decode_item(const Params& p, int id) {
-    Item it;
-    if (id < p.n_glob) {
-        it.global = 1;
-        it.split = id % p.NS;
-        const int r = id / p.NS;
-        it.tile = r % p.RT;
-        it.bh = r / p.RT;
-    } else {
-        const int id2 = id - p.n_glob;
-        it.global = 0;
-        it.split = 0;
-        it.tile = id2 % p.NT;
-        it.bh = id2 / p.NT;
-    }
-    it.b = it.bh / p.H;
-    it.h = it.bh % p.H;
-    it.r0 = it.tile * kBM;
-    return it;
-}
+struct Plan {
+    int id;       // item id, -1 = no more items
+    int global;
+    int b, h, bh, rt;
+    int g;        // leading global count (valid sample iff g <= w)
+    Tile t[2];
+    int nloads;
+    int e1, lo_min;  // band pair: loads are [0, e1) then lo_min, lo_min + 1, ...
+    int zero_only[2]; // band tile with no work but rows to zero (padded rows)
+};
 
 // Leading 0.0 entries of global_mask[b, :] capped at w + 1 (whole warp).
 __device__ int leading_globals(const Params& p, int b) {
@@ -129,32 +201,129 @@ __device__ int leading_globals(const Params& p, int b) {
     return cap;
 }
 
-struct Blocks {
-    int n;        // number of key blocks
-    int glob_hi;  // blocks [0, glob_hi) are global-key blocks
-    int band_lo;  // then blocks band_lo, band_lo + 1, ...
-};
-
-__device__ __forceinline__ Blocks block_list(const Params& p, const Item& it, int g) {
-    Blocks bl{0, 0, 0};
-    if (g > p.w) return bl;  // invalid sample: no compute
-    if (it.global) {
-        if (it.r0 >= g) return bl;
-        bl.band_lo = it.split * kChunkBlocks;
-        const int hi = min(p.NKB, bl.band_lo + kChunkBlocks) - 1;
-        bl.n = hi - bl.band_lo + 1;
-        return bl;
+// Whole warp: does band tile [r0, r0+128) have a row g <= i < L that is not
+// padded?  Also reports whether it has padded rows in [g, L).
+__device__ void band_rows(const Params& p, int b, int r0, int g, int& work, int& padded) {
+    const int lane = threadIdx.x & 31;
+    const float* lm = p.local_mask + (size_t)b * p.L;
+    bool w_ = false, pd = false;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const int i = r0 + lane + 32 * k;
+        if (i < p.L && i >= g) {
+            const bool tok = lm[i] == 1.0f;
+            w_ |= tok;
+            pd |= !tok;
+        }
     }
-    const int lo = it.r0 - p.w;
-    bl.band_lo = lo <= 0 ? 0 : lo / kBN;
-    const int hi = min(p.NKB - 1, (it.r0 + kBM - 1 + p.w) / kBN);
-    bl.glob_hi = min((g + kBN - 1) / kBN, bl.band_lo);
-    bl.n = bl.glob_hi + hi - bl.band_lo + 1;
-    return bl;
+    work = __any_sync(0xffffffffu, w_);
+    padded = __any_sync(0xffffffffu, pd);
 }
 
-__device__ __forceinline__ int block_at(const Blocks& bl, int n) {
-    return n < bl.glob_hi ? n : bl.band_lo + (n - bl.glob_hi);
+// Whole warp: the item's plan (identical in every role).
+__device__ Plan make_plan(const Params& p, int id, int& cached_b, int& g) {
+    Plan pl;
+    pl.id = id;
+    if (id >= p.n_band) {
+        const int id2 = id - p.n_band;
+        pl.global = 1;
+        const int sp = id2 % p.NSP;
+        const int r = id2 / p.NSP;
+        pl.rt = r % p.RT;
+        pl.bh = r / p.RT;
+        pl.t[0].split = 2 * sp;
+        pl.t[1].split = 2 * sp + 1;
+    } else {
+        pl.global = 0;
+        pl.rt = 0;
+        const int tp = id % p.NTP;
+        pl.bh = id / p.NTP;
+        pl.t[0].r0 = 2 * tp * kBM;
+        pl.t[1].r0 = (2 * tp + 1) * kBM;
+    }
+    pl.b = pl.bh / p.H;
+    pl.h = pl.bh % p.H;
+    if (pl.b != cached_b) {
+        g = leading_globals(p, pl.b);
+        cached_b = pl.b;
+    }
+    pl.g = g;
+    pl.nloads = 0;
+    pl.e1 = 0;
+    pl.lo_min = 0;
+    pl.zero_only[0] = pl.zero_only[1] = 0;
+    for (int x = 0; x < 2; ++x) {
+        pl.t[x].present = 0;
+        pl.t[x].glob_hi = pl.t[x].lo = 0;
+        pl.t[x].hi = -1;
+    }
+    if (g > p.w) return pl;  // invalid sample: zero output only
+    if (pl.global) {
+        const int r0 = pl.rt * kBM;
+        for (int x = 0; x < 2; ++x) {
+            Tile& t = pl.t[x];
+            t.r0 = r0;
+            if (r0 < g && t.split < p.NS) {
+                t.present = 1;
+                t.lo = t.split * kChunkBlocks;
+                t.hi = min(p.NKB, t.lo + kChunkBlocks) - 1;
+            }
+        }
+        const int nA = pl.t[0].present ? pl.t[0].hi - pl.t[0].lo + 1 : 0;
+        const int nB = pl.t[1].present ? pl.t[1].hi - pl.t[1].lo + 1 : 0;
+        pl.nloads = nA + nB;
+        return pl;
+    }
+    int G = 0, lo_min = 1 << 30, hi_max = -1;
+    for (int x = 0; x < 2; ++x) {
+        Tile& t = pl.t[x];
+        t.split = 0;
+        if (t.r0 >= p.L) continue;
+        int work, padded;
+        band_rows(p, pl.b, t.r0, g, work, padded);
+        if (!work) {
+            pl.zero_only[x] = padded;
+            continue;
+        }
+        t.present = 1;
+        const int lo = t.r0 - p.w;
+        t.lo = lo <= 0 ? 0 : lo / kBN;
+        t.hi = min(p.NKB - 1, (t.r0 + kBM - 1 + p.w) / kBN);
+        t.glob_hi = min((g + kBN - 1) / kBN, t.lo);
+        G = max(G, t.glob_hi);
+        lo_min = min(lo_min, t.lo);
+        hi_max = max(hi_max, t.hi);
+    }
+    if (hi_max < 0) return pl;
+    pl.e1 = min(G, lo_min);
+    pl.lo_min = lo_min;
+    pl.nloads = pl.e1 + (hi_max - lo_min + 1);
+    return pl;
+}
+
+__device__ __forceinline__ void load_at(const Plan& pl, int q, int& kb, int& needA, int& needB) {
+    if (pl.global) {
+        const int nA = pl.t[0].present ? pl.t[0].hi - pl.t[0].lo + 1 : 0;
+        const int nB = pl.t[1].present ? pl.t[1].hi - pl.t[1].lo + 1 : 0;
+        const int m = min(nA, nB);
+        int x, idx;
+        if (q < 2 * m) {
+            x = q & 1;
+            idx = q >> 1;
+        } else {
+            x = nA > nB ? 0 : 1;
+            idx = m + (q - 2 * m);
+        }
+        kb = pl.t[x].lo + idx;
+        needA = x == 0;
+        needB = x == 1;
+        return;
+    }
+    kb = q < pl.e1 ? q : pl.lo_min + (q - pl.e1);
+    const Tile& A = pl.t[0];
+    const Tile& Bt = pl.t[1];
+    needA = A.present && (kb < A.glob_hi || (kb >= A.lo && kb <= A.hi));
+    needB = Bt.present && (kb < Bt.glob_hi || (kb >= Bt.lo && kb <= Bt.hi));
 }
 
 template <typename T>
@@ -196,6 +365,131 @@ __device__ __forceinline__ void store_zero_row(void* out_base, size_t elem_off, 
     for (int c = 0; c < 8; ++c) dst[c] = make_uint4(0, 0, 0, 0);
 }
 
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
+}
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+}
+// Same as tmem_ld32 into float registers (bit patterns are kept).
+__device__ __forceinline__ void tmem_ld32f(uint32_t taddr, float (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=f"(r[0]), "=f"(r[1]), "=f"(r[2]), "=f"(r[3]), "=f"(r[4]), "=f"(r[5]), "=f"(r[6]), "=f"(r[7]),
+          "=f"(r[8]), "=f"(r[9]), "=f"(r[10]), "=f"(r[11]), "=f"(r[12]), "=f"(r[13]), "=f"(r[14]), "=f"(r[15]),
+          "=f"(r[16]), "=f"(r[17]), "=f"(r[18]), "=f"(r[19]), "=f"(r[20]), "=f"(r[21]), "=f"(r[22]), "=f"(r[23]),
+          "=f"(r[24]), "=f"(r[25]), "=f"(r[26]), "=f"(r[27]), "=f"(r[28]), "=f"(r[29]), "=f"(r[30]), "=f"(r[31])
+        : "r"(taddr));
+}
+__device__ __forceinline__ float fast_rcp(float x) {
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
+        "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
+        "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+        : "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// D[tmem] (+)= A[tmem] * B[smem desc], kind::f16.
+__device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                           uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+template <uint32_t N>
+__device__ __forceinline__ void regs_dec() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void regs_inc() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+__device__ __forceinline__ float max3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+enum : int { kSkip = 0, kFull = 1, kPart = 2 };
+
+// Packed fp32 pair arithmetic (fma.rn.f32x2 / add.f32x2, sm_100).
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+        "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return d;
+}
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "add.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+
+// 2^x for a pair on the FMA/ALU pipes, to take load off the MUFU unit
+// (16 results per clock per SM).  Cody-Waite reduction x = n + f with
+// n = round(x) (|f| <= 1/2, via the 1.5 * 2^23 rounding constant), then a
+// cubic for 2^f whose coefficients were fitted for this kernel by iteratively
+// reweighted least squares (Lawson) on Chebyshev nodes of [-1/2, 1/2]
+// (max relative error 7.5e-5, below the rounding of P to fp16/bf16); the
+// exponent n is added to the bits of the result.  x is clamped at -126 so the
+// result stays a normal number (2^-126 rounds to 0 in fp16).
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+    const float2 t = make_float2(fmaxf(x.x, -126.0f), fmaxf(x.y, -126.0f));
+    const float2 rnd = make_float2(12582912.0f, 12582912.0f);
+    const float2 j = fadd2(t, rnd);                                       // n in the low mantissa bits
+    const float2 nf = fadd2(j, make_float2(-12582912.0f, -12582912.0f));  // n as a float
+    const float2 f = ffma2(nf, make_float2(-1.0f, -1.0f), t);             // t - n, exact
+    float2 q = ffma2(make_float2(0.0551716648f, 0.0551716648f), f, make_float2(0.2426111251f, 0.2426111251f));
+    q = ffma2(q, f, make_float2(0.6932609677f, 0.6932609677f));
+    q = ffma2(q, f, make_float2(0.9999280572f, 0.9999280572f));
+    return make_float2(__uint_as_float(__float_as_uint(q.x) + (__float_as_uint(j.x) << 23)),
+                       __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(j.y) << 23)));
+}
+
+// Bits 0..n-1 set (n clamped to [0, 32]).
+__device__ __forceinline__ uint32_t low_bits(int n) {
+    n = min(max(n, 0), 32);
+    return (uint32_t)((1ull << n) - 1ull);
+}
+// Bits lo..hi set (inclusive, clamped to [0, 31]; empty when lo > hi).
+__device__ __forceinline__ uint32_t range_bits(int lo, int hi) {
+    return low_bits(hi + 1) & ~low_bits(lo);
+}
+
 template <typename T>
 __global__ void __launch_bounds__(kThreads, 1)
 attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Params p) {
@@ -205,12 +499,17 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
     uint64_t* q_full = bars + 0;
     uint64_t* q_empty = bars + 2;
     uint64_t* kv_full = bars + 4;
-    uint64_t* kv_empty = bars + 4 + kStages;
-    uint64_t* s_full = bars + 4 + 2 * kStages;
-    uint64_t* p_full = s_full + 2;
-    uint64_t* pv_full = p_full + 2;
-    uint64_t* pv_free = pv_full + 2;
-    uint64_t* drain = pv_free + 2;
+    uint64_t* kv_empty = kv_full + kStages;
+    uint64_t* s_full = kv_empty + kStages;  // [tile]
+    uint64_t* p_full = s_full + 2;          // [tile]
+    uint64_t* o_done = p_full + 2;          // [tile]
+    uint64_t* o_free = o_done + 2;          // [tile]
+    uint64_t* item_full = o_free + 2;       // [kRing]
+    uint64_t* item_empty = item_full + kRing;
+    uint64_t* drain = item_empty + kRing;
+    uint64_t* tma_done = drain + 1;  // the TMA warp finished issuing an item's loads
+    Plan* plans = reinterpret_cast<Plan*>(smem + kOffPlans);
+    static_assert(sizeof(Plan) <= 128, "plan slot");
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
 
@@ -222,14 +521,19 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
             mbar_init(&q_empty[i], 1);
             mbar_init(&s_full[i], 1);
             mbar_init(&p_full[i], 4);
-            mbar_init(&pv_full[i], 1);
-            mbar_init(&pv_free[i], 4);
+            mbar_init(&o_done[i], 1);
+            mbar_init(&o_free[i], 4);
         }
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&kv_full[s], 1);
             mbar_init(&kv_empty[s], 1);
         }
+        for (int s = 0; s < kRing; ++s) {
+            mbar_init(&item_full[s], 1);
+            mbar_init(&item_empty[s], kItemConsumers);
+        }
         mbar_init(drain, 1);
+        mbar_init(tma_done, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -249,319 +553,574 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    if (threadIdx.x == 0) TRACE(11, 1, 0, 0, 0);
 
+    if (warp < kSoftmaxWarp0) {
+    regs_dec<kRegsProducer>();
     if (warp == 0) {
-        // ------------------------------------------------------------ TMA producer
+        // ------------------------------------------------------------ scheduler + TMA producer
+        TDECL;
         uint32_t kv_cnt = 0, item_cnt = 0;
-        int cached_b = -1, g = 0;
         bool ok = true;
-        for (int id = blockIdx.x; id < p.n_items && ok; id += gridDim.x) {
-            const Item it = decode_item(p, id);
-            if (it.b != cached_b) {
-                g = leading_globals(p, it.b);
-                cached_b = it.b;
+        for (uint32_t k = 0; ok; ++k) {
+            const uint32_t slot = k % kRing;
+            if (lane == 0) TIMED(0, ok = mbar_wait(&item_full[slot], (k / kRing) & 1, abort_flag));
+            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+            if (!ok) break;
+            __syncwarp();                 // lane 0's acquire orders the reads below
+            const Plan pl = plans[slot];  // published by the planner before item_full
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&item_empty[slot]);
+            const int id = pl.id;
+            if (id < 0) break;
+            if (pl.nloads == 0) {
+                if (lane == 0) mbar_arrive(tma_done);
+                continue;
             }
-            const Blocks bl = block_list(p, it, g);
-            if (bl.n == 0) continue;
             if (lane == 0) {
                 const uint32_t qb = item_cnt & 1;
-                ok = mbar_wait(&q_empty[qb], ((item_cnt >> 1) & 1) ^ 1, abort_flag);
+                TRACE(0, 12, id, item_cnt, 0);
+                TIMED(2, ok = mbar_wait(&q_empty[qb], ((item_cnt >> 1) & 1) ^ 1, abort_flag));
                 if (ok) {
-                    mbar_arrive_expect_tx(&q_full[qb], kTileBytes);
-                    tma_load_3d(smem + kOffQ + qb * kTileBytes, it.global ? &maps.qg : &maps.q, &q_full[qb], 0,
-                                it.r0, it.bh);
+                    const int nq = pl.t[0].present + pl.t[1].present;
+                    mbar_arrive_expect_tx(&q_full[qb], nq * kTileBytes);
+                    for (int x = 0; x < 2; ++x)
+                        if (pl.t[x].present)
+                            tma_load_3d(smem + kOffQ + (qb * 2 + x) * kTileBytes, pl.global ? &maps.qg : &maps.q,
+                                        &q_full[qb], 0, pl.t[x].r0, pl.bh);
                 }
-                for (int n = 0; n < bl.n && ok; ++n) {
+                for (int q = 0; q < pl.nloads && ok; ++q) {
+                    int kb, nA, nB;
+                    load_at(pl, q, kb, nA, nB);
+                    if (!nA && !nB) continue;
                     const uint32_t st = kv_cnt % kStages;
-                    ok = mbar_wait(&kv_empty[st], ((kv_cnt / kStages) & 1) ^ 1, abort_flag);
+                    TRACE(0, 13, id, q, kv_cnt);
+                    TIMED(3, ok = mbar_wait(&kv_empty[st], ((kv_cnt / kStages) & 1) ^ 1, abort_flag));
                     if (!ok) break;
-                    const int kb = block_at(bl, n);
                     mbar_arrive_expect_tx(&kv_full[st], 2 * kTileBytes);
-                    tma_load_3d(smem + kOffK + st * kTileBytes, it.global ? &maps.kg : &maps.k, &kv_full[st], 0,
-                                kb * kBN, it.bh);
-                    tma_load_3d(smem + kOffV + st * kTileBytes, it.global ? &maps.vg : &maps.v, &kv_full[st], 0,
-                                kb * kBN, it.bh);
+                    tma_load_3d(smem + kOffK + st * kTileBytes, pl.global ? &maps.kg : &maps.k, &kv_full[st], 0,
+                                kb * kBN, pl.bh);
+                    tma_load_3d(smem + kOffV + st * kTileBytes, pl.global ? &maps.vg : &maps.v, &kv_full[st], 0,
+                                kb * kBN, pl.bh);
                     ++kv_cnt;
                 }
+                if (ok) mbar_arrive(tma_done);
             }
             ++item_cnt;
             ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
         }
-        // Wind-down: let issued copies land before the CTA can exit.
-        if (lane == 0 && !ok) {
+        if (lane == 0) TRACE(0, 19, ok ? 1 : 0, item_cnt, kv_cnt);
+        if (lane == 0) TDUMP(0);
+        if (lane == 0 && !ok) {  // wind-down: let issued copies land
             for (uint32_t c = (kv_cnt > kStages ? kv_cnt - kStages : 0); c < kv_cnt; ++c) {
                 volatile int never = 0;
                 mbar_wait(&kv_full[c % kStages], (c / kStages) & 1, &never, 200000000ull);
             }
         }
+    } else if (warp == 2) {
+        // ------------------------------------------------------------ planner
+        // Takes items from the global counter, works out each item's plan
+        // (reads of the masks included) once and publishes it through the
+        // ring, running up to kRing items ahead of the other roles.
+        int cached_b = -1, g = 0;
+        bool ok = true;
+        for (uint32_t k = 0; ok; ++k) {
+            const uint32_t slot = k % kRing;
+            int id = -1;
+            if (lane == 0) {
+                // Take item k only once the TMA warp has issued every load of
+                // item k-1: a CTA holds at most one item in reserve, taken a
+                // few K/V stages before it is needed, so items are not hoarded
+                // by early CTAs while others idle.
+                if (k > 0) ok = mbar_wait(tma_done, (k - 1) & 1, abort_flag);
+                if (ok) ok = mbar_wait(&item_empty[slot], ((k / kRing) & 1) ^ 1, abort_flag);
+                if (ok) {
+                    id = atomicAdd(p.sched, 1);
+                    if (id >= p.n_items) id = -1;
+                }
+            }
+            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+            id = __shfl_sync(0xffffffffu, id, 0);
+            if (!ok) break;
+            Plan pl;
+            if (id >= 0) pl = make_plan(p, id, cached_b, g);
+            else pl.id = -1;
+            if (lane == 0) {
+                plans[slot] = pl;
+                mbar_arrive(&item_full[slot]);
+            }
+            if (id < 0) break;
+        }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         constexpr uint32_t idesc_qk = idesc_f16(Pack<T>::fmt, kBM, kBN, 0, 0);
         constexpr uint32_t idesc_pv = idesc_f16(Pack<T>::fmt, kBM, kHD, 0, 1);
-        uint32_t kv_cnt = 0, blk = 0, item_cnt = 0;
-        int cached_b = -1, g = 0;
+        uint32_t kv_cnt = 0, item_cnt = 0;
+        TDECL;
+        uint32_t pcnt[2] = {0, 0};   // P blocks consumed per tile
+        uint32_t icnt[2] = {0, 0};   // items with work per tile
         bool ok = true;
-        for (int id = blockIdx.x; id < p.n_items && ok; id += gridDim.x) {
-            const Item it = decode_item(p, id);
-            if (it.b != cached_b) {
-                g = leading_globals(p, it.b);
-                cached_b = it.b;
+        for (uint32_t k = 0; ok; ++k) {
+            const uint32_t slot = k % kRing;
+            if (lane == 0) {
+                TRACE(warp == 1 ? 1 : 2 + warp - kSoftmaxWarp0, warp == 1 ? 20 : 30, k, 0, 0);
+                TIMED(0, ok = mbar_wait(&item_full[slot], (k / kRing) & 1, abort_flag));
             }
-            const Blocks bl = block_list(p, it, g);
-            if (bl.n == 0) continue;
+            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+            if (!ok) break;
+            __syncwarp();                 // lane 0's acquire orders the reads below
+            const Plan pl = plans[slot];  // published by the producer before item_full
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&item_empty[slot]);
+            const int id = pl.id;
+            if (id < 0) break;
+            const int g = pl.g;
+            if (pl.nloads == 0) continue;
             if (lane == 0) {
                 const uint32_t qb = item_cnt & 1;
-                ok = mbar_wait(&q_full[qb], (item_cnt >> 1) & 1, abort_flag);
+                TRACE(1, 22, id, item_cnt, 0);
+                TIMED(2, ok = mbar_wait(&q_full[qb], (item_cnt >> 1) & 1, abort_flag));
                 tc_fence_after();
-                const uint32_t q_addr = smem_u32(smem + kOffQ + qb * kTileBytes);
-                uint32_t prev_st = 0;
-                for (int n = 0; n <= bl.n && ok; ++n) {
-                    uint32_t st = 0;
-                    if (n < bl.n) {
-                        st = kv_cnt % kStages;
-                        ok = mbar_wait(&kv_full[st], (kv_cnt / kStages) & 1, abort_flag);
+                int pend[2] = {-1, -1};
+                bool first[2] = {true, true};
+                int refc[kStages];
+#pragma unroll
+                for (int s = 0; s < kStages; ++s) refc[s] = 0;
+                // O_X += P_X V[st]; releases the stage when its last user is done.
+                auto issue_pv = [&](int x, int st) -> bool {
+                    TRACE(1, 24, id, x, pcnt[x]);
+                    bool w_ok;
+                    TIMED(4, w_ok = mbar_wait(&p_full[x], pcnt[x] & 1, abort_flag));
+                    if (!w_ok) return false;
+                    ++pcnt[x];
+                    TRACE(1, 25, id, x, icnt[x]);
+                    if (first[x]) {
+                        TIMED(5, w_ok = mbar_wait(&o_free[x], (icnt[x] & 1) ^ 1, abort_flag));
+                        if (!w_ok) return false;
+                    }
+                    tc_fence_after();
+                    const uint32_t v_addr = smem_u32(smem + kOffV + st * kTileBytes);
+#pragma unroll
+                    for (int kk = 0; kk < kBN / 16; ++kk)
+                        mma_f16_ts(tmem + kTmemO + x * kHD, tmem + x * kBN + kk * 8, desc_sw128(v_addr + kk * 2048, 0),
+                                   idesc_pv, (first[x] && kk == 0) ? 0u : 1u);
+                    first[x] = false;
+                    if (--refc[st] == 0) tc_commit(&kv_empty[st]);
+                    return true;
+                };
+                for (int q = 0; q < pl.nloads && ok; ++q) {
+                    int kb, need[2];
+                    load_at(pl, q, kb, need[0], need[1]);
+                    if (!need[0] && !need[1]) continue;
+                    const int st = kv_cnt % kStages;
+                    TRACE(1, 23, id, q, kv_cnt);
+                    TIMED(3, ok = mbar_wait(&kv_full[st], (kv_cnt / kStages) & 1, abort_flag));
+                    if (!ok) break;
+                    tc_fence_after();
+                    refc[st] = need[0] + need[1];
+                    const uint32_t k_addr = smem_u32(smem + kOffK + st * kTileBytes);
+                    for (int x = 0; x < 2 && ok; ++x) {
+                        if (!need[x]) continue;
+                        if (pend[x] >= 0) ok = issue_pv(x, pend[x]);
                         if (!ok) break;
-                        tc_fence_after();
-                        const uint32_t sb = (blk + n) & 1;
-                        const uint32_t k_addr = smem_u32(smem + kOffK + st * kTileBytes);
+                        const uint32_t q_addr = smem_u32(smem + kOffQ + (qb * 2 + x) * kTileBytes);
 #pragma unroll
                         for (int kk = 0; kk < kHD / 16; ++kk)
-                            mma_f16_ss(tmem + kTmemS + sb * kBN, desc_sw128(q_addr + kk * 32),
-                                       desc_sw128(k_addr + kk * 32), idesc_qk, kk > 0);
-                        tc_commit(&s_full[sb]);
-                        if (n == bl.n - 1) tc_commit(&q_empty[qb]);
+                            mma_f16_ss(tmem + x * kBN, desc_sw128(q_addr + kk * 32), desc_sw128(k_addr + kk * 32),
+                                       idesc_qk, kk > 0);
+                        tc_commit(&s_full[x]);
+                        pend[x] = st;
                     }
-                    if (n >= 1) {
-                        const uint32_t j = blk + n - 1;
-                        const uint32_t pb = j & 1;
-                        ok = mbar_wait(&p_full[pb], (j >> 1) & 1, abort_flag);
-                        if (ok) ok = mbar_wait(&pv_free[pb], ((j >> 1) & 1) ^ 1, abort_flag);
-                        if (!ok) break;
-                        tc_fence_after();
-                        const uint32_t p_addr = smem_u32(smem + kOffP + pb * kPBytes);
-                        const uint32_t v_addr = smem_u32(smem + kOffV + prev_st * kTileBytes);
-#pragma unroll
-                        for (int kk = 0; kk < kBN / 16; ++kk)
-                            mma_f16_ss(tmem + kTmemPV + pb * kHD,
-                                       desc_sw128(p_addr + (kk >> 2) * (kBM * 128) + (kk & 3) * 32),
-                                       desc_sw128(v_addr + kk * 2048, 0), idesc_pv, kk > 0);
-                        tc_commit(&pv_full[pb]);
-                        tc_commit(&kv_empty[prev_st]);
-                    }
-                    if (n < bl.n) {
-                        prev_st = st;
-                        ++kv_cnt;
-                    }
+                    ++kv_cnt;
                 }
+                for (int x = 0; x < 2 && ok; ++x) {
+                    if (pend[x] < 0) continue;
+                    ok = issue_pv(x, pend[x]);
+                    if (ok) tc_commit(&o_done[x]);
+                }
+                tc_commit(&q_empty[qb]);
+                for (int x = 0; x < 2; ++x)
+                    if (pl.t[x].present) ++icnt[x];
             }
-            blk += bl.n;
             ++item_cnt;
             ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
         }
-        // Wind-down after an abort: wait for the MMAs already issued.
-        if (lane == 0 && !ok) {
+        if (lane == 0) TRACE(1, 29, ok ? 1 : 0, item_cnt, kv_cnt);
+        if (lane == 0) TDUMP(1);
+        if (lane == 0 && !ok) {  // wind-down: wait for the MMAs already issued
             tc_commit(drain);
             volatile int never = 0;
             mbar_wait(drain, 0, &never, 200000000ull);
         }
+    }
     } else {
-        // ------------------------------------------------------------ softmax / epilogue
-        const int sp = warp & 3;            // TMEM sub-partition of this warp
-        const int r = sp * 32 + lane;       // query row within the tile
+        regs_inc<kRegsSoftmax>();
+        // ------------------------------------------------------------ softmax / epilogue warps
+        const int x = (warp - kSoftmaxWarp0) >> 2;  // tile handled by this warpgroup
+        const int sp = warp & 3;           // TMEM sub-partition (rows sp*32 .. +31)
+        const int r = sp * 32 + lane;      // query row within the tile
         const uint32_t lane_off = (uint32_t)(sp * 32) << 16;
-        float* bias_w = reinterpret_cast<float*>(smem + kOffBias) + sp * 2 * kBN;  // this warp's copy
-        uint32_t blk = 0;
-        int cached_b = -1, g = 0;
+        const uint32_t tS = tmem + lane_off + x * kBN;
+        const uint32_t tO = tmem + lane_off + kTmemO + x * kHD;
+        float* bias_w = reinterpret_cast<float*>(smem + kOffBias) + (warp - kSoftmaxWarp0) * kBN;
+        TDECL;
+        uint32_t scnt = 0, icnt = 0;
         bool ok = true;
-        for (int id = blockIdx.x; id < p.n_items && ok; id += gridDim.x) {
-            const Item it = decode_item(p, id);
-            if (it.b != cached_b) {
-                g = leading_globals(p, it.b);
-                cached_b = it.b;
+        for (uint32_t k = 0; ok; ++k) {
+            const uint32_t slot = k % kRing;
+            if (lane == 0) {
+                TRACE(warp == 1 ? 1 : 2 + warp - kSoftmaxWarp0, warp == 1 ? 20 : 30, k, 0, 0);
+                TIMED(0, ok = mbar_wait(&item_full[slot], (k / kRing) & 1, abort_flag));
             }
-            const float* lm = p.local_mask + (size_t)it.b * p.L;
-            const int i = it.r0 + r;
-            if (g > p.w) {  // invalid sample: zero output, record once
-                if (!it.global) {
-                    if (i < p.L) store_zero_row(p.out, ((size_t)(it.b * p.L + i) * p.H + it.h) * kHD, sizeof(T));
-                    if (r == 0 && it.tile == 0 && it.h == 0) record_status(p.status, it.b, LF_ERR_G_GT_W);
+            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+            if (!ok) break;
+            __syncwarp();                 // lane 0's acquire orders the reads below
+            const Plan pl = plans[slot];  // published by the producer before item_full
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&item_empty[slot]);
+            const int id = pl.id;
+            if (id < 0) break;
+            const int g = pl.g;
+            const Tile& me = pl.t[x];
+            const float* lm = p.local_mask + (size_t)pl.b * p.L;
+            const int i = me.r0 + r;
+            if (!pl.global) {
+                if (g > p.w) {  // invalid sample: zero output, record once
+                    if (me.r0 < p.L && i < p.L)
+                        store_zero_row(p.out, ((size_t)(pl.b * p.L + i) * p.H + pl.h) * kHD, sizeof(T));
+                    if (x == 0 && r == 0 && me.r0 == 0 && pl.h == 0) record_status(p.status, pl.b, LF_ERR_G_GT_W);
+                    continue;
                 }
-                continue;
+                if (me.r0 < p.L && i < p.L && i >= g && p.global_mask[(size_t)pl.b * p.L + i] == 0.0f)
+                    record_status(p.status, pl.b, LF_ERR_GLOBAL_NOT_PREFIX);
+                if (pl.zero_only[x]) {
+                    if (i < p.L && i >= g && lm[i] != 1.0f)
+                        store_zero_row(p.out, ((size_t)(pl.b * p.L + i) * p.H + pl.h) * kHD, sizeof(T));
+                    continue;
+                }
             }
-            const Blocks bl = block_list(p, it, g);
-            if (bl.n == 0) continue;
-            if (!it.global && i < p.L && i >= g && p.global_mask[(size_t)it.b * p.L + i] == 0.0f)
-                record_status(p.status, it.b, LF_ERR_GLOBAL_NOT_PREFIX);
+            if (!me.present) continue;
+            // This tile's key blocks in load order: [0, glob_hi) then lo..hi.
+            // Only these few scalars stay live through the block loop.
+            const int is_global = pl.global;
+            const int nblk = me.glob_hi + (me.hi - me.lo + 1);
+            const int blk_gh = me.glob_hi, blk_lo = me.lo;
+            const int pb = pl.b, ph = pl.h, pbh = pl.bh, prt = pl.rt, psplit = me.split;
 
-            float o[kHD];
-#pragma unroll
-            for (int c = 0; c < kHD; ++c) o[c] = 0.0f;
-            float m_run = -INFINITY, l_run = 0.0f, a_prev = 0.0f;
+            // Does this warp have rows whose output is kept?
+            const int wr0 = me.r0 + sp * 32;
+            const bool row_kept = is_global ? (i < g && lm[i] == 1.0f) : (i < p.L && i >= g && lm[i] == 1.0f);
+            const bool warp_active = __any_sync(0xffffffffu, row_kept);
 
-            for (int n = 0; n <= bl.n && ok; ++n) {
-                float a_cur = 0.0f;
-                if (n < bl.n) {
-                    const uint32_t j = blk + n;
-                    const uint32_t sb = j & 1;
-                    const int kb = block_at(bl, n);
-                    const int c0 = kb * kBN;
+            float m_used = -INFINITY, l_run = 0.0f;
+            bool first = true;
+            // local_mask of the next block's keys, loaded one block ahead so
+            // that the load latency is off the critical path
+            float mv_next[4] = {1.0f, 1.0f, 1.0f, 1.0f};
+            auto load_mv = [&](int n2) {
+                const int c2 = (n2 < blk_gh ? n2 : blk_lo + (n2 - blk_gh)) * kBN;
 #pragma unroll
-                    for (int t = 0; t < kBN / 32; ++t) {
-                        const int key = c0 + t * 32 + lane;
-                        bias_w[sb * kBN + t * 32 + lane] =
-                            key < p.L ? fmaf(lm[key], 10000.0f, -10000.0f) * kLog2e : -INFINITY;
+                for (int t = 0; t < 4; ++t) {
+                    const int key = c2 + t * 32 + lane;
+                    mv_next[t] = key < p.L ? lm[key] : 1.0f;
+                }
+            };
+            if (warp_active && nblk > 0) load_mv(0);
+            for (int n = 0; n < nblk && ok; ++n) {
+                const int kb = n < blk_gh ? n : blk_lo + (n - blk_gh);
+                const int c0 = kb * kBN;
+                // Padding bias of the block's keys (keys >= L are masked instead).
+                bool has_pad = false;
+                if (warp_active) {
+                    float mv[4];
+#pragma unroll
+                    for (int t = 0; t < 4; ++t) mv[t] = mv_next[t];
+                    if (n + 1 < nblk) load_mv(n + 1);
+                    const bool pad = mv[0] != 1.0f || mv[1] != 1.0f || mv[2] != 1.0f || mv[3] != 1.0f;
+                    has_pad = __any_sync(0xffffffffu, pad);
+                    if (has_pad) {
+#pragma unroll
+                        for (int t = 0; t < 4; ++t) bias_w[t * 32 + lane] = fmaf(mv[t], 10000.0f, -10000.0f) * p.inv_scale;
                     }
                     __syncwarp();
-                    ok = mbar_wait(&s_full[sb], (j >> 1) & 1, abort_flag);
-                    if (!ok) break;
-                    tc_fence_after();
-
-                    // Mask geometry for this row and block.
-                    const int d0 = it.r0 + r - c0;           // i - c0
-                    const bool full = it.global ||
-                                      (max(it.r0 + kBM - 1 - c0, c0 + kBN - 1 - it.r0) <= p.w);
-                    const int lo_c = d0 - p.w, hi_c = d0 + p.w, gl_c = g - c0;
-
-                    float x[kBN];
-                    const float* bias = bias_w + sb * kBN;
-#pragma unroll
-                    for (int ch = 0; ch < kBN / 32; ++ch) {
-                        uint32_t raw[32];
-                        tmem_ld32(tmem + lane_off + kTmemS + sb * kBN + ch * 32, raw);
-                        tmem_ld_wait();
-#pragma unroll
-                        for (int c = 0; c < 32; ++c) {
-                            const int cc = ch * 32 + c;
-                            float v = fmaf(__uint_as_float(raw[c]), p.scale_log2, bias[cc]);
-                            if (!full) {
-                                const bool allowed = (cc < gl_c) || (cc >= lo_c && cc <= hi_c);
-                                v = allowed ? v : -INFINITY;
-                            }
-                            x[cc] = v;
-                        }
-                    }
-                    float mb = -INFINITY;
-#pragma unroll
-                    for (int c = 0; c < kBN; ++c) mb = fmaxf(mb, x[c]);
-                    const float m_new = fmaxf(m_run, mb);
-                    const float m_use = m_new == -INFINITY ? 0.0f : m_new;
-                    a_cur = ex2(m_run - m_use);
-                    float sum = 0.0f;
-                    uint8_t* pbuf = smem + kOffP + sb * kPBytes;
-#pragma unroll
-                    for (int chunk = 0; chunk < kBN / 8; ++chunk) {
-                        float e[8];
-#pragma unroll
-                        for (int t = 0; t < 8; ++t) {
-                            e[t] = ex2(x[chunk * 8 + t] - m_use);
-                            sum += e[t];
-                        }
-                        uint4 u;
-                        u.x = Pack<T>::two(e[0], e[1]);
-                        u.y = Pack<T>::two(e[2], e[3]);
-                        u.z = Pack<T>::two(e[4], e[5]);
-                        u.w = Pack<T>::two(e[6], e[7]);
-                        const int atom = chunk >> 3, cidx = chunk & 7;
-                        *reinterpret_cast<uint4*>(pbuf + atom * (kBM * 128) + r * 128 + ((cidx ^ (r & 7)) << 4)) = u;
-                    }
-                    l_run = l_run * a_cur + sum;
-                    m_run = m_new;
-                    fence_proxy_async_smem();
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&p_full[sb]);
                 }
-                if (n >= 1) {
-                    const uint32_t j = blk + n - 1;
-                    const uint32_t pb = j & 1;
-                    ok = mbar_wait(&pv_full[pb], (j >> 1) & 1, abort_flag);
-                    if (!ok) break;
-                    tc_fence_after();
-                    uint32_t pv0[32], pv1[32];
-                    tmem_ld32(tmem + lane_off + kTmemPV + pb * kHD, pv0);
-                    tmem_ld32(tmem + lane_off + kTmemPV + pb * kHD + 32, pv1);
+                if (lane == 0) TRACE(2 + warp - kSoftmaxWarp0, 32, id, n, scnt);
+                // every lane waits; the result is made warp-uniform so that an
+                // abort never splits the warp before a .sync.aligned instruction
+                TIMED(2, ok = __all_sync(0xffffffffu, mbar_wait(&s_full[x], scnt & 1, abort_flag)));
+                const long long tc0_ = clock64();
+                ++scnt;
+                if (!ok) break;
+                tc_fence_after();
+                if (warp_active) {
+                    // Chunk states (warp-uniform): skip / full / masked.
+                    int state[4];
+#pragma unroll
+                    for (int ch = 0; ch < 4; ++ch) {
+                        const int cj0 = c0 + ch * 32;
+                        int s;
+                        if (cj0 >= p.L) {
+                            s = kSkip;
+                        } else if (is_global) {
+                            s = (cj0 + 31 < p.L) ? kFull : kPart;
+                        } else {
+                            const bool any_g = cj0 < g;
+                            const bool all_g = cj0 + 31 < g;
+                            const bool overlap = cj0 <= wr0 + 31 + p.w && cj0 + 31 >= wr0 - p.w;
+                            const bool inside = (wr0 + 31 - cj0 <= p.w) && (cj0 + 31 - wr0 <= p.w);
+                            if (!any_g && !overlap) s = kSkip;
+                            else if ((all_g || inside) && cj0 + 31 < p.L) s = kFull;
+                            else s = kPart;
+                        }
+                        state[ch] = s;
+                    }
+                    // All TMEM loads of the block first, one wait: the load
+                    // latency is paid once per block, not once per chunk.
+                    float xv[kBN];
+#pragma unroll
+                    for (int ch = 0; ch < 4; ++ch) {
+                        if (state[ch] == kSkip) continue;
+                        tmem_ld32f(tS + ch * 32, *reinterpret_cast<float(*)[32]>(&xv[ch * 32]));
+                    }
                     tmem_ld_wait();
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&pv_free[pb]);
+#if LF_TRACE
+                    const long long ts1_ = clock64();
+                    tacc[6] += ts1_ - tc0_;
+#endif
+                    // Raw scores (+ padding bias in raw units), mask; row max with
+                    // four independent accumulators.  The scale is applied once
+                    // to the max and folded into the exponent's FMA below.
+                    const int d0 = i - c0;
+                    const int lo_c = d0 - p.w, hi_c = d0 + p.w, gl_c = g - c0, lim_c = p.L - c0;
+                    float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-                    for (int c = 0; c < 32; ++c) {
-                        o[c] = fmaf(o[c], a_prev, __uint_as_float(pv0[c]));
-                        o[c + 32] = fmaf(o[c + 32], a_prev, __uint_as_float(pv1[c]));
+                    for (int ch = 0; ch < 4; ++ch) {
+                        if (state[ch] == kSkip) continue;
+                        if (has_pad) {
+#pragma unroll
+                            for (int c = 0; c < 32; c += 4) {
+                                const float4 b4 = *reinterpret_cast<const float4*>(bias_w + ch * 32 + c);
+                                xv[ch * 32 + c] += b4.x;
+                                xv[ch * 32 + c + 1] += b4.y;
+                                xv[ch * 32 + c + 2] += b4.z;
+                                xv[ch * 32 + c + 3] += b4.w;
+                            }
+                        }
+                        if (state[ch] == kPart) {
+                            // allowed columns of this row in the chunk as one bit
+                            // mask (no per-element branches)
+                            const int b0 = ch * 32;
+                            uint32_t bits = low_bits(lim_c - b0);
+                            if (!is_global)
+                                bits &= low_bits(gl_c - b0) | range_bits(lo_c - b0, hi_c - b0);
+#pragma unroll
+                            for (int c = 0; c < 32; ++c)
+                                xv[b0 + c] = ((bits >> c) & 1u) ? xv[b0 + c] : -INFINITY;
+                        }
+#pragma unroll
+                        for (int c = 0; c < 32; c += 8) {
+                            mx[0] = max3(mx[0], xv[ch * 32 + c], xv[ch * 32 + c + 1]);
+                            mx[1] = max3(mx[1], xv[ch * 32 + c + 2], xv[ch * 32 + c + 3]);
+                            mx[2] = max3(mx[2], xv[ch * 32 + c + 4], xv[ch * 32 + c + 5]);
+                            mx[3] = max3(mx[3], xv[ch * 32 + c + 6], xv[ch * 32 + c + 7]);
+                        }
                     }
+                    const float mb = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * p.scale_log2;
+#if LF_TRACE
+                    const long long ts2_ = clock64();
+                    tacc[7] += ts2_ - ts1_;
+#endif
+                    // Running max with lazy rescaling of the TMEM accumulator.
+                    // The decision is per row, but tcgen05.ld/st are warp-wide
+                    // (.sync.aligned): the whole warp rescales when any row
+                    // needs it, rows that do not use factor 1.
+                    if (first) {
+                        m_used = mb;
+                    } else {
+                        const bool need = mb > m_used + kRescaleThreshold;
+                        if (__any_sync(0xffffffffu, need)) {
+                            const float factor = !need ? 1.0f : (m_used == -INFINITY ? 0.0f : ex2(m_used - mb));
+                            if (need) {
+                                l_run *= factor;
+                                m_used = mb;
+                            }
+#pragma unroll
+                            for (int c0o = 0; c0o < kHD; c0o += 16) {
+                                uint32_t ob[16];
+                                tmem_ld16(tO + c0o, ob);
+                                tmem_ld_wait();
+#pragma unroll
+                                for (int c = 0; c < 16; ++c)
+                                    ob[c] = __float_as_uint(__uint_as_float(ob[c]) * factor);
+                                tmem_st16(tO + c0o, ob);
+                            }
+                        }
+                    }
+                    const float m_use = m_used == -INFINITY ? 0.0f : m_used;
+#if LF_TRACE
+                    const long long ts3_ = clock64();
+                    tacc[8] += ts3_ - ts2_;
+#endif
+                    // p = 2^(raw * scale_log2 - m): one packed FMA per pair
+                    const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
+                    const float2 nm2 = make_float2(-m_use, -m_use);
+                    float2 sm2[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
+#pragma unroll
+                    for (int ch = 0; ch < 4; ++ch) {
+                        uint32_t pk[16];
+                        if (state[ch] == kSkip) {
+#pragma unroll
+                            for (int c = 0; c < 16; ++c) pk[c] = 0u;
+                        } else {
+#pragma unroll
+                            for (int c = 0; c < 16; ++c) {
+                                const float2 a = ffma2(make_float2(xv[ch * 32 + 2 * c], xv[ch * 32 + 2 * c + 1]), sc2, nm2);
+                                // about a third of the pairs on the FMA pipe, the rest on MUFU
+                                const float2 e = (c % 3 == 2) ? exp2_poly2(a) : make_float2(ex2(a.x), ex2(a.y));
+                                sm2[c & 1] = fadd2(sm2[c & 1], e);
+                                pk[c] = Pack<T>::two(e.x, e.y);
+                            }
+                        }
+                        tmem_st16(tS + ch * 16, pk);
+                    }
+                    l_run += (sm2[0].x + sm2[0].y) + (sm2[1].x + sm2[1].y);
+#if LF_TRACE
+                    const long long ts4_ = clock64();
+                    tacc[9] += ts4_ - ts3_;
+#endif
+                    tmem_st_wait();
+#if LF_TRACE
+                    tacc[10] += clock64() - ts4_;
+#endif
                 }
-                a_prev = a_cur;
+                first = false;
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&p_full[x]);
+#if LF_TRACE
+                tacc[3] += clock64() - tc0_;
+                tacc[4] += 1;
+#endif
             }
             if (!ok) break;
-            blk += bl.n;
 
             // ---------------------------------------------------- epilogue
-            if (!it.global) {
-                if (i < p.L && i >= g) {
-                    const size_t off = ((size_t)(it.b * p.L + i) * p.H + it.h) * kHD;
-                    if (fmaf(lm[i], 10000.0f, -10000.0f) != 0.0f) store_zero_row(p.out, off, sizeof(T));
-                    else store_row<T>(p.out, off, o, 1.0f / l_run);
+            if (lane == 0) TRACE(2 + warp - kSoftmaxWarp0, 33, id, icnt, 0);
+            TIMED(5, ok = __all_sync(0xffffffffu, mbar_wait(&o_done[x], icnt & 1, abort_flag)));
+            ++icnt;
+            if (!ok) break;
+            tc_fence_after();
+            float o[kHD];
+            {
+                uint32_t o0[32], o1[32];
+                tmem_ld32(tO, o0);
+                tmem_ld32(tO + 32, o1);
+                tmem_ld_wait();
+#pragma unroll
+                for (int c = 0; c < 32; ++c) {
+                    o[c] = __uint_as_float(o0[c]);
+                    o[c + 32] = __uint_as_float(o1[c]);
                 }
-            } else if (it.r0 + sp * 32 < g) {
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&o_free[x]);
+
+            if (!is_global) {
+                if (i < p.L && i >= g) {
+                    const size_t off = ((size_t)(pb * p.L + i) * p.H + ph) * kHD;
+                    if (lm[i] != 1.0f) store_zero_row(p.out, off, sizeof(T));
+                    else store_row<T>(p.out, off, o, fast_rcp(l_run));
+                }
+            } else if (wr0 < g) {
                 // Split-KV partials of this warp's 32 rows; the warp that
                 // completes the last split of its row group merges them.
-                const int slot = (it.bh * p.RT + it.tile) * p.NS + it.split;
+                const int slot0 = (pbh * p.RT + prt) * p.NS;
+                const int sl = slot0 + psplit;
                 if (i < g) {
-                    float4* po = reinterpret_cast<float4*>(p.part_o + ((size_t)slot * kBM + r) * kHD);
+                    float4* po = reinterpret_cast<float4*>(p.part_o + ((size_t)sl * kBM + r) * kHD);
 #pragma unroll
                     for (int c = 0; c < kHD / 4; ++c)
                         __stcg(po + c, make_float4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]));
-                    __stcg(reinterpret_cast<float2*>(p.part_ml + ((size_t)slot * kBM + r) * 2),
-                           make_float2(m_run, l_run));
+                    __stcg(reinterpret_cast<float2*>(p.part_ml + ((size_t)sl * kBM + r) * 2),
+                           make_float2(m_used, l_run));
                 }
                 __threadfence();
                 __syncwarp();
-                int* counter = p.counters + (it.bh * p.RT + it.tile) * 4 + sp;
+                int* counter = p.counters + (pbh * p.RT + prt) * 4 + sp;
                 int last = 0;
                 if (lane == 0) last = (atomicAdd(counter, 1) == p.NS - 1) ? 1 : 0;
                 last = __shfl_sync(0xffffffffu, last, 0);
                 if (last) {
                     __threadfence();
                     if (i < g) {
-                        const size_t off = ((size_t)(it.b * p.L + i) * p.H + it.h) * kHD;
-                        if (fmaf(lm[i], 10000.0f, -10000.0f) != 0.0f) {
+                        const size_t off = ((size_t)(pb * p.L + i) * p.H + ph) * kHD;
+                        if (lm[i] != 1.0f) {
                             store_zero_row(p.out, off, sizeof(T));
                         } else {
-                            const int slot0 = (it.bh * p.RT + it.tile) * p.NS;
                             float M = -INFINITY;
                             for (int s = 0; s < p.NS; ++s)
                                 M = fmaxf(M, __ldcg(p.part_ml + ((size_t)(slot0 + s) * kBM + r) * 2));
-                            float acc[kHD];
-#pragma unroll
-                            for (int c = 0; c < kHD; ++c) acc[c] = 0.0f;
                             float lsum = 0.0f;
                             for (int s = 0; s < p.NS; ++s) {
                                 const float2 ml = __ldcg(
                                     reinterpret_cast<const float2*>(p.part_ml + ((size_t)(slot0 + s) * kBM + r) * 2));
-                                const float wgt = ml.x == -INFINITY ? 0.0f : ex2(ml.x - M);
-                                lsum = fmaf(ml.y, wgt, lsum);
-                                const float4* po =
-                                    reinterpret_cast<const float4*>(p.part_o + ((size_t)(slot0 + s) * kBM + r) * kHD);
+                                lsum = fmaf(ml.y, ml.x == -INFINITY ? 0.0f : ex2(ml.x - M), lsum);
+                            }
+                            const float inv = fast_rcp(lsum);
+                            // merge 16 channels at a time to keep registers low
+                            for (int cq = 0; cq < kHD; cq += 16) {
+                                float acc[16];
 #pragma unroll
-                                for (int c = 0; c < kHD / 4; ++c) {
-                                    const float4 t4 = __ldcg(po + c);
-                                    acc[4 * c] = fmaf(t4.x, wgt, acc[4 * c]);
-                                    acc[4 * c + 1] = fmaf(t4.y, wgt, acc[4 * c + 1]);
-                                    acc[4 * c + 2] = fmaf(t4.z, wgt, acc[4 * c + 2]);
-                                    acc[4 * c + 3] = fmaf(t4.w, wgt, acc[4 * c + 3]);
+                                for (int c = 0; c < 16; ++c) acc[c] = 0.0f;
+                                for (int s = 0; s < p.NS; ++s) {
+                                    const float mx = __ldcg(p.part_ml + ((size_t)(slot0 + s) * kBM + r) * 2);
+                                    const float wgt = mx == -INFINITY ? 0.0f : ex2(mx - M);
+                                    const float4* po = reinterpret_cast<const float4*>(
+                                        p.part_o + ((size_t)(slot0 + s) * kBM + r) * kHD + cq);
+#pragma unroll
+                                    for (int c = 0; c < 4; ++c) {
+                                        const float4 t4 = __ldcg(po + c);
+                                        acc[4 * c] = fmaf(t4.x, wgt, acc[4 * c]);
+                                        acc[4 * c + 1] = fmaf(t4.y, wgt, acc[4 * c + 1]);
+                                        acc[4 * c + 2] = fmaf(t4.z, wgt, acc[4 * c + 2]);
+                                        acc[4 * c + 3] = fmaf(t4.w, wgt, acc[4 * c + 3]);
+                                    }
+                                }
+                                uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<T*>(p.out) + off + cq);
+#pragma unroll
+                                for (int c = 0; c < 2; ++c) {
+                                    uint4 u;
+                                    u.x = Pack<T>::two(acc[8 * c + 0] * inv, acc[8 * c + 1] * inv);
+                                    u.y = Pack<T>::two(acc[8 * c + 2] * inv, acc[8 * c + 3] * inv);
+                                    u.z = Pack<T>::two(acc[8 * c + 4] * inv, acc[8 * c + 5] * inv);
+                                    u.w = Pack<T>::two(acc[8 * c + 6] * inv, acc[8 * c + 7] * inv);
+                                    dst[c] = u;
                                 }
                             }
-                            store_row<T>(p.out, off, acc, 1.0f / lsum);
                         }
                     }
                     if (lane == 0) *counter = 0;
                 }
             }
         }
+        if (lane == 0) TDUMP(2 + warp - kSoftmaxWarp0);
     }
 
+    if (warp >= kSoftmaxWarp0 && lane == 0) TRACE(2 + warp - kSoftmaxWarp0, 39, 0, 0, 0);
     __syncthreads();
-    if (*abort_flag && threadIdx.x == 0) record_status(p.status, 0, LF_ERR_DEVICE_TIMEOUT);
+    if (threadIdx.x == 0) {
+        TRACE(10, 98, *abort_flag, 0, 0);
+        if (*abort_flag) record_status(p.status, 0, LF_ERR_DEVICE_TIMEOUT);
+        // The last CTA to finish resets the scheduler for the next launch.
+        __threadfence();
+        if (atomicAdd(p.sched + 1, 1) == (int)gridDim.x - 1) {
+            p.sched[0] = 0;
+            p.sched[1] = 0;
+            __threadfence();
+        }
+        TRACE(10, 99, 0, 0, 0);
+    }
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
@@ -601,8 +1160,8 @@ bool make_map(CUtensorMap* m, const void* base, int BH, int L) {
 }
 
 struct Geometry {
-    int NKB, NT, RT, NS;
-    size_t counters_bytes, part_o_bytes, part_ml_bytes;
+    int NKB, NT, RT, NS, NSP, NTP;
+    size_t sched_bytes, counters_bytes, part_o_bytes, part_ml_bytes;
 };
 
 Geometry geometry(int B, int H, int L, int w) {
@@ -611,7 +1170,10 @@ Geometry geometry(int B, int H, int L, int w) {
     g.NT = (L + kBM - 1) / kBM;
     g.RT = (w + kBM - 1) / kBM;
     g.NS = (g.NKB + kChunkBlocks - 1) / kChunkBlocks;
+    g.NSP = (g.NS + 1) / 2;
+    g.NTP = (g.NT + 1) / 2;
     const size_t slots = (size_t)B * H * g.RT * g.NS;
+    g.sched_bytes = 256;
     g.counters_bytes = (((size_t)B * H * g.RT * 4 * sizeof(int)) + 255) & ~size_t(255);
     g.part_o_bytes = slots * kBM * kHD * sizeof(float);
     g.part_ml_bytes = slots * kBM * 2 * sizeof(float);
@@ -622,7 +1184,7 @@ Geometry geometry(int B, int H, int L, int w) {
 
 size_t attention_tc_scratch_bytes(int B, int H, int L, int w) {
     const Geometry g = geometry(B, H, L, w);
-    return g.counters_bytes + g.part_o_bytes + g.part_ml_bytes;
+    return g.sched_bytes + g.counters_bytes + g.part_o_bytes + g.part_ml_bytes;
 }
 
 lf_status launch_attention_tc(const void* q, const void* k, const void* v, const void* qg, const void* kg,
@@ -644,20 +1206,27 @@ lf_status launch_attention_tc(const void* q, const void* k, const void* v, const
     p.NT = geo.NT;
     p.RT = geo.RT;
     p.NS = geo.NS;
-    p.n_glob = BH * geo.RT * geo.NS;
-    p.n_items = p.n_glob + BH * geo.NT;
+    p.NSP = geo.NSP;
+    p.NTP = geo.NTP;
+    p.n_band = BH * geo.NTP;
+    p.n_items = p.n_band + BH * geo.RT * geo.NSP;
     p.scale_log2 = scale * kLog2e;
+    p.inv_scale = 1.0f / scale;
     p.local_mask = local_mask;
     p.global_mask = global_mask;
     p.out = out;
     uint8_t* s = reinterpret_cast<uint8_t*>(scratch);
-    p.counters = reinterpret_cast<int*>(s);
-    p.part_o = reinterpret_cast<float*>(s + geo.counters_bytes);
-    p.part_ml = reinterpret_cast<float*>(s + geo.counters_bytes + geo.part_o_bytes);
+    p.sched = reinterpret_cast<int*>(s);
+    p.counters = reinterpret_cast<int*>(s + geo.sched_bytes);
+    p.part_o = reinterpret_cast<float*>(s + geo.sched_bytes + geo.counters_bytes);
+    p.part_ml = reinterpret_cast<float*>(s + geo.sched_bytes + geo.counters_bytes + geo.part_o_bytes);
     p.status = status;
+    p.trace = nullptr;
+#if LF_TRACE
+    if (const char* a = getenv("LF_TRACE_ADDR")) p.trace = reinterpret_cast<int*>(strtoull(a, nullptr, 10));
+#endif
 
     const int grid = p.n_items < sm_count ? p.n_items : sm_count;
-    cudaError_t err;
     if (dtype == LF_F16) {
         static bool attr = false;
         if (!attr) {
@@ -674,8 +1243,7 @@ lf_status launch_attention_tc(const void* q, const void* k, const void* v, const
         }
         attention_tc_kernel<__nv_bfloat16><<<grid, kThreads, kSmemBytes, stream>>>(maps, p);
     }
-    err = cudaGetLastError();
-    return err == cudaSuccess ? LF_OK : LF_ERR_CUDA;
+    return cudaGetLastError() == cudaSuccess ? LF_OK : LF_ERR_CUDA;
 }
 
 }  // namespace lf

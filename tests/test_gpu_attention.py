@@ -149,6 +149,23 @@ def test_attention_bitwise_invariant_outside_window(dtype):
     assert torch.equal(pert[0, i], base[0, i])
 
 
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+def test_attention_growing_scores_rescale(dtype):
+    """Scores that grow along the sequence, so the running row max rises by
+    far more than 2^8 between key blocks: exercises the accumulator
+    rescaling of the tensor-core path."""
+    B, H, L, w = 1, 2, 2048, 256
+    t = inputs.attention_inputs(B, H, L, dtype, seed=8)
+    direction = torch.ones(64) / 8.0
+    ramp = torch.linspace(0, 24, L)[:, None] * direction[None, :]
+    for n in ("q", "qg"):
+        t[n] = (t[n].float() + direction * 8).to(t[n].dtype)
+    for n in ("k", "kg"):
+        t[n] = (t[n].float() + ramp).to(t[n].dtype)
+    lm, gm = inputs.masks(B, L, [40], [100])
+    _compare_full(t, lm, gm, w, TDT[dtype])
+
+
 def test_attention_device_status_errors():
     B, H, L, w = 2, 1, 512, 64
     t = inputs.attention_inputs(B, H, L, "f16", seed=6)
