@@ -853,8 +853,9 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
                 if (!ok) break;
                 tc_fence_after();
                 if (warp_active) {
-                    // Chunk states (warp-uniform): skip / full / masked.
-                    int state[4];
+                    // Chunk states (warp-uniform): skip / full / masked, two bits
+                    // per chunk so that a rolled loop can index them.
+                    uint32_t states = 0;
 #pragma unroll
                     for (int ch = 0; ch < 4; ++ch) {
                         const int cj0 = c0 + ch * 32;
@@ -872,63 +873,61 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
                             else if ((all_g || inside) && cj0 + 31 < p.L) s = kFull;
                             else s = kPart;
                         }
-                        state[ch] = s;
+                        states |= (uint32_t)s << (2 * ch);
                     }
-                    // All TMEM loads of the block first, one wait: the load
-                    // latency is paid once per block, not once per chunk.
-                    float xv[kBN];
-#pragma unroll
-                    for (int ch = 0; ch < 4; ++ch) {
-                        if (state[ch] == kSkip) continue;
-                        tmem_ld32f(tS + ch * 32, *reinterpret_cast<float(*)[32]>(&xv[ch * 32]));
-                    }
-                    tmem_ld_wait();
-#if LF_TRACE
-                    const long long ts1_ = clock64();
-                    tacc[6] += ts1_ - tc0_;
-#endif
-                    // Raw scores (+ padding bias in raw units), mask; row max with
-                    // four independent accumulators.  The scale is applied once
-                    // to the max and folded into the exponent's FMA below.
+                    auto state_of = [&](int ch) -> int { return (int)((states >> (2 * ch)) & 3u); };
+                    // Two passes over S in 32-column chunks with a rolled loop
+                    // (compact code, 32 live scores): pass 1 takes the row max,
+                    // pass 2 reloads each chunk from TMEM (cheap: ~100 cycles
+                    // for 16 KB) and writes P.  Pad bias and mask are applied
+                    // in both passes.
                     const int d0 = i - c0;
                     const int lo_c = d0 - p.w, hi_c = d0 + p.w, gl_c = g - c0, lim_c = p.L - c0;
-                    float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-                    for (int ch = 0; ch < 4; ++ch) {
-                        if (state[ch] == kSkip) continue;
+                    auto chunk_bits = [&](int ch) -> uint32_t {
+                        const int b0 = ch * 32;
+                        uint32_t bits = low_bits(lim_c - b0);
+                        if (!is_global) bits &= low_bits(gl_c - b0) | range_bits(lo_c - b0, hi_c - b0);
+                        return bits;
+                    };
+                    // bias and mask of chunk ch, applied to raw scores in r
+                    auto fix_chunk = [&](int ch, float (&r)[32]) {
                         if (has_pad) {
+                            const float4* b4p = reinterpret_cast<const float4*>(bias_w + ch * 32);
 #pragma unroll
                             for (int c = 0; c < 32; c += 4) {
-                                const float4 b4 = *reinterpret_cast<const float4*>(bias_w + ch * 32 + c);
-                                xv[ch * 32 + c] += b4.x;
-                                xv[ch * 32 + c + 1] += b4.y;
-                                xv[ch * 32 + c + 2] += b4.z;
-                                xv[ch * 32 + c + 3] += b4.w;
+                                const float4 b4 = b4p[c / 4];
+                                r[c] += b4.x;
+                                r[c + 1] += b4.y;
+                                r[c + 2] += b4.z;
+                                r[c + 3] += b4.w;
                             }
                         }
-                        if (state[ch] == kPart) {
-                            // allowed columns of this row in the chunk as one bit
-                            // mask (no per-element branches)
-                            const int b0 = ch * 32;
-                            uint32_t bits = low_bits(lim_c - b0);
-                            if (!is_global)
-                                bits &= low_bits(gl_c - b0) | range_bits(lo_c - b0, hi_c - b0);
+                        if (state_of(ch) == kPart) {
+                            const uint32_t bits = chunk_bits(ch);
 #pragma unroll
-                            for (int c = 0; c < 32; ++c)
-                                xv[b0 + c] = ((bits >> c) & 1u) ? xv[b0 + c] : -INFINITY;
+                            for (int c = 0; c < 32; ++c) r[c] = ((bits >> c) & 1u) ? r[c] : -INFINITY;
                         }
+                    };
+                    float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll 1
+                    for (int ch = 0; ch < 4; ++ch) {
+                        if (state_of(ch) == kSkip) continue;
+                        float r[32];
+                        tmem_ld32f(tS + ch * 32, r);
+                        tmem_ld_wait();
+                        fix_chunk(ch, r);
 #pragma unroll
                         for (int c = 0; c < 32; c += 8) {
-                            mx[0] = max3(mx[0], xv[ch * 32 + c], xv[ch * 32 + c + 1]);
-                            mx[1] = max3(mx[1], xv[ch * 32 + c + 2], xv[ch * 32 + c + 3]);
-                            mx[2] = max3(mx[2], xv[ch * 32 + c + 4], xv[ch * 32 + c + 5]);
-                            mx[3] = max3(mx[3], xv[ch * 32 + c + 6], xv[ch * 32 + c + 7]);
+                            mx[0] = max3(mx[0], r[c], r[c + 1]);
+                            mx[1] = max3(mx[1], r[c + 2], r[c + 3]);
+                            mx[2] = max3(mx[2], r[c + 4], r[c + 5]);
+                            mx[3] = max3(mx[3], r[c + 6], r[c + 7]);
                         }
                     }
                     const float mb = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * p.scale_log2;
 #if LF_TRACE
                     const long long ts2_ = clock64();
-                    tacc[7] += ts2_ - ts1_;
+                    tacc[7] += ts2_ - tc0_;
 #endif
                     // Running max with lazy rescaling of the TMEM accumulator.
                     // The decision is per row, but tcgen05.ld/st are warp-wide
@@ -965,21 +964,29 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
                     const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
                     const float2 nm2 = make_float2(-m_use, -m_use);
                     float2 sm2[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
+                    // exponentials of one chunk, packed to 16 words of P
+                    auto exp_chunk = [&](float (&r)[32], uint32_t (&pk)[16]) {
 #pragma unroll
+                        for (int c = 0; c < 16; ++c) {
+                            const float2 a = ffma2(make_float2(r[2 * c], r[2 * c + 1]), sc2, nm2);
+                            // about a third of the pairs on the FMA pipe, the rest on MUFU
+                            const float2 e = (c % 3 == 2) ? exp2_poly2(a) : make_float2(ex2(a.x), ex2(a.y));
+                            sm2[c & 1] = fadd2(sm2[c & 1], e);
+                            pk[c] = Pack<T>::two(e.x, e.y);
+                        }
+                    };
+#pragma unroll 1
                     for (int ch = 0; ch < 4; ++ch) {
                         uint32_t pk[16];
-                        if (state[ch] == kSkip) {
+                        if (state_of(ch) == kSkip) {
 #pragma unroll
                             for (int c = 0; c < 16; ++c) pk[c] = 0u;
                         } else {
-#pragma unroll
-                            for (int c = 0; c < 16; ++c) {
-                                const float2 a = ffma2(make_float2(xv[ch * 32 + 2 * c], xv[ch * 32 + 2 * c + 1]), sc2, nm2);
-                                // about a third of the pairs on the FMA pipe, the rest on MUFU
-                                const float2 e = (c % 3 == 2) ? exp2_poly2(a) : make_float2(ex2(a.x), ex2(a.y));
-                                sm2[c & 1] = fadd2(sm2[c & 1], e);
-                                pk[c] = Pack<T>::two(e.x, e.y);
-                            }
+                            float r[32];
+                            tmem_ld32f(tS + ch * 32, r);
+                            tmem_ld_wait();
+                            fix_chunk(ch, r);
+                            exp_chunk(r, pk);
                         }
                         tmem_st16(tS + ch * 16, pk);
                     }
