@@ -50,7 +50,8 @@ typedef enum {
     LF_ERR_DEVICE_TIMEOUT = 10,      /* a bounded device-side wait expired */
     LF_ERR_UNSUPPORTED_DEVICE = 11,  /* current device is not compute capability 10.0 */
     LF_ERR_WORKSPACE = 12,           /* workspace pointer/size too small */
-    LF_ERR_TOO_LARGE = 13            /* a size exceeds the documented maximum */
+    LF_ERR_TOO_LARGE = 13,           /* a size exceeds the documented maximum */
+    LF_ERR_SCRATCH_LIMIT = 14        /* shape needs more scratch than lf_attention_forward_noalloc holds */
 } lf_status;
 
 typedef enum { LF_F32 = 0, LF_F16 = 1, LF_BF16 = 2 } lf_dtype;
@@ -139,6 +140,34 @@ size_t lf_attention_scratch_bytes(int B, int H, int L, int w, lf_dtype dtype);
 
 /* Free the library-owned scratch of the current device (synchronises it). */
 lf_status lf_release_scratch(void);
+
+/*
+ * lf_attention_forward_noalloc -- lf_attention_forward for callers that
+ * cannot allocate device memory.  The pages describe no such entry point: it
+ * exists for code that may not call cudaMalloc (for example code running
+ * inside another framework's device-memory pool, or allocation-free real-time
+ * paths) and so cannot let the library grow its scratch buffer.
+ *
+ * Same arguments, layouts and results as lf_attention_forward, for LF_F16 and
+ * LF_BF16 only (LF_F32 needs no scratch: use lf_attention_forward).  The
+ * caller still provides every input and the output.  This call allocates
+ * nothing: its scratch is a fixed 32 MiB array in the library's device image,
+ * held on every device that has run it until the process exits.  A shape
+ * whose scratch (lf_attention_scratch_bytes) exceeds 32 MiB returns
+ * LF_ERR_SCRATCH_LIMIT before anything is launched.  The first call on a
+ * device looks up the array's device address (cudaGetSymbolAddress); make
+ * that first call before any stream capture.  Each call clears the array's
+ * counter region on `stream` (cudaMemsetAsync) before its kernel.  All calls
+ * share the one array: calls that overlap on the GPU (different streams)
+ * race and must not overlap.  Content errors (g_b > w, globals not a prefix)
+ * are recorded in a device word of this entry point that the library does
+ * not expose; validate masks beforehand when that matters.
+ */
+lf_status lf_attention_forward_noalloc(const void* q, const void* k, const void* v,
+                                       const void* qg, const void* kg, const void* vg,
+                                       const float* local_mask, const float* global_mask,
+                                       int B, int H, int L, int w, lf_dtype dtype,
+                                       lf_stream_t stream, void* out);
 
 #ifdef __cplusplus
 }

@@ -101,6 +101,7 @@ const char* lf_status_string(int s) {
         case LF_ERR_UNSUPPORTED_DEVICE: return "LF_ERR_UNSUPPORTED_DEVICE: needs compute capability 10.0 (B200)";
         case LF_ERR_WORKSPACE: return "LF_ERR_WORKSPACE: workspace missing or too small";
         case LF_ERR_TOO_LARGE: return "LF_ERR_TOO_LARGE: size beyond the supported maximum";
+        case LF_ERR_SCRATCH_LIMIT: return "LF_ERR_SCRATCH_LIMIT: shape needs more than the 32 MiB scratch of the no-allocation entry point";
         default: return "unknown lf_status";
     }
 }

@@ -1194,6 +1194,11 @@ size_t attention_tc_scratch_bytes(int B, int H, int L, int w) {
     return g.sched_bytes + g.counters_bytes + g.part_o_bytes + g.part_ml_bytes;
 }
 
+size_t attention_tc_scratch_zero_bytes(int B, int H, int L, int w) {
+    const Geometry g = geometry(B, H, L, w);
+    return g.sched_bytes + g.counters_bytes;
+}
+
 lf_status launch_attention_tc(const void* q, const void* k, const void* v, const void* qg, const void* kg,
                               const void* vg, const float* local_mask, const float* global_mask, int B, int H,
                               int L, int w, float scale, lf_dtype dtype, void* out, void* scratch, int* status,

@@ -51,6 +51,9 @@ lf_status launch_attention_simt_f32(const float* q, const float* k, const float*
 // attention_tc_scratch_bytes(B, H, L, w) bytes whose counter region is zero
 // on entry (the kernel leaves it zero).
 size_t attention_tc_scratch_bytes(int B, int H, int L, int w);
+// Leading part of that scratch (scheduler and split counters) that must be
+// zero when a launch starts.
+size_t attention_tc_scratch_zero_bytes(int B, int H, int L, int w);
 lf_status launch_attention_tc(const void* q, const void* k, const void* v, const void* qg,
                               const void* kg, const void* vg, const float* local_mask,
                               const float* global_mask, int B, int H, int L, int w, float scale,

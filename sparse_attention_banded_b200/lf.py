@@ -50,6 +50,8 @@ def lib():
         L.lf_attention_scratch_bytes.argtypes = [i, i, i, i, i]
         L.lf_attention_scratch_bytes.restype = ctypes.c_size_t
         L.lf_release_scratch.restype = st
+        L.lf_attention_forward_noalloc.argtypes = [vp] * 8 + [i, i, i, i, i, vp, vp]
+        L.lf_attention_forward_noalloc.restype = st
         _lib = L
     return _lib
 
@@ -126,3 +128,17 @@ def lf_attention_scratch_bytes(B: int, H: int, L: int, w: int, dtype) -> int:
 
 def lf_release_scratch():
     _check(lib().lf_release_scratch(), "lf_release_scratch")
+
+
+def lf_attention_forward_noalloc(q, k, v, qg, kg, vg, local_mask, global_mask, w: int, out=None, stream=None):
+    """Same as :func:`lf_attention_forward` through the entry point that
+    allocates no device memory (fp16/bf16; scratch limited to 32 MiB)."""
+    B, H, L, _ = q.shape
+    if out is None:
+        out = torch.empty(B, L, H * 64, dtype=q.dtype, device=q.device)
+    code = DTYPE_CODE.get(q.dtype, 99)
+    st = lib().lf_attention_forward_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(qg), _ptr(kg), _ptr(vg),
+                                            _ptr(local_mask), _ptr(global_mask), B, H, L, w, code,
+                                            _stream(stream), _ptr(out))
+    _check(st, "lf_attention_forward_noalloc")
+    return out
