@@ -142,6 +142,58 @@ size_t lf_attention_scratch_bytes(int B, int H, int L, int w, lf_dtype dtype);
 lf_status lf_release_scratch(void);
 
 /*
+ * One Longformer encoder layer: FTL §Longformer Encoder 计算流程 / 每个
+ * Transformer 层, steps 1-6 (LongformerEncoder::forwardLayer):
+ *   [q k v kg vg] = x W^T + b      (step 1; the five weights contiguous, as
+ *                                    §PyTorch OP requires)   -> [B,H,L,64] (step 2)
+ *   qg            = x W_qg^T + b_qg over the rows that can be global (i <
+ *                   ceil(w/128)*128), as the page's separate Qg GEMM
+ *   a             = attention(q, k, v, qg, kg, vg)   (steps 3-5, scale attn_scale)
+ *   h             = LN1(a W_o^T + b_o + x)           (step 5, AddBiasResidualLayerNorm)
+ *   y             = LN2(GELU(h W_1^T + b_1) W_2^T + b_2 + h)   (step 6, GeluFfnLayer)
+ * GELU is the erf form; LN uses the population variance and ln_eps.
+ * All weights use the nn.Linear layout [out_features][in_features] in the
+ * layer's dtype; LayerNorm parameters are fp32.  D = H*64.
+ */
+typedef struct {
+    int ffn_dim;                 /* F: FFN inner size (multiple of 128) */
+    const void* W_qkv_kgvg;      /* [5][D][D]: q, k, v, kg, vg weights, contiguous */
+    const void* b_qkv_kgvg;      /* [5][D] */
+    const void* W_qg;            /* [D][D] */
+    const void* b_qg;            /* [D] */
+    const void* W_o;             /* [D][D] */
+    const void* b_o;             /* [D] */
+    const float* ln1_gamma;      /* [D] */
+    const float* ln1_beta;       /* [D] */
+    const void* W_1;             /* [F][D] */
+    const void* b_1;             /* [F] */
+    const void* W_2;             /* [D][F] */
+    const void* b_2;             /* [D] */
+    const float* ln2_gamma;      /* [D] */
+    const float* ln2_beta;       /* [D] */
+} lf_layer_weights;
+
+/* Bytes of device workspace lf_encoder_layer_forward needs (0 on bad sizes). */
+size_t lf_encoder_layer_workspace_bytes(int B, int H, int L, int w, int ffn_dim, lf_dtype dtype);
+
+/*
+ * lf_encoder_layer_forward -- the layer above.  x and out are [B, L, D] of
+ * `dtype` (LF_F16 or LF_BF16), masks as lf_attention_forward.  `workspace`
+ * is caller-owned device memory of at least
+ * lf_encoder_layer_workspace_bytes(...) bytes, 256-byte aligned; its
+ * contents need not be initialised and are overwritten.  Shape rules: those
+ * of lf_attention_forward, plus D = H*64 a multiple of 128 (H even),
+ * D <= 1024 (LayerNorm keeps a row in registers) and F a multiple of 128.
+ * Errors: LF_ERR_WORKSPACE if the workspace is missing, misaligned or too
+ * small; otherwise as lf_attention_forward.  Asynchronous on `stream`.
+ */
+lf_status lf_encoder_layer_forward(const void* x, const float* local_mask, const float* global_mask,
+                                   const lf_layer_weights* weights, int B, int H, int L, int w,
+                                   float attn_scale, float ln_eps, lf_dtype dtype,
+                                   void* workspace, size_t workspace_bytes,
+                                   lf_stream_t stream, void* out);
+
+/*
  * lf_attention_forward_noalloc -- lf_attention_forward for callers that
  * cannot allocate device memory.  The pages describe no such entry point: it
  * exists for code that may not call cudaMalloc (for example code running

@@ -169,24 +169,28 @@ def to_heads(y, H):
 
 
 def encoder_layer(x, local_mask, global_mask, weights: dict, H: int, w: int,
-                  scale: float, eps: float, round_attention_inputs=None):
+                  scale: float, eps: float, round_attention_inputs=None, round_stored=None):
     """x: [B, L, H*64]; weights: float64 arrays with keys
     W_qkv_kgvg [5, D, D], b_qkv_kgvg [5, D], W_qg [D, D], b_qg [D],
     W_o [D, D], b_o [D], ln1_gamma, ln1_beta [D], W_1 [D, F], b_1 [F],
     W_2 [F, D], b_2 [D], ln2_gamma, ln2_beta [D].
 
     round_attention_inputs: optional function applied to each projected
-    [B, H, L, 64] tensor before attention (the device stores them in its
-    compute dtype).  Returns float64 [B, L, D]."""
+    [B, H, L, 64] tensor before attention; round_stored: optional function
+    applied to the attention output, to h and to the FFN intermediate.  The
+    page's LongformerEncoder<T> keeps every intermediate buffer in T (FTL
+    §Longformer Encoder 计算流程), so the comparison rounds where values are
+    stored; all arithmetic stays float64.  Returns float64 [B, L, D]."""
     x = _f64(x)
     W = {k: _f64(v) for k, v in weights.items()}
     rnd = round_attention_inputs or (lambda a: a)
+    keep = round_stored or (lambda a: a)
     proj = [to_heads(x @ W["W_qkv_kgvg"][n] + W["b_qkv_kgvg"][n], H) for n in range(5)]
     q, k, v, kg, vg = [rnd(p) for p in proj]
     qg = rnd(to_heads(x @ W["W_qg"] + W["b_qg"], H))
     att = attention(q, k, v, qg, kg, vg, local_mask, global_mask, w, scale)
     B, L = x.shape[:2]
-    att = att.reshape(B, L, H * D)
-    h = layer_norm(att @ W["W_o"] + W["b_o"] + x, W["ln1_gamma"], W["ln1_beta"], eps)
-    f = gelu(h @ W["W_1"] + W["b_1"])
+    att = keep(att.reshape(B, L, H * D))
+    h = keep(layer_norm(att @ W["W_o"] + W["b_o"] + x, W["ln1_gamma"], W["ln1_beta"], eps))
+    f = keep(gelu(h @ W["W_1"] + W["b_1"]))
     return layer_norm(f @ W["W_2"] + W["b_2"] + h, W["ln2_gamma"], W["ln2_beta"], eps)

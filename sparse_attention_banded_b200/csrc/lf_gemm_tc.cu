@@ -1,0 +1,357 @@
+// Dense GEMM with fused epilogues on the sm_100a tensor cores, for the
+// projections, the output projection and the FFN of one encoder layer
+// (FasterTransformer Longformer page, §Longformer Encoder 计算流程 / 每个
+// Transformer 层 steps 1, 2, 5 and 6).
+//
+//   C[b, m, n] = sum_k A[b, m, k] * W[n, k]      (W in nn.Linear layout [out, in])
+//
+// A is [batches][rows][K] (rows of one batch contiguous, the batch stride may
+// exceed rows so that only the first rows of each sample are multiplied),
+// both operands K-major fp16/bf16, fp32 accumulation in TMEM.  Tiles are
+// 128 x 128 with 64-wide K steps through a kStages-deep TMA ring.  One
+// persistent CTA per SM: warp 0 issues TMA loads, warp 1 issues tcgen05.mma
+// into one of two TMEM accumulators, warps 4-7 run the epilogue of the
+// previous tile (one thread per row) while the next tile accumulates.
+//
+// Epilogues:
+//   kEpiHeads  : + bias, round, scatter column n to head layout
+//                out[n / D][b][h][m][d] with h = (n % D) / 64, d = n % 64
+//                (AddBiasTransposeToMultiHead, step 2)
+//   kEpiGelu   : + bias, GELU (erf form), round, row-major out[b*rows + m][n]
+//   kEpiResid  : + bias + residual (same dtype, row-major [.., N]), fp32
+//                row-major out (the LayerNorm kernel reads it)
+// Roofline: tensor-bound (2*M*N*K flops over (M*K + N*K)*2 + out bytes).
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include <mutex>
+
+#include "lf_internal.h"
+#include "sm100.cuh"
+
+namespace lf {
+namespace {
+
+using namespace sm100;
+
+constexpr int kTM = 128, kTN = 128, kTK = 64;
+constexpr int kStages = 6;
+constexpr int kThreads = 256;  // 8 warps: 0 TMA, 1 MMA, 2-3 idle, 4-7 epilogue
+constexpr uint32_t kABytes = kTM * kTK * 2;  // 16 KB
+constexpr uint32_t kBBytes = kTN * kTK * 2;  // 16 KB
+constexpr uint32_t kOffA = 0;
+constexpr uint32_t kOffB = kOffA + kStages * kABytes;
+constexpr uint32_t kOffBias = kOffB + kStages * kBBytes;        // 4 warps x 128 floats
+constexpr uint32_t kOffBar = kOffBias + 4 * kTN * 4;
+constexpr uint32_t kNumBars = 2 * kStages + 4 + 1;
+constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
+constexpr uint32_t kSmemBytes = kOffMisc + 64 + 1024;
+constexpr uint32_t kTmemCols = 256;  // two 128-column fp32 accumulators
+
+struct GemmParams {
+    int batches, rows, K, N;  // per batch: rows x N outputs
+    int mtiles, ntiles, ktiles, tiles;
+    int mode;
+    const void* bias;    // [N] of T
+    const void* resid;   // kEpiResid: [batches*rows][N] of T
+    void* out;
+    int heads_D;         // kEpiHeads: columns per output tensor (H*64)
+    int heads_H;
+    int heads_L;         // rows of the head-layout tensors (L)
+    int* status;
+};
+
+template <typename T>
+struct Cvt;
+template <>
+struct Cvt<__half> {
+    static constexpr uint32_t fmt = 0;
+    __device__ static float to_f(__half x) { return __half2float(x); }
+    __device__ static uint32_t two(float a, float b) {
+        __half2 h = __floats2half2_rn(a, b);
+        return *reinterpret_cast<uint32_t*>(&h);
+    }
+};
+template <>
+struct Cvt<__nv_bfloat16> {
+    static constexpr uint32_t fmt = 1;
+    __device__ static float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
+    __device__ static uint32_t two(float a, float b) {
+        __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+        return *reinterpret_cast<uint32_t*>(&h);
+    }
+};
+
+__device__ __forceinline__ void tmem_ld32v(uint32_t taddr, float (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=f"(r[0]), "=f"(r[1]), "=f"(r[2]), "=f"(r[3]), "=f"(r[4]), "=f"(r[5]), "=f"(r[6]), "=f"(r[7]),
+          "=f"(r[8]), "=f"(r[9]), "=f"(r[10]), "=f"(r[11]), "=f"(r[12]), "=f"(r[13]), "=f"(r[14]), "=f"(r[15]),
+          "=f"(r[16]), "=f"(r[17]), "=f"(r[18]), "=f"(r[19]), "=f"(r[20]), "=f"(r[21]), "=f"(r[22]), "=f"(r[23]),
+          "=f"(r[24]), "=f"(r[25]), "=f"(r[26]), "=f"(r[27]), "=f"(r[28]), "=f"(r[29]), "=f"(r[30]), "=f"(r[31])
+        : "r"(taddr));
+}
+
+__device__ __forceinline__ float gelu_erf(float x) { return 0.5f * x * (1.0f + erff(x * 0.70710678118654752f)); }
+
+template <typename T>
+__global__ void __launch_bounds__(kThreads, 1)
+gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_w,
+               const __grid_constant__ GemmParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
+    uint64_t* full = bars;
+    uint64_t* empty = bars + kStages;
+    uint64_t* acc_full = bars + 2 * kStages;
+    uint64_t* acc_empty = acc_full + 2;
+    uint64_t* drain = acc_empty + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&acc_full[i], 1);
+            mbar_init(&acc_empty[i], 4);
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tensormap(&map_a);
+        prefetch_tensormap(&map_w);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            uint32_t kc = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < p.tiles && ok; t += gridDim.x) {
+                const int nt = t % p.ntiles;
+                const int bm = t / p.ntiles;
+                const int mt = bm % p.mtiles, b = bm / p.mtiles;
+                for (int kt = 0; kt < p.ktiles && ok; ++kt, ++kc) {
+                    const uint32_t st = kc % kStages;
+                    ok = mbar_wait(&empty[st], ((kc / kStages) & 1) ^ 1, abort_flag);
+                    if (!ok) break;
+                    mbar_arrive_expect_tx(&full[st], kABytes + kBBytes);
+                    tma_load_3d(smem + kOffA + st * kABytes, &map_a, &full[st], kt * kTK, mt * kTM, b);
+                    tma_load_2d(smem + kOffB + st * kBBytes, &map_w, &full[st], kt * kTK, nt * kTN);
+                }
+            }
+            if (!ok) {  // wind-down: let issued copies land
+                for (uint32_t c = (kc > kStages ? kc - kStages : 0); c < kc; ++c) {
+                    volatile int never = 0;
+                    mbar_wait(&full[c % kStages], (c / kStages) & 1, &never, 200000000ull);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            constexpr uint32_t idesc = idesc_f16(Cvt<T>::fmt, kTM, kTN, 0, 0);
+            uint32_t kc = 0, tc = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < p.tiles && ok; t += gridDim.x, ++tc) {
+                const uint32_t ab = tc & 1;
+                ok = mbar_wait(&acc_empty[ab], ((tc >> 1) & 1) ^ 1, abort_flag);
+                if (!ok) break;
+                tc_fence_after();
+                for (int kt = 0; kt < p.ktiles && ok; ++kt, ++kc) {
+                    const uint32_t st = kc % kStages;
+                    ok = mbar_wait(&full[st], (kc / kStages) & 1, abort_flag);
+                    if (!ok) break;
+                    tc_fence_after();
+                    const uint32_t a_addr = smem_u32(smem + kOffA + st * kABytes);
+                    const uint32_t b_addr = smem_u32(smem + kOffB + st * kBBytes);
+#pragma unroll
+                    for (int kk = 0; kk < kTK / 16; ++kk)
+                        mma_f16_ss(tmem + ab * kTN, desc_sw128(a_addr + kk * 32), desc_sw128(b_addr + kk * 32), idesc,
+                                   (kt > 0 || kk > 0) ? 1u : 0u);
+                    tc_commit(&empty[st]);
+                }
+                if (ok) tc_commit(&acc_full[ab]);
+            }
+            if (!ok) {
+                tc_commit(drain);
+                volatile int never = 0;
+                mbar_wait(drain, 0, &never, 200000000ull);
+            }
+        }
+    } else if (warp >= 4) {
+        const int sp = warp & 3;
+        const int r = sp * 32 + lane;
+        const uint32_t lane_off = (uint32_t)(sp * 32) << 16;
+        float* bias_w = reinterpret_cast<float*>(smem + kOffBias) + sp * kTN;
+        const T* bias = reinterpret_cast<const T*>(p.bias);
+        uint32_t tc = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < p.tiles && ok; t += gridDim.x, ++tc) {
+            const int nt = t % p.ntiles;
+            const int bm = t / p.ntiles;
+            const int mt = bm % p.mtiles, b = bm / p.mtiles;
+            const int n0 = nt * kTN;
+            // this warp's copy of the tile's bias
+#pragma unroll
+            for (int c = 0; c < kTN / 32; ++c) bias_w[c * 32 + lane] = Cvt<T>::to_f(bias[n0 + c * 32 + lane]);
+            __syncwarp();
+            const uint32_t ab = tc & 1;
+            ok = __all_sync(0xffffffffu, mbar_wait(&acc_full[ab], (tc >> 1) & 1, abort_flag));
+            if (!ok) break;
+            tc_fence_after();
+            const int m = mt * kTM + r;  // row within the batch
+            const bool row_ok = m < p.rows;
+            const size_t grow = (size_t)b * p.rows + m;  // global row (row-major outputs)
+#pragma unroll 1
+            for (int c0 = 0; c0 < kTN; c0 += 32) {
+                float acc[32];
+                __syncwarp();  // tcgen05.ld is .sync.aligned: whole warp, converged
+                tmem_ld32v(tmem + lane_off + ab * kTN + c0, acc);
+                tmem_ld_wait();
+#pragma unroll
+                for (int c = 0; c < 32; ++c) acc[c] += bias_w[c0 + c];
+                const int n = n0 + c0;
+                if (p.mode == kEpiGelu) {
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) acc[c] = gelu_erf(acc[c]);
+                }
+                if (!row_ok) {
+                } else if (p.mode == kEpiResid) {
+                    const uint4* rs = reinterpret_cast<const uint4*>(reinterpret_cast<const T*>(p.resid) + grow * p.N + n);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        uint4 u = rs[q];
+                        const T* e = reinterpret_cast<const T*>(&u);
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) acc[q * 8 + j] += Cvt<T>::to_f(e[j]);
+                    }
+                    float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) + grow * p.N + n);
+#pragma unroll
+                    for (int q = 0; q < 8; ++q)
+                        dst[q] = make_float4(acc[4 * q], acc[4 * q + 1], acc[4 * q + 2], acc[4 * q + 3]);
+                } else {
+                    T* dst;
+                    if (p.mode == kEpiHeads) {
+                        const int which = n / p.heads_D;
+                        const int h = (n % p.heads_D) / 64, d = n % 64;
+                        dst = reinterpret_cast<T*>(p.out) +
+                              ((((size_t)which * p.batches + b) * p.heads_H + h) * p.heads_L + m) * 64 + d;
+                    } else {
+                        dst = reinterpret_cast<T*>(p.out) + grow * p.N + n;
+                    }
+                    uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        uint4 u;
+                        u.x = Cvt<T>::two(acc[8 * q + 0], acc[8 * q + 1]);
+                        u.y = Cvt<T>::two(acc[8 * q + 2], acc[8 * q + 3]);
+                        u.z = Cvt<T>::two(acc[8 * q + 4], acc[8 * q + 5]);
+                        u.w = Cvt<T>::two(acc[8 * q + 6], acc[8 * q + 7]);
+                        d4[q] = u;
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[ab]);
+        }
+    }
+
+    __syncthreads();
+    if (threadIdx.x == 0 && *abort_flag) record_status(p.status, 0, LF_ERR_DEVICE_TIMEOUT);
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    });
+    return fn;
+}
+
+template <typename T>
+lf_status launch_t(const GemmArgs& g, int sm_count, cudaStream_t stream) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return LF_ERR_CUDA;
+    CUtensorMap ma, mw;
+    // A: [batches][batch_stride rows][K], tiles over the first `rows` of each batch
+    cuuint64_t adims[3] = {(cuuint64_t)g.K, (cuuint64_t)g.rows, (cuuint64_t)g.batches};
+    cuuint64_t astr[2] = {(cuuint64_t)g.K * 2, (cuuint64_t)g.batch_stride * g.K * 2};
+    cuuint32_t abox[3] = {(cuuint32_t)kTK, (cuuint32_t)kTM, 1};
+    cuuint32_t e3[3] = {1, 1, 1};
+    if (enc(&ma, CU_TENSOR_MAP_DATA_TYPE_UINT16, 3, const_cast<void*>(g.A), adims, astr, abox, e3,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return LF_ERR_CUDA;
+    cuuint64_t wdims[2] = {(cuuint64_t)g.K, (cuuint64_t)g.N};
+    cuuint64_t wstr[1] = {(cuuint64_t)g.K * 2};
+    cuuint32_t wbox[2] = {(cuuint32_t)kTK, (cuuint32_t)kTN};
+    if (enc(&mw, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void*>(g.W), wdims, wstr, wbox, e3,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return LF_ERR_CUDA;
+    GemmParams p;
+    p.batches = g.batches;
+    p.rows = g.rows;
+    p.K = g.K;
+    p.N = g.N;
+    p.mtiles = (g.rows + kTM - 1) / kTM;
+    p.ntiles = g.N / kTN;
+    p.ktiles = g.K / kTK;
+    p.tiles = g.batches * p.mtiles * p.ntiles;
+    p.mode = g.mode;
+    p.bias = g.bias;
+    p.resid = g.resid;
+    p.out = g.out;
+    p.heads_D = g.heads_D;
+    p.heads_H = g.heads_H;
+    p.heads_L = g.heads_L;
+    p.status = g.status;
+    static bool attr = false;
+    if (!attr) {
+        cudaFuncSetAttribute(gemm_tc_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+        attr = true;
+    }
+    const int grid = p.tiles < sm_count ? p.tiles : sm_count;
+    gemm_tc_kernel<T><<<grid, kThreads, kSmemBytes, stream>>>(ma, mw, p);
+    return cudaGetLastError() == cudaSuccess ? LF_OK : LF_ERR_CUDA;
+}
+
+}  // namespace
+
+lf_status launch_gemm_tc(const GemmArgs& g, lf_dtype dtype, int sm_count, cudaStream_t stream) {
+    if (g.N % kTN != 0 || g.K % kTK != 0 || g.rows <= 0 || g.batches <= 0) return LF_ERR_BAD_DIM;
+    if (dtype == LF_F16) return launch_t<__half>(g, sm_count, stream);
+    if (dtype == LF_BF16) return launch_t<__nv_bfloat16>(g, sm_count, stream);
+    return LF_ERR_DTYPE;
+}
+
+}  // namespace lf

@@ -60,4 +60,25 @@ lf_status launch_attention_tc(const void* q, const void* k, const void* v, const
                               lf_dtype dtype, void* out, void* scratch, int* status,
                               int sm_count, cudaStream_t stream);
 
+// ---- dense GEMM with fused epilogues (encoder layer) ----
+enum { kEpiHeads = 0, kEpiGelu = 1, kEpiResid = 2 };
+struct GemmArgs {
+    const void* A;     // [batches][batch_stride][K], K-major
+    int batches, rows, batch_stride, K;
+    const void* W;     // [N][K] (nn.Linear layout)
+    int N;
+    const void* bias;  // [N]
+    int mode;          // kEpi*
+    const void* resid; // kEpiResid: [batches*rows][N]
+    void* out;
+    int heads_D, heads_H, heads_L;  // kEpiHeads
+    int* status;
+};
+// N % 128 == 0, K % 64 == 0; fp16 / bf16.
+lf_status launch_gemm_tc(const GemmArgs& g, lf_dtype dtype, int sm_count, cudaStream_t stream);
+
+// LayerNorm over rows of an fp32 [rows][N] matrix into dtype (N % 32 == 0, N <= 1024).
+lf_status launch_layernorm(const float* z, const float* gamma, const float* beta, int rows, int N, float eps,
+                           lf_dtype dtype, void* out, cudaStream_t stream);
+
 }  // namespace lf

@@ -1,0 +1,123 @@
+// One Longformer encoder layer on the tensor cores: the composition of the
+// FasterTransformer Longformer page, §Longformer Encoder 计算流程 / 每个
+// Transformer 层 steps 1-6, as a sequence of this library's kernels on one
+// stream (no host synchronisation):
+//   GEMM(x, W_qkv_kgvg) + bias -> q, k, v, kg, vg in head layout
+//   GEMM(x rows < ceil(w/128)*128, W_qg) + bias -> qg in head layout
+//   banded + global attention -> a [B, L, D]
+//   GEMM(a, W_o) + b_o + x -> z (fp32);  LayerNorm -> h
+//   GEMM(h, W_1) + b_1, GELU -> f;  GEMM(f, W_2) + b_2 + h -> z;  LayerNorm -> out
+#include "lf_internal.h"
+
+namespace lf {
+namespace {
+
+struct Workspace {
+    size_t qkv, qg, att, z, h, f, scratch, total;
+};
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+Workspace layout(int B, int H, int L, int w, int F, int elem) {
+    const size_t D = (size_t)H * 64, rows = (size_t)B * L;
+    Workspace s;
+    size_t o = 0;
+    s.qkv = o; o += align256(5 * rows * D * elem);
+    s.qg = o; o += align256(rows * D * elem);
+    s.att = o; o += align256(rows * D * elem);
+    s.z = o; o += align256(rows * D * 4);
+    s.h = o; o += align256(rows * D * elem);
+    s.f = o; o += align256(rows * (size_t)F * elem);
+    s.scratch = o; o += align256(attention_tc_scratch_bytes(B, H, L, w));
+    s.total = o;
+    return s;
+}
+
+lf_status check_layer(int B, int H, int L, int w, int F, lf_dtype dtype) {
+    lf_status st = check_shape(B, H, L, w);
+    if (st != LF_OK) return st;
+    if (dtype != LF_F16 && dtype != LF_BF16) return LF_ERR_DTYPE;
+    const int D = H * 64;
+    if (D % 128 != 0 || D > 1024 || F <= 0 || F % 128 != 0) return LF_ERR_BAD_DIM;
+    return LF_OK;
+}
+
+}  // namespace
+}  // namespace lf
+
+using namespace lf;
+
+extern "C" size_t lf_encoder_layer_workspace_bytes(int B, int H, int L, int w, int ffn_dim, lf_dtype dtype) {
+    if (check_layer(B, H, L, w, ffn_dim, dtype) != LF_OK) return 0;
+    return layout(B, H, L, w, ffn_dim, 2).total;
+}
+
+extern "C" lf_status lf_encoder_layer_forward(const void* x, const float* local_mask, const float* global_mask,
+                                              const lf_layer_weights* wt, int B, int H, int L, int w,
+                                              float attn_scale, float ln_eps, lf_dtype dtype, void* workspace,
+                                              size_t workspace_bytes, lf_stream_t stream, void* out) {
+    if (!x || !local_mask || !global_mask || !wt || !out) return LF_ERR_NULL;
+    const int F = wt->ffn_dim;
+    lf_status st = check_layer(B, H, L, w, F, dtype);
+    if (st != LF_OK) return st;
+    const void* wptrs[] = {wt->W_qkv_kgvg, wt->b_qkv_kgvg, wt->W_qg, wt->b_qg, wt->W_o, wt->b_o,
+                           wt->ln1_gamma, wt->ln1_beta, wt->W_1, wt->b_1, wt->W_2, wt->b_2,
+                           wt->ln2_gamma, wt->ln2_beta};
+    for (const void* p : wptrs) {
+        if (!p) return LF_ERR_NULL;
+        if (!aligned16(p)) return LF_ERR_MISALIGNED;
+    }
+    const void* ptrs[] = {x, local_mask, global_mask, out};
+    for (const void* p : ptrs)
+        if (!aligned16(p)) return LF_ERR_MISALIGNED;
+    const Workspace ws = layout(B, H, L, w, F, 2);
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < ws.total)
+        return LF_ERR_WORKSPACE;
+    DeviceCtx* d = current_device(&st);
+    if (!d) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    uint8_t* base = reinterpret_cast<uint8_t*>(workspace);
+    const int D = H * 64;
+    const size_t head_elems = (size_t)B * H * L * 64;
+    uint8_t* qkv = base + ws.qkv;  // [5][B][H][L][64]
+    auto slot = [&](int i) { return qkv + (size_t)i * head_elems * 2; };
+
+    // steps 1-2: the five projections with bias, scattered to head layout
+    GemmArgs g{};
+    g.A = x; g.batches = B; g.rows = L; g.batch_stride = L; g.K = D;
+    g.W = wt->W_qkv_kgvg; g.N = 5 * D; g.bias = wt->b_qkv_kgvg; g.mode = kEpiHeads;
+    g.out = qkv; g.heads_D = D; g.heads_H = H; g.heads_L = L; g.status = d->status;
+    if ((st = launch_gemm_tc(g, dtype, d->sm_count, s)) != LF_OK) return st;
+    // Qg over the rows that can be global tokens (g_b <= w)
+    const int qrows = ((w + 127) / 128) * 128 < L ? ((w + 127) / 128) * 128 : L;
+    g.rows = qrows; g.W = wt->W_qg; g.N = D; g.bias = wt->b_qg; g.out = base + ws.qg;
+    if ((st = launch_gemm_tc(g, dtype, d->sm_count, s)) != LF_OK) return st;
+    // steps 3-5: attention (its split counters must start at zero)
+    if (cudaMemsetAsync(base + ws.scratch, 0, attention_tc_scratch_zero_bytes(B, H, L, w), s) != cudaSuccess)
+        return LF_ERR_CUDA;
+    if ((st = launch_attention_tc(slot(0), slot(1), slot(2), base + ws.qg, slot(3), slot(4), local_mask, global_mask,
+                                  B, H, L, w, attn_scale, dtype, base + ws.att, base + ws.scratch, d->status,
+                                  d->sm_count, s)) != LF_OK)
+        return st;
+    // step 5: output projection + bias + residual, LayerNorm
+    GemmArgs o{};
+    o.A = base + ws.att; o.batches = B; o.rows = L; o.batch_stride = L; o.K = D;
+    o.W = wt->W_o; o.N = D; o.bias = wt->b_o; o.mode = kEpiResid; o.resid = x; o.out = base + ws.z;
+    o.status = d->status;
+    if ((st = launch_gemm_tc(o, dtype, d->sm_count, s)) != LF_OK) return st;
+    if ((st = launch_layernorm(reinterpret_cast<float*>(base + ws.z), wt->ln1_gamma, wt->ln1_beta, B * L, D, ln_eps,
+                               dtype, base + ws.h, s)) != LF_OK)
+        return st;
+    // step 6: GELU FFN + bias + residual, LayerNorm
+    GemmArgs f1{};
+    f1.A = base + ws.h; f1.batches = B; f1.rows = L; f1.batch_stride = L; f1.K = D;
+    f1.W = wt->W_1; f1.N = F; f1.bias = wt->b_1; f1.mode = kEpiGelu; f1.out = base + ws.f; f1.status = d->status;
+    if ((st = launch_gemm_tc(f1, dtype, d->sm_count, s)) != LF_OK) return st;
+    GemmArgs f2{};
+    f2.A = base + ws.f; f2.batches = B; f2.rows = L; f2.batch_stride = L; f2.K = F;
+    f2.W = wt->W_2; f2.N = D; f2.bias = wt->b_2; f2.mode = kEpiResid; f2.resid = base + ws.h; f2.out = base + ws.z;
+    f2.status = d->status;
+    if ((st = launch_gemm_tc(f2, dtype, d->sm_count, s)) != LF_OK) return st;
+    return launch_layernorm(reinterpret_cast<float*>(base + ws.z), wt->ln2_gamma, wt->ln2_beta, B * L, D, ln_eps,
+                            dtype, out, s);
+}

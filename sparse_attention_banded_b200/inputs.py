@@ -96,28 +96,41 @@ def workload_inputs(cid: int, device: str = "cpu"):
     return wl, t, lm.to(device), gm.to(device)
 
 
-def layer_inputs(cid: int = 5, hidden: int = 1024, ffn: int = 4096, device: str = "cpu"):
-    """Encoder-layer input x [B, L, hidden] and weights (y = x @ W + b, W
-    stored [in, out]; q k v kg vg weights contiguous as [5, hidden, hidden])."""
+def layer_inputs(cid: int = 5, hidden: int = 1024, ffn: int = 4096, device: str = "cpu", B=None, L=None,
+                 dtype=None, g=None, pad=None, seed=None, bias_scale: float = 0.0, ln_scale: float = 0.0):
+    """Encoder-layer input x [B, L, hidden] and weights in the nn.Linear
+    layout [out, in] (y = x @ W.T + b; q k v kg vg weights contiguous as
+    [5, hidden, hidden]).  Workload 5 by default; B, L, dtype, g, pad and
+    seed override it for smaller test layers; bias_scale > 0 draws biases
+    ~ N(0, bias_scale^2) and ln_scale > 0 draws gamma ~ 1 + N(0, ln_scale^2),
+    beta ~ N(0, ln_scale^2) (workload 5 itself has zero biases, gamma 1,
+    beta 0)."""
     wl = workload(cid)
-    dt = TORCH_DTYPES[wl.dtype]
-    gen = torch.Generator().manual_seed(wl.seed)
-    x = torch.randn(wl.B, wl.L, hidden, generator=gen)
+    B = wl.B if B is None else B
+    L = wl.L if L is None else L
+    g = wl.g if g is None else g
+    pad = wl.pad if pad is None else pad
+    dt = TORCH_DTYPES[wl.dtype if dtype is None else dtype]
+    gen = torch.Generator().manual_seed(wl.seed if seed is None else seed)
+    x = torch.randn(B, L, hidden, generator=gen)
     w = {}
     mats = [("W_q", (hidden, hidden)), ("W_k", (hidden, hidden)), ("W_v", (hidden, hidden)),
             ("W_kg", (hidden, hidden)), ("W_vg", (hidden, hidden)), ("W_qg", (hidden, hidden)),
-            ("W_o", (hidden, hidden)), ("W_1", (hidden, ffn)), ("W_2", (ffn, hidden))]
+            ("W_o", (hidden, hidden)), ("W_1", (ffn, hidden)), ("W_2", (hidden, ffn))]
     for n, shp in mats:
         w[n] = torch.randn(*shp, generator=gen) * 0.02
+    def vec(n, scale, base=0.0):
+        return base + torch.randn(n, generator=gen) * scale if scale > 0 else torch.full((n,), base)
+
     weights = {
         "W_qkv_kgvg": torch.stack([w["W_q"], w["W_k"], w["W_v"], w["W_kg"], w["W_vg"]]).to(dt),
-        "b_qkv_kgvg": torch.zeros(5, hidden).to(dt),
-        "W_qg": w["W_qg"].to(dt), "b_qg": torch.zeros(hidden).to(dt),
-        "W_o": w["W_o"].to(dt), "b_o": torch.zeros(hidden).to(dt),
-        "ln1_gamma": torch.ones(hidden), "ln1_beta": torch.zeros(hidden),
-        "W_1": w["W_1"].to(dt), "b_1": torch.zeros(ffn).to(dt),
-        "W_2": w["W_2"].to(dt), "b_2": torch.zeros(hidden).to(dt),
-        "ln2_gamma": torch.ones(hidden), "ln2_beta": torch.zeros(hidden),
+        "b_qkv_kgvg": vec(5 * hidden, bias_scale).reshape(5, hidden).to(dt),
+        "W_qg": w["W_qg"].to(dt), "b_qg": vec(hidden, bias_scale).to(dt),
+        "W_o": w["W_o"].to(dt), "b_o": vec(hidden, bias_scale).to(dt),
+        "ln1_gamma": vec(hidden, ln_scale, 1.0), "ln1_beta": vec(hidden, ln_scale),
+        "W_1": w["W_1"].to(dt), "b_1": vec(ffn, bias_scale).to(dt),
+        "W_2": w["W_2"].to(dt), "b_2": vec(hidden, bias_scale).to(dt),
+        "ln2_gamma": vec(hidden, ln_scale, 1.0), "ln2_beta": vec(hidden, ln_scale),
     }
-    lm, gm = masks(wl.B, wl.L, wl.g, wl.pad)
+    lm, gm = masks(B, L, g, pad)
     return wl, x.to(dt).to(device), {k: v.to(device) for k, v in weights.items()}, lm.to(device), gm.to(device)

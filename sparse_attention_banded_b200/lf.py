@@ -23,6 +23,14 @@ DTYPE_CODE = {torch.float32: LF_F32, torch.float16: LF_F16, torch.bfloat16: LF_B
 
 _lib = None
 
+LAYER_FIELDS = ("W_qkv_kgvg", "b_qkv_kgvg", "W_qg", "b_qg", "W_o", "b_o", "ln1_gamma", "ln1_beta",
+                "W_1", "b_1", "W_2", "b_2", "ln2_gamma", "ln2_beta")
+
+
+class LayerWeights(ctypes.Structure):
+    """lf_layer_weights of include/lf.h."""
+    _fields_ = [("ffn_dim", ctypes.c_int)] + [(n, ctypes.c_void_p) for n in LAYER_FIELDS]
+
 
 class LFError(RuntimeError):
     def __init__(self, status: int, where: str):
@@ -52,6 +60,11 @@ def lib():
         L.lf_release_scratch.restype = st
         L.lf_attention_forward_noalloc.argtypes = [vp] * 8 + [i, i, i, i, i, vp, vp]
         L.lf_attention_forward_noalloc.restype = st
+        L.lf_encoder_layer_workspace_bytes.argtypes = [i, i, i, i, i, i]
+        L.lf_encoder_layer_workspace_bytes.restype = ctypes.c_size_t
+        L.lf_encoder_layer_forward.argtypes = [vp, vp, vp, ctypes.POINTER(LayerWeights), i, i, i, i,
+                                               ctypes.c_float, ctypes.c_float, i, vp, ctypes.c_size_t, vp, vp]
+        L.lf_encoder_layer_forward.restype = st
         _lib = L
     return _lib
 
@@ -141,4 +154,30 @@ def lf_attention_forward_noalloc(q, k, v, qg, kg, vg, local_mask, global_mask, w
                                             _ptr(local_mask), _ptr(global_mask), B, H, L, w, code,
                                             _stream(stream), _ptr(out))
     _check(st, "lf_attention_forward_noalloc")
+    return out
+
+
+def lf_encoder_layer_workspace_bytes(B: int, H: int, L: int, w: int, ffn_dim: int, dtype) -> int:
+    return lib().lf_encoder_layer_workspace_bytes(B, H, L, w, ffn_dim, DTYPE_CODE[dtype])
+
+
+def lf_encoder_layer_forward(x, local_mask, global_mask, weights: dict, H: int, w: int, attn_scale: float = 0.125,
+                             ln_eps: float = 1e-5, out=None, workspace=None, stream=None):
+    """One encoder layer; x [B, L, H*64]; weights: tensors named as the
+    fields of lf_layer_weights (nn.Linear layout [out, in]), LayerNorm
+    parameters fp32.  Returns out [B, L, H*64]."""
+    B, L, D = x.shape
+    ffn = weights["W_1"].shape[0]
+    wt = LayerWeights(ffn, *[weights[n].data_ptr() for n in LAYER_FIELDS])
+    for n in LAYER_FIELDS:
+        _ptr(weights[n])
+    if out is None:
+        out = torch.empty_like(x)
+    need = lf_encoder_layer_workspace_bytes(B, H, L, w, ffn, x.dtype)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=x.device)
+    st = lib().lf_encoder_layer_forward(_ptr(x), _ptr(local_mask), _ptr(global_mask), ctypes.byref(wt), B, H, L,
+                                        w, attn_scale, ln_eps, DTYPE_CODE.get(x.dtype, 99), _ptr(workspace),
+                                        workspace.numel(), _stream(stream), _ptr(out))
+    _check(st, "lf_encoder_layer_forward")
     return out
