@@ -6,8 +6,8 @@
 // masked-softmax kernel and a transpose kernel.  Here it is ONE persistent
 // kernel per call.
 //
-// Work items (taken from a global atomic counter; band pairs first, then the
-// smaller global pairs, so that the last items handed out are short):
+// Work items (taken from a global atomic counter; global pairs first, so that
+// their split merges overlap the band pairs that follow):
 //   global pair (b, h, row tile rt, splits 2s and 2s+1): rows i < g_b attend
 //       to every key through qg/kg/vg.  Keys are cut into chunks of
 //       kChunkBlocks 128-key blocks; each split leaves (m, l, O) partials in
@@ -26,8 +26,8 @@
 // its registers over; warpgroups 1 and 2
 // are the softmax warpgroups of tile A and tile B (one thread per query row).
 // Registers are rebalanced with setmaxnreg: launched at 168 per thread,
-// warpgroup 0 drops to 64 and the softmax warpgroups rise to 216
-// (4*32*64 + 8*32*216 = 63488 <= 384*168 = 64512).  Per tile X and key block:
+// warpgroup 0 drops to 96 and the softmax warpgroups rise to 200
+// (4*32*96 + 8*32*200 = 63488 <= 384*168 = 64512).  Per tile X and key block:
 //   S_X = Q_X K^T           (TMEM, fp32)
 //   softmax warps: read S_X, scale, padding bias, mask, row max; rescale the
 //   TMEM accumulator O_X only when the running max grows by more than 8 (in
@@ -61,8 +61,8 @@ constexpr int kRing = 4;          // item-id ring depth
 constexpr int kWarps = 12;
 constexpr int kThreads = kWarps * 32;
 constexpr int kSoftmaxWarp0 = 4;
-constexpr uint32_t kRegsProducer = 64;
-constexpr uint32_t kRegsSoftmax = 216;
+constexpr uint32_t kRegsProducer = 96;
+constexpr uint32_t kRegsSoftmax = 200;
 static_assert(4 * 32 * kRegsProducer + 8 * 32 * kRegsSoftmax <= kThreads * 168, "register split");
 constexpr int kItemConsumers = 1 + 1 + 8;  // TMA warp + MMA warp + 8 softmax warps
 constexpr uint32_t kTileBytes = kBM * kHD * 2;  // 16 KB
@@ -92,7 +92,8 @@ struct Params {
     int NS;      // key splits per global row tile
     int NSP;     // split pairs per global row tile
     int NTP;     // tile pairs per head
-    int n_band;  // band pair items (they come first; global pairs follow)
+    int n_glob;  // global pair items (they come first: their split merges
+                 // then overlap band work instead of trailing the kernel)
     int n_items;
     float scale_log2;  // scale * log2(e)
     float inv_scale;   // 1 / scale: the padding bias in raw score units
@@ -224,8 +225,8 @@ __device__ void band_rows(const Params& p, int b, int r0, int g, int& work, int&
 __device__ Plan make_plan(const Params& p, int id, int& cached_b, int& g) {
     Plan pl;
     pl.id = id;
-    if (id >= p.n_band) {
-        const int id2 = id - p.n_band;
+    if (id < p.n_glob) {
+        const int id2 = id;
         pl.global = 1;
         const int sp = id2 % p.NSP;
         const int r = id2 / p.NSP;
@@ -234,10 +235,11 @@ __device__ Plan make_plan(const Params& p, int id, int& cached_b, int& g) {
         pl.t[0].split = 2 * sp;
         pl.t[1].split = 2 * sp + 1;
     } else {
+        const int id2 = id - p.n_glob;
         pl.global = 0;
         pl.rt = 0;
-        const int tp = id % p.NTP;
-        pl.bh = id / p.NTP;
+        const int tp = id2 % p.NTP;
+        pl.bh = id2 / p.NTP;
         pl.t[0].r0 = 2 * tp * kBM;
         pl.t[1].r0 = (2 * tp + 1) * kBM;
     }
@@ -1065,15 +1067,18 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
                         if (lm[i] != 1.0f) {
                             store_zero_row(p.out, off, sizeof(T));
                         } else {
+                            // all (m, l) of the row first, in flight together
+                            constexpr int kMaxNS = 64;
+                            float2 mls[kMaxNS];
+                            const int ns = min(p.NS, kMaxNS);
                             float M = -INFINITY;
-                            for (int s = 0; s < p.NS; ++s)
-                                M = fmaxf(M, __ldcg(p.part_ml + ((size_t)(slot0 + s) * kBM + r) * 2));
-                            float lsum = 0.0f;
-                            for (int s = 0; s < p.NS; ++s) {
-                                const float2 ml = __ldcg(
+                            for (int s = 0; s < ns; ++s)
+                                mls[s] = __ldcg(
                                     reinterpret_cast<const float2*>(p.part_ml + ((size_t)(slot0 + s) * kBM + r) * 2));
-                                lsum = fmaf(ml.y, ml.x == -INFINITY ? 0.0f : ex2(ml.x - M), lsum);
-                            }
+                            for (int s = 0; s < ns; ++s) M = fmaxf(M, mls[s].x);
+                            float lsum = 0.0f;
+                            for (int s = 0; s < ns; ++s)
+                                lsum = fmaf(mls[s].y, mls[s].x == -INFINITY ? 0.0f : ex2(mls[s].x - M), lsum);
                             const float inv = fast_rcp(lsum);
                             // merge 16 channels at a time to keep registers low
                             for (int cq = 0; cq < kHD; cq += 16) {
@@ -1220,8 +1225,8 @@ lf_status launch_attention_tc(const void* q, const void* k, const void* v, const
     p.NS = geo.NS;
     p.NSP = geo.NSP;
     p.NTP = geo.NTP;
-    p.n_band = BH * geo.NTP;
-    p.n_items = p.n_band + BH * geo.RT * geo.NSP;
+    p.n_glob = BH * geo.RT * geo.NSP;
+    p.n_items = p.n_glob + BH * geo.NTP;
     p.scale_log2 = scale * kLog2e;
     p.inv_scale = 1.0f / scale;
     p.local_mask = local_mask;
