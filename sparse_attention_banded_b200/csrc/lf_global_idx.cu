@@ -1,7 +1,7 @@
 // Global-token index partition (invokeInitLongformerIdx of the
 // FasterTransformer Longformer page, §Longformer Encoder 计算流程 / 预处理).
 //
-// One CTA per sample walks the row in chunks of kThreads * 4 positions.  Each
+// One CTA (1024 threads) per sample walks the row in chunks of 4096 positions.  Each
 // thread flags its 4 positions (global_mask == 0.0f), a block-wide exclusive
 // scan of the per-thread counts gives every flagged position its slot at the
 // front (ascending) and every unflagged one its slot at the back
@@ -17,7 +17,7 @@
 namespace lf {
 namespace {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 1024;
 constexpr int kItems = 4;
 
 __global__ void __launch_bounds__(kThreads)
@@ -28,7 +28,7 @@ global_idx_kernel(const float* __restrict__ global_mask, int L, int w, int32_t* 
     int32_t* idx = global_idx + (size_t)b * L;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
-    __shared__ int warp_tot[kThreads / 32];
+    __shared__ int warp_tot[kThreads / 32 + 1];
     __shared__ int first_unflagged;
     if (tid == 0) first_unflagged = L;
     __syncthreads();
@@ -62,13 +62,19 @@ global_idx_kernel(const float* __restrict__ global_mask, int L, int w, int32_t* 
         }
         if (lane == 31) warp_tot[warp] = incl;
         __syncthreads();
-        int warp_base = 0, chunk_tot = 0;
+        if (warp == 0) {  // exclusive scan of the 32 warp totals; slot 32 = chunk total
+            const int t = warp_tot[lane];
+            int x = t;
 #pragma unroll
-        for (int i = 0; i < kThreads / 32; ++i) {
-            int t = warp_tot[i];
-            if (i < warp) warp_base += t;
-            chunk_tot += t;
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, x, o);
+                if (lane >= o) x += y;
+            }
+            warp_tot[lane] = x - t;
+            if (lane == 31) warp_tot[32] = x;
         }
+        __syncthreads();
+        const int warp_base = warp_tot[warp], chunk_tot = warp_tot[32];
         int sel = base + warp_base + incl - cnt;  // flagged before position j0
 #pragma unroll
         for (int t = 0; t < kItems; ++t) {
