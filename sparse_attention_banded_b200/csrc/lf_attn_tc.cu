@@ -6,11 +6,13 @@
 // masked-softmax kernel and a transpose kernel.  Here it is ONE persistent
 // kernel per call.
 //
-// Work items (taken from a global atomic counter; global pairs first, so that
-// their split merges overlap the band pairs that follow):
+// Work items, taken from a global atomic counter longest first: band pairs
+// away from the sequence ends, then global pairs (their split merges overlap
+// the band work that follows), then the band pairs at the sequence ends:
 //   global pair (b, h, row tile rt, splits 2s and 2s+1): rows i < g_b attend
-//       to every key through qg/kg/vg.  Keys are cut into chunks of
-//       kChunkBlocks 128-key blocks; each split leaves (m, l, O) partials in
+//       to every key through qg/kg/vg.  Keys are cut into chunks of `chunk`
+//       128-key blocks (picked per shape on the host so that the items pack
+//       evenly onto the SMs); each split leaves (m, l, O) partials in
 //       scratch and the warp that finishes the last split of its 32 rows
 //       merges them (log-sum-exp) and writes the rows.
 //   band pair (b, h, tiles 2p and 2p+1 of 128 query rows): each tile visits
@@ -42,7 +44,10 @@
 
 #include <stdlib.h>
 
+#include <algorithm>
+#include <functional>
 #include <mutex>
+#include <vector>
 
 #include "lf_internal.h"
 #include "sm100.cuh"
@@ -56,7 +61,8 @@ constexpr int kBM = 128;          // query rows per tile
 constexpr int kBN = 128;          // keys per block
 constexpr int kHD = 64;           // head dim
 constexpr int kStages = 4;        // K/V ring depth
-constexpr int kChunkBlocks = 4;   // key blocks per global-row split
+constexpr int kMinChunk = 4;      // key blocks per global-row split: chosen per
+constexpr int kMaxChunk = 16;     // shape in [kMinChunk, kMaxChunk] on the host
 constexpr int kRing = 4;          // item-id ring depth
 constexpr int kWarps = 12;
 constexpr int kThreads = kWarps * 32;
@@ -92,8 +98,10 @@ struct Params {
     int NS;      // key splits per global row tile
     int NSP;     // split pairs per global row tile
     int NTP;     // tile pairs per head
-    int n_glob;  // global pair items (they come first: their split merges
-                 // then overlap band work instead of trailing the kernel)
+    int chunk;   // key blocks per global-row split
+    int n_inner; // band pairs away from the sequence ends (first in the order)
+    int n_glob;  // global pair items (next: their split merges then overlap
+                 // the band pairs at the ends of the sequences, which are last)
     int n_items;
     float scale_log2;  // scale * log2(e)
     float inv_scale;   // 1 / scale: the padding bias in raw score units
@@ -225,8 +233,12 @@ __device__ void band_rows(const Params& p, int b, int r0, int g, int& work, int&
 __device__ Plan make_plan(const Params& p, int id, int& cached_b, int& g) {
     Plan pl;
     pl.id = id;
-    if (id < p.n_glob) {
-        const int id2 = id;
+    // Item order, longest first: interior band pairs (the most key blocks),
+    // then global pairs, then the band pairs at both ends of each sequence.
+    const int inner_per = p.NTP > 2 ? p.NTP - 2 : 0;
+    const int edge_per = p.NTP < 2 ? p.NTP : 2;
+    if (id >= p.n_inner && id < p.n_inner + p.n_glob) {
+        const int id2 = id - p.n_inner;
         pl.global = 1;
         const int sp = id2 % p.NSP;
         const int r = id2 / p.NSP;
@@ -235,11 +247,17 @@ __device__ Plan make_plan(const Params& p, int id, int& cached_b, int& g) {
         pl.t[0].split = 2 * sp;
         pl.t[1].split = 2 * sp + 1;
     } else {
-        const int id2 = id - p.n_glob;
+        int tp;
+        if (id < p.n_inner) {
+            tp = 1 + id % inner_per;
+            pl.bh = id / inner_per;
+        } else {
+            const int e = id - p.n_inner - p.n_glob;
+            tp = (e % edge_per == 0) ? 0 : p.NTP - 1;
+            pl.bh = e / edge_per;
+        }
         pl.global = 0;
         pl.rt = 0;
-        const int tp = id2 % p.NTP;
-        pl.bh = id2 / p.NTP;
         pl.t[0].r0 = 2 * tp * kBM;
         pl.t[1].r0 = (2 * tp + 1) * kBM;
     }
@@ -267,8 +285,8 @@ __device__ Plan make_plan(const Params& p, int id, int& cached_b, int& g) {
             t.r0 = r0;
             if (r0 < g && t.split < p.NS) {
                 t.present = 1;
-                t.lo = t.split * kChunkBlocks;
-                t.hi = min(p.NKB, t.lo + kChunkBlocks) - 1;
+                t.lo = t.split * p.chunk;
+                t.hi = min(p.NKB, t.lo + p.chunk) - 1;
             }
         }
         const int nA = pl.t[0].present ? pl.t[0].hi - pl.t[0].lo + 1 : 0;
@@ -399,17 +417,6 @@ __device__ __forceinline__ float fast_rcp(float x) {
     float y;
     asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
-}
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
-        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
-        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
-        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
-        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
-        "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
-        "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
-        : "memory");
 }
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
@@ -556,6 +563,17 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     if (threadIdx.x == 0) TRACE(11, 1, 0, 0, 0);
+#if LF_TRACE
+    if (threadIdx.x == 0 && p.trace) {  // CTA start time and SM id
+        const unsigned long long t = globaltimer();
+        volatile int* d_ = p.trace + gridDim.x * 16 * 4 + (blockIdx.x * 16 + 12) * 16;
+        d_[0] = (int)(t & 0xffffffffu);
+        d_[1] = (int)(t >> 32);
+        unsigned smid;
+        asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
+        d_[4] = (int)smid;
+    }
+#endif
 
     if (warp < kSoftmaxWarp0) {
     regs_dec<kRegsProducer>();
@@ -676,7 +694,6 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
             if (lane == 0) mbar_arrive(&item_empty[slot]);
             const int id = pl.id;
             if (id < 0) break;
-            const int g = pl.g;
             if (pl.nloads == 0) continue;
             if (lane == 0) {
                 const uint32_t qb = item_cnt & 1;
@@ -917,6 +934,7 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
                         float r[32];
                         tmem_ld32f(tS + ch * 32, r);
                         tmem_ld_wait();
+                        regs_ready<32>(r);
                         fix_chunk(ch, r);
 #pragma unroll
                         for (int c = 0; c < 32; c += 8) {
@@ -950,6 +968,7 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
                                 uint32_t ob[16];
                                 tmem_ld16(tO + c0o, ob);
                                 tmem_ld_wait();
+                                regs_ready<16>(ob);
 #pragma unroll
                                 for (int c = 0; c < 16; ++c)
                                     ob[c] = __float_as_uint(__uint_as_float(ob[c]) * factor);
@@ -987,6 +1006,7 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
                             float r[32];
                             tmem_ld32f(tS + ch * 32, r);
                             tmem_ld_wait();
+                            regs_ready<32>(r);
                             fix_chunk(ch, r);
                             exp_chunk(r, pk);
                         }
@@ -1025,6 +1045,8 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
                 tmem_ld32(tO, o0);
                 tmem_ld32(tO + 32, o1);
                 tmem_ld_wait();
+                regs_ready<32>(o0);
+                regs_ready<32>(o1);
 #pragma unroll
                 for (int c = 0; c < 32; ++c) {
                     o[c] = __uint_as_float(o0[c]);
@@ -1075,10 +1097,18 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
                             for (int s = 0; s < ns; ++s)
                                 mls[s] = __ldcg(
                                     reinterpret_cast<const float2*>(p.part_ml + ((size_t)(slot0 + s) * kBM + r) * 2));
-                            for (int s = 0; s < ns; ++s) M = fmaxf(M, mls[s].x);
+                            // splits beyond the batch are read again where used
+                            auto ml_of = [&](int s) -> float2 {
+                                return s < ns ? mls[s]
+                                              : __ldcg(reinterpret_cast<const float2*>(
+                                                    p.part_ml + ((size_t)(slot0 + s) * kBM + r) * 2));
+                            };
+                            for (int s = 0; s < p.NS; ++s) M = fmaxf(M, ml_of(s).x);
                             float lsum = 0.0f;
-                            for (int s = 0; s < ns; ++s)
-                                lsum = fmaf(mls[s].y, mls[s].x == -INFINITY ? 0.0f : ex2(mls[s].x - M), lsum);
+                            for (int s = 0; s < p.NS; ++s) {
+                                const float2 ml = ml_of(s);
+                                lsum = fmaf(ml.y, ml.x == -INFINITY ? 0.0f : ex2(ml.x - M), lsum);
+                            }
                             const float inv = fast_rcp(lsum);
                             // merge 16 channels at a time to keep registers low
                             for (int cq = 0; cq < kHD; cq += 16) {
@@ -1132,6 +1162,14 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
             __threadfence();
         }
         TRACE(10, 99, 0, 0, 0);
+#if LF_TRACE
+        if (p.trace) {  // CTA end time
+            const unsigned long long t = globaltimer();
+            volatile int* d_ = p.trace + gridDim.x * 16 * 4 + (blockIdx.x * 16 + 12) * 16;
+            d_[2] = (int)(t & 0xffffffffu);
+            d_[3] = (int)(t >> 32);
+        }
+#endif
     }
     if (warp == 1) {
         tc_fence_after();
@@ -1171,17 +1209,119 @@ bool make_map(CUtensorMap* m, const void* base, int BH, int L) {
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Global-row split size.  Items are taken from a counter by the CTAs as they
+// free up, so the kernel ends when the last CTA finishes its last item; with
+// only a few items per CTA the split size decides how evenly the work packs.
+// The host replays that list schedule for each candidate size with a cost
+// model of the kernel (per item: a fixed part plus its longer tile's key
+// blocks; a global pair adds its merge; relative weights 80 : 60 per block :
+// 30, from event traces of the kernel on B200) and keeps the size with the
+// earliest finish.  Leading
+// globals are taken as g <= 128 (one global row tile with work, one block of
+// global keys per band tile); the choice only affects speed.
+int choose_chunk(int B, int H, int L, int w, int sm_count) {
+    const int NKB = (L + kBN - 1) / kBN;
+    const int NT = (L + kBM - 1) / kBM;
+    const int NTP = (NT + 1) / 2;
+    const int RT = (w + kBM - 1) / kBM;
+    const int BH = B * H;
+    const int lo_c = kMinChunk < NKB ? kMinChunk : NKB;
+    const int hi_c = kMaxChunk < NKB ? kMaxChunk : NKB;
+    const long long n_band = (long long)BH * NTP;
+    if (sm_count <= 0 || n_band * (hi_c - lo_c + 1) > 4000000LL) return lo_c;
+    struct Key {
+        int B, H, L, w, sm, chunk;
+    };
+    static std::mutex mu;
+    static Key cache[16];
+    static int n_cache = 0;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        for (int i = 0; i < n_cache; ++i)
+            if (cache[i].B == B && cache[i].H == H && cache[i].L == L && cache[i].w == w && cache[i].sm == sm_count)
+                return cache[i].chunk;
+    }
+    constexpr long long kBlock = 60, kItem = 80, kMerge = 30, kEmpty = 10;
+    auto band_blocks = [&](int r0) -> int {
+        if (r0 >= L) return 0;
+        const int lo = (r0 - w <= 0 ? 0 : r0 - w) / kBN;
+        const int hi = (r0 + kBM - 1 + w) / kBN < NKB - 1 ? (r0 + kBM - 1 + w) / kBN : NKB - 1;
+        return (lo > 0 ? 1 : 0) + hi - lo + 1;
+    };
+    auto pair_cost = [&](int tp) -> long long {
+        const int a = band_blocks(2 * tp * kBM), b = band_blocks((2 * tp + 1) * kBM);
+        return (a > b ? a : b) * kBlock + kItem;
+    };
+    std::vector<long long> costs;
+    std::vector<long long> heap;
+    long long best = -1;
+    int best_c = lo_c;
+    for (int c = lo_c; c <= hi_c; ++c) {
+        const int NS = (NKB + c - 1) / c, NSP = (NS + 1) / 2;
+        costs.clear();
+        for (int bh = 0; bh < BH; ++bh)
+            for (int tp = 1; tp + 1 < NTP; ++tp) costs.push_back(pair_cost(tp));
+        for (int bh = 0; bh < BH; ++bh)
+            for (int rt = 0; rt < RT; ++rt)
+                for (int sp = 0; sp < NSP; ++sp) {
+                    if (rt > 0) {
+                        costs.push_back(kEmpty);
+                        continue;
+                    }
+                    int m = 0;
+                    for (int s = 2 * sp; s < 2 * sp + 2 && s < NS; ++s) {
+                        const int n = (NKB < s * c + c ? NKB : s * c + c) - s * c;
+                        m = n > m ? n : m;
+                    }
+                    costs.push_back(m * kBlock + kItem + kMerge);
+                }
+        for (int bh = 0; bh < BH; ++bh) {
+            costs.push_back(pair_cost(0));
+            if (NTP > 1) costs.push_back(pair_cost(NTP - 1));
+        }
+        heap.assign(sm_count, 0);  // min-heap of CTA finish times
+        for (long long cst : costs) {
+            std::pop_heap(heap.begin(), heap.end(), std::greater<long long>());
+            heap.back() += cst;
+            std::push_heap(heap.begin(), heap.end(), std::greater<long long>());
+        }
+        const long long span = *std::max_element(heap.begin(), heap.end());
+        if (best < 0 || span < best) {
+            best = span;
+            best_c = c;
+        }
+    }
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        if (n_cache < 16) cache[n_cache++] = Key{B, H, L, w, sm_count, best_c};
+    }
+    return best_c;
+}
+
+int current_sm_count() {
+    static int sms[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+    if (sms[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+        sms[dev] = n;
+    }
+    return sms[dev];
+}
+
 struct Geometry {
-    int NKB, NT, RT, NS, NSP, NTP;
+    int NKB, NT, RT, NS, NSP, NTP, chunk;
     size_t sched_bytes, counters_bytes, part_o_bytes, part_ml_bytes;
 };
 
-Geometry geometry(int B, int H, int L, int w) {
+Geometry geometry(int B, int H, int L, int w, int sm_count) {
     Geometry g;
     g.NKB = (L + kBN - 1) / kBN;
     g.NT = (L + kBM - 1) / kBM;
     g.RT = (w + kBM - 1) / kBM;
-    g.NS = (g.NKB + kChunkBlocks - 1) / kChunkBlocks;
+    g.chunk = choose_chunk(B, H, L, w, sm_count);
+    g.NS = (g.NKB + g.chunk - 1) / g.chunk;
     g.NSP = (g.NS + 1) / 2;
     g.NTP = (g.NT + 1) / 2;
     const size_t slots = (size_t)B * H * g.RT * g.NS;
@@ -1195,12 +1335,12 @@ Geometry geometry(int B, int H, int L, int w) {
 }  // namespace
 
 size_t attention_tc_scratch_bytes(int B, int H, int L, int w) {
-    const Geometry g = geometry(B, H, L, w);
+    const Geometry g = geometry(B, H, L, w, current_sm_count());
     return g.sched_bytes + g.counters_bytes + g.part_o_bytes + g.part_ml_bytes;
 }
 
 size_t attention_tc_scratch_zero_bytes(int B, int H, int L, int w) {
-    const Geometry g = geometry(B, H, L, w);
+    const Geometry g = geometry(B, H, L, w, current_sm_count());
     return g.sched_bytes + g.counters_bytes;
 }
 
@@ -1208,7 +1348,7 @@ lf_status launch_attention_tc(const void* q, const void* k, const void* v, const
                               const void* vg, const float* local_mask, const float* global_mask, int B, int H,
                               int L, int w, float scale, lf_dtype dtype, void* out, void* scratch, int* status,
                               int sm_count, cudaStream_t stream) {
-    const Geometry geo = geometry(B, H, L, w);
+    const Geometry geo = geometry(B, H, L, w, sm_count);
     Maps maps;
     const int BH = B * H;
     if (!make_map(&maps.q, q, BH, L) || !make_map(&maps.k, k, BH, L) || !make_map(&maps.v, v, BH, L) ||
@@ -1225,6 +1365,8 @@ lf_status launch_attention_tc(const void* q, const void* k, const void* v, const
     p.NS = geo.NS;
     p.NSP = geo.NSP;
     p.NTP = geo.NTP;
+    p.chunk = geo.chunk;
+    p.n_inner = BH * (geo.NTP > 2 ? geo.NTP - 2 : 0);
     p.n_glob = BH * geo.RT * geo.NSP;
     p.n_items = p.n_glob + BH * geo.NTP;
     p.scale_log2 = scale * kLog2e;

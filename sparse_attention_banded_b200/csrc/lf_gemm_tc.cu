@@ -223,6 +223,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
                 __syncwarp();  // tcgen05.ld is .sync.aligned: whole warp, converged
                 tmem_ld32v(tmem + lane_off + ab * kTN + c0, acc);
                 tmem_ld_wait();
+                regs_ready<32>(acc);
 #pragma unroll
                 for (int c = 0; c < 32; ++c) acc[c] += bias_w[c0 + c];
                 const int n = n0 + c0;

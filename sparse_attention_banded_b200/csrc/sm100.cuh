@@ -46,6 +46,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
+// Non-blocking test of a phase (never suspends the thread).
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 // Bounded wait.  Returns false when `abort` is raised by another thread or
 // when the wait exceeds `limit_ns`; in the second case it raises `abort`
 // itself so that every role of the CTA winds down.
@@ -156,6 +169,20 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
         : "r"(taddr));
 }
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// tcgen05.ld fills its registers asynchronously; they are valid only after
+// tcgen05.wait::ld.  Passing them through an empty volatile asm after the
+// wait keeps the compiler from moving any use of them above the wait.
+template <int N>
+__device__ __forceinline__ void regs_ready(float* r) {
+#pragma unroll
+    for (int c = 0; c < N; ++c) asm volatile("" : "+f"(r[c]));
+}
+template <int N>
+__device__ __forceinline__ void regs_ready(uint32_t* r) {
+#pragma unroll
+    for (int c = 0; c < N; ++c) asm volatile("" : "+r"(r[c]));
+}
 
 __device__ __forceinline__ float ex2(float x) {
     float y;
