@@ -9,8 +9,12 @@ footprint (~50 MB) fits in L2, so L2 is flushed (a 2 x L2 write) before
 every timed step, outside the step's event pair.
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+                       [--workload N]
 Under torchrun each rank runs its own replica of the workload (weak scaling,
 no collective on the data path); timings are the max over ranks.
+--workload selects another of the synthetic configurations (1: fp32
+attention, 3: bf16 batched, 4: fp16 L=16384, 5: one fp16 encoder layer with
+its projections, LayerNorms and FFN); 2 is the default and the headline.
 """
 from __future__ import annotations
 
@@ -46,6 +50,7 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=50)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", type=int, default=WORKLOAD_ID, choices=[1, 2, 3, 4, 5])
     return ap.parse_args()
 
 
@@ -171,21 +176,38 @@ def run_ours(args):
     if world > 1:
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
-    wl, t_cpu, lm_cpu, gm_cpu = inputs.workload_inputs(WORKLOAD_ID)
-    t = {n: t_cpu[n].to(dev) for n in inputs.NAMES}
+    layer = args.workload == 5
+    if layer:
+        wl, x_cpu, wts_cpu, lm_cpu, gm_cpu = inputs.layer_inputs(5)
+        x = x_cpu.to(dev)
+        wts = {n: v.to(dev) for n, v in wts_cpu.items()}
+        ffn = wts["W_1"].shape[0]
+        ws = torch.empty(max(256, lf.lf_encoder_layer_workspace_bytes(wl.B, wl.H, wl.L, wl.w, ffn, x.dtype)),
+                         dtype=torch.uint8, device=dev)
+        args_in = [x]
+        t_cpu = None
+    else:
+        wl, t_cpu, lm_cpu, gm_cpu = inputs.workload_inputs(args.workload)
+        t = {n: t_cpu[n].to(dev) for n in inputs.NAMES}
+        args_in = [t[n] for n in inputs.NAMES]
     lm, gm = lm_cpu.to(dev), gm_cpu.to(dev)
-    out = torch.empty(wl.B, wl.L, wl.H * 64, dtype=t["q"].dtype, device=dev)
+    out = torch.empty(wl.B, wl.L, wl.H * 64, dtype=args_in[0].dtype, device=dev)
     gidx = torch.empty(wl.B, wl.L, dtype=torch.int32, device=dev)
     gnum = torch.empty(wl.B, dtype=torch.int32, device=dev)
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     flush = torch.empty(max(2 * l2, 256 << 20) // 4, dtype=torch.float32, device=dev)
-    args_in = [t[n] for n in inputs.NAMES]
+
+    def compute(ins, lm_, gm_):
+        if layer:
+            lf.lf_encoder_layer_forward(ins[0], lm_, gm_, wts, wl.H, wl.w, out=out, workspace=ws)
+        else:
+            lf.lf_attention_forward(*ins, lm_, gm_, wl.w, out=out)
 
     def step(ev_a=None):
         lf.lf_init_global_idx(gm, wl.w, gidx, gnum, sync=False)
         if ev_a is not None:
             ev_a.record()
-        lf.lf_attention_forward(*args_in, lm, gm, wl.w, out=out)
+        compute(args_in, lm, gm)
 
     lf.lf_device_status(reset=True)
     for _ in range(max(args.warmup, 3)):
@@ -233,11 +255,13 @@ def run_ours(args):
     h2d = sum(x.numel() * x.element_size() for x in h_in)
     d2h = h_out.numel() * h_out.element_size()
 
+    n_t = len(args_in)
+
     def e2e_step():
         for h, d in zip(h_in, d_in):
             d.copy_(h, non_blocking=True)
-        lf.lf_init_global_idx(d_in[7], wl.w, gidx, gnum, sync=False)
-        lf.lf_attention_forward(*d_in[:6], d_in[6], d_in[7], wl.w, out=out)
+        lf.lf_init_global_idx(d_in[n_t + 1], wl.w, gidx, gnum, sync=False)
+        compute(d_in[:n_t], d_in[n_t], d_in[n_t + 1])
         h_out.copy_(out, non_blocking=True)
 
     for _ in range(3):
@@ -259,11 +283,26 @@ def run_ours(args):
         raise RuntimeError("device status after timing: %s" % lf.status_string(st))
 
     pk, pk_kind = peaks()
-    F = metrics.flops(wl.B, wl.H, wl.L, wl.w, wl.g, wl.pad)
-    By = metrics.algorithmic_bytes(wl.B, wl.H, wl.L, wl.w, wl.g, wl.dtype)
+    if layer:
+        F = metrics.layer_flops(wl.B, wl.H, wl.L, wl.w, wl.g, wl.pad, ffn)
+        wbytes = sum(v.numel() * v.element_size() for v in wts.values())
+        By = float(wbytes + 2 * x.numel() * x.element_size() + 2 * wl.B * wl.L * 4)
+    else:
+        F = metrics.flops(wl.B, wl.H, wl.L, wl.w, wl.g, wl.pad)
+        By = metrics.algorithmic_bytes(wl.B, wl.H, wl.L, wl.w, wl.g, wl.dtype)
     t_attn = attn_avg_ms * 1e-3
     tokens = wl.B * wl.L
     value = world * tokens * K / (total_ms * 1e-3)
+    tensor_path = wl.dtype in ("f16", "bf16")
+    if layer:
+        roof = {"bound": "tensor", "achieved": F / t_attn / 1e12, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": F / t_attn / 1e12 / pk["bf16_tflops"], "traffic": None, "peak_kind": pk_kind,
+                "algorithmic_bytes_per_launch": By, "flops_per_launch": F}
+    else:
+        roof = {"bound": "hbm", "achieved": By / t_attn / 1e9, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": By / t_attn / 1e9 / pk["hbm_gbs"],
+                "traffic": traffic_from_profile(kernel_source_hash()) if args.workload == WORKLOAD_ID else None,
+                "peak_kind": pk_kind, "algorithmic_bytes_per_launch": By, "flops_per_launch": F}
     res = {
         "metric": METRIC,
         "value": value,
@@ -275,36 +314,27 @@ def run_ours(args):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "f16",
-        "data": "synthetic (seeded N(0,1)*0.5 inputs of the workload's shape)",
+        "dtype": wl.dtype,
+        "data": "synthetic (seeded inputs of the workload's shape%s)" %
+                (": x ~ N(0,1), weights ~ N(0, 0.02)" if layer else ", N(0,1)*0.5"),
         "config": {"workload": wl.name, "B": wl.B, "H": wl.H, "L": wl.L, "w": wl.w, "g": wl.g,
                    "pad": wl.pad, "head_dim": 64, "l2": "flushed before every timed step (2 x L2 write)",
                    "parallelism": "replica per GPU (weak)" if world > 1 else "single GPU"},
         "tflops": F / (total_ms * 1e-3 / K) / 1e12,
-        "attention_kernel": {
+        ("layer" if layer else "attention_kernel"): {
             "avg_us": attn_avg_ms * 1e3,
             "tflops": F / t_attn / 1e12,
-            "tensor_peak_frac": F / t_attn / 1e12 / pk["bf16_tflops"],
+            "tensor_peak_frac": F / t_attn / 1e12 / pk["bf16_tflops"] if tensor_path else None,
             "tensor_peak_tflops": pk["bf16_tflops"],
             "note": "fp16 and bf16 dense tensor rates are equal; peak = measured bf16 burst (%s)" % pk_kind,
         },
-        "roofline": {
-            "bound": "hbm",
-            "achieved": By / t_attn / 1e9,
-            "peak": pk["hbm_gbs"],
-            "unit": "GB/s",
-            "frac": By / t_attn / 1e9 / pk["hbm_gbs"],
-            "traffic": traffic_from_profile(kernel_source_hash()),
-            "peak_kind": pk_kind,
-            "algorithmic_bytes_per_launch": By,
-            "flops_per_launch": F,
-        },
+        "roofline": roof,
         "e2e": {"value": world * tokens / (e2e_ms * 1e-3), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": 2 * K,
+        "gpu_launches": (1 + (8 if layer else 1)) * K,
         "clocks": clocks,
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not layer:
         res["cpu_baseline"] = cpu_baseline(wl, t_cpu, lm_cpu, gm_cpu)
     if world > 1:
         torch.distributed.destroy_process_group()

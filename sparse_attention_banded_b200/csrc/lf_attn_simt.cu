@@ -4,9 +4,10 @@
 // Transformer 层 steps 3-5.  fp32 inputs have no tensor-core path that keeps
 // the 1e-4 error bound, so this kernel computes the same function as the
 // tensor-core kernel with plain FMAs:
-//   one warp per output row (b, h, i); the row's key set is walked in chunks
-//   of 32 keys (lane = key) with an online softmax; lane c then owns output
-//   channels c and c + 32.
+//   one CTA per output row (b, h, i); its warps walk interleaved chunks of
+//   32 keys of the row's key set (lane = key) with an online softmax each,
+//   lane c owning output channels c and c + 32, and the partial results are
+//   merged (log-sum-exp) in shared memory.
 // Key set (local row i >= g_b): [0, g_b) then [max(i - w, g_b), min(i + w,
 // L - 1)], each key once; global row i < g_b: [0, L) with qg/kg/vg.  Score
 // = scale * <q_i, k_j> + lb[j], lb[j] = fmaf(local_mask[j], 1e4, -1e4).
@@ -44,56 +45,66 @@ struct RowState {
     float m, l, o0, o1;
 };
 
-// Process keys [j_begin, j_end] (inclusive) of one row.
-__device__ __forceinline__ void process_range(RowState& st, const float* sq, const float* K, const float* V,
-                                              const float* lm_row, int j_begin, int j_end, float scale,
-                                              int lane) {
-    for (int base = j_begin; base <= j_end; base += 32) {
-        const int j = base + lane;
-        const bool valid = j <= j_end;
-        float s = -INFINITY;
-        if (valid) {
-            const float4* kr = reinterpret_cast<const float4*>(K + (size_t)j * 64);
-            float acc = 0.0f;
+// Keys at list positions [pos0, pos0 + 32) of one row (lane = key): the
+// row's key list is [0, g_seg) followed by [lo, hi], each key once.
+__device__ __forceinline__ void process_chunk(RowState& st, const float* sq, const float* K, const float* V,
+                                              const float* lm_row, int pos0, int g_seg, int lo, int n_keys,
+                                              float scale, int lane) {
+    const int pos = pos0 + lane;
+    const bool valid = pos < n_keys;
+    const int j = valid ? (pos < g_seg ? pos : lo + (pos - g_seg)) : 0;
+    float s = -INFINITY;
+    if (valid) {
+        const float4* kr = reinterpret_cast<const float4*>(K + (size_t)j * 64);
+        // four partial sums over interleaved columns, added at the end
+        float a4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
-            for (int c = 0; c < 16; ++c) {
-                const float4 kv = kr[c];
-                acc = fmaf(sq[4 * c + 0], kv.x, acc);
-                acc = fmaf(sq[4 * c + 1], kv.y, acc);
-                acc = fmaf(sq[4 * c + 2], kv.z, acc);
-                acc = fmaf(sq[4 * c + 3], kv.w, acc);
-            }
-            s = fmaf(acc, scale, fmaf(lm_row[j], 10000.0f, -10000.0f));
+        for (int c = 0; c < 16; ++c) {
+            const float4 kv = kr[c];
+            a4[c & 3] = fmaf(sq[4 * c + 0], kv.x, a4[c & 3]);
+            a4[c & 3] = fmaf(sq[4 * c + 1], kv.y, a4[c & 3]);
+            a4[c & 3] = fmaf(sq[4 * c + 2], kv.z, a4[c & 3]);
+            a4[c & 3] = fmaf(sq[4 * c + 3], kv.w, a4[c & 3]);
         }
-        const float m_new = fmaxf(st.m, warp_max(s));
-        const float alpha = (st.m == -INFINITY) ? 0.0f : expf(st.m - m_new);
-        const float p = valid ? expf(s - m_new) : 0.0f;
-        st.l = st.l * alpha + warp_sum(p);
-        st.o0 *= alpha;
-        st.o1 *= alpha;
-        const int n = min(32, j_end - base + 1);
-        for (int t = 0; t < n; ++t) {
-            const float pt = __shfl_sync(0xffffffffu, p, t);
-            const float* vr = V + (size_t)(base + t) * 64;
-            st.o0 = fmaf(pt, vr[lane], st.o0);
-            st.o1 = fmaf(pt, vr[lane + 32], st.o1);
-        }
-        st.m = m_new;
+        const float acc = (a4[0] + a4[1]) + (a4[2] + a4[3]);
+        s = fmaf(acc, scale, fmaf(lm_row[j], 10000.0f, -10000.0f));
     }
+    const float m_new = fmaxf(st.m, warp_max(s));
+    const float alpha = (st.m == -INFINITY) ? 0.0f : expf(st.m - m_new);
+    const float p = valid ? expf(s - m_new) : 0.0f;
+    st.l = st.l * alpha + warp_sum(p);
+    st.o0 *= alpha;
+    st.o1 *= alpha;
+    // fixed trip count so that the V-row loads are issued together; keys
+    // past the end have p = 0 and read key 0
+#pragma unroll 8
+    for (int t = 0; t < 32; ++t) {
+        const float pt = __shfl_sync(0xffffffffu, p, t);
+        const int jt = __shfl_sync(0xffffffffu, j, t);
+        const float* vr = V + (size_t)jt * 64;
+        st.o0 = fmaf(pt, vr[lane], st.o0);
+        st.o1 = fmaf(pt, vr[lane + 32], st.o1);
+    }
+    st.m = m_new;
 }
 
-__global__ void __launch_bounds__(kWarps * 32)
+// One CTA per output row (b, h, i): the kWarps warps take interleaved
+// 32-key chunks of the row's key list (warp w: chunks w, w + kWarps, ...),
+// each with its own online softmax, and warp 0 merges the partial (m, l, o)
+// through shared memory.  Many short chains per SM instead of one long one
+// keep the L2 latency of the K/V rows hidden, global rows included.
+__global__ void __launch_bounds__(kWarps * 32, 4)
 attention_simt_kernel(const float* __restrict__ q, const float* __restrict__ k, const float* __restrict__ v,
                       const float* __restrict__ qg, const float* __restrict__ kg,
                       const float* __restrict__ vg, const float* __restrict__ local_mask,
                       const float* __restrict__ global_mask, int B, int H, int L, int w, float scale,
                       float* __restrict__ out, int* status) {
-    __shared__ __align__(16) float sq_all[kWarps][64];
+    __shared__ __align__(16) float sq[64];
+    __shared__ float part_ml[kWarps][2];
+    __shared__ float part_o[kWarps][64];
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-    float* sq = sq_all[wid];
     const long long total = (long long)B * H * L;
-    const long long nwarps = (long long)gridDim.x * kWarps;
-    for (long long r = (long long)blockIdx.x * kWarps + wid; r < total; r += nwarps) {
+    for (long long r = blockIdx.x; r < total; r += gridDim.x) {
         const int i = (int)(r % L);
         const int h = (int)((r / L) % H);
         const int b = (int)(r / ((long long)L * H));
@@ -101,37 +112,70 @@ attention_simt_kernel(const float* __restrict__ q, const float* __restrict__ k, 
         const float* gm_row = global_mask + (size_t)b * L;
         float* o = out + (((size_t)b * L + i) * H + h) * 64;
 
-        const int g = leading_globals(gm_row, L, w, lane);
+        const int g = leading_globals(gm_row, L, w, lane);  // same in every warp
         const bool bad_sample = g > w;
-        if (bad_sample && lane == 0 && h == 0 && i == 0) record_status(status, b, LF_ERR_G_GT_W);
-        if (!bad_sample && i >= g && gm_row[i] == 0.0f && lane == 0 && h == 0)
-            record_status(status, b, LF_ERR_GLOBAL_NOT_PREFIX);
+        if (wid == 0) {
+            if (bad_sample && lane == 0 && h == 0 && i == 0) record_status(status, b, LF_ERR_G_GT_W);
+            if (!bad_sample && i >= g && gm_row[i] == 0.0f && lane == 0 && h == 0)
+                record_status(status, b, LF_ERR_GLOBAL_NOT_PREFIX);
+        }
         if (bad_sample || fmaf(lm_row[i], 10000.0f, -10000.0f) != 0.0f) {
-            o[lane] = 0.0f;
-            o[lane + 32] = 0.0f;
-            continue;
+            if (wid == 0) {
+                o[lane] = 0.0f;
+                o[lane + 32] = 0.0f;
+            }
+            continue;  // uniform over the CTA
         }
         const bool global_row = i < g;
         const size_t head = ((size_t)b * H + h) * (size_t)L * 64;
         const float* Q = (global_row ? qg : q) + head;
         const float* K = (global_row ? kg : k) + head;
         const float* V = (global_row ? vg : v) + head;
-        sq[lane] = Q[(size_t)i * 64 + lane];
-        sq[lane + 32] = Q[(size_t)i * 64 + lane + 32];
-        __syncwarp();
-
-        RowState st{-INFINITY, 0.0f, 0.0f, 0.0f};
-        if (global_row) {
-            process_range(st, sq, K, V, lm_row, 0, L - 1, scale, lane);
-        } else {
-            const int lo = max(i - w, g), hi = min(i + w, L - 1);
-            if (g > 0) process_range(st, sq, K, V, lm_row, 0, g - 1, scale, lane);
-            process_range(st, sq, K, V, lm_row, lo, hi, scale, lane);
+        if (wid == 0) {
+            sq[lane] = Q[(size_t)i * 64 + lane];
+            sq[lane + 32] = Q[(size_t)i * 64 + lane + 32];
         }
-        const float inv = 1.0f / st.l;
-        o[lane] = st.o0 * inv;
-        o[lane + 32] = st.o1 * inv;
-        __syncwarp();
+        __syncthreads();
+
+        // key list: global row [0, L); local row [0, g) then [max(i - w, g), min(i + w, L - 1)]
+        int g_seg, lo, n_keys;
+        if (global_row) {
+            g_seg = 0;
+            lo = 0;
+            n_keys = L;
+        } else {
+            lo = max(i - w, g);
+            g_seg = g;
+            n_keys = g + (min(i + w, L - 1) - lo + 1);
+        }
+        RowState st{-INFINITY, 0.0f, 0.0f, 0.0f};
+        for (int pos0 = wid * 32; pos0 < n_keys; pos0 += kWarps * 32)
+            process_chunk(st, sq, K, V, lm_row, pos0, g_seg, lo, n_keys, scale, lane);
+        if (lane == 0) {
+            part_ml[wid][0] = st.m;
+            part_ml[wid][1] = st.l;
+        }
+        part_o[wid][lane] = st.o0;
+        part_o[wid][lane + 32] = st.o1;
+        __syncthreads();
+        if (wid == 0) {
+            float M = -INFINITY;
+#pragma unroll
+            for (int u = 0; u < kWarps; ++u) M = fmaxf(M, part_ml[u][0]);
+            float lsum = 0.0f, o0 = 0.0f, o1 = 0.0f;
+#pragma unroll
+            for (int u = 0; u < kWarps; ++u) {
+                const float mu = part_ml[u][0];
+                const float f = mu == -INFINITY ? 0.0f : expf(mu - M);
+                lsum = fmaf(part_ml[u][1], f, lsum);
+                o0 = fmaf(part_o[u][lane], f, o0);
+                o1 = fmaf(part_o[u][lane + 32], f, o1);
+            }
+            const float inv = 1.0f / lsum;
+            o[lane] = o0 * inv;
+            o[lane + 32] = o1 * inv;
+        }
+        __syncthreads();  // shared buffers are reused by the next row
     }
 }
 
@@ -142,8 +186,8 @@ lf_status launch_attention_simt_f32(const float* q, const float* k, const float*
                                     const float* global_mask, int B, int H, int L, int w, float scale,
                                     float* out, int* status, cudaStream_t stream) {
     const long long rows = (long long)B * H * L;
-    long long blocks = (rows + kWarps - 1) / kWarps;
-    if (blocks > 148 * 16) blocks = 148 * 16;
+    long long blocks = rows;
+    if (blocks > 148 * 64) blocks = 148 * 64;
     attention_simt_kernel<<<(int)blocks, kWarps * 32, 0, stream>>>(q, k, v, qg, kg, vg, local_mask, global_mask,
                                                                   B, H, L, w, scale, out, status);
     return cudaGetLastError() == cudaSuccess ? LF_OK : LF_ERR_CUDA;

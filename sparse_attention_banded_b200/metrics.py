@@ -1,5 +1,10 @@
 """Algorithmic work counts used for the roofline numbers (host-side only).
 
+Encoder layer (one Longformer layer, hidden D = 64 H, FFN width Fw):
+    F_layer = 2 L D (5 D) + 2 g_max D D + 2 L D D + 2 L D Fw + 2 L Fw D + F
+per sample: the five q k v kg vg projections, the qg projection of the
+global rows, the output projection, the two FFN GEMMs and the attention.
+
 FLOPs count the band + global work of unpadded query rows:
     F = 4 * 64 * H * sum_b [ sum_{i valid, i >= g_b} |K_i| + sum_{i valid, i < g_b} L ]
 with K_i = [max(0, i - w), min(L - 1, i + w)] united with [0, g_b) (each key
@@ -39,3 +44,10 @@ def algorithmic_bytes(B: int, H: int, L: int, w: int, g_list, dtype: str) -> flo
     masks = 2 * B * L * 4
     out = B * L * H * 64 * e
     return float(full + qg + masks + out)
+
+
+def layer_flops(B: int, H: int, L: int, w: int, g_list, pad_list, ffn: int) -> float:
+    D = 64 * H
+    gemm = B * (2.0 * L * D * 5 * D + 2.0 * L * D * D + 4.0 * L * D * ffn)
+    gemm += 2.0 * max(g_list) * D * D * B
+    return gemm + flops(B, H, L, w, g_list, pad_list)
