@@ -70,6 +70,24 @@ def dist_env():
     return rank, world, local
 
 
+def max_over_ranks(values, device="cpu"):
+    """Element-wise max of `values` over all ranks of the default process
+    group (every rank calls it with the same length); the values themselves
+    on a single rank."""
+    import torch.distributed as dist
+    if not dist.is_available() or not dist.is_initialized() or dist.get_world_size() == 1:
+        return [float(v) for v in values]
+    x = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(x, op=dist.ReduceOp.MAX)
+    return x.tolist()
+
+
+def job_throughput(world: int, units_per_rank: float, steps: int, max_total_ms: float) -> float:
+    """Whole-job units/s: every rank processed units_per_rank per step, the
+    job took the slowest rank's time."""
+    return world * units_per_rank * steps / (max_total_ms * 1e-3)
+
+
 # ---------------------------------------------------------------- clocks
 
 class ClockSampler:
@@ -241,10 +259,7 @@ def run_ours(args):
     attn_ms = [ev_a[k].elapsed_time(ev_e[k]) for k in range(K)]
     total_ms = sum(step_ms)
     attn_avg_ms = sum(attn_ms) / K
-    if world > 1:
-        x = torch.tensor([total_ms, attn_avg_ms], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(x, op=torch.distributed.ReduceOp.MAX)
-        total_ms, attn_avg_ms = x.tolist()
+    total_ms, attn_avg_ms = max_over_ranks([total_ms, attn_avg_ms], dev)
 
     # end to end through the public call: pinned host inputs -> device ->
     # partition + attention -> output back to pinned host memory
@@ -274,10 +289,7 @@ def run_ours(args):
     e1.record()
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1) / E
-    if world > 1:
-        x = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(x, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = x.item()
+    e2e_ms = max_over_ranks([e2e_ms], dev)[0]
     st = lf.lf_device_status(reset=True)
     if st != 0:
         raise RuntimeError("device status after timing: %s" % lf.status_string(st))
@@ -292,7 +304,7 @@ def run_ours(args):
         By = metrics.algorithmic_bytes(wl.B, wl.H, wl.L, wl.w, wl.g, wl.dtype)
     t_attn = attn_avg_ms * 1e-3
     tokens = wl.B * wl.L
-    value = world * tokens * K / (total_ms * 1e-3)
+    value = job_throughput(world, tokens, K, total_ms)
     tensor_path = wl.dtype in ("f16", "bf16")
     if layer:
         roof = {"bound": "tensor", "achieved": F / t_attn / 1e12, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
@@ -329,7 +341,7 @@ def run_ours(args):
             "note": "fp16 and bf16 dense tensor rates are equal; peak = measured bf16 burst (%s)" % pk_kind,
         },
         "roofline": roof,
-        "e2e": {"value": world * tokens / (e2e_ms * 1e-3), "unit": "tokens/s",
+        "e2e": {"value": job_throughput(world, tokens, 1, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": (1 + (8 if layer else 1)) * K,
         "clocks": clocks,
