@@ -8,10 +8,16 @@
 // A is [batches][rows][K] (rows of one batch contiguous, the batch stride may
 // exceed rows so that only the first rows of each sample are multiplied),
 // both operands K-major fp16/bf16, fp32 accumulation in TMEM.  Tiles are
-// 128 x 128 with 64-wide K steps through a kStages-deep TMA ring.  One
+// 128 x 256 (one M=128, N=256 tcgen05.mma per 16-wide K step: per byte
+// brought in from L2 this does a third more math than 128 x 128 tiles, which
+// the L2 bandwidth of the projections' and FFN's operands needs) with 64-wide
+// K steps through a kStages-deep TMA ring; N only needs to be a multiple of
+// 128 (the last tile's second half is zero-filled by TMA and not stored).  One
 // persistent CTA per SM: warp 0 issues TMA loads, warp 1 issues tcgen05.mma
-// into one of two TMEM accumulators, warps 4-7 run the epilogue of the
-// previous tile (one thread per row) while the next tile accumulates.
+// into one of two TMEM accumulators, warps 4-11 run the epilogue of the
+// previous tile while the next tile accumulates (one thread per row, two
+// warps per TMEM lane quarter, each taking half of the tile's columns, so
+// that the GELU epilogue keeps up with the MMAs).
 //
 // Epilogues:
 //   kEpiHeads  : + bias, round, scatter column n to head layout
@@ -34,19 +40,20 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kTM = 128, kTN = 128, kTK = 64;
-constexpr int kStages = 6;
-constexpr int kThreads = 256;  // 8 warps: 0 TMA, 1 MMA, 2-3 idle, 4-7 epilogue
+constexpr int kTM = 128, kTN = 256, kTK = 64;
+constexpr int kStages = 4;
+constexpr int kThreads = 384;  // 12 warps: 0 TMA, 1 MMA, 2-3 idle, 4-11 epilogue
+constexpr int kEpiWarps = 8;
 constexpr uint32_t kABytes = kTM * kTK * 2;  // 16 KB
-constexpr uint32_t kBBytes = kTN * kTK * 2;  // 16 KB
+constexpr uint32_t kBBytes = kTN * kTK * 2;  // 32 KB
 constexpr uint32_t kOffA = 0;
 constexpr uint32_t kOffB = kOffA + kStages * kABytes;
-constexpr uint32_t kOffBias = kOffB + kStages * kBBytes;        // 4 warps x 128 floats
-constexpr uint32_t kOffBar = kOffBias + 4 * kTN * 4;
+constexpr uint32_t kOffBias = kOffB + kStages * kBBytes;        // epilogue warps x kTN / 2 floats
+constexpr uint32_t kOffBar = kOffBias + kEpiWarps * (kTN / 2) * 4;
 constexpr uint32_t kNumBars = 2 * kStages + 4 + 1;
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
 constexpr uint32_t kSmemBytes = kOffMisc + 64 + 1024;
-constexpr uint32_t kTmemCols = 256;  // two 128-column fp32 accumulators
+constexpr uint32_t kTmemCols = 512;  // two 256-column fp32 accumulators
 
 struct GemmParams {
     int batches, rows, K, N;  // per batch: rows x N outputs
@@ -119,7 +126,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&acc_full[i], 1);
-            mbar_init(&acc_empty[i], 4);
+            mbar_init(&acc_empty[i], kEpiWarps);
         }
         mbar_init(drain, 1);
         *abort_flag = 0;
@@ -194,10 +201,11 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
             }
         }
     } else if (warp >= 4) {
-        const int sp = warp & 3;
+        const int sp = warp & 3;               // TMEM lane quarter
+        const int half = (warp - 4) >> 2;      // which half of the tile's columns
         const int r = sp * 32 + lane;
         const uint32_t lane_off = (uint32_t)(sp * 32) << 16;
-        float* bias_w = reinterpret_cast<float*>(smem + kOffBias) + sp * kTN;
+        float* bias_w = reinterpret_cast<float*>(smem + kOffBias) + (warp - 4) * (kTN / 2);
         const T* bias = reinterpret_cast<const T*>(p.bias);
         uint32_t tc = 0;
         bool ok = true;
@@ -205,10 +213,13 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
             const int nt = t % p.ntiles;
             const int bm = t / p.ntiles;
             const int mt = bm % p.mtiles, b = bm / p.mtiles;
-            const int n0 = nt * kTN;
-            // this warp's copy of the tile's bias
+            const int n0 = nt * kTN + half * (kTN / 2);  // this warp's columns
+            int ncols = p.N - n0 < kTN / 2 ? p.N - n0 : kTN / 2;  // a multiple of 32, maybe <= 0
+            if (ncols < 0) ncols = 0;
+            // this warp's copy of its columns' bias
 #pragma unroll
-            for (int c = 0; c < kTN / 32; ++c) bias_w[c * 32 + lane] = Cvt<T>::to_f(bias[n0 + c * 32 + lane]);
+            for (int c = 0; c < kTN / 64; ++c)
+                if (c * 32 < ncols) bias_w[c * 32 + lane] = Cvt<T>::to_f(bias[n0 + c * 32 + lane]);
             __syncwarp();
             const uint32_t ab = tc & 1;
             ok = __all_sync(0xffffffffu, mbar_wait(&acc_full[ab], (tc >> 1) & 1, abort_flag));
@@ -218,10 +229,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
             const bool row_ok = m < p.rows;
             const size_t grow = (size_t)b * p.rows + m;  // global row (row-major outputs)
 #pragma unroll 1
-            for (int c0 = 0; c0 < kTN; c0 += 32) {
+            for (int c0 = 0; c0 < ncols; c0 += 32) {
                 float acc[32];
                 __syncwarp();  // tcgen05.ld is .sync.aligned: whole warp, converged
-                tmem_ld32v(tmem + lane_off + ab * kTN + c0, acc);
+                tmem_ld32v(tmem + lane_off + ab * kTN + half * (kTN / 2) + c0, acc);
                 tmem_ld_wait();
                 regs_ready<32>(acc);
 #pragma unroll
@@ -325,7 +336,7 @@ lf_status launch_t(const GemmArgs& g, int sm_count, cudaStream_t stream) {
     p.K = g.K;
     p.N = g.N;
     p.mtiles = (g.rows + kTM - 1) / kTM;
-    p.ntiles = g.N / kTN;
+    p.ntiles = (g.N + kTN - 1) / kTN;
     p.ktiles = g.K / kTK;
     p.tiles = g.batches * p.mtiles * p.ntiles;
     p.mode = g.mode;
@@ -349,7 +360,7 @@ lf_status launch_t(const GemmArgs& g, int sm_count, cudaStream_t stream) {
 }  // namespace
 
 lf_status launch_gemm_tc(const GemmArgs& g, lf_dtype dtype, int sm_count, cudaStream_t stream) {
-    if (g.N % kTN != 0 || g.K % kTK != 0 || g.rows <= 0 || g.batches <= 0) return LF_ERR_BAD_DIM;
+    if (g.N % 128 != 0 || g.K % kTK != 0 || g.rows <= 0 || g.batches <= 0) return LF_ERR_BAD_DIM;
     if (dtype == LF_F16) return launch_t<__half>(g, sm_count, stream);
     if (dtype == LF_BF16) return launch_t<__nv_bfloat16>(g, sm_count, stream);
     return LF_ERR_DTYPE;

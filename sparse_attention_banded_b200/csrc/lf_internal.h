@@ -26,6 +26,10 @@ struct DeviceCtx {
     int* status = nullptr;  // device word, see LF_STATUS_CLEAR
     void* scratch = nullptr;
     size_t scratch_bytes = 0;
+    // encoder layer: a second stream (and its fork/join events) on which a
+    // small GEMM runs beside a large one
+    cudaStream_t side = nullptr;
+    cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
 };
 
 // Current device's context (initialised on first use; NULL + status on error).

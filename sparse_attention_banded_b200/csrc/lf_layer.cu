@@ -3,7 +3,10 @@
 // Transformer 层 steps 1-6, as a sequence of this library's kernels on one
 // stream (no host synchronisation):
 //   GEMM(x, W_qkv_kgvg) + bias -> q, k, v, kg, vg in head layout
-//   GEMM(x rows < ceil(w/128)*128, W_qg) + bias -> qg in head layout
+//   GEMM(x rows < ceil(w/128)*128, W_qg) + bias -> qg in head layout, on a
+//     second stream (forked from and joined back into the caller's stream)
+//     so that its few tiles run on the SMs the large GEMM's last wave leaves
+//     free
 //   banded + global attention -> a [B, L, D]
 //   GEMM(a, W_o) + b_o + x -> z (fp32);  LayerNorm -> h
 //   GEMM(h, W_1) + b_1, GELU -> f;  GEMM(f, W_2) + b_2 + h -> z;  LayerNorm -> out
@@ -82,16 +85,26 @@ extern "C" lf_status lf_encoder_layer_forward(const void* x, const float* local_
     uint8_t* qkv = base + ws.qkv;  // [5][B][H][L][64]
     auto slot = [&](int i) { return qkv + (size_t)i * head_elems * 2; };
 
+    if (!d->side) {
+        if (cudaStreamCreateWithFlags(&d->side, cudaStreamNonBlocking) != cudaSuccess ||
+            cudaEventCreateWithFlags(&d->ev_fork, cudaEventDisableTiming) != cudaSuccess ||
+            cudaEventCreateWithFlags(&d->ev_join, cudaEventDisableTiming) != cudaSuccess)
+            return LF_ERR_CUDA;
+    }
     // steps 1-2: the five projections with bias, scattered to head layout
     GemmArgs g{};
     g.A = x; g.batches = B; g.rows = L; g.batch_stride = L; g.K = D;
     g.W = wt->W_qkv_kgvg; g.N = 5 * D; g.bias = wt->b_qkv_kgvg; g.mode = kEpiHeads;
     g.out = qkv; g.heads_D = D; g.heads_H = H; g.heads_L = L; g.status = d->status;
+    if (cudaEventRecord(d->ev_fork, s) != cudaSuccess || cudaStreamWaitEvent(d->side, d->ev_fork, 0) != cudaSuccess)
+        return LF_ERR_CUDA;
     if ((st = launch_gemm_tc(g, dtype, d->sm_count, s)) != LF_OK) return st;
-    // Qg over the rows that can be global tokens (g_b <= w)
+    // Qg over the rows that can be global tokens (g_b <= w), beside the above
     const int qrows = ((w + 127) / 128) * 128 < L ? ((w + 127) / 128) * 128 : L;
     g.rows = qrows; g.W = wt->W_qg; g.N = D; g.bias = wt->b_qg; g.out = base + ws.qg;
-    if ((st = launch_gemm_tc(g, dtype, d->sm_count, s)) != LF_OK) return st;
+    if ((st = launch_gemm_tc(g, dtype, d->sm_count, d->side)) != LF_OK) return st;
+    if (cudaEventRecord(d->ev_join, d->side) != cudaSuccess || cudaStreamWaitEvent(s, d->ev_join, 0) != cudaSuccess)
+        return LF_ERR_CUDA;
     // steps 3-5: attention (its split counters must start at zero)
     if (cudaMemsetAsync(base + ws.scratch, 0, attention_tc_scratch_zero_bytes(B, H, L, w), s) != cudaSuccess)
         return LF_ERR_CUDA;
