@@ -3,8 +3,8 @@
 // and 6): the GEMM epilogue has already added bias and residual into an fp32
 // row; this kernel normalises each row with the population variance,
 // y = gamma * (z - mean) / sqrt(var + eps) + beta, and rounds to the dtype.
-// One warp per row, the row held in registers; HBM-bound (4 bytes read and
-// 2 written per element).
+// One warp per row, the row held in registers (16-byte loads, 8-byte
+// stores); memory-bound (4 bytes read and 2 written per element).
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -20,6 +20,21 @@ __device__ __forceinline__ __half from_f<__half>(float x) { return __float2half_
 template <>
 __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
 
+template <typename T>
+__device__ __forceinline__ uint32_t pack2(float a, float b);
+template <>
+__device__ __forceinline__ uint32_t pack2<__half>(float a, float b) {
+    __half2 h = __floats2half2_rn(a, b);
+    return *reinterpret_cast<uint32_t*>(&h);
+}
+template <>
+__device__ __forceinline__ uint32_t pack2<__nv_bfloat16>(float a, float b) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// VPL = N / 128: lane l holds columns 4 (k 32 + l) .. +3 for k < VPL, read
+// and written with 16- and 8-byte accesses.
 template <typename T, int VPL>
 __global__ void __launch_bounds__(256) layernorm_kernel(const float* __restrict__ z, const float* __restrict__ gamma,
                                                         const float* __restrict__ beta, int rows, int N, float eps,
@@ -27,13 +42,13 @@ __global__ void __launch_bounds__(256) layernorm_kernel(const float* __restrict_
     const int lane = threadIdx.x & 31;
     const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
     if (row >= rows) return;
-    const float* zr = z + (size_t)row * N;
-    float v[VPL];
+    const float4* zr = reinterpret_cast<const float4*>(z + (size_t)row * N);
+    float4 v[VPL];
     float s = 0.0f;
 #pragma unroll
     for (int k = 0; k < VPL; ++k) {
         v[k] = zr[k * 32 + lane];
-        s += v[k];
+        s += (v[k].x + v[k].y) + (v[k].z + v[k].w);
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
@@ -41,17 +56,23 @@ __global__ void __launch_bounds__(256) layernorm_kernel(const float* __restrict_
     float q = 0.0f;
 #pragma unroll
     for (int k = 0; k < VPL; ++k) {
-        const float d = v[k] - mean;
-        q = fmaf(d, d, q);
+        const float a = v[k].x - mean, b = v[k].y - mean, c = v[k].z - mean, d = v[k].w - mean;
+        q = fmaf(a, a, fmaf(b, b, fmaf(c, c, fmaf(d, d, q))));
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) q += __shfl_xor_sync(0xffffffffu, q, o);
     const float inv = rsqrtf(q / (float)N + eps);
-    T* orow = out + (size_t)row * N;
+    uint2* orow = reinterpret_cast<uint2*>(out + (size_t)row * N);
+    const float4* g4 = reinterpret_cast<const float4*>(gamma);
+    const float4* b4 = reinterpret_cast<const float4*>(beta);
 #pragma unroll
     for (int k = 0; k < VPL; ++k) {
         const int c = k * 32 + lane;
-        orow[c] = from_f<T>(fmaf((v[k] - mean) * inv, gamma[c], beta[c]));
+        const float4 g = g4[c], bb = b4[c];
+        uint2 u;
+        u.x = pack2<T>(fmaf((v[k].x - mean) * inv, g.x, bb.x), fmaf((v[k].y - mean) * inv, g.y, bb.y));
+        u.y = pack2<T>(fmaf((v[k].z - mean) * inv, g.z, bb.z), fmaf((v[k].w - mean) * inv, g.w, bb.w));
+        orow[c] = u;
     }
 }
 
@@ -60,15 +81,15 @@ lf_status launch_t(const float* z, const float* gamma, const float* beta, int ro
                    cudaStream_t stream) {
     const int blocks = (rows + 7) / 8;
     T* o = reinterpret_cast<T*>(out);
-    switch (N / 32) {
+    switch (N / 128) {
+        case 1: layernorm_kernel<T, 1><<<blocks, 256, 0, stream>>>(z, gamma, beta, rows, N, eps, o); break;
+        case 2: layernorm_kernel<T, 2><<<blocks, 256, 0, stream>>>(z, gamma, beta, rows, N, eps, o); break;
+        case 3: layernorm_kernel<T, 3><<<blocks, 256, 0, stream>>>(z, gamma, beta, rows, N, eps, o); break;
         case 4: layernorm_kernel<T, 4><<<blocks, 256, 0, stream>>>(z, gamma, beta, rows, N, eps, o); break;
+        case 5: layernorm_kernel<T, 5><<<blocks, 256, 0, stream>>>(z, gamma, beta, rows, N, eps, o); break;
+        case 6: layernorm_kernel<T, 6><<<blocks, 256, 0, stream>>>(z, gamma, beta, rows, N, eps, o); break;
+        case 7: layernorm_kernel<T, 7><<<blocks, 256, 0, stream>>>(z, gamma, beta, rows, N, eps, o); break;
         case 8: layernorm_kernel<T, 8><<<blocks, 256, 0, stream>>>(z, gamma, beta, rows, N, eps, o); break;
-        case 12: layernorm_kernel<T, 12><<<blocks, 256, 0, stream>>>(z, gamma, beta, rows, N, eps, o); break;
-        case 16: layernorm_kernel<T, 16><<<blocks, 256, 0, stream>>>(z, gamma, beta, rows, N, eps, o); break;
-        case 20: layernorm_kernel<T, 20><<<blocks, 256, 0, stream>>>(z, gamma, beta, rows, N, eps, o); break;
-        case 24: layernorm_kernel<T, 24><<<blocks, 256, 0, stream>>>(z, gamma, beta, rows, N, eps, o); break;
-        case 28: layernorm_kernel<T, 28><<<blocks, 256, 0, stream>>>(z, gamma, beta, rows, N, eps, o); break;
-        case 32: layernorm_kernel<T, 32><<<blocks, 256, 0, stream>>>(z, gamma, beta, rows, N, eps, o); break;
         default: return LF_ERR_BAD_DIM;
     }
     return cudaGetLastError() == cudaSuccess ? LF_OK : LF_ERR_CUDA;
