@@ -25,7 +25,7 @@ def test_exports_every_declared_function(L):
 
 
 def test_status_strings(L):
-    for code in range(14):
+    for code in range(15):
         assert lf.status_string(code).startswith("LF_")
     assert lf.status_string(999) == "unknown lf_status"
 
@@ -48,6 +48,8 @@ def _attn(L, B=1, H=1, Ln=512, w=64, dtype=1, ptrs=None, out=FAKE):
     (dict(dtype=7), 7),
     (dict(ptrs=[FAKE + 8] + [FAKE] * 7), 8),
     (dict(out=FAKE + 2), 8),
+    (dict(B=1, H=1 << 16, Ln=1 << 16, w=64), 13),   # B*H*L >= 2^31
+    (dict(B=1 << 23, H=1, Ln=128, w=64), 13),
 ])
 def test_attention_host_validation(L, kw, status):
     assert _attn(L, **kw) == status
@@ -59,6 +61,7 @@ def test_attention_host_validation(L, kw, status):
     ((FAKE, 1, 500, 64, FAKE, FAKE), 3),
     ((FAKE, 1, 64, 64, FAKE, FAKE), 4),
     ((FAKE, 1, 512, 64, FAKE + 4, FAKE), 8),
+    ((FAKE, 1 << 16, 1 << 16, 64, FAKE, FAKE), 13),  # B*L >= 2^31
 ])
 def test_global_idx_host_validation(L, args, status):
     gm, B, Ln, w, idx, nums = args
@@ -71,3 +74,47 @@ def test_scratch_bytes_host_only(L):
     assert lf.lf_attention_scratch_bytes(1, 16, 4096, 256, torch.float16) > 0
     assert lf.lf_attention_scratch_bytes(1, 2, 512, 64, torch.float32) == 0
     assert lf.lf_attention_scratch_bytes(1, 2, 500, 64, torch.float16) == 0
+
+
+def _layer(L, B=1, H=4, Ln=512, w=64, ffn=512, dtype=1, ws_bytes=1 << 30, weights="ok", x=FAKE, ws=FAKE):
+    if weights == "null":
+        wp = None
+    else:
+        vals = [FAKE] * len(lf.LAYER_FIELDS)
+        if weights == "one_null":
+            vals[4] = 0  # W_o
+        if weights == "misaligned":
+            vals[2] = FAKE + 2
+        wp = ctypes.byref(lf.LayerWeights(ffn, *vals))
+    return L.lf_encoder_layer_forward(ctypes.c_void_p(x), ctypes.c_void_p(FAKE), ctypes.c_void_p(FAKE), wp,
+                                      B, H, Ln, w, 0.125, 1e-5, dtype, ctypes.c_void_p(ws), ws_bytes, None,
+                                      ctypes.c_void_p(FAKE))
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(weights="null"), 1),
+    (dict(weights="one_null"), 1),
+    (dict(x=0), 1),
+    (dict(B=0), 2),
+    (dict(H=1), 2),             # hidden 64 is not a multiple of 128
+    (dict(H=32), 2),            # hidden 2048 > 1024
+    (dict(ffn=200), 2),         # FFN width not a multiple of 128
+    (dict(Ln=500), 3),
+    (dict(Ln=64), 4),
+    (dict(dtype=0), 7),         # fp32 layer: no tensor-core path
+    (dict(weights="misaligned"), 8),
+    (dict(ws_bytes=1024), 12),  # workspace smaller than lf_encoder_layer_workspace_bytes
+    (dict(ws=FAKE + 16), 12),   # workspace not 256-byte aligned
+])
+def test_layer_host_validation(L, kw, status):
+    assert _layer(L, **kw) == status
+
+
+def test_layer_workspace_bytes_host_only(L):
+    import torch
+    n = lf.lf_encoder_layer_workspace_bytes(1, 16, 4096, 256, 4096, torch.float16)
+    # five projections + qg + attention output + fp32 residual sum + h + FFN intermediate + scratch
+    D, rows = 1024, 4096
+    assert n >= (5 + 1 + 1 + 2 + 1) * rows * D * 2 + rows * 4096 * 2
+    assert lf.lf_encoder_layer_workspace_bytes(1, 1, 512, 64, 512, torch.float16) == 0   # hidden 64
+    assert lf.lf_encoder_layer_workspace_bytes(1, 4, 512, 64, 512, torch.float32) == 0
