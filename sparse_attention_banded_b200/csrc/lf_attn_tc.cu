@@ -355,6 +355,7 @@ struct Pack<__half> {
         __half2 h = __floats2half2_rn(a, b);
         return *reinterpret_cast<uint32_t*>(&h);
     }
+    __device__ static float2 unpack(uint32_t u) { return __half22float2(*reinterpret_cast<__half2*>(&u)); }
 };
 template <>
 struct Pack<__nv_bfloat16> {
@@ -363,6 +364,7 @@ struct Pack<__nv_bfloat16> {
         __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
         return *reinterpret_cast<uint32_t*>(&h);
     }
+    __device__ static float2 unpack(uint32_t u) { return __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&u)); }
 };
 
 template <typename T>
@@ -927,66 +929,19 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
                             for (int c = 0; c < 32; ++c) r[c] = ((bits >> c) & 1u) ? r[c] : -INFINITY;
                         }
                     };
-                    float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll 1
-                    for (int ch = 0; ch < 4; ++ch) {
-                        if (state_of(ch) == kSkip) continue;
-                        float r[32];
-                        tmem_ld32f(tS + ch * 32, r);
-                        tmem_ld_wait();
-                        regs_ready<32>(r);
-                        fix_chunk(ch, r);
-#pragma unroll
-                        for (int c = 0; c < 32; c += 8) {
-                            mx[0] = max3(mx[0], r[c], r[c + 1]);
-                            mx[1] = max3(mx[1], r[c + 2], r[c + 3]);
-                            mx[2] = max3(mx[2], r[c + 4], r[c + 5]);
-                            mx[3] = max3(mx[3], r[c + 6], r[c + 7]);
-                        }
-                    }
-                    const float mb = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * p.scale_log2;
-#if LF_TRACE
-                    const long long ts2_ = clock64();
-                    tacc[7] += ts2_ - tc0_;
-#endif
-                    // Running max with lazy rescaling of the TMEM accumulator.
-                    // The decision is per row, but tcgen05.ld/st are warp-wide
-                    // (.sync.aligned): the whole warp rescales when any row
-                    // needs it, rows that do not use factor 1.
-                    if (first) {
-                        m_used = mb;
-                    } else {
-                        const bool need = mb > m_used + kRescaleThreshold;
-                        if (__any_sync(0xffffffffu, need)) {
-                            const float factor = !need ? 1.0f : (m_used == -INFINITY ? 0.0f : ex2(m_used - mb));
-                            if (need) {
-                                l_run *= factor;
-                                m_used = mb;
-                            }
-#pragma unroll
-                            for (int c0o = 0; c0o < kHD; c0o += 16) {
-                                uint32_t ob[16];
-                                tmem_ld16(tO + c0o, ob);
-                                tmem_ld_wait();
-                                regs_ready<16>(ob);
-#pragma unroll
-                                for (int c = 0; c < 16; ++c)
-                                    ob[c] = __float_as_uint(__uint_as_float(ob[c]) * factor);
-                                tmem_st16(tO + c0o, ob);
-                            }
-                        }
-                    }
-                    const float m_use = m_used == -INFINITY ? 0.0f : m_used;
-#if LF_TRACE
-                    const long long ts3_ = clock64();
-                    tacc[8] += ts3_ - ts2_;
-#endif
-                    // p = 2^(raw * scale_log2 - m): one packed FMA per pair
+                    // One pass over S in 32-column chunks (rolled loop, 32 live
+                    // scores): each chunk is read once, biased and masked, and
+                    // exponentiated against the running row max m.  m only
+                    // moves when a row's max grows by more than 8 (log2 units,
+                    // so P <= 2^8); the whole warp then rescales (tcgen05.ld/st
+                    // are .sync.aligned): the sums so far, this block's P
+                    // chunks already in TMEM and, past the item's first block,
+                    // the O accumulator (whose previous P V has completed: it
+                    // ran before this block's S).
                     const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
-                    const float2 nm2 = make_float2(-m_use, -m_use);
                     float2 sm2[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
                     // exponentials of one chunk, packed to 16 words of P
-                    auto exp_chunk = [&](float (&r)[32], uint32_t (&pk)[16]) {
+                    auto exp_chunk = [&](float (&r)[32], uint32_t (&pk)[16], float2 nm2) {
 #pragma unroll
                         for (int c = 0; c < 16; ++c) {
                             const float2 a = ffma2(make_float2(r[2 * c], r[2 * c + 1]), sc2, nm2);
@@ -996,6 +951,10 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
                             pk[c] = Pack<T>::two(e.x, e.y);
                         }
                     };
+#if LF_TRACE
+                    const long long ts2_ = clock64();
+                    tacc[7] += ts2_ - tc0_;
+#endif
 #pragma unroll 1
                     for (int ch = 0; ch < 4; ++ch) {
                         uint32_t pk[16];
@@ -1008,14 +967,62 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
                             tmem_ld_wait();
                             regs_ready<32>(r);
                             fix_chunk(ch, r);
-                            exp_chunk(r, pk);
+                            float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+                            for (int c = 0; c < 32; c += 8) {
+                                mx[0] = max3(mx[0], r[c], r[c + 1]);
+                                mx[1] = max3(mx[1], r[c + 2], r[c + 3]);
+                                mx[2] = max3(mx[2], r[c + 4], r[c + 5]);
+                                mx[3] = max3(mx[3], r[c + 6], r[c + 7]);
+                            }
+                            const float cm = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * p.scale_log2;
+                            const bool need = cm > m_used + kRescaleThreshold;
+                            if (__any_sync(0xffffffffu, need)) {
+                                // rows with a finite previous max rescale what they
+                                // have so far; rows at -inf have nothing yet (zeros)
+                                const bool real = need && m_used != -INFINITY;
+                                if (__any_sync(0xffffffffu, real)) {
+                                    const float factor = real ? ex2(m_used - cm) : 1.0f;
+                                    l_run *= factor;
+                                    sm2[0] = make_float2(sm2[0].x * factor, sm2[0].y * factor);
+                                    sm2[1] = make_float2(sm2[1].x * factor, sm2[1].y * factor);
+                                    for (int pc = 0; pc < ch; ++pc) {  // this block's earlier P
+                                        uint32_t pb16[16];
+                                        tmem_ld16(tS + pc * 16, pb16);
+                                        tmem_ld_wait();
+                                        regs_ready<16>(pb16);
+#pragma unroll
+                                        for (int c = 0; c < 16; ++c) {
+                                            const float2 v = Pack<T>::unpack(pb16[c]);
+                                            pb16[c] = Pack<T>::two(v.x * factor, v.y * factor);
+                                        }
+                                        tmem_st16(tS + pc * 16, pb16);
+                                    }
+                                    if (!first) {
+#pragma unroll
+                                        for (int c0o = 0; c0o < kHD; c0o += 16) {
+                                            uint32_t ob[16];
+                                            tmem_ld16(tO + c0o, ob);
+                                            tmem_ld_wait();
+                                            regs_ready<16>(ob);
+#pragma unroll
+                                            for (int c = 0; c < 16; ++c)
+                                                ob[c] = __float_as_uint(__uint_as_float(ob[c]) * factor);
+                                            tmem_st16(tO + c0o, ob);
+                                        }
+                                    }
+                                }
+                                if (need) m_used = cm;
+                            }
+                            const float m_use = m_used == -INFINITY ? 0.0f : m_used;
+                            exp_chunk(r, pk, make_float2(-m_use, -m_use));
                         }
                         tmem_st16(tS + ch * 16, pk);
                     }
                     l_run += (sm2[0].x + sm2[0].y) + (sm2[1].x + sm2[1].y);
 #if LF_TRACE
                     const long long ts4_ = clock64();
-                    tacc[9] += ts4_ - ts3_;
+                    tacc[9] += ts4_ - ts2_;
 #endif
                     tmem_st_wait();
 #if LF_TRACE
