@@ -865,6 +865,30 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
                     }
                     __syncwarp();
                 }
+                // Chunk states (warp-uniform): skip / full / masked, two bits
+                // per chunk so that a rolled loop can index them.  They depend
+                // only on where the block lies, so they are worked out before
+                // the wait for its S, not after.
+                uint32_t states = 0;
+#pragma unroll
+                for (int ch = 0; ch < 4; ++ch) {
+                    const int cj0 = c0 + ch * 32;
+                    int s;
+                    if (cj0 >= p.L) {
+                        s = kSkip;
+                    } else if (is_global) {
+                        s = (cj0 + 31 < p.L) ? kFull : kPart;
+                    } else {
+                        const bool any_g = cj0 < g;
+                        const bool all_g = cj0 + 31 < g;
+                        const bool overlap = cj0 <= wr0 + 31 + p.w && cj0 + 31 >= wr0 - p.w;
+                        const bool inside = (wr0 + 31 - cj0 <= p.w) && (cj0 + 31 - wr0 <= p.w);
+                        if (!any_g && !overlap) s = kSkip;
+                        else if ((all_g || inside) && cj0 + 31 < p.L) s = kFull;
+                        else s = kPart;
+                    }
+                    states |= (uint32_t)s << (2 * ch);
+                }
                 if (lane == 0) TRACE(2 + warp - kSoftmaxWarp0, 32, id, n, scnt);
                 // every lane waits; the result is made warp-uniform so that an
                 // abort never splits the warp before a .sync.aligned instruction
@@ -874,28 +898,6 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
                 if (!ok) break;
                 tc_fence_after();
                 if (warp_active) {
-                    // Chunk states (warp-uniform): skip / full / masked, two bits
-                    // per chunk so that a rolled loop can index them.
-                    uint32_t states = 0;
-#pragma unroll
-                    for (int ch = 0; ch < 4; ++ch) {
-                        const int cj0 = c0 + ch * 32;
-                        int s;
-                        if (cj0 >= p.L) {
-                            s = kSkip;
-                        } else if (is_global) {
-                            s = (cj0 + 31 < p.L) ? kFull : kPart;
-                        } else {
-                            const bool any_g = cj0 < g;
-                            const bool all_g = cj0 + 31 < g;
-                            const bool overlap = cj0 <= wr0 + 31 + p.w && cj0 + 31 >= wr0 - p.w;
-                            const bool inside = (wr0 + 31 - cj0 <= p.w) && (cj0 + 31 - wr0 <= p.w);
-                            if (!any_g && !overlap) s = kSkip;
-                            else if ((all_g || inside) && cj0 + 31 < p.L) s = kFull;
-                            else s = kPart;
-                        }
-                        states |= (uint32_t)s << (2 * ch);
-                    }
                     auto state_of = [&](int ch) -> int { return (int)((states >> (2 * ch)) & 3u); };
                     // Two passes over S in 32-column chunks with a rolled loop
                     // (compact code, 32 live scores): pass 1 takes the row max,
