@@ -64,13 +64,16 @@ constexpr int kStages = 4;        // K/V ring depth
 constexpr int kMinChunk = 4;      // key blocks per global-row split: chosen per
 constexpr int kMaxChunk = 16;     // shape in [kMinChunk, kMaxChunk] on the host
 constexpr int kRing = 4;          // item-id ring depth
-constexpr int kWarps = 12;
+constexpr int kSBuf = 3;          // S buffers in TMEM, rotating over the two tiles
+constexpr int kWarps = 16;
 constexpr int kThreads = kWarps * 32;
-constexpr int kSoftmaxWarp0 = 4;
+constexpr int kSoftmaxWarp0 = 4;  // warps 4-7: tile A, 8-11: tile B
+constexpr int kEpiWarp0 = 12;     // warps 12-15: epilogue of both tiles
 constexpr uint32_t kRegsProducer = 96;
-constexpr uint32_t kRegsSoftmax = 200;
-static_assert(4 * 32 * kRegsProducer + 8 * 32 * kRegsSoftmax <= kThreads * 168, "register split");
-constexpr int kItemConsumers = 1 + 1 + 8;  // TMA warp + MMA warp + 8 softmax warps
+constexpr uint32_t kRegsSoftmax = 160;
+constexpr uint32_t kRegsEpi = 96;
+static_assert(4 * 32 * kRegsProducer + 8 * 32 * kRegsSoftmax + 4 * 32 * kRegsEpi <= 65536, "register split");
+constexpr int kItemConsumers = 1 + 1 + 8 + 4;  // TMA + MMA + softmax + epilogue warps
 constexpr uint32_t kTileBytes = kBM * kHD * 2;  // 16 KB
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;
@@ -80,15 +83,18 @@ constexpr uint32_t kOffQ = 0;                                 // [2 parity][2 ti
 constexpr uint32_t kOffK = kOffQ + 4 * kTileBytes;            // kStages x 16 KB
 constexpr uint32_t kOffV = kOffK + kStages * kTileBytes;      // kStages x 16 KB
 constexpr uint32_t kOffBias = kOffV + kStages * kTileBytes;   // 8 warps x 128 floats
-constexpr uint32_t kOffPlans = kOffBias + 8 * kBN * 4;        // kRing plans
+constexpr uint32_t kOffStats = kOffBias + 8 * kBN * 4;        // [2 tiles][128 rows] (m, l)
+constexpr uint32_t kOffPlans = kOffStats + 2 * kBM * 8;       // kRing plans
 constexpr uint32_t kOffBar = kOffPlans + kRing * 128;
-constexpr uint32_t kNumBars = 2 + 2 + 2 * kStages + 2 * 4 + 2 * kRing + 2;
+constexpr uint32_t kNumBars = 2 + 2 + 2 * kStages + 2 * kSBuf + kSBuf + 2 + 2 + 2 + 2 + 2 * kRing + 2;
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
 constexpr uint32_t kSmemBytes = kOffMisc + 64 + 1024;  // + alignment slack
 
-// TMEM columns: S_A [0,128), S_B [128,256), O_A [256,320), O_B [320,384).
+// TMEM columns: S buffers [0,128), [128,256), [256,384); O_A [384,448),
+// O_B [448,512).
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kTmemO = 256;
+constexpr uint32_t kTmemO = kSBuf * kBN;
+static_assert(kTmemO + 2 * kHD <= kTmemCols, "TMEM budget");
 
 struct Params {
     int B, H, L, w;
@@ -121,11 +127,12 @@ struct Params {
 #ifndef LF_TRACE
 #define LF_TRACE 0
 #endif
+// Wait-site states (each write is a system-scope fence: for locating a hang,
+// not for timing).
 #ifndef LF_TRACE_STATES
-#define LF_TRACE_STATES 1
+#define LF_TRACE_STATES 0
 #endif
-#if LF_TRACE
-#if LF_TRACE_STATES
+#if LF_TRACE && LF_TRACE_STATES
 #define TRACE(role, state, item, a, b)                                                 \
     do {                                                                               \
         if (p.trace) {                                                                 \
@@ -142,33 +149,37 @@ struct Params {
     do {                               \
     } while (0)
 #endif
+#if LF_TRACE
 // Cycle accounting per role: TIMED(k, stmt) adds the clock64() cycles of
 // stmt to slot k; TDUMP(role) writes the 16 slots after the state words.
-#define TIMED(k, stmt)                    \
-    do {                                  \
-        const long long t0_ = clock64();  \
-        stmt;                             \
-        tacc[k] += clock64() - t0_;       \
+#define TDECL                  \
+    long long tacc[16] = {0}; \
+    const long long tstart_ = clock64()
+#define TIMED(k, stmt)                   \
+    do {                                 \
+        const long long t0_ = clock64(); \
+        stmt;                            \
+        tacc[k] += clock64() - t0_;      \
     } while (0)
-#define TDECL long long tacc[16] = {0}; const long long tstart_ = clock64()
-#define TDUMP(role)                                                                               \
-    do {                                                                                          \
-        if (p.trace) {                                                                            \
-            tacc[15] = clock64() - tstart_;                                                       \
-            volatile int* d_ = p.trace + gridDim.x * 16 * 4 + (blockIdx.x * 16 + (role)) * 16;    \
-            for (int k_ = 0; k_ < 16; ++k_) d_[k_] = (int)tacc[k_];                               \
-        }                                                                                         \
+#define TCOUNT(k) (tacc[k] += 1)
+#define TDUMP(role)                                                                             \
+    do {                                                                                        \
+        if (p.trace) {                                                                          \
+            tacc[15] = clock64() - tstart_;                                                     \
+            volatile int* d_ = p.trace + gridDim.x * 16 * 4 + (blockIdx.x * 16 + (role)) * 16;  \
+            for (int k_ = 0; k_ < 16; ++k_) d_[k_] = (int)tacc[k_];                             \
+        }                                                                                       \
     } while (0)
 #else
-#define TRACE(role, state, item, a, b) \
-    do {                               \
+#define TDECL \
+    do {      \
     } while (0)
 #define TIMED(k, stmt) \
     do {               \
         stmt;          \
     } while (0)
-#define TDECL \
-    do {      \
+#define TCOUNT(k) \
+    do {          \
     } while (0)
 #define TDUMP(role) \
     do {            \
@@ -198,35 +209,62 @@ struct Plan {
 };
 
 // Leading 0.0 entries of global_mask[b, :] capped at w + 1 (whole warp).
+// 256 entries per round, all loads of a round in flight together.
 __device__ int leading_globals(const Params& p, int b) {
     const int lane = threadIdx.x & 31;
     const float* row = p.global_mask + (size_t)b * p.L;
     const int cap = min(p.w + 1, p.L);
-    for (int c0 = 0; c0 < cap; c0 += 32) {
-        const int j = c0 + lane;
-        const unsigned m = __ballot_sync(0xffffffffu, j < cap && row[j] != 0.0f);
-        if (m) return c0 + __ffs(m) - 1;
+    for (int c0 = 0; c0 < cap; c0 += 256) {
+        float v[8];
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+            const int j = c0 + 32 * t + lane;
+            v[t] = j < cap ? row[j] : 0.0f;
+        }
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+            const unsigned m = __ballot_sync(0xffffffffu, v[t] != 0.0f);
+            if (m) return c0 + 32 * t + __ffs(m) - 1;
+        }
     }
     return cap;
 }
 
-// Whole warp: does band tile [r0, r0+128) have a row g <= i < L that is not
-// padded?  Also reports whether it has padded rows in [g, L).
-__device__ void band_rows(const Params& p, int b, int r0, int g, int& work, int& padded) {
+// Whole warp: for each of the two band tiles starting at r0[x], does it have
+// a row g <= i < L that is not padded (work), and padded rows in [g, L)?
+// The local_mask loads of both tiles are issued before the global count is
+// needed, so the first plan of a sample costs one round of loads.
+__device__ void band_rows2(const Params& p, int b, const int (&r0)[2], int& cached_b, int& g, int (&work)[2],
+                           int (&padded)[2]) {
     const int lane = threadIdx.x & 31;
     const float* lm = p.local_mask + (size_t)b * p.L;
-    bool w_ = false, pd = false;
+    float v[2][4];
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        const int i = r0 + lane + 32 * k;
-        if (i < p.L && i >= g) {
-            const bool tok = lm[i] == 1.0f;
-            w_ |= tok;
-            pd |= !tok;
+    for (int x = 0; x < 2; ++x)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int i = r0[x] + lane + 32 * k;
+            v[x][k] = i < p.L ? lm[i] : 1.0f;
         }
+    if (b != cached_b) {
+        g = leading_globals(p, b);
+        cached_b = b;
     }
-    work = __any_sync(0xffffffffu, w_);
-    padded = __any_sync(0xffffffffu, pd);
+#pragma unroll
+    for (int x = 0; x < 2; ++x) {
+        bool w_ = false, pd = false;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int i = r0[x] + lane + 32 * k;
+            if (i < p.L && i >= g) {
+                const bool tok = v[x][k] == 1.0f;
+                w_ |= tok;
+                pd |= !tok;
+            }
+        }
+        work[x] = __any_sync(0xffffffffu, w_);
+        padded[x] = __any_sync(0xffffffffu, pd);
+    }
 }
 
 // Whole warp: the item's plan (identical in every role).
@@ -263,9 +301,15 @@ __device__ Plan make_plan(const Params& p, int id, int& cached_b, int& g) {
     }
     pl.b = pl.bh / p.H;
     pl.h = pl.bh % p.H;
-    if (pl.b != cached_b) {
-        g = leading_globals(p, pl.b);
-        cached_b = pl.b;
+    int work[2] = {0, 0}, padded[2] = {0, 0};
+    if (pl.global) {
+        if (pl.b != cached_b) {
+            g = leading_globals(p, pl.b);
+            cached_b = pl.b;
+        }
+    } else {
+        const int r0[2] = {pl.t[0].r0, pl.t[1].r0};
+        band_rows2(p, pl.b, r0, cached_b, g, work, padded);
     }
     pl.g = g;
     pl.nloads = 0;
@@ -299,10 +343,8 @@ __device__ Plan make_plan(const Params& p, int id, int& cached_b, int& g) {
         Tile& t = pl.t[x];
         t.split = 0;
         if (t.r0 >= p.L) continue;
-        int work, padded;
-        band_rows(p, pl.b, t.r0, g, work, padded);
-        if (!work) {
-            pl.zero_only[x] = padded;
+        if (!work[x]) {
+            pl.zero_only[x] = padded[x];
             continue;
         }
         t.present = 1;
@@ -344,6 +386,34 @@ __device__ __forceinline__ void load_at(const Plan& pl, int q, int& kb, int& nee
     const Tile& Bt = pl.t[1];
     needA = A.present && (kb < A.glob_hi || (kb >= A.lo && kb <= A.hi));
     needB = Bt.present && (kb < Bt.glob_hi || (kb >= Bt.lo && kb <= Bt.hi));
+}
+
+// Key blocks of one tile of an item.
+__device__ __forceinline__ int tile_blocks(const Tile& t) { return t.present ? t.glob_hi + (t.hi - t.lo + 1) : 0; }
+// Key block of a tile's j-th block: [0, glob_hi) then lo, lo + 1, ...
+__device__ __forceinline__ int block_kb(const Tile& t, int j) { return j < t.glob_hi ? j : t.lo + (j - t.glob_hi); }
+// An item's S products are computed in the order A0 B0 A1 B1 ... while both
+// tiles have blocks left, then the rest of the longer tile.
+__device__ __forceinline__ void seq_at(int pos, int nA, int nB, int& x, int& j) {
+    const int m = min(nA, nB);
+    if (pos < 2 * m) {
+        x = pos & 1;
+        j = pos >> 1;
+    } else {
+        x = nA > nB ? 0 : 1;
+        j = pos - m;
+    }
+}
+__device__ __forceinline__ int seq_pos(int x, int j, int nA, int nB) {
+    const int m = min(nA, nB);
+    return j < m ? 2 * j + x : m + j;
+}
+// Index, in the item's K/V load order, of tile x's j-th block.  Global pairs
+// load in sequence order; band pairs load [0, e1) then lo_min, lo_min + 1, ...
+__device__ __forceinline__ int load_of(const Plan& pl, int x, int j, int nA, int nB) {
+    if (pl.global) return seq_pos(x, j, nA, nB);
+    const int kb = block_kb(pl.t[x], j);
+    return kb < pl.e1 ? kb : pl.e1 + (kb - pl.lo_min);
 }
 
 template <typename T>
@@ -511,29 +581,45 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
     uint64_t* q_empty = bars + 2;
     uint64_t* kv_full = bars + 4;
     uint64_t* kv_empty = kv_full + kStages;
-    uint64_t* s_full = kv_empty + kStages;  // [tile]
-    uint64_t* p_full = s_full + 2;          // [tile]
-    uint64_t* o_done = p_full + 2;          // [tile]
-    uint64_t* o_free = o_done + 2;          // [tile]
-    uint64_t* item_full = o_free + 2;       // [kRing]
+    uint64_t* s_full = kv_empty + kStages;   // [tile][S buffer]: QK of that tile into that buffer done
+    uint64_t* p_full = s_full + 2 * kSBuf;   // [S buffer]: P written by the 4 warps of its tile
+    uint64_t* pv_done = p_full + kSBuf;      // [tile]: one phase per P V product of the tile
+    uint64_t* o_free = pv_done + 2;          // [tile]: the epilogue has read O
+    uint64_t* st_full = o_free + 2;          // [tile]: row (m, l) of an item written
+    uint64_t* st_free = st_full + 2;         // [tile]: ... and read by the epilogue
+    uint64_t* item_full = st_free + 2;       // [kRing]
     uint64_t* item_empty = item_full + kRing;
     uint64_t* drain = item_empty + kRing;
     uint64_t* tma_done = drain + 1;  // the TMA warp finished issuing an item's loads
+    static_assert(2 + 2 + 2 * kStages + 2 * kSBuf + kSBuf + 2 + 2 + 2 + 2 + 2 * kRing + 2 == kNumBars, "barriers");
     Plan* plans = reinterpret_cast<Plan*>(smem + kOffPlans);
     static_assert(sizeof(Plan) <= 128, "plan slot");
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+#if LF_TRACE
+    if (threadIdx.x == 0 && p.trace) {  // kernel entry time
+        volatile int* d_ = p.trace + gridDim.x * 16 * 4 + (blockIdx.x * 16 + 15) * 16;
+        const unsigned long long t = globaltimer();
+        d_[0] = (int)(t & 0xffffffffu);
+        d_[1] = (int)(t >> 32);
+    }
+#endif
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < 2; ++i) {
             mbar_init(&q_full[i], 1);
             mbar_init(&q_empty[i], 1);
-            mbar_init(&s_full[i], 1);
-            mbar_init(&p_full[i], 4);
-            mbar_init(&o_done[i], 1);
+            mbar_init(&pv_done[i], 1);
             mbar_init(&o_free[i], 4);
+            mbar_init(&st_full[i], 4);
+            mbar_init(&st_free[i], 4);
+        }
+        for (int b = 0; b < kSBuf; ++b) {
+            mbar_init(&s_full[b], 1);
+            mbar_init(&s_full[kSBuf + b], 1);
+            mbar_init(&p_full[b], 4);
         }
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&kv_full[s], 1);
@@ -564,45 +650,49 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    if (threadIdx.x == 0) TRACE(11, 1, 0, 0, 0);
 #if LF_TRACE
-    if (threadIdx.x == 0 && p.trace) {  // CTA start time and SM id
+    if (threadIdx.x == 0 && p.trace) {
+        volatile int* d_ = p.trace + gridDim.x * 16 * 4 + (blockIdx.x * 16 + 14) * 16;
         const unsigned long long t = globaltimer();
-        volatile int* d_ = p.trace + gridDim.x * 16 * 4 + (blockIdx.x * 16 + 12) * 16;
         d_[0] = (int)(t & 0xffffffffu);
         d_[1] = (int)(t >> 32);
-        unsigned smid;
-        asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
-        d_[4] = (int)smid;
     }
 #endif
+
+    // Every role but the planner reads the item plans from the ring in order.
+    auto next_plan = [&](uint32_t k, Plan& pl) -> bool {
+        const uint32_t slot = k % kRing;
+        bool ok = true;
+        if (lane == 0) ok = mbar_wait(&item_full[slot], (k / kRing) & 1, abort_flag);
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        if (!ok) return false;
+        __syncwarp();       // lane 0's acquire orders the reads below
+        pl = plans[slot];   // published by the planner before item_full
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&item_empty[slot]);
+        return true;
+    };
 
     if (warp < kSoftmaxWarp0) {
     regs_dec<kRegsProducer>();
     if (warp == 0) {
-        // ------------------------------------------------------------ scheduler + TMA producer
+        // ------------------------------------------------------------ TMA producer
         TDECL;
         uint32_t kv_cnt = 0, item_cnt = 0;
         bool ok = true;
         for (uint32_t k = 0; ok; ++k) {
-            const uint32_t slot = k % kRing;
-            if (lane == 0) TIMED(0, ok = mbar_wait(&item_full[slot], (k / kRing) & 1, abort_flag));
-            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+            Plan pl;
+            TIMED(0, ok = next_plan(k, pl));
             if (!ok) break;
-            __syncwarp();                 // lane 0's acquire orders the reads below
-            const Plan pl = plans[slot];  // published by the planner before item_full
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&item_empty[slot]);
-            const int id = pl.id;
-            if (id < 0) break;
+            if (pl.id < 0) break;
             if (pl.nloads == 0) {
                 if (lane == 0) mbar_arrive(tma_done);
                 continue;
             }
             if (lane == 0) {
                 const uint32_t qb = item_cnt & 1;
-                TRACE(0, 12, id, item_cnt, 0);
-                TIMED(2, ok = mbar_wait(&q_empty[qb], ((item_cnt >> 1) & 1) ^ 1, abort_flag));
+                TRACE(0, 12, pl.id, item_cnt, 0);
+                TIMED(1, ok = mbar_wait(&q_empty[qb], ((item_cnt >> 1) & 1) ^ 1, abort_flag));
                 if (ok) {
                     const int nq = pl.t[0].present + pl.t[1].present;
                     mbar_arrive_expect_tx(&q_full[qb], nq * kTileBytes);
@@ -611,13 +701,14 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
                             tma_load_3d(smem + kOffQ + (qb * 2 + x) * kTileBytes, pl.global ? &maps.qg : &maps.q,
                                         &q_full[qb], 0, pl.t[x].r0, pl.bh);
                 }
+                // Every load of the plan is issued (the MMA warp maps a tile's
+                // blocks to ring stages by load index).
                 for (int q = 0; q < pl.nloads && ok; ++q) {
                     int kb, nA, nB;
                     load_at(pl, q, kb, nA, nB);
-                    if (!nA && !nB) continue;
                     const uint32_t st = kv_cnt % kStages;
-                    TRACE(0, 13, id, q, kv_cnt);
-                    TIMED(3, ok = mbar_wait(&kv_empty[st], ((kv_cnt / kStages) & 1) ^ 1, abort_flag));
+                    TRACE(0, 13, pl.id, q, kv_cnt);
+                    TIMED(2, ok = mbar_wait(&kv_empty[st], ((kv_cnt / kStages) & 1) ^ 1, abort_flag));
                     if (!ok) break;
                     mbar_arrive_expect_tx(&kv_full[st], 2 * kTileBytes);
                     tma_load_3d(smem + kOffK + st * kTileBytes, pl.global ? &maps.kg : &maps.k, &kv_full[st], 0,
@@ -657,7 +748,10 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
                 if (k > 0) ok = mbar_wait(tma_done, (k - 1) & 1, abort_flag);
                 if (ok) ok = mbar_wait(&item_empty[slot], ((k / kRing) & 1) ^ 1, abort_flag);
                 if (ok) {
-                    id = atomicAdd(p.sched, 1);
+                    // The first item of CTA c is item c (no atomic on the
+                    // critical path of the start); later ones come from the
+                    // counter, which counts past the first gridDim.x items.
+                    id = k == 0 ? (int)blockIdx.x : (int)gridDim.x + atomicAdd(p.sched, 1);
                     if (id >= p.n_items) id = -1;
                 }
             }
@@ -675,98 +769,176 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
+        // One sequence of S products over all items: product n goes to S
+        // buffer n % 3, and is issued right after the P V of product n - 3
+        // (which read that buffer; the tensor pipe runs in issue order).  So
+        // a tile's next S is computed while its softmax works on the current
+        // one, and P V of a block runs while the other tile's softmax runs.
+        // Lane 0 issues; its bookkeeping lives in packed registers.
         constexpr uint32_t idesc_qk = idesc_f16(Pack<T>::fmt, kBM, kBN, 0, 0);
         constexpr uint32_t idesc_pv = idesc_f16(Pack<T>::fmt, kBM, kHD, 0, 1);
-        uint32_t kv_cnt = 0, item_cnt = 0;
+        // Descriptors of the first Q / K / V tile; the others are reached by
+        // adding (byte offset >> 4) to the start-address field.
+        const uint64_t dq0 = desc_sw128(smem_u32(smem + kOffQ));
+        const uint64_t dk0 = desc_sw128(smem_u32(smem + kOffK));
+        const uint64_t dv0 = desc_sw128(smem_u32(smem + kOffV), 0);
+        constexpr uint32_t kTileStep = kTileBytes >> 4;
         TDECL;
-        uint32_t pcnt[2] = {0, 0};   // P blocks consumed per tile
-        uint32_t icnt[2] = {0, 0};   // items with work per tile
+        uint32_t kv_cnt = 0, item_cnt = 0;
+        uint32_t n_qk = 0, n_pv = 0;   // S products issued / P V products issued
+        uint32_t b_qk = 0, b_pv = 0;   // their S buffers (n % 3)
+        uint32_t pf_par = 0;           // bit b: phase of the next p_full[b] wait
+        uint32_t of_par = 0;           // bit x: phase of the next o_free[x] wait, flipped
+        uint32_t pend = 0;             // per S buffer, 4 bits: tile | stage << 1 | first << 3
+        uint32_t refc = 0;             // per K/V stage, 2 bits: P V products still to read it
+        // O_X (+)= P V for the oldest pending product; releases the K/V stage
+        // when its last user is done.
+        auto issue_pv = [&]() -> bool {
+            const uint32_t b = b_pv;
+            const uint32_t e = (pend >> (4 * b)) & 15u;
+            const uint32_t x = e & 1u, st = (e >> 1) & 3u, first = e >> 3;
+            bool w_ok;
+            TIMED(3, w_ok = mbar_wait(&p_full[b], (pf_par >> b) & 1u, abort_flag));
+            if (!w_ok) return false;
+            pf_par ^= 1u << b;
+            TCOUNT(5);
+            if (first) {
+                TIMED(4, w_ok = mbar_wait(&o_free[x], ((of_par >> x) & 1u) ^ 1u, abort_flag));
+                if (!w_ok) return false;
+                of_par ^= 1u << x;
+            }
+            tc_fence_after();
+            const uint64_t dv = dv0 + st * kTileStep;
+            const uint32_t d_tm = tmem + kTmemO + x * kHD, a_tm = tmem + b * kBN;
+#if LF_TRACE
+            const long long tp0_ = clock64();
+#endif
+#pragma unroll
+            for (int kk = 0; kk < kBN / 16; ++kk)
+                mma_f16_ts(d_tm, a_tm + kk * 8, dv + kk * (2048 >> 4), idesc_pv, (first && kk == 0) ? 0u : 1u);
+#if LF_TRACE
+            const long long tp1_ = clock64();
+            tacc[8] += tp1_ - tp0_;
+#endif
+            tc_commit(&pv_done[x]);
+            refc -= 1u << (2 * st);
+            if (((refc >> (2 * st)) & 3u) == 0) tc_commit(&kv_empty[st]);
+#if LF_TRACE
+            tacc[9] += clock64() - tp1_;
+#endif
+            ++n_pv;
+            b_pv = b_pv == kSBuf - 1 ? 0 : b_pv + 1;
+            return true;
+        };
+        // Waits for `bar` while issuing each pending P V as soon as its P is
+        // ready: a P V must never wait behind a plan, a Q tile or a K/V load,
+        // since the epilogue (which frees plan slots) and the softmax warps
+        // wait for it.
+        auto wait_issuing = [&](uint64_t* bar, uint32_t parity) -> bool {
+            if (mbar_test(bar, parity)) return true;
+            const uint64_t t0 = globaltimer();
+            for (uint32_t it = 1;; ++it) {
+                if (n_pv < n_qk && mbar_test(&p_full[b_pv], (pf_par >> b_pv) & 1u)) {
+                    if (!issue_pv()) return false;
+                } else {
+                    __nanosleep(20);
+                }
+                if (mbar_test(bar, parity)) return true;
+                if ((it & 63u) == 0) {
+                    if (*abort_flag) return false;
+                    if (globaltimer() - t0 > 2000000000ull) {
+                        *abort_flag = 1;
+                        return false;
+                    }
+                }
+            }
+        };
         bool ok = true;
         for (uint32_t k = 0; ok; ++k) {
-            const uint32_t slot = k % kRing;
-            if (lane == 0) {
-                TRACE(warp == 1 ? 1 : 2 + warp - kSoftmaxWarp0, warp == 1 ? 20 : 30, k, 0, 0);
-                TIMED(0, ok = mbar_wait(&item_full[slot], (k / kRing) & 1, abort_flag));
+            Plan pl;
+            {
+                const uint32_t slot = k % kRing;
+                if (lane == 0) TIMED(0, ok = wait_issuing(&item_full[slot], (k / kRing) & 1));
+                ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+                if (!ok) break;
+                __syncwarp();
+                pl = plans[slot];
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&item_empty[slot]);
             }
-            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-            if (!ok) break;
-            __syncwarp();                 // lane 0's acquire orders the reads below
-            const Plan pl = plans[slot];  // published by the producer before item_full
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&item_empty[slot]);
-            const int id = pl.id;
-            if (id < 0) break;
+            if (pl.id < 0) break;
             if (pl.nloads == 0) continue;
             if (lane == 0) {
                 const uint32_t qb = item_cnt & 1;
-                TRACE(1, 22, id, item_cnt, 0);
-                TIMED(2, ok = mbar_wait(&q_full[qb], (item_cnt >> 1) & 1, abort_flag));
-                tc_fence_after();
-                int pend[2] = {-1, -1};
-                bool first[2] = {true, true};
-                int refc[kStages];
-#pragma unroll
-                for (int s = 0; s < kStages; ++s) refc[s] = 0;
-                // O_X += P_X V[st]; releases the stage when its last user is done.
-                auto issue_pv = [&](int x, int st) -> bool {
-                    TRACE(1, 24, id, x, pcnt[x]);
-                    bool w_ok;
-                    TIMED(4, w_ok = mbar_wait(&p_full[x], pcnt[x] & 1, abort_flag));
-                    if (!w_ok) return false;
-                    ++pcnt[x];
-                    TRACE(1, 25, id, x, icnt[x]);
-                    if (first[x]) {
-                        TIMED(5, w_ok = mbar_wait(&o_free[x], (icnt[x] & 1) ^ 1, abort_flag));
-                        if (!w_ok) return false;
+                TIMED(1, ok = wait_issuing(&q_full[qb], (item_cnt >> 1) & 1));
+                // The item as scalars (no indexed accesses in the loop).
+                const int nA = tile_blocks(pl.t[0]), nB = tile_blocks(pl.t[1]);
+                const int m = min(nA, nB), xl = nA > nB ? 0 : 1, ntot = nA + nB;
+                const int glob = pl.global, e1 = pl.e1, lo_min = pl.lo_min;
+                const int ghA = pl.t[0].glob_hi, loA = pl.t[0].lo, hiA = pl.t[0].hi, prA = pl.t[0].present;
+                const int ghB = pl.t[1].glob_hi, loB = pl.t[1].lo, hiB = pl.t[1].hi, prB = pl.t[1].present;
+                const uint64_t dq = dq0 + qb * 2 * kTileStep;
+                int q_ready = -1;
+                for (int pos = 0; pos < ntot && ok; ++pos) {
+                    const bool inter = pos < 2 * m;
+                    const uint32_t x = inter ? (uint32_t)(pos & 1) : (uint32_t)xl;
+                    const int j = inter ? pos >> 1 : pos - m;
+                    if (n_qk - n_pv == (uint32_t)kSBuf) {  // free the buffer of product n_qk
+                        ok = issue_pv();
+                        if (!ok) break;
                     }
-                    tc_fence_after();
-                    const uint32_t v_addr = smem_u32(smem + kOffV + st * kTileBytes);
-#pragma unroll
-                    for (int kk = 0; kk < kBN / 16; ++kk)
-                        mma_f16_ts(tmem + kTmemO + x * kHD, tmem + x * kBN + kk * 8, desc_sw128(v_addr + kk * 2048, 0),
-                                   idesc_pv, (first[x] && kk == 0) ? 0u : 1u);
-                    first[x] = false;
-                    if (--refc[st] == 0) tc_commit(&kv_empty[st]);
-                    return true;
-                };
-                for (int q = 0; q < pl.nloads && ok; ++q) {
-                    int kb, need[2];
-                    load_at(pl, q, kb, need[0], need[1]);
-                    if (!need[0] && !need[1]) continue;
-                    const int st = kv_cnt % kStages;
-                    TRACE(1, 23, id, q, kv_cnt);
-                    TIMED(3, ok = mbar_wait(&kv_full[st], (kv_cnt / kStages) & 1, abort_flag));
+                    int q;
+                    if (glob) {
+                        q = pos;
+                    } else {
+                        const int gh = x ? ghB : ghA, lo = x ? loB : loA;
+                        const int kb = j < gh ? j : lo + (j - gh);
+                        q = kb < e1 ? kb : e1 + (kb - lo_min);
+                    }
+                    while (q_ready < q && ok) {
+                        ++q_ready;
+                        const uint32_t c = kv_cnt + q_ready, st = c % kStages;
+                        TIMED(2, ok = wait_issuing(&kv_full[st], (c / kStages) & 1));
+                        uint32_t users = 1;
+                        if (!glob) {
+                            const int kb = q_ready < e1 ? q_ready : lo_min + (q_ready - e1);
+                            users = (uint32_t)(prA && (kb < ghA || (kb >= loA && kb <= hiA))) +
+                                    (uint32_t)(prB && (kb < ghB || (kb >= loB && kb <= hiB)));
+                        }
+                        refc = (refc & ~(3u << (2 * st))) | (users << (2 * st));
+                        if (ok && users == 0) tc_commit(&kv_empty[st]);
+                    }
                     if (!ok) break;
                     tc_fence_after();
-                    refc[st] = need[0] + need[1];
-                    const uint32_t k_addr = smem_u32(smem + kOffK + st * kTileBytes);
-                    for (int x = 0; x < 2 && ok; ++x) {
-                        if (!need[x]) continue;
-                        if (pend[x] >= 0) ok = issue_pv(x, pend[x]);
-                        if (!ok) break;
-                        const uint32_t q_addr = smem_u32(smem + kOffQ + (qb * 2 + x) * kTileBytes);
+                    const uint32_t b = b_qk, st = (kv_cnt + q) % kStages;
+                    const uint64_t dqx = dq + x * kTileStep, dk = dk0 + st * kTileStep;
+#if LF_TRACE
+                    const long long tq0_ = clock64();
+#endif
 #pragma unroll
-                        for (int kk = 0; kk < kHD / 16; ++kk)
-                            mma_f16_ss(tmem + x * kBN, desc_sw128(q_addr + kk * 32), desc_sw128(k_addr + kk * 32),
-                                       idesc_qk, kk > 0);
-                        tc_commit(&s_full[x]);
-                        pend[x] = st;
-                    }
-                    ++kv_cnt;
+                    for (int kk = 0; kk < kHD / 16; ++kk)
+                        mma_f16_ss(tmem + b * kBN, dqx + kk * 2, dk + kk * 2, idesc_qk, kk > 0);
+#if LF_TRACE
+                    const long long tq1_ = clock64();
+                    tacc[7] += tq1_ - tq0_;
+#endif
+                    tc_commit(&s_full[x * kSBuf + b]);
+#if LF_TRACE
+                    tacc[10] += clock64() - tq1_;
+#endif
+                    TCOUNT(6);
+                    pend = (pend & ~(15u << (4 * b))) | ((x | (st << 1) | ((j == 0 ? 1u : 0u) << 3)) << (4 * b));
+                    ++n_qk;
+                    b_qk = b_qk == kSBuf - 1 ? 0 : b_qk + 1;
                 }
-                for (int x = 0; x < 2 && ok; ++x) {
-                    if (pend[x] < 0) continue;
-                    ok = issue_pv(x, pend[x]);
-                    if (ok) tc_commit(&o_done[x]);
-                }
-                tc_commit(&q_empty[qb]);
-                for (int x = 0; x < 2; ++x)
-                    if (pl.t[x].present) ++icnt[x];
+                if (ok) tc_commit(&q_empty[qb]);
             }
             ++item_cnt;
+            kv_cnt += pl.nloads;
             ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
         }
-        if (lane == 0) TRACE(1, 29, ok ? 1 : 0, item_cnt, kv_cnt);
+        if (lane == 0)
+            while (ok && n_pv < n_qk) ok = issue_pv();
         if (lane == 0) TDUMP(1);
         if (lane == 0 && !ok) {  // wind-down: wait for the MMAs already issued
             tc_commit(drain);
@@ -774,59 +946,41 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
             mbar_wait(drain, 0, &never, 200000000ull);
         }
     }
-    } else {
+    } else if (warp < kEpiWarp0) {
         regs_inc<kRegsSoftmax>();
-        // ------------------------------------------------------------ softmax / epilogue warps
+        // ------------------------------------------------------------ softmax warps
         const int x = (warp - kSoftmaxWarp0) >> 2;  // tile handled by this warpgroup
         const int sp = warp & 3;           // TMEM sub-partition (rows sp*32 .. +31)
         const int r = sp * 32 + lane;      // query row within the tile
         const uint32_t lane_off = (uint32_t)(sp * 32) << 16;
-        const uint32_t tS = tmem + lane_off + x * kBN;
         const uint32_t tO = tmem + lane_off + kTmemO + x * kHD;
         float* bias_w = reinterpret_cast<float*>(smem + kOffBias) + (warp - kSoftmaxWarp0) * kBN;
+        float2* stats = reinterpret_cast<float2*>(smem + kOffStats) + x * kBM;
+        uint32_t nqk = 0;     // S products of earlier items (both tiles)
+        uint32_t npv = 0;     // this tile's blocks in earlier items (its P V products)
+        uint32_t s_par = 0;   // bit b: phase of this tile's next use of S buffer b
+        uint32_t st_cnt = 0;  // items in which this tile had blocks
         TDECL;
-        uint32_t scnt = 0, icnt = 0;
         bool ok = true;
         for (uint32_t k = 0; ok; ++k) {
-            const uint32_t slot = k % kRing;
-            if (lane == 0) {
-                TRACE(warp == 1 ? 1 : 2 + warp - kSoftmaxWarp0, warp == 1 ? 20 : 30, k, 0, 0);
-                TIMED(0, ok = mbar_wait(&item_full[slot], (k / kRing) & 1, abort_flag));
-            }
-            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+            Plan pl;
+            TIMED(0, ok = next_plan(k, pl));
             if (!ok) break;
-            __syncwarp();                 // lane 0's acquire orders the reads below
-            const Plan pl = plans[slot];  // published by the producer before item_full
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&item_empty[slot]);
-            const int id = pl.id;
-            if (id < 0) break;
+            if (pl.id < 0) break;
+            if (pl.nloads == 0) continue;
+            const int nA = tile_blocks(pl.t[0]), nB = tile_blocks(pl.t[1]);
+            const int nblk = x == 0 ? nA : nB;
+            if (nblk == 0) {
+                nqk += nA + nB;
+                continue;
+            }
             const int g = pl.g;
             const Tile& me = pl.t[x];
             const float* lm = p.local_mask + (size_t)pl.b * p.L;
             const int i = me.r0 + r;
-            if (!pl.global) {
-                if (g > p.w) {  // invalid sample: zero output, record once
-                    if (me.r0 < p.L && i < p.L)
-                        store_zero_row(p.out, ((size_t)(pl.b * p.L + i) * p.H + pl.h) * kHD, sizeof(T));
-                    if (x == 0 && r == 0 && me.r0 == 0 && pl.h == 0) record_status(p.status, pl.b, LF_ERR_G_GT_W);
-                    continue;
-                }
-                if (me.r0 < p.L && i < p.L && i >= g && p.global_mask[(size_t)pl.b * p.L + i] == 0.0f)
-                    record_status(p.status, pl.b, LF_ERR_GLOBAL_NOT_PREFIX);
-                if (pl.zero_only[x]) {
-                    if (i < p.L && i >= g && lm[i] != 1.0f)
-                        store_zero_row(p.out, ((size_t)(pl.b * p.L + i) * p.H + pl.h) * kHD, sizeof(T));
-                    continue;
-                }
-            }
-            if (!me.present) continue;
-            // This tile's key blocks in load order: [0, glob_hi) then lo..hi.
             // Only these few scalars stay live through the block loop.
             const int is_global = pl.global;
-            const int nblk = me.glob_hi + (me.hi - me.lo + 1);
             const int blk_gh = me.glob_hi, blk_lo = me.lo;
-            const int pb = pl.b, ph = pl.h, pbh = pl.bh, prt = pl.rt, psplit = me.split;
 
             // Does this warp have rows whose output is kept?
             const int wr0 = me.r0 + sp * 32;
@@ -834,7 +988,6 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
             const bool warp_active = __any_sync(0xffffffffu, row_kept);
 
             float m_used = -INFINITY, l_run = 0.0f;
-            bool first = true;
             // local_mask of the next block's keys, loaded one block ahead so
             // that the load latency is off the critical path
             float mv_next[4] = {1.0f, 1.0f, 1.0f, 1.0f};
@@ -846,10 +999,16 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
                     mv_next[t] = key < p.L ? lm[key] : 1.0f;
                 }
             };
-            if (warp_active && nblk > 0) load_mv(0);
+            if (warp_active) load_mv(0);
             for (int n = 0; n < nblk && ok; ++n) {
+#if LF_TRACE
+                const long long tpro_ = clock64();
+#endif
+                const bool first = n == 0;
                 const int kb = n < blk_gh ? n : blk_lo + (n - blk_gh);
                 const int c0 = kb * kBN;
+                const uint32_t sb = (nqk + (uint32_t)seq_pos(x, n, nA, nB)) % kSBuf;
+                const uint32_t tS = tmem + lane_off + sb * kBN;
                 // Padding bias of the block's keys (keys >= L are masked instead).
                 bool has_pad = false;
                 if (warp_active) {
@@ -889,21 +1048,23 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
                     }
                     states |= (uint32_t)s << (2 * ch);
                 }
-                if (lane == 0) TRACE(2 + warp - kSoftmaxWarp0, 32, id, n, scnt);
+                if (lane == 0) TRACE(2 + warp - kSoftmaxWarp0, 32, pl.id, n, sb);
                 // every lane waits; the result is made warp-uniform so that an
                 // abort never splits the warp before a .sync.aligned instruction
-                TIMED(2, ok = __all_sync(0xffffffffu, mbar_wait(&s_full[x], scnt & 1, abort_flag)));
-                const long long tc0_ = clock64();
-                ++scnt;
+#if LF_TRACE
+                const long long tsw_ = clock64();
+                tacc[10] += tsw_ - tpro_;
+#endif
+                TIMED(1, ok = __all_sync(0xffffffffu, mbar_wait(&s_full[x * kSBuf + sb], (s_par >> sb) & 1u, abort_flag)));
+#if LF_TRACE
+                const long long tb0_ = clock64();
+                if (first) tacc[9] += tb0_ - tsw_;
+#endif
+                s_par ^= 1u << sb;
                 if (!ok) break;
                 tc_fence_after();
                 if (warp_active) {
                     auto state_of = [&](int ch) -> int { return (int)((states >> (2 * ch)) & 3u); };
-                    // Two passes over S in 32-column chunks with a rolled loop
-                    // (compact code, 32 live scores): pass 1 takes the row max,
-                    // pass 2 reloads each chunk from TMEM (cheap: ~100 cycles
-                    // for 16 KB) and writes P.  Pad bias and mask are applied
-                    // in both passes.
                     const int d0 = i - c0;
                     const int lo_c = d0 - p.w, hi_c = d0 + p.w, gl_c = g - c0, lim_c = p.L - c0;
                     auto chunk_bits = [&](int ch) -> uint32_t {
@@ -938,8 +1099,7 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
                     // so P <= 2^8); the whole warp then rescales (tcgen05.ld/st
                     // are .sync.aligned): the sums so far, this block's P
                     // chunks already in TMEM and, past the item's first block,
-                    // the O accumulator (whose previous P V has completed: it
-                    // ran before this block's S).
+                    // the O accumulator, once the previous block's P V is done.
                     const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
                     float2 sm2[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
                     // exponentials of one chunk, packed to 16 words of P
@@ -953,10 +1113,6 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
                             pk[c] = Pack<T>::two(e.x, e.y);
                         }
                     };
-#if LF_TRACE
-                    const long long ts2_ = clock64();
-                    tacc[7] += ts2_ - tc0_;
-#endif
 #pragma unroll 1
                     for (int ch = 0; ch < 4; ++ch) {
                         uint32_t pk[16];
@@ -1001,8 +1157,16 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
                                         tmem_st16(tS + pc * 16, pb16);
                                     }
                                     if (!first) {
+                                        // O holds the tile's blocks so far once the
+                                        // previous block's P V has completed
+                                        bool w_ok;
+                                        TIMED(7, w_ok = __all_sync(
+                                            0xffffffffu, mbar_wait(&pv_done[x], (npv + n - 1) & 1u, abort_flag)));
+                                        TCOUNT(8);
+                                        if (!w_ok) ok = false;
+                                        tc_fence_after();
 #pragma unroll
-                                        for (int c0o = 0; c0o < kHD; c0o += 16) {
+                                        for (int c0o = 0; c0o < kHD && w_ok; c0o += 16) {
                                             uint32_t ob[16];
                                             tmem_ld16(tO + c0o, ob);
                                             tmem_ld_wait();
@@ -1022,168 +1186,233 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
                         tmem_st16(tS + ch * 16, pk);
                     }
                     l_run += (sm2[0].x + sm2[0].y) + (sm2[1].x + sm2[1].y);
-#if LF_TRACE
-                    const long long ts4_ = clock64();
-                    tacc[9] += ts4_ - ts2_;
-#endif
                     tmem_st_wait();
-#if LF_TRACE
-                    tacc[10] += clock64() - ts4_;
-#endif
                 }
-                first = false;
+                // The previous block's P V has completed before this block's P
+                // is handed over: every later wait on pv_done is then at most
+                // one phase behind the barrier.
+#if LF_TRACE
+                tacc[2] += clock64() - tb0_;
+                TCOUNT(5);
+#endif
+                if (npv + n > 0)
+                    TIMED(3, ok = ok && __all_sync(0xffffffffu, mbar_wait(&pv_done[x], (npv + n - 1) & 1u, abort_flag)));
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&p_full[x]);
-#if LF_TRACE
-                tacc[3] += clock64() - tc0_;
-                tacc[4] += 1;
-#endif
+                if (lane == 0) mbar_arrive(&p_full[sb]);
             }
             if (!ok) break;
-
-            // ---------------------------------------------------- epilogue
-            if (lane == 0) TRACE(2 + warp - kSoftmaxWarp0, 33, id, icnt, 0);
-            TIMED(5, ok = __all_sync(0xffffffffu, mbar_wait(&o_done[x], icnt & 1, abort_flag)));
-            ++icnt;
+            // Row (m, l) to the epilogue warps.
+            TIMED(4, ok = __all_sync(0xffffffffu, mbar_wait(&st_free[x], (st_cnt & 1) ^ 1, abort_flag)));
+            TCOUNT(6);
             if (!ok) break;
-            tc_fence_after();
-            float o[kHD];
-            {
-                uint32_t o0[32], o1[32];
-                tmem_ld32(tO, o0);
-                tmem_ld32(tO + 32, o1);
-                tmem_ld_wait();
-                regs_ready<32>(o0);
-                regs_ready<32>(o1);
-#pragma unroll
-                for (int c = 0; c < 32; ++c) {
-                    o[c] = __uint_as_float(o0[c]);
-                    o[c + 32] = __uint_as_float(o1[c]);
-                }
-            }
-            tc_fence_before();
+            stats[r] = make_float2(m_used, l_run);
             __syncwarp();
-            if (lane == 0) mbar_arrive(&o_free[x]);
-
-            if (!is_global) {
-                if (i < p.L && i >= g) {
-                    const size_t off = ((size_t)(pb * p.L + i) * p.H + ph) * kHD;
-                    if (lm[i] != 1.0f) store_zero_row(p.out, off, sizeof(T));
-                    else store_row<T>(p.out, off, o, fast_rcp(l_run));
+            if (lane == 0) mbar_arrive(&st_full[x]);
+            ++st_cnt;
+            nqk += nA + nB;
+            npv += nblk;
+        }
+        if (lane == 0) TDUMP(2 + warp - kSoftmaxWarp0);
+    } else {
+        regs_dec<kRegsEpi>();
+        // ------------------------------------------------------------ epilogue warps
+        // Per item and tile: wait for the tile's last P V, read O and the row
+        // (m, l), hand O back, then write the rows (band tiles), or the
+        // split-KV partials and, for the last split of a row group, the
+        // merged rows (global tiles).  Also zeroes padded rows of tiles
+        // without key blocks and rows of samples that break the constraints.
+        const int sp = warp & 3;
+        const int r = sp * 32 + lane;
+        const uint32_t lane_off = (uint32_t)(sp * 32) << 16;
+        const float2* stats = reinterpret_cast<const float2*>(smem + kOffStats);
+        uint32_t npv[2] = {0, 0}, st_cnt[2] = {0, 0};
+        TDECL;
+        bool ok = true;
+        for (uint32_t k = 0; ok; ++k) {
+            Plan pl;
+            TIMED(0, ok = next_plan(k, pl));
+            if (!ok) break;
+            if (pl.id < 0) break;
+            const int g = pl.g;
+            const float* lm = p.local_mask + (size_t)pl.b * p.L;
+            for (int x = 0; x < 2 && ok; ++x) {
+                const Tile& me = pl.t[x];
+                const int i = me.r0 + r;
+                if (!pl.global) {
+                    if (g > p.w) {  // invalid sample: zero output, record once
+                        if (me.r0 < p.L && i < p.L)
+                            store_zero_row(p.out, ((size_t)(pl.b * p.L + i) * p.H + pl.h) * kHD, sizeof(T));
+                        if (x == 0 && r == 0 && me.r0 == 0 && pl.h == 0) record_status(p.status, pl.b, LF_ERR_G_GT_W);
+                        continue;
+                    }
+                    if (me.r0 < p.L && i < p.L && i >= g && p.global_mask[(size_t)pl.b * p.L + i] == 0.0f)
+                        record_status(p.status, pl.b, LF_ERR_GLOBAL_NOT_PREFIX);
+                    if (pl.zero_only[x]) {
+                        if (i < p.L && i >= g && lm[i] != 1.0f)
+                            store_zero_row(p.out, ((size_t)(pl.b * p.L + i) * p.H + pl.h) * kHD, sizeof(T));
+                        continue;
+                    }
                 }
-            } else if (wr0 < g) {
-                // Split-KV partials of this warp's 32 rows; the warp that
-                // completes the last split of its row group merges them.
-                const int slot0 = (pbh * p.RT + prt) * p.NS;
-                const int sl = slot0 + psplit;
-                if (i < g) {
-                    float4* po = reinterpret_cast<float4*>(p.part_o + ((size_t)sl * kBM + r) * kHD);
+                const int nblk = tile_blocks(me);
+                if (nblk == 0) continue;
+                // (m, l) first: they are written after the tile's last block,
+                // whose P V is then at most one phase ahead of this wait.
+                if (lane == 0) TRACE(10 + sp, 40 + x, pl.id, st_cnt[x], npv[x]);
+                TIMED(1, ok = __all_sync(0xffffffffu, mbar_wait(&st_full[x], st_cnt[x] & 1, abort_flag)));
+                if (!ok) break;
+                const float2 ml = stats[x * kBM + r];
+                TIMED(2, ok = __all_sync(0xffffffffu, mbar_wait(&pv_done[x], (npv[x] + nblk - 1) & 1u, abort_flag)));
+                if (!ok) break;
+                tc_fence_after();
+                float o[kHD];
+                {
+                    const uint32_t tO = tmem + lane_off + kTmemO + x * kHD;
+                    uint32_t o0[32], o1[32];
+                    tmem_ld32(tO, o0);
+                    tmem_ld32(tO + 32, o1);
+                    tmem_ld_wait();
+                    regs_ready<32>(o0);
+                    regs_ready<32>(o1);
 #pragma unroll
-                    for (int c = 0; c < kHD / 4; ++c)
-                        __stcg(po + c, make_float4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]));
-                    __stcg(reinterpret_cast<float2*>(p.part_ml + ((size_t)sl * kBM + r) * 2),
-                           make_float2(m_used, l_run));
+                    for (int c = 0; c < 32; ++c) {
+                        o[c] = __uint_as_float(o0[c]);
+                        o[c + 32] = __uint_as_float(o1[c]);
+                    }
                 }
-                __threadfence();
+                tc_fence_before();
                 __syncwarp();
-                int* counter = p.counters + (pbh * p.RT + prt) * 4 + sp;
-                int last = 0;
-                if (lane == 0) last = (atomicAdd(counter, 1) == p.NS - 1) ? 1 : 0;
-                last = __shfl_sync(0xffffffffu, last, 0);
-                if (last) {
-                    __threadfence();
+                if (lane == 0) {
+                    mbar_arrive(&o_free[x]);
+                    mbar_arrive(&st_free[x]);
+                }
+                ++st_cnt[x];
+                npv[x] += nblk;
+
+                if (!pl.global) {
+                    if (i < p.L && i >= g) {
+                        const size_t off = ((size_t)(pl.b * p.L + i) * p.H + pl.h) * kHD;
+                        if (lm[i] != 1.0f) store_zero_row(p.out, off, sizeof(T));
+                        else store_row<T>(p.out, off, o, fast_rcp(ml.y));
+                    }
+                } else if (me.r0 + sp * 32 < g) {
+                    // Split-KV partials of this warp's 32 rows; the warp that
+                    // completes the last split of its row group merges them.
+                    const int slot0 = (pl.bh * p.RT + pl.rt) * p.NS;
+                    const int sl = slot0 + me.split;
                     if (i < g) {
-                        const size_t off = ((size_t)(pb * p.L + i) * p.H + ph) * kHD;
-                        if (lm[i] != 1.0f) {
-                            store_zero_row(p.out, off, sizeof(T));
-                        } else {
-                            // all (m, l) of the row first, in flight together
-                            constexpr int kMaxNS = 64;
-                            float2 mls[kMaxNS];
-                            const int ns = min(p.NS, kMaxNS);
-                            float M = -INFINITY;
-                            for (int s = 0; s < ns; ++s)
-                                mls[s] = __ldcg(
-                                    reinterpret_cast<const float2*>(p.part_ml + ((size_t)(slot0 + s) * kBM + r) * 2));
-                            // splits beyond the batch are read again where used
-                            auto ml_of = [&](int s) -> float2 {
-                                return s < ns ? mls[s]
-                                              : __ldcg(reinterpret_cast<const float2*>(
-                                                    p.part_ml + ((size_t)(slot0 + s) * kBM + r) * 2));
-                            };
-                            for (int s = 0; s < p.NS; ++s) M = fmaxf(M, ml_of(s).x);
-                            float lsum = 0.0f;
-                            for (int s = 0; s < p.NS; ++s) {
-                                const float2 ml = ml_of(s);
-                                lsum = fmaf(ml.y, ml.x == -INFINITY ? 0.0f : ex2(ml.x - M), lsum);
-                            }
-                            const float inv = fast_rcp(lsum);
-                            // merge 16 channels at a time to keep registers low
-                            for (int cq = 0; cq < kHD; cq += 16) {
-                                float acc[16];
+                        float4* po = reinterpret_cast<float4*>(p.part_o + ((size_t)sl * kBM + r) * kHD);
 #pragma unroll
-                                for (int c = 0; c < 16; ++c) acc[c] = 0.0f;
+                        for (int c = 0; c < kHD / 4; ++c)
+                            __stcg(po + c, make_float4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]));
+                        __stcg(reinterpret_cast<float2*>(p.part_ml + ((size_t)sl * kBM + r) * 2), ml);
+                    }
+                    __threadfence();
+                    __syncwarp();
+                    int* counter = p.counters + (pl.bh * p.RT + pl.rt) * 4 + sp;
+                    int last = 0;
+                    if (lane == 0) last = (atomicAdd(counter, 1) == p.NS - 1) ? 1 : 0;
+                    last = __shfl_sync(0xffffffffu, last, 0);
+                    if (last) {
+                        __threadfence();
+                        if (i < g) {
+                            const size_t off = ((size_t)(pl.b * p.L + i) * p.H + pl.h) * kHD;
+                            if (lm[i] != 1.0f) {
+                                store_zero_row(p.out, off, sizeof(T));
+                            } else {
+                                auto ml_of = [&](int s) -> float2 {
+                                    return __ldcg(reinterpret_cast<const float2*>(
+                                        p.part_ml + ((size_t)(slot0 + s) * kBM + r) * 2));
+                                };
+                                float M = -INFINITY;
+                                for (int s = 0; s < p.NS; ++s) M = fmaxf(M, ml_of(s).x);
+                                float lsum = 0.0f;
                                 for (int s = 0; s < p.NS; ++s) {
-                                    const float mx = __ldcg(p.part_ml + ((size_t)(slot0 + s) * kBM + r) * 2);
-                                    const float wgt = mx == -INFINITY ? 0.0f : ex2(mx - M);
-                                    const float4* po = reinterpret_cast<const float4*>(
-                                        p.part_o + ((size_t)(slot0 + s) * kBM + r) * kHD + cq);
-#pragma unroll
-                                    for (int c = 0; c < 4; ++c) {
-                                        const float4 t4 = __ldcg(po + c);
-                                        acc[4 * c] = fmaf(t4.x, wgt, acc[4 * c]);
-                                        acc[4 * c + 1] = fmaf(t4.y, wgt, acc[4 * c + 1]);
-                                        acc[4 * c + 2] = fmaf(t4.z, wgt, acc[4 * c + 2]);
-                                        acc[4 * c + 3] = fmaf(t4.w, wgt, acc[4 * c + 3]);
-                                    }
+                                    const float2 m2 = ml_of(s);
+                                    lsum = fmaf(m2.y, m2.x == -INFINITY ? 0.0f : ex2(m2.x - M), lsum);
                                 }
-                                uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<T*>(p.out) + off + cq);
+                                const float inv = fast_rcp(lsum);
+                                // merge 16 channels at a time to keep registers low
+                                for (int cq = 0; cq < kHD; cq += 16) {
+                                    float acc[16];
 #pragma unroll
-                                for (int c = 0; c < 2; ++c) {
-                                    uint4 u;
-                                    u.x = Pack<T>::two(acc[8 * c + 0] * inv, acc[8 * c + 1] * inv);
-                                    u.y = Pack<T>::two(acc[8 * c + 2] * inv, acc[8 * c + 3] * inv);
-                                    u.z = Pack<T>::two(acc[8 * c + 4] * inv, acc[8 * c + 5] * inv);
-                                    u.w = Pack<T>::two(acc[8 * c + 6] * inv, acc[8 * c + 7] * inv);
-                                    dst[c] = u;
+                                    for (int c = 0; c < 16; ++c) acc[c] = 0.0f;
+                                    for (int s = 0; s < p.NS; ++s) {
+                                        const float mx = ml_of(s).x;
+                                        const float wgt = mx == -INFINITY ? 0.0f : ex2(mx - M);
+                                        const float4* po = reinterpret_cast<const float4*>(
+                                            p.part_o + ((size_t)(slot0 + s) * kBM + r) * kHD + cq);
+#pragma unroll
+                                        for (int c = 0; c < 4; ++c) {
+                                            const float4 t4 = __ldcg(po + c);
+                                            acc[4 * c] = fmaf(t4.x, wgt, acc[4 * c]);
+                                            acc[4 * c + 1] = fmaf(t4.y, wgt, acc[4 * c + 1]);
+                                            acc[4 * c + 2] = fmaf(t4.z, wgt, acc[4 * c + 2]);
+                                            acc[4 * c + 3] = fmaf(t4.w, wgt, acc[4 * c + 3]);
+                                        }
+                                    }
+                                    uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<T*>(p.out) + off + cq);
+#pragma unroll
+                                    for (int c = 0; c < 2; ++c) {
+                                        uint4 u;
+                                        u.x = Pack<T>::two(acc[8 * c + 0] * inv, acc[8 * c + 1] * inv);
+                                        u.y = Pack<T>::two(acc[8 * c + 2] * inv, acc[8 * c + 3] * inv);
+                                        u.z = Pack<T>::two(acc[8 * c + 4] * inv, acc[8 * c + 5] * inv);
+                                        u.w = Pack<T>::two(acc[8 * c + 6] * inv, acc[8 * c + 7] * inv);
+                                        dst[c] = u;
+                                    }
                                 }
                             }
                         }
+                        if (lane == 0) *counter = 0;
                     }
-                    if (lane == 0) *counter = 0;
                 }
             }
         }
-        if (lane == 0) TDUMP(2 + warp - kSoftmaxWarp0);
+        if (lane == 0) TDUMP(10 + sp);
     }
 
-    if (warp >= kSoftmaxWarp0 && lane == 0) TRACE(2 + warp - kSoftmaxWarp0, 39, 0, 0, 0);
+#if LF_TRACE
+    if (threadIdx.x == 0 && p.trace) {  // CTA start/end time
+        volatile int* d_ = p.trace + gridDim.x * 16 * 4 + (blockIdx.x * 16 + 14) * 16;
+        const unsigned long long t = globaltimer();
+        d_[2] = (int)(t & 0xffffffffu);
+        d_[3] = (int)(t >> 32);
+    }
+#endif
     __syncthreads();
+    volatile int* last_cta = abort_flag + 1;
     if (threadIdx.x == 0) {
-        TRACE(10, 98, *abort_flag, 0, 0);
         if (*abort_flag) record_status(p.status, 0, LF_ERR_DEVICE_TIMEOUT);
-        // The last CTA to finish resets the scheduler for the next launch.
         __threadfence();
-        if (atomicAdd(p.sched + 1, 1) == (int)gridDim.x - 1) {
+        *last_cta = atomicAdd(p.sched + 1, 1) == (int)gridDim.x - 1;
+    }
+    __syncthreads();
+    if (*last_cta) {
+        // The last CTA to finish resets the scheduler and the split counters
+        // for the next launch (the counters are already zero unless a
+        // launch was aborted part-way).
+        __threadfence();
+        const int n_counters = p.B * p.H * p.RT * 4;
+        for (int c = threadIdx.x; c < n_counters; c += kThreads) p.counters[c] = 0;
+        if (threadIdx.x == 0) {
             p.sched[0] = 0;
             p.sched[1] = 0;
-            __threadfence();
         }
-        TRACE(10, 99, 0, 0, 0);
-#if LF_TRACE
-        if (p.trace) {  // CTA end time
-            const unsigned long long t = globaltimer();
-            volatile int* d_ = p.trace + gridDim.x * 16 * 4 + (blockIdx.x * 16 + 12) * 16;
-            d_[2] = (int)(t & 0xffffffffu);
-            d_[3] = (int)(t >> 32);
-        }
-#endif
+        __threadfence();
     }
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
+#if LF_TRACE
+    if (threadIdx.x == 32 && p.trace) {  // exit time (after the TMEM release)
+        volatile int* d_ = p.trace + gridDim.x * 16 * 4 + (blockIdx.x * 16 + 15) * 16;
+        const unsigned long long t = globaltimer();
+        d_[2] = (int)(t & 0xffffffffu);
+        d_[3] = (int)(t >> 32);
+    }
+#endif
 }
 
 // ---------------------------------------------------------------- host side
