@@ -69,9 +69,9 @@ constexpr int kWarps = 16;
 constexpr int kThreads = kWarps * 32;
 constexpr int kSoftmaxWarp0 = 4;  // warps 4-7: tile A, 8-11: tile B
 constexpr int kEpiWarp0 = 12;     // warps 12-15: epilogue of both tiles
-constexpr uint32_t kRegsProducer = 96;
-constexpr uint32_t kRegsSoftmax = 160;
-constexpr uint32_t kRegsEpi = 96;
+constexpr uint32_t kRegsProducer = 88;
+constexpr uint32_t kRegsSoftmax = 152;
+constexpr uint32_t kRegsEpi = 120;
 static_assert(4 * 32 * kRegsProducer + 8 * 32 * kRegsSoftmax + 4 * 32 * kRegsEpi <= 65536, "register split");
 constexpr int kItemConsumers = 1 + 1 + 8 + 4;  // TMA + MMA + softmax + epilogue warps
 constexpr uint32_t kTileBytes = kBM * kHD * 2;  // 16 KB
@@ -106,8 +106,8 @@ struct Params {
     int NTP;     // tile pairs per head
     int chunk;   // key blocks per global-row split
     int n_inner; // band pairs away from the sequence ends (first in the order)
-    int n_glob;  // global pair items (next: their split merges then overlap
-                 // the band pairs at the ends of the sequences, which are last)
+    int n_glob;  // global pair items (after the interior band pairs, before
+                 // the band pairs at the ends of the sequences)
     int n_items;
     float scale_log2;  // scale * log2(e)
     float inv_scale;   // 1 / scale: the padding bias in raw score units
@@ -271,8 +271,10 @@ __device__ void band_rows2(const Params& p, int b, const int (&r0)[2], int& cach
 __device__ Plan make_plan(const Params& p, int id, int& cached_b, int& g) {
     Plan pl;
     pl.id = id;
-    // Item order, longest first: interior band pairs (the most key blocks),
-    // then global pairs, then the band pairs at both ends of each sequence.
+    // Item order: interior band pairs (the most key blocks), then the global
+    // pairs (the epilogue warps merge their splits while the softmax warps
+    // already run the next item), then the band pairs at both ends of each
+    // sequence, which are short and end the launch.
     const int inner_per = p.NTP > 2 ? p.NTP - 2 : 0;
     const int edge_per = p.NTP < 2 ? p.NTP : 2;
     if (id >= p.n_inner && id < p.n_inner + p.n_glob) {
@@ -284,6 +286,7 @@ __device__ Plan make_plan(const Params& p, int id, int& cached_b, int& g) {
         pl.bh = r / p.RT;
         pl.t[0].split = 2 * sp;
         pl.t[1].split = 2 * sp + 1;
+        pl.t[0].r0 = pl.t[1].r0 = pl.rt * kBM;  // set before any early return: every role reads it
     } else {
         int tp;
         if (id < p.n_inner) {
@@ -298,6 +301,7 @@ __device__ Plan make_plan(const Params& p, int id, int& cached_b, int& g) {
         pl.rt = 0;
         pl.t[0].r0 = 2 * tp * kBM;
         pl.t[1].r0 = (2 * tp + 1) * kBM;
+        pl.t[0].split = pl.t[1].split = 0;
     }
     pl.b = pl.bh / p.H;
     pl.h = pl.bh % p.H;
@@ -1239,23 +1243,37 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
             for (int x = 0; x < 2 && ok; ++x) {
                 const Tile& me = pl.t[x];
                 const int i = me.r0 + r;
+#if LF_TRACE
+                const long long te0_ = clock64();
+#endif
+                // This row's mask values, loaded before any wait so that
+                // their latency is hidden; a global_mask 0.0 past the prefix
+                // is recorded at the end of the tile.
+                const bool in_row = me.r0 < p.L && i < p.L;
+                const float lmi = in_row ? lm[i] : 1.0f;
+                const float gmi = (in_row && !pl.global) ? p.global_mask[(size_t)pl.b * p.L + i] : 1.0f;
+                const bool not_prefix = !pl.global && g <= p.w && in_row && i >= g;
                 if (!pl.global) {
                     if (g > p.w) {  // invalid sample: zero output, record once
-                        if (me.r0 < p.L && i < p.L)
-                            store_zero_row(p.out, ((size_t)(pl.b * p.L + i) * p.H + pl.h) * kHD, sizeof(T));
+                        if (in_row) store_zero_row(p.out, ((size_t)(pl.b * p.L + i) * p.H + pl.h) * kHD, sizeof(T));
                         if (x == 0 && r == 0 && me.r0 == 0 && pl.h == 0) record_status(p.status, pl.b, LF_ERR_G_GT_W);
                         continue;
                     }
-                    if (me.r0 < p.L && i < p.L && i >= g && p.global_mask[(size_t)pl.b * p.L + i] == 0.0f)
-                        record_status(p.status, pl.b, LF_ERR_GLOBAL_NOT_PREFIX);
                     if (pl.zero_only[x]) {
-                        if (i < p.L && i >= g && lm[i] != 1.0f)
+                        if (in_row && i >= g && lmi != 1.0f)
                             store_zero_row(p.out, ((size_t)(pl.b * p.L + i) * p.H + pl.h) * kHD, sizeof(T));
+                        if (not_prefix && gmi == 0.0f) record_status(p.status, pl.b, LF_ERR_GLOBAL_NOT_PREFIX);
                         continue;
                     }
                 }
                 const int nblk = tile_blocks(me);
-                if (nblk == 0) continue;
+#if LF_TRACE
+                tacc[7] += clock64() - te0_;
+#endif
+                if (nblk == 0) {
+                    if (not_prefix && gmi == 0.0f) record_status(p.status, pl.b, LF_ERR_GLOBAL_NOT_PREFIX);
+                    continue;
+                }
                 // (m, l) first: they are written after the tile's last block,
                 // whose P V is then at most one phase ahead of this wait.
                 if (lane == 0) TRACE(10 + sp, 40 + x, pl.id, st_cnt[x], npv[x]);
@@ -1265,20 +1283,17 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
                 TIMED(2, ok = __all_sync(0xffffffffu, mbar_wait(&pv_done[x], (npv[x] + nblk - 1) & 1u, abort_flag)));
                 if (!ok) break;
                 tc_fence_after();
+                // O of this tile's rows, read once; P V is complete.
+#if LF_TRACE
+                const long long te1_ = clock64();
+#endif
                 float o[kHD];
                 {
                     const uint32_t tO = tmem + lane_off + kTmemO + x * kHD;
-                    uint32_t o0[32], o1[32];
-                    tmem_ld32(tO, o0);
-                    tmem_ld32(tO + 32, o1);
+                    tmem_ld32f(tO, *reinterpret_cast<float(*)[32]>(&o[0]));
+                    tmem_ld32f(tO + 32, *reinterpret_cast<float(*)[32]>(&o[32]));
                     tmem_ld_wait();
-                    regs_ready<32>(o0);
-                    regs_ready<32>(o1);
-#pragma unroll
-                    for (int c = 0; c < 32; ++c) {
-                        o[c] = __uint_as_float(o0[c]);
-                        o[c + 32] = __uint_as_float(o1[c]);
-                    }
+                    regs_ready<kHD>(o);
                 }
                 tc_fence_before();
                 __syncwarp();
@@ -1288,13 +1303,22 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
                 }
                 ++st_cnt[x];
                 npv[x] += nblk;
+#if LF_TRACE
+                const long long te2_ = clock64();
+                tacc[3] += te2_ - te1_;
+#endif
 
                 if (!pl.global) {
-                    if (i < p.L && i >= g) {
+                    if (in_row && i >= g) {
                         const size_t off = ((size_t)(pl.b * p.L + i) * p.H + pl.h) * kHD;
-                        if (lm[i] != 1.0f) store_zero_row(p.out, off, sizeof(T));
+                        if (lmi != 1.0f) store_zero_row(p.out, off, sizeof(T));
                         else store_row<T>(p.out, off, o, fast_rcp(ml.y));
                     }
+                    if (not_prefix && gmi == 0.0f) record_status(p.status, pl.b, LF_ERR_GLOBAL_NOT_PREFIX);
+#if LF_TRACE
+                    tacc[4] += clock64() - te2_;
+                    TCOUNT(8);
+#endif
                 } else if (me.r0 + sp * 32 < g) {
                     // Split-KV partials of this warp's 32 rows; the warp that
                     // completes the last split of its row group merges them.
@@ -1313,58 +1337,74 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
                     int last = 0;
                     if (lane == 0) last = (atomicAdd(counter, 1) == p.NS - 1) ? 1 : 0;
                     last = __shfl_sync(0xffffffffu, last, 0);
+#if LF_TRACE
+                    const long long te3_ = clock64();
+                    tacc[5] += te3_ - te2_;
+                    TCOUNT(9);
+#endif
                     if (last) {
                         __threadfence();
                         if (i < g) {
                             const size_t off = ((size_t)(pl.b * p.L + i) * p.H + pl.h) * kHD;
-                            if (lm[i] != 1.0f) {
+                            if (lmi != 1.0f) {
                                 store_zero_row(p.out, off, sizeof(T));
                             } else {
-                                auto ml_of = [&](int s) -> float2 {
-                                    return __ldcg(reinterpret_cast<const float2*>(
-                                        p.part_ml + ((size_t)(slot0 + s) * kBM + r) * 2));
-                                };
+                                // Merge by log-sum-exp, with the loads of a
+                                // round in flight together: the (m, l) of up
+                                // to 16 splits, then per column half each
+                                // split's 32 values with its (m, l).
+                                const float2* pml = reinterpret_cast<const float2*>(p.part_ml) + (size_t)slot0 * kBM + r;
                                 float M = -INFINITY;
-                                for (int s = 0; s < p.NS; ++s) M = fmaxf(M, ml_of(s).x);
-                                float lsum = 0.0f;
-                                for (int s = 0; s < p.NS; ++s) {
-                                    const float2 m2 = ml_of(s);
-                                    lsum = fmaf(m2.y, m2.x == -INFINITY ? 0.0f : ex2(m2.x - M), lsum);
+                                for (int s0 = 0; s0 < p.NS; s0 += 16) {
+                                    float mx[16];
+#pragma unroll
+                                    for (int u = 0; u < 16; ++u)
+                                        mx[u] = s0 + u < p.NS ? __ldcg(pml + (size_t)(s0 + u) * kBM).x : -INFINITY;
+#pragma unroll
+                                    for (int u = 0; u < 16; ++u) M = fmaxf(M, mx[u]);
                                 }
-                                const float inv = fast_rcp(lsum);
-                                // merge 16 channels at a time to keep registers low
-                                for (int cq = 0; cq < kHD; cq += 16) {
-                                    float acc[16];
+                                float lsum = 0.0f;
+                                for (int h = 0; h < 2; ++h) {
+                                    float acc[32];
 #pragma unroll
-                                    for (int c = 0; c < 16; ++c) acc[c] = 0.0f;
-                                    for (int s = 0; s < p.NS; ++s) {
-                                        const float mx = ml_of(s).x;
-                                        const float wgt = mx == -INFINITY ? 0.0f : ex2(mx - M);
+                                    for (int c = 0; c < 32; ++c) acc[c] = 0.0f;
+                                    for (int s1 = 0; s1 < p.NS; ++s1) {
                                         const float4* po = reinterpret_cast<const float4*>(
-                                            p.part_o + ((size_t)(slot0 + s) * kBM + r) * kHD + cq);
+                                            p.part_o + ((size_t)(slot0 + s1) * kBM + r) * kHD + 32 * h);
+                                        float4 t4[8];
 #pragma unroll
-                                        for (int c = 0; c < 4; ++c) {
-                                            const float4 t4 = __ldcg(po + c);
-                                            acc[4 * c] = fmaf(t4.x, wgt, acc[4 * c]);
-                                            acc[4 * c + 1] = fmaf(t4.y, wgt, acc[4 * c + 1]);
-                                            acc[4 * c + 2] = fmaf(t4.z, wgt, acc[4 * c + 2]);
-                                            acc[4 * c + 3] = fmaf(t4.w, wgt, acc[4 * c + 3]);
+                                        for (int c = 0; c < 8; ++c) t4[c] = __ldcg(po + c);
+                                        const float2 m2 = __ldcg(pml + (size_t)s1 * kBM);
+                                        const float wgt = m2.x == -INFINITY ? 0.0f : ex2(m2.x - M);
+                                        if (h == 0) lsum = fmaf(m2.y, wgt, lsum);
+#pragma unroll
+                                        for (int c = 0; c < 8; ++c) {
+                                            acc[4 * c] = fmaf(t4[c].x, wgt, acc[4 * c]);
+                                            acc[4 * c + 1] = fmaf(t4[c].y, wgt, acc[4 * c + 1]);
+                                            acc[4 * c + 2] = fmaf(t4[c].z, wgt, acc[4 * c + 2]);
+                                            acc[4 * c + 3] = fmaf(t4[c].w, wgt, acc[4 * c + 3]);
                                         }
                                     }
-                                    uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<T*>(p.out) + off + cq);
+                                    // lsum is complete after the first half
+                                    const float inv = fast_rcp(lsum);
+                                    uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<T*>(p.out) + off + 32 * h);
 #pragma unroll
-                                    for (int c = 0; c < 2; ++c) {
-                                        uint4 u;
-                                        u.x = Pack<T>::two(acc[8 * c + 0] * inv, acc[8 * c + 1] * inv);
-                                        u.y = Pack<T>::two(acc[8 * c + 2] * inv, acc[8 * c + 3] * inv);
-                                        u.z = Pack<T>::two(acc[8 * c + 4] * inv, acc[8 * c + 5] * inv);
-                                        u.w = Pack<T>::two(acc[8 * c + 6] * inv, acc[8 * c + 7] * inv);
-                                        dst[c] = u;
+                                    for (int c = 0; c < 4; ++c) {
+                                        uint4 u4;
+                                        u4.x = Pack<T>::two(acc[8 * c + 0] * inv, acc[8 * c + 1] * inv);
+                                        u4.y = Pack<T>::two(acc[8 * c + 2] * inv, acc[8 * c + 3] * inv);
+                                        u4.z = Pack<T>::two(acc[8 * c + 4] * inv, acc[8 * c + 5] * inv);
+                                        u4.w = Pack<T>::two(acc[8 * c + 6] * inv, acc[8 * c + 7] * inv);
+                                        dst[c] = u4;
                                     }
                                 }
                             }
                         }
                         if (lane == 0) *counter = 0;
+#if LF_TRACE
+                        tacc[6] += clock64() - te3_;
+                        TCOUNT(10);
+#endif
                     }
                 }
             }
@@ -1450,13 +1490,14 @@ bool make_map(CUtensorMap* m, const void* base, int BH, int L) {
 // Global-row split size.  Items are taken from a counter by the CTAs as they
 // free up, so the kernel ends when the last CTA finishes its last item; with
 // only a few items per CTA the split size decides how evenly the work packs.
-// The host replays that list schedule for each candidate size with a cost
-// model of the kernel (per item: a fixed part plus its longer tile's key
-// blocks; a global pair adds its merge; relative weights 80 : 60 per block :
-// 30, from event traces of the kernel on B200) and keeps the size with the
-// earliest finish.  Leading
-// globals are taken as g <= 128 (one global row tile with work, one block of
-// global keys per band tile); the choice only affects speed.
+// The host replays that list schedule (inner band pairs, global pairs, edge
+// pairs) for each candidate size with a cost model of the kernel and keeps
+// the size with the earliest finish.  Relative costs, from per-role cycle
+// counts of the kernel on B200: a band key block 60, a global key block 75
+// (every chunk of it is computed), an item 25 (its first S and the
+// epilogue), a split merge 15.  Leading globals are taken as g <= 128 (one
+// global row tile with work, one block of global keys per band tile); the
+// choice only affects speed.
 int choose_chunk(int B, int H, int L, int w, int sm_count) {
     const int NKB = (L + kBN - 1) / kBN;
     const int NT = (L + kBM - 1) / kBM;
@@ -1479,7 +1520,7 @@ int choose_chunk(int B, int H, int L, int w, int sm_count) {
             if (cache[i].B == B && cache[i].H == H && cache[i].L == L && cache[i].w == w && cache[i].sm == sm_count)
                 return cache[i].chunk;
     }
-    constexpr long long kBlock = 60, kItem = 80, kMerge = 30, kEmpty = 10;
+    constexpr long long kBlock = 60, kGlobBlock = 75, kItem = 25, kMerge = 15, kEmpty = 2;
     auto band_blocks = [&](int r0) -> int {
         if (r0 >= L) return 0;
         const int lo = (r0 - w <= 0 ? 0 : r0 - w) / kBN;
@@ -1511,7 +1552,7 @@ int choose_chunk(int B, int H, int L, int w, int sm_count) {
                         const int n = (NKB < s * c + c ? NKB : s * c + c) - s * c;
                         m = n > m ? n : m;
                     }
-                    costs.push_back(m * kBlock + kItem + kMerge);
+                    costs.push_back(m * kGlobBlock + kItem + kMerge);
                 }
         for (int bh = 0; bh < BH; ++bh) {
             costs.push_back(pair_cost(0));
