@@ -64,7 +64,6 @@ constexpr int kStages = 4;        // K/V ring depth
 constexpr int kMinChunk = 4;      // key blocks per global-row split: chosen per
 constexpr int kMaxChunk = 16;     // shape in [kMinChunk, kMaxChunk] on the host
 constexpr int kRing = 4;          // item-id ring depth
-constexpr int kSBuf = 3;          // S buffers in TMEM, rotating over the two tiles
 constexpr int kWarps = 16;
 constexpr int kThreads = kWarps * 32;
 constexpr int kSoftmaxWarp0 = 4;  // warps 4-7: tile A, 8-11: tile B
@@ -73,7 +72,7 @@ constexpr uint32_t kRegsProducer = 88;
 constexpr uint32_t kRegsSoftmax = 152;
 constexpr uint32_t kRegsEpi = 120;
 static_assert(4 * 32 * kRegsProducer + 8 * 32 * kRegsSoftmax + 4 * 32 * kRegsEpi <= 65536, "register split");
-constexpr int kItemConsumers = 1 + 1 + 8 + 4;  // TMA + MMA + softmax + epilogue warps
+constexpr int kItemConsumers = 1 + 2 + 8 + 4;  // TMA + 2 MMA + softmax + epilogue warps
 constexpr uint32_t kTileBytes = kBM * kHD * 2;  // 16 KB
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;
@@ -86,15 +85,17 @@ constexpr uint32_t kOffBias = kOffV + kStages * kTileBytes;   // 8 warps x 128 f
 constexpr uint32_t kOffStats = kOffBias + 8 * kBN * 4;        // [2 tiles][128 rows] (m, l)
 constexpr uint32_t kOffPlans = kOffStats + 2 * kBM * 8;       // kRing plans
 constexpr uint32_t kOffBar = kOffPlans + kRing * 128;
-constexpr uint32_t kNumBars = 2 + 2 + 2 * kStages + 2 * kSBuf + kSBuf + 2 + 2 + 2 + 2 + 2 * kRing + 2;
+constexpr uint32_t kNumBars = 2 + 2 + 2 * kStages + 2 * 7 + 2 * kRing + 2 + 1;
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
 constexpr uint32_t kSmemBytes = kOffMisc + 64 + 1024;  // + alignment slack
 
-// TMEM columns: S buffers [0,128), [128,256), [256,384); O_A [384,448),
-// O_B [448,512).
+// TMEM columns per tile x (base x * 256): S [0,128) fp32, P [128,192)
+// fp16/bf16 pairs, O [192,256) fp32.
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kTmemO = kSBuf * kBN;
-static_assert(kTmemO + 2 * kHD <= kTmemCols, "TMEM budget");
+constexpr uint32_t kTmemTile = 256;
+constexpr uint32_t kTmemP = 128;
+constexpr uint32_t kTmemO = 192;
+static_assert(2 * kTmemTile <= kTmemCols && kTmemO + kHD <= kTmemTile, "TMEM budget");
 
 struct Params {
     int B, H, L, w;
@@ -396,30 +397,6 @@ __device__ __forceinline__ void load_at(const Plan& pl, int q, int& kb, int& nee
 __device__ __forceinline__ int tile_blocks(const Tile& t) { return t.present ? t.glob_hi + (t.hi - t.lo + 1) : 0; }
 // Key block of a tile's j-th block: [0, glob_hi) then lo, lo + 1, ...
 __device__ __forceinline__ int block_kb(const Tile& t, int j) { return j < t.glob_hi ? j : t.lo + (j - t.glob_hi); }
-// An item's S products are computed in the order A0 B0 A1 B1 ... while both
-// tiles have blocks left, then the rest of the longer tile.
-__device__ __forceinline__ void seq_at(int pos, int nA, int nB, int& x, int& j) {
-    const int m = min(nA, nB);
-    if (pos < 2 * m) {
-        x = pos & 1;
-        j = pos >> 1;
-    } else {
-        x = nA > nB ? 0 : 1;
-        j = pos - m;
-    }
-}
-__device__ __forceinline__ int seq_pos(int x, int j, int nA, int nB) {
-    const int m = min(nA, nB);
-    return j < m ? 2 * j + x : m + j;
-}
-// Index, in the item's K/V load order, of tile x's j-th block.  Global pairs
-// load in sequence order; band pairs load [0, e1) then lo_min, lo_min + 1, ...
-__device__ __forceinline__ int load_of(const Plan& pl, int x, int j, int nA, int nB) {
-    if (pl.global) return seq_pos(x, j, nA, nB);
-    const int kb = block_kb(pl.t[x], j);
-    return kb < pl.e1 ? kb : pl.e1 + (kb - pl.lo_min);
-}
-
 template <typename T>
 struct Pack;
 template <>
@@ -585,17 +562,18 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
     uint64_t* q_empty = bars + 2;
     uint64_t* kv_full = bars + 4;
     uint64_t* kv_empty = kv_full + kStages;
-    uint64_t* s_full = kv_empty + kStages;   // [tile][S buffer]: QK of that tile into that buffer done
-    uint64_t* p_full = s_full + 2 * kSBuf;   // [S buffer]: P written by the 4 warps of its tile
-    uint64_t* pv_done = p_full + kSBuf;      // [tile]: one phase per P V product of the tile
-    uint64_t* o_free = pv_done + 2;          // [tile]: the epilogue has read O
-    uint64_t* st_full = o_free + 2;          // [tile]: row (m, l) of an item written
-    uint64_t* st_free = st_full + 2;         // [tile]: ... and read by the epilogue
-    uint64_t* item_full = st_free + 2;       // [kRing]
+    uint64_t* s_full = kv_empty + kStages;  // [tile]: S of the tile's next block computed
+    uint64_t* s_free = s_full + 2;          // [tile]: its 4 softmax warps have read S
+    uint64_t* p_full = s_free + 2;          // [tile]: ... and written P
+    uint64_t* pv_done = p_full + 2;         // [tile]: one phase per P V product of the tile
+    uint64_t* o_free = pv_done + 2;         // [tile]: the epilogue has read O
+    uint64_t* st_full = o_free + 2;         // [tile]: row (m, l) of an item written
+    uint64_t* st_free = st_full + 2;        // [tile]: ... and read by the epilogue
+    uint64_t* item_full = st_free + 2;      // [kRing]
     uint64_t* item_empty = item_full + kRing;
-    uint64_t* drain = item_empty + kRing;
-    uint64_t* tma_done = drain + 1;  // the TMA warp finished issuing an item's loads
-    static_assert(2 + 2 + 2 * kStages + 2 * kSBuf + kSBuf + 2 + 2 + 2 + 2 + 2 * kRing + 2 == kNumBars, "barriers");
+    uint64_t* drain = item_empty + kRing;   // [tile]: wind-down of an MMA warp
+    uint64_t* tma_done = drain + 2;         // the TMA warp finished issuing an item's loads
+    static_assert(2 + 2 + 2 * kStages + 2 * 7 + 2 * kRing + 2 + 1 == kNumBars, "barriers");
     Plan* plans = reinterpret_cast<Plan*>(smem + kOffPlans);
     static_assert(sizeof(Plan) <= 128, "plan slot");
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
@@ -614,26 +592,24 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
     if (threadIdx.x == 0) {
         for (int i = 0; i < 2; ++i) {
             mbar_init(&q_full[i], 1);
-            mbar_init(&q_empty[i], 1);
+            mbar_init(&q_empty[i], 2);  // one arrival per MMA warp
+            mbar_init(&s_full[i], 1);
+            mbar_init(&s_free[i], 4);
+            mbar_init(&p_full[i], 4);
             mbar_init(&pv_done[i], 1);
             mbar_init(&o_free[i], 4);
             mbar_init(&st_full[i], 4);
             mbar_init(&st_free[i], 4);
-        }
-        for (int b = 0; b < kSBuf; ++b) {
-            mbar_init(&s_full[b], 1);
-            mbar_init(&s_full[kSBuf + b], 1);
-            mbar_init(&p_full[b], 4);
+            mbar_init(&drain[i], 1);
         }
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&kv_full[s], 1);
-            mbar_init(&kv_empty[s], 1);
+            mbar_init(&kv_empty[s], 2);  // one arrival per MMA warp
         }
         for (int s = 0; s < kRing; ++s) {
             mbar_init(&item_full[s], 1);
             mbar_init(&item_empty[s], kItemConsumers);
         }
-        mbar_init(drain, 1);
         mbar_init(tma_done, 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -771,14 +747,16 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
             }
             if (id < 0) break;
         }
-    } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer
-        // One sequence of S products over all items: product n goes to S
-        // buffer n % 3, and is issued right after the P V of product n - 3
-        // (which read that buffer; the tensor pipe runs in issue order).  So
-        // a tile's next S is computed while its softmax works on the current
-        // one, and P V of a block runs while the other tile's softmax runs.
-        // Lane 0 issues; its bookkeeping lives in packed registers.
+    } else {
+        // ------------------------------------------------------------ MMA issuers
+        // Warp 1 issues the tensor-core work of tile A, warp 3 that of tile B.
+        // Per block j of its tile: S_j = Q K_j^T into the tile's S columns as
+        // soon as the softmax warps have read S_(j-1), then O += P_(j-1) V_(j-1)
+        // once they have written P_(j-1).  So a tile's next S is computed while
+        // its softmax still works on the current block, and neither tile
+        // waits on the other.  Every K/V stage is released by both warps: by a
+        // commit after its P V where the tile used it, else at once.
+        const int x = warp == 1 ? 0 : 1;
         constexpr uint32_t idesc_qk = idesc_f16(Pack<T>::fmt, kBM, kBN, 0, 0);
         constexpr uint32_t idesc_pv = idesc_f16(Pack<T>::fmt, kBM, kHD, 0, 1);
         // Descriptors of the first Q / K / V tile; the others are reached by
@@ -787,167 +765,123 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
         const uint64_t dk0 = desc_sw128(smem_u32(smem + kOffK));
         const uint64_t dv0 = desc_sw128(smem_u32(smem + kOffV), 0);
         constexpr uint32_t kTileStep = kTileBytes >> 4;
+        const uint32_t t_s = tmem + x * kTmemTile, t_p = t_s + kTmemP, t_o = t_s + kTmemO;
         TDECL;
         uint32_t kv_cnt = 0, item_cnt = 0;
-        uint32_t n_qk = 0, n_pv = 0;   // S products issued / P V products issued
-        uint32_t b_qk = 0, b_pv = 0;   // their S buffers (n % 3)
-        uint32_t pf_par = 0;           // bit b: phase of the next p_full[b] wait
-        uint32_t of_par = 0;           // bit x: phase of the next o_free[x] wait, flipped
-        uint32_t pend = 0;             // per S buffer, 4 bits: tile | stage << 1 | first << 3
-        uint32_t refc = 0;             // per K/V stage, 2 bits: P V products still to read it
-        // O_X (+)= P V for the oldest pending product; releases the K/V stage
-        // when its last user is done.
-        auto issue_pv = [&]() -> bool {
-            const uint32_t b = b_pv;
-            const uint32_t e = (pend >> (4 * b)) & 15u;
-            const uint32_t x = e & 1u, st = (e >> 1) & 3u, first = e >> 3;
+        uint32_t s_use = 0;  // S products issued (s_free phases)
+        uint32_t p_use = 0;  // P blocks consumed (p_full phases)
+        uint32_t o_use = 0;  // items with blocks (o_free phases)
+        // O (+)= P V for the tile's block j read from stage st; the stage is
+        // released when the product is done.
+        auto issue_pv = [&](int j, uint32_t st) -> bool {
             bool w_ok;
-            TIMED(3, w_ok = mbar_wait(&p_full[b], (pf_par >> b) & 1u, abort_flag));
+            TIMED(3, w_ok = mbar_wait(&p_full[x], p_use & 1u, abort_flag));
             if (!w_ok) return false;
-            pf_par ^= 1u << b;
+            ++p_use;
             TCOUNT(5);
-            if (first) {
-                TIMED(4, w_ok = mbar_wait(&o_free[x], ((of_par >> x) & 1u) ^ 1u, abort_flag));
+            if (j == 0) {
+                TIMED(4, w_ok = mbar_wait(&o_free[x], (o_use & 1u) ^ 1u, abort_flag));
                 if (!w_ok) return false;
-                of_par ^= 1u << x;
+                ++o_use;
             }
             tc_fence_after();
             const uint64_t dv = dv0 + st * kTileStep;
-            const uint32_t d_tm = tmem + kTmemO + x * kHD, a_tm = tmem + b * kBN;
 #if LF_TRACE
             const long long tp0_ = clock64();
 #endif
 #pragma unroll
             for (int kk = 0; kk < kBN / 16; ++kk)
-                mma_f16_ts(d_tm, a_tm + kk * 8, dv + kk * (2048 >> 4), idesc_pv, (first && kk == 0) ? 0u : 1u);
-#if LF_TRACE
-            const long long tp1_ = clock64();
-            tacc[8] += tp1_ - tp0_;
-#endif
+                mma_f16_ts(t_o, t_p + kk * 8, dv + kk * (2048 >> 4), idesc_pv, (j == 0 && kk == 0) ? 0u : 1u);
             tc_commit(&pv_done[x]);
-            refc -= 1u << (2 * st);
-            if (((refc >> (2 * st)) & 3u) == 0) tc_commit(&kv_empty[st]);
+            tc_commit(&kv_empty[st]);
 #if LF_TRACE
-            tacc[9] += clock64() - tp1_;
+            tacc[8] += clock64() - tp0_;
 #endif
-            ++n_pv;
-            b_pv = b_pv == kSBuf - 1 ? 0 : b_pv + 1;
             return true;
-        };
-        // Waits for `bar` while issuing each pending P V as soon as its P is
-        // ready: a P V must never wait behind a plan, a Q tile or a K/V load,
-        // since the epilogue (which frees plan slots) and the softmax warps
-        // wait for it.
-        auto wait_issuing = [&](uint64_t* bar, uint32_t parity) -> bool {
-            if (mbar_test(bar, parity)) return true;
-            const uint64_t t0 = globaltimer();
-            for (uint32_t it = 1;; ++it) {
-                if (n_pv < n_qk && mbar_test(&p_full[b_pv], (pf_par >> b_pv) & 1u)) {
-                    if (!issue_pv()) return false;
-                } else {
-                    __nanosleep(20);
-                }
-                if (mbar_test(bar, parity)) return true;
-                if ((it & 63u) == 0) {
-                    if (*abort_flag) return false;
-                    if (globaltimer() - t0 > 2000000000ull) {
-                        *abort_flag = 1;
-                        return false;
-                    }
-                }
-            }
         };
         bool ok = true;
         for (uint32_t k = 0; ok; ++k) {
             Plan pl;
-            {
-                const uint32_t slot = k % kRing;
-                if (lane == 0) TIMED(0, ok = wait_issuing(&item_full[slot], (k / kRing) & 1));
-                ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-                if (!ok) break;
-                __syncwarp();
-                pl = plans[slot];
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&item_empty[slot]);
-            }
+            TIMED(0, ok = next_plan(k, pl));
+            if (!ok) break;
             if (pl.id < 0) break;
             if (pl.nloads == 0) continue;
             if (lane == 0) {
                 const uint32_t qb = item_cnt & 1;
-                TIMED(1, ok = wait_issuing(&q_full[qb], (item_cnt >> 1) & 1));
-                // The item as scalars (no indexed accesses in the loop).
                 const int nA = tile_blocks(pl.t[0]), nB = tile_blocks(pl.t[1]);
-                const int m = min(nA, nB), xl = nA > nB ? 0 : 1, ntot = nA + nB;
+                const int nx = x ? nB : nA;
                 const int glob = pl.global, e1 = pl.e1, lo_min = pl.lo_min;
-                const int ghA = pl.t[0].glob_hi, loA = pl.t[0].lo, hiA = pl.t[0].hi, prA = pl.t[0].present;
-                const int ghB = pl.t[1].glob_hi, loB = pl.t[1].lo, hiB = pl.t[1].hi, prB = pl.t[1].present;
-                const uint64_t dq = dq0 + qb * 2 * kTileStep;
+                const int gh = pl.t[x].glob_hi, lo = pl.t[x].lo, hi = pl.t[x].hi;
+                const int m = min(nA, nB);
+                // load index of this tile's block j
+                auto load_idx = [&](int j) -> int {
+                    if (glob) return j < m ? 2 * j + x : m + j;
+                    const int kb = j < gh ? j : lo + (j - gh);
+                    return kb < e1 ? kb : e1 + (kb - lo_min);
+                };
+                // is load q one of this tile's blocks?
+                auto mine = [&](int q) -> bool {
+                    if (nx == 0) return false;
+                    if (glob) return q < 2 * m ? (q & 1) == x : nx > m;
+                    const int kb = q < e1 ? q : lo_min + (q - e1);
+                    return kb < gh || (kb >= lo && kb <= hi);
+                };
                 int q_ready = -1;
-                for (int pos = 0; pos < ntot && ok; ++pos) {
-                    const bool inter = pos < 2 * m;
-                    const uint32_t x = inter ? (uint32_t)(pos & 1) : (uint32_t)xl;
-                    const int j = inter ? pos >> 1 : pos - m;
-                    if (n_qk - n_pv == (uint32_t)kSBuf) {  // free the buffer of product n_qk
-                        ok = issue_pv();
-                        if (!ok) break;
-                    }
-                    int q;
-                    if (glob) {
-                        q = pos;
-                    } else {
-                        const int gh = x ? ghB : ghA, lo = x ? loB : loA;
-                        const int kb = j < gh ? j : lo + (j - gh);
-                        q = kb < e1 ? kb : e1 + (kb - lo_min);
-                    }
-                    while (q_ready < q && ok) {
+                // wait for loads up to q; loads this tile does not use are released at once
+                auto take_loads = [&](int q) -> bool {
+                    while (q_ready < q) {
                         ++q_ready;
                         const uint32_t c = kv_cnt + q_ready, st = c % kStages;
-                        TIMED(2, ok = wait_issuing(&kv_full[st], (c / kStages) & 1));
-                        uint32_t users = 1;
-                        if (!glob) {
-                            const int kb = q_ready < e1 ? q_ready : lo_min + (q_ready - e1);
-                            users = (uint32_t)(prA && (kb < ghA || (kb >= loA && kb <= hiA))) +
-                                    (uint32_t)(prB && (kb < ghB || (kb >= loB && kb <= hiB)));
-                        }
-                        refc = (refc & ~(3u << (2 * st))) | (users << (2 * st));
-                        if (ok && users == 0) tc_commit(&kv_empty[st]);
+                        bool w_ok;
+                        TIMED(2, w_ok = mbar_wait(&kv_full[st], (c / kStages) & 1, abort_flag));
+                        if (!w_ok) return false;
+                        if (!mine(q_ready)) mbar_arrive(&kv_empty[st]);
                     }
+                    return true;
+                };
+                if (nx > 0) TIMED(1, ok = mbar_wait(&q_full[qb], (item_cnt >> 1) & 1, abort_flag));
+                const uint64_t dqx = dq0 + (qb * 2 + x) * kTileStep;
+                uint32_t st_prev = 0;
+                for (int j = 0; j < nx && ok; ++j) {
+                    const int q = load_idx(j);
+                    ok = take_loads(q);
                     if (!ok) break;
+                    // the softmax warps have read the previous S
+                    TIMED(6, ok = mbar_wait(&s_free[x], (s_use & 1u) ^ 1u, abort_flag));
+                    if (!ok) break;
+                    ++s_use;
                     tc_fence_after();
-                    const uint32_t b = b_qk, st = (kv_cnt + q) % kStages;
-                    const uint64_t dqx = dq + x * kTileStep, dk = dk0 + st * kTileStep;
+                    const uint32_t st = (kv_cnt + q) % kStages;
+                    const uint64_t dk = dk0 + st * kTileStep;
 #if LF_TRACE
                     const long long tq0_ = clock64();
 #endif
 #pragma unroll
                     for (int kk = 0; kk < kHD / 16; ++kk)
-                        mma_f16_ss(tmem + b * kBN, dqx + kk * 2, dk + kk * 2, idesc_qk, kk > 0);
+                        mma_f16_ss(t_s, dqx + kk * 2, dk + kk * 2, idesc_qk, kk > 0);
+                    tc_commit(&s_full[x]);
 #if LF_TRACE
-                    const long long tq1_ = clock64();
-                    tacc[7] += tq1_ - tq0_;
+                    tacc[7] += clock64() - tq0_;
 #endif
-                    tc_commit(&s_full[x * kSBuf + b]);
-#if LF_TRACE
-                    tacc[10] += clock64() - tq1_;
-#endif
-                    TCOUNT(6);
-                    pend = (pend & ~(15u << (4 * b))) | ((x | (st << 1) | ((j == 0 ? 1u : 0u) << 3)) << (4 * b));
-                    ++n_qk;
-                    b_qk = b_qk == kSBuf - 1 ? 0 : b_qk + 1;
+                    if (j > 0) ok = issue_pv(j - 1, st_prev);
+                    st_prev = st;
                 }
-                if (ok) tc_commit(&q_empty[qb]);
+                if (ok && nx > 0) ok = issue_pv(nx - 1, st_prev);
+                if (ok) ok = take_loads(pl.nloads - 1);
+                if (ok) {
+                    if (nx > 0) tc_commit(&q_empty[qb]);
+                    else mbar_arrive(&q_empty[qb]);
+                }
             }
             ++item_cnt;
             kv_cnt += pl.nloads;
             ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
         }
-        if (lane == 0)
-            while (ok && n_pv < n_qk) ok = issue_pv();
-        if (lane == 0) TDUMP(1);
+        if (lane == 0) TDUMP(1 + 2 * x);
         if (lane == 0 && !ok) {  // wind-down: wait for the MMAs already issued
-            tc_commit(drain);
+            tc_commit(&drain[x]);
             volatile int never = 0;
-            mbar_wait(drain, 0, &never, 200000000ull);
+            mbar_wait(&drain[x], 0, &never, 200000000ull);
         }
     }
     } else if (warp < kEpiWarp0) {
@@ -957,12 +891,10 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
         const int sp = warp & 3;           // TMEM sub-partition (rows sp*32 .. +31)
         const int r = sp * 32 + lane;      // query row within the tile
         const uint32_t lane_off = (uint32_t)(sp * 32) << 16;
-        const uint32_t tO = tmem + lane_off + kTmemO + x * kHD;
+        const uint32_t tS = tmem + lane_off + x * kTmemTile, tP = tS + kTmemP, tO = tS + kTmemO;
         float* bias_w = reinterpret_cast<float*>(smem + kOffBias) + (warp - kSoftmaxWarp0) * kBN;
         float2* stats = reinterpret_cast<float2*>(smem + kOffStats) + x * kBM;
-        uint32_t nqk = 0;     // S products of earlier items (both tiles)
         uint32_t npv = 0;     // this tile's blocks in earlier items (its P V products)
-        uint32_t s_par = 0;   // bit b: phase of this tile's next use of S buffer b
         uint32_t st_cnt = 0;  // items in which this tile had blocks
         TDECL;
         bool ok = true;
@@ -974,10 +906,7 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
             if (pl.nloads == 0) continue;
             const int nA = tile_blocks(pl.t[0]), nB = tile_blocks(pl.t[1]);
             const int nblk = x == 0 ? nA : nB;
-            if (nblk == 0) {
-                nqk += nA + nB;
-                continue;
-            }
+            if (nblk == 0) continue;
             const int g = pl.g;
             const Tile& me = pl.t[x];
             const float* lm = p.local_mask + (size_t)pl.b * p.L;
@@ -1011,8 +940,6 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
                 const bool first = n == 0;
                 const int kb = n < blk_gh ? n : blk_lo + (n - blk_gh);
                 const int c0 = kb * kBN;
-                const uint32_t sb = (nqk + (uint32_t)seq_pos(x, n, nA, nB)) % kSBuf;
-                const uint32_t tS = tmem + lane_off + sb * kBN;
                 // Padding bias of the block's keys (keys >= L are masked instead).
                 bool has_pad = false;
                 if (warp_active) {
@@ -1052,21 +979,48 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
                     }
                     states |= (uint32_t)s << (2 * ch);
                 }
-                if (lane == 0) TRACE(2 + warp - kSoftmaxWarp0, 32, pl.id, n, sb);
+                if (lane == 0) TRACE(2 + warp - kSoftmaxWarp0, 32, pl.id, n, 0);
                 // every lane waits; the result is made warp-uniform so that an
                 // abort never splits the warp before a .sync.aligned instruction
 #if LF_TRACE
                 const long long tsw_ = clock64();
                 tacc[10] += tsw_ - tpro_;
 #endif
-                TIMED(1, ok = __all_sync(0xffffffffu, mbar_wait(&s_full[x * kSBuf + sb], (s_par >> sb) & 1u, abort_flag)));
+                TIMED(1, ok = __all_sync(0xffffffffu, mbar_wait(&s_full[x], (npv + n) & 1u, abort_flag)));
 #if LF_TRACE
                 const long long tb0_ = clock64();
                 if (first) tacc[9] += tb0_ - tsw_;
 #endif
-                s_par ^= 1u << sb;
                 if (!ok) break;
                 tc_fence_after();
+                // P of the previous block is read by its P V product until
+                // that completes: waited once, before this block's first P
+                // write or O access.  (It also keeps every later wait on
+                // pv_done within one phase of the barrier.)
+                bool pv_ok = npv + n == 0;
+                auto ensure_pv = [&]() {
+                    if (!pv_ok) {
+                        bool w_ok;
+                        TIMED(3, w_ok = __all_sync(0xffffffffu, mbar_wait(&pv_done[x], (npv + n - 1) & 1u, abort_flag)));
+                        if (!w_ok) ok = false;
+                        tc_fence_after();
+                        pv_ok = true;
+                    }
+                };
+                // S is handed back to the MMA warp once its last chunk this warp
+                // reads has landed in registers (or at once when it reads none).
+                int last_ld = -1;
+                if (warp_active) {
+#pragma unroll
+                    for (int ch = 0; ch < 4; ++ch)
+                        if (((states >> (2 * ch)) & 3u) != kSkip) last_ld = ch;
+                }
+                auto release_s = [&]() {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&s_free[x]);
+                };
+                if (last_ld < 0) release_s();
                 if (warp_active) {
                     auto state_of = [&](int ch) -> int { return (int)((states >> (2 * ch)) & 3u); };
                     const int d0 = i - c0;
@@ -1128,6 +1082,7 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
                             tmem_ld32f(tS + ch * 32, r);
                             tmem_ld_wait();
                             regs_ready<32>(r);
+                            if (ch == last_ld) release_s();
                             fix_chunk(ch, r);
                             float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
@@ -1150,7 +1105,7 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
                                     sm2[1] = make_float2(sm2[1].x * factor, sm2[1].y * factor);
                                     for (int pc = 0; pc < ch; ++pc) {  // this block's earlier P
                                         uint32_t pb16[16];
-                                        tmem_ld16(tS + pc * 16, pb16);
+                                        tmem_ld16(tP + pc * 16, pb16);
                                         tmem_ld_wait();
                                         regs_ready<16>(pb16);
 #pragma unroll
@@ -1158,19 +1113,15 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
                                             const float2 v = Pack<T>::unpack(pb16[c]);
                                             pb16[c] = Pack<T>::two(v.x * factor, v.y * factor);
                                         }
-                                        tmem_st16(tS + pc * 16, pb16);
+                                        tmem_st16(tP + pc * 16, pb16);
                                     }
                                     if (!first) {
                                         // O holds the tile's blocks so far once the
                                         // previous block's P V has completed
-                                        bool w_ok;
-                                        TIMED(7, w_ok = __all_sync(
-                                            0xffffffffu, mbar_wait(&pv_done[x], (npv + n - 1) & 1u, abort_flag)));
+                                        ensure_pv();
                                         TCOUNT(8);
-                                        if (!w_ok) ok = false;
-                                        tc_fence_after();
 #pragma unroll
-                                        for (int c0o = 0; c0o < kHD && w_ok; c0o += 16) {
+                                        for (int c0o = 0; c0o < kHD && ok; c0o += 16) {
                                             uint32_t ob[16];
                                             tmem_ld16(tO + c0o, ob);
                                             tmem_ld_wait();
@@ -1187,23 +1138,20 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
                             const float m_use = m_used == -INFINITY ? 0.0f : m_used;
                             exp_chunk(r, pk, make_float2(-m_use, -m_use));
                         }
-                        tmem_st16(tS + ch * 16, pk);
+                        ensure_pv();
+                        tmem_st16(tP + ch * 16, pk);
                     }
                     l_run += (sm2[0].x + sm2[0].y) + (sm2[1].x + sm2[1].y);
                     tmem_st_wait();
                 }
-                // The previous block's P V has completed before this block's P
-                // is handed over: every later wait on pv_done is then at most
-                // one phase behind the barrier.
 #if LF_TRACE
                 tacc[2] += clock64() - tb0_;
                 TCOUNT(5);
 #endif
-                if (npv + n > 0)
-                    TIMED(3, ok = ok && __all_sync(0xffffffffu, mbar_wait(&pv_done[x], (npv + n - 1) & 1u, abort_flag)));
+                ensure_pv();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&p_full[sb]);
+                if (lane == 0) mbar_arrive(&p_full[x]);
             }
             if (!ok) break;
             // Row (m, l) to the epilogue warps.
@@ -1214,7 +1162,6 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
             __syncwarp();
             if (lane == 0) mbar_arrive(&st_full[x]);
             ++st_cnt;
-            nqk += nA + nB;
             npv += nblk;
         }
         if (lane == 0) TDUMP(2 + warp - kSoftmaxWarp0);
@@ -1289,7 +1236,7 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
 #endif
                 float o[kHD];
                 {
-                    const uint32_t tO = tmem + lane_off + kTmemO + x * kHD;
+                    const uint32_t tO = tmem + lane_off + x * kTmemTile + kTmemO;
                     tmem_ld32f(tO, *reinterpret_cast<float(*)[32]>(&o[0]));
                     tmem_ld32f(tO + 32, *reinterpret_cast<float(*)[32]>(&o[32]));
                     tmem_ld_wait();
