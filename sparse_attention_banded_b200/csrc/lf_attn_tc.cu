@@ -921,18 +921,31 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
             const bool warp_active = __any_sync(0xffffffffu, row_kept);
 
             float m_used = -INFINITY, l_run = 0.0f;
-            // local_mask of the next block's keys, loaded one block ahead so
-            // that the load latency is off the critical path
-            float mv_next[4] = {1.0f, 1.0f, 1.0f, 1.0f};
-            auto load_mv = [&](int n2) {
-                const int c2 = (n2 < blk_gh ? n2 : blk_lo + (n2 - blk_gh)) * kBN;
+            // Which of the tile's key blocks hold padded keys (bit j for block
+            // j < 32; later blocks are always treated as padded): worked out
+            // once per item, eight blocks' loads in flight at a time, while
+            // the first S of the item is still being computed.
+            uint32_t padbits = 0;
+            if (warp_active) {
+                for (int j0 = 0; j0 < nblk && j0 < 32; j0 += 8) {
+                    float v[8][4];
 #pragma unroll
-                for (int t = 0; t < 4; ++t) {
-                    const int key = c2 + t * 32 + lane;
-                    mv_next[t] = key < p.L ? lm[key] : 1.0f;
+                    for (int u = 0; u < 8; ++u) {
+                        const int j = j0 + u;
+                        const int c2 = (j < blk_gh ? j : blk_lo + (j - blk_gh)) * kBN;
+#pragma unroll
+                        for (int t = 0; t < 4; ++t) {
+                            const int key = c2 + t * 32 + lane;
+                            v[u][t] = (j < nblk && key < p.L) ? lm[key] : 1.0f;
+                        }
+                    }
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        const bool pad = v[u][0] != 1.0f || v[u][1] != 1.0f || v[u][2] != 1.0f || v[u][3] != 1.0f;
+                        if (__any_sync(0xffffffffu, pad)) padbits |= 1u << (j0 + u);
+                    }
                 }
-            };
-            if (warp_active) load_mv(0);
+            }
             for (int n = 0; n < nblk && ok; ++n) {
 #if LF_TRACE
                 const long long tpro_ = clock64();
@@ -941,17 +954,13 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
                 const int kb = n < blk_gh ? n : blk_lo + (n - blk_gh);
                 const int c0 = kb * kBN;
                 // Padding bias of the block's keys (keys >= L are masked instead).
-                bool has_pad = false;
-                if (warp_active) {
-                    float mv[4];
+                const bool has_pad = warp_active && (n >= 32 || ((padbits >> n) & 1u));
+                if (has_pad) {
 #pragma unroll
-                    for (int t = 0; t < 4; ++t) mv[t] = mv_next[t];
-                    if (n + 1 < nblk) load_mv(n + 1);
-                    const bool pad = mv[0] != 1.0f || mv[1] != 1.0f || mv[2] != 1.0f || mv[3] != 1.0f;
-                    has_pad = __any_sync(0xffffffffu, pad);
-                    if (has_pad) {
-#pragma unroll
-                        for (int t = 0; t < 4; ++t) bias_w[t * 32 + lane] = fmaf(mv[t], 10000.0f, -10000.0f) * p.inv_scale;
+                    for (int t = 0; t < 4; ++t) {
+                        const int key = c0 + t * 32 + lane;
+                        const float mv = key < p.L ? lm[key] : 1.0f;
+                        bias_w[t * 32 + lane] = fmaf(mv, 10000.0f, -10000.0f) * p.inv_scale;
                     }
                     __syncwarp();
                 }
