@@ -106,9 +106,8 @@ struct Params {
     int NSP;     // split pairs per global row tile
     int NTP;     // tile pairs per head
     int chunk;   // key blocks per global-row split
-    int n_inner; // band pairs away from the sequence ends (first in the order)
-    int n_glob;  // global pair items (after the interior band pairs, before
-                 // the band pairs at the ends of the sequences)
+    int n_inner; // band pairs away from the sequence ends (after the global pairs)
+    int n_glob;  // global pair items (first in the order)
     int n_items;
     float scale_log2;  // scale * log2(e)
     float inv_scale;   // 1 / scale: the padding bias in raw score units
@@ -272,14 +271,15 @@ __device__ void band_rows2(const Params& p, int b, const int (&r0)[2], int& cach
 __device__ Plan make_plan(const Params& p, int id, int& cached_b, int& g) {
     Plan pl;
     pl.id = id;
-    // Item order: interior band pairs (the most key blocks), then the global
-    // pairs (the epilogue warps merge their splits while the softmax warps
-    // already run the next item), then the band pairs at both ends of each
-    // sequence, which are short and end the launch.
+    // Item order: the global pairs first (the longest items; the epilogue
+    // warps merge their splits while the softmax warps already run band
+    // work, so no merge is left at the end of the launch), then the interior
+    // band pairs, then the band pairs at both ends of each sequence, which
+    // are short and end the launch.
     const int inner_per = p.NTP > 2 ? p.NTP - 2 : 0;
     const int edge_per = p.NTP < 2 ? p.NTP : 2;
-    if (id >= p.n_inner && id < p.n_inner + p.n_glob) {
-        const int id2 = id - p.n_inner;
+    if (id < p.n_glob) {
+        const int id2 = id;
         pl.global = 1;
         const int sp = id2 % p.NSP;
         const int r = id2 / p.NSP;
@@ -290,9 +290,9 @@ __device__ Plan make_plan(const Params& p, int id, int& cached_b, int& g) {
         pl.t[0].r0 = pl.t[1].r0 = pl.rt * kBM;  // set before any early return: every role reads it
     } else {
         int tp;
-        if (id < p.n_inner) {
-            tp = 1 + id % inner_per;
-            pl.bh = id / inner_per;
+        if (id < p.n_glob + p.n_inner) {
+            tp = 1 + (id - p.n_glob) % inner_per;
+            pl.bh = (id - p.n_glob) / inner_per;
         } else {
             const int e = id - p.n_inner - p.n_glob;
             tp = (e % edge_per == 0) ? 0 : p.NTP - 1;
@@ -1189,11 +1189,17 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
         uint32_t npv[2] = {0, 0}, st_cnt[2] = {0, 0};
         TDECL;
         bool ok = true;
+#if LF_TRACE
+        const unsigned long long tent_ = globaltimer();
+#endif
         for (uint32_t k = 0; ok; ++k) {
             Plan pl;
             TIMED(0, ok = next_plan(k, pl));
             if (!ok) break;
             if (pl.id < 0) break;
+#if LF_TRACE
+            if (k < 3) tacc[11 + k] = (long long)(globaltimer() - tent_);
+#endif
             const int g = pl.g;
             const float* lm = p.local_mask + (size_t)pl.b * p.L;
             for (int x = 0; x < 2 && ok; ++x) {
@@ -1365,6 +1371,9 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
                 }
             }
         }
+#if LF_TRACE
+        tacc[14] = (long long)(globaltimer() - tent_);
+#endif
         if (lane == 0) TDUMP(10 + sp);
     }
 
@@ -1446,7 +1455,7 @@ bool make_map(CUtensorMap* m, const void* base, int BH, int L) {
 // Global-row split size.  Items are taken from a counter by the CTAs as they
 // free up, so the kernel ends when the last CTA finishes its last item; with
 // only a few items per CTA the split size decides how evenly the work packs.
-// The host replays that list schedule (inner band pairs, global pairs, edge
+// The host replays that list schedule (global pairs, inner band pairs, edge
 // pairs) for each candidate size with a cost model of the kernel and keeps
 // the size with the earliest finish.  Relative costs, from per-role cycle
 // counts of the kernel on B200: a band key block 60, a global key block 75
@@ -1495,8 +1504,6 @@ int choose_chunk(int B, int H, int L, int w, int sm_count) {
         const int NS = (NKB + c - 1) / c, NSP = (NS + 1) / 2;
         costs.clear();
         for (int bh = 0; bh < BH; ++bh)
-            for (int tp = 1; tp + 1 < NTP; ++tp) costs.push_back(pair_cost(tp));
-        for (int bh = 0; bh < BH; ++bh)
             for (int rt = 0; rt < RT; ++rt)
                 for (int sp = 0; sp < NSP; ++sp) {
                     if (rt > 0) {
@@ -1510,6 +1517,8 @@ int choose_chunk(int B, int H, int L, int w, int sm_count) {
                     }
                     costs.push_back(m * kGlobBlock + kItem + kMerge);
                 }
+        for (int bh = 0; bh < BH; ++bh)
+            for (int tp = 1; tp + 1 < NTP; ++tp) costs.push_back(pair_cost(tp));
         for (int bh = 0; bh < BH; ++bh) {
             costs.push_back(pair_cost(0));
             if (NTP > 1) costs.push_back(pair_cost(NTP - 1));
