@@ -6,15 +6,16 @@
 // masked-softmax kernel and a transpose kernel.  Here it is ONE persistent
 // kernel per call.
 //
-// Work items, taken from a global atomic counter longest first: band pairs
-// away from the sequence ends, then global pairs (their split merges overlap
-// the band work that follows), then the band pairs at the sequence ends:
+// Work items: CTA c takes item c first, later ones come from a global atomic
+// counter.  Global pairs come first (the longest items; their split merges
+// then overlap the band work that follows), then the band pairs away from
+// the sequence ends, then the band pairs at the sequence ends:
 //   global pair (b, h, row tile rt, splits 2s and 2s+1): rows i < g_b attend
 //       to every key through qg/kg/vg.  Keys are cut into chunks of `chunk`
 //       128-key blocks (picked per shape on the host so that the items pack
 //       evenly onto the SMs); each split leaves (m, l, O) partials in
-//       scratch and the warp that finishes the last split of its 32 rows
-//       merges them (log-sum-exp) and writes the rows.
+//       scratch and the epilogue warp that finishes the last split of its 32
+//       rows merges them (log-sum-exp) and writes the rows.
 //   band pair (b, h, tiles 2p and 2p+1 of 128 query rows): each tile visits
 //       the 128-key blocks that meet its rows' windows |i - j| <= w and the
 //       blocks of global keys 0..g_b-1 seen outside the window, with the mask
@@ -22,23 +23,22 @@
 //       window counts once.  The two tiles share every K/V block they both
 //       need (loaded once).
 //
-// Roles (384 threads = 3 warpgroups): warp 2 fetches items and publishes
-// their plans through a ring; warp 0 issues TMA loads (Q of both tiles, K/V
-// blocks into a kStages ring); warp 1 issues tcgen05.mma; warp 3 only hands
-// its registers over; warpgroups 1 and 2
-// are the softmax warpgroups of tile A and tile B (one thread per query row).
-// Registers are rebalanced with setmaxnreg: launched at 168 per thread,
-// warpgroup 0 drops to 96 and the softmax warpgroups rise to 200
-// (4*32*96 + 8*32*200 = 63488 <= 384*168 = 64512).  Per tile X and key block:
-//   S_X = Q_X K^T           (TMEM, fp32)
+// Roles (512 threads = 4 warpgroups): warp 0 issues TMA loads (Q of both
+// tiles, K/V blocks into a kStages ring); warp 2 fetches items and publishes
+// their plans through a ring; warps 1 and 3 issue the tcgen05.mma work of
+// tile A and tile B; warpgroups 1 and 2 are the softmax warps of tiles A and
+// B (one thread per query row); warpgroup 3 is the epilogue of both tiles.
+// Registers are rebalanced with setmaxnreg from 128 per thread to 88, 152
+// and 120.  Each tile owns 256 TMEM columns: S (fp32), P (fp16/bf16 pairs)
+// and O (fp32).  Per tile X and key block j:
+//   S_X = Q_X K_j^T            (issued once the softmax has read S of j - 1)
 //   softmax warps: read S_X, scale, padding bias, mask, row max; rescale the
 //   TMEM accumulator O_X only when the running max grows by more than 8 (in
-//   log2 units, so P <= 2^8); P = exp2(x - m) written back into TMEM over S_X
-//   as fp16/bf16 pairs
-//   O_X += P_X V            (tcgen05.mma with A from TMEM)
-// The MMA warp alternates the two tiles, so one tile's MMAs run while the
-// other tile's softmax runs.  All waits are bounded; on expiry the CTA
-// records LF_ERR_DEVICE_TIMEOUT and winds down.
+//   log2 units, so P <= 2^8); write P = exp2(x - m) as fp16/bf16 pairs
+//   O_X += P_X V_j             (tcgen05.mma with A from TMEM)
+// so a tile's next S runs while its softmax works on the current block, and
+// the two tiles never wait on each other.  All waits are bounded; on expiry
+// the CTA records LF_ERR_DEVICE_TIMEOUT and winds down.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -119,11 +119,13 @@ struct Params {
     int* counters;   // [B*H*RT][4]: per 32-row group of a global row tile
     int* sched;      // [0] next item, [1] finished CTAs
     int* status;
-    int* trace;      // diagnostic builds only: [CTA][16 roles][state, item, a, b]
+    int* trace;      // diagnostic builds only: [CTA][16 roles][4] wait sites, then [CTA][16 roles][16] cycle counts
 };
 
-// Diagnostic builds (-DLF_TRACE=1) record, per CTA and role, the wait site
-// each role is at into host-mapped memory, readable while the kernel runs.
+// Diagnostic builds (-DLF_TRACE=1) record per CTA and role the cycles spent
+// in each wait and phase (written at the end of the role); with
+// -DLF_TRACE_STATES=1 they also record the wait site each role is at, into
+// host-mapped memory readable while the kernel runs (for locating a hang).
 #ifndef LF_TRACE
 #define LF_TRACE 0
 #endif
