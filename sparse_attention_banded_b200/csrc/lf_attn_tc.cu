@@ -1459,9 +1459,10 @@ bool make_map(CUtensorMap* m, const void* base, int BH, int L) {
 // only a few items per CTA the split size decides how evenly the work packs.
 // The host replays that list schedule (global pairs, inner band pairs, edge
 // pairs) for each candidate size with a cost model of the kernel and keeps
-// the size with the earliest finish.  Relative costs, from per-role cycle
-// counts of the kernel on B200: a band key block 60, a global key block 75
-// (every chunk of it is computed), an item 25 (its first S and the
+// the size with the earliest finish.  Relative costs, fitted to split-size
+// sweeps of the kernel on B200 (workloads of 4096 and 16384 tokens): a key
+// block 60 (band or global: a global block has no skipped chunks, but only
+// the warps holding rows i < g work on it), an item 25 (its first S and the
 // epilogue), a split merge 15.  Leading globals are taken as g <= 128 (one
 // global row tile with work, one block of global keys per band tile); the
 // choice only affects speed.
@@ -1487,7 +1488,7 @@ int choose_chunk(int B, int H, int L, int w, int sm_count) {
             if (cache[i].B == B && cache[i].H == H && cache[i].L == L && cache[i].w == w && cache[i].sm == sm_count)
                 return cache[i].chunk;
     }
-    constexpr long long kBlock = 60, kGlobBlock = 75, kItem = 25, kMerge = 15, kEmpty = 2;
+    constexpr long long kBlock = 60, kGlobBlock = 60, kItem = 25, kMerge = 15, kEmpty = 2;
     auto band_blocks = [&](int r0) -> int {
         if (r0 >= L) return 0;
         const int lo = (r0 - w <= 0 ? 0 : r0 - w) / kBN;
