@@ -51,6 +51,9 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=50)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--workload", type=int, default=WORKLOAD_ID, choices=[1, 2, 3, 4, 5])
+    ap.add_argument("--layers", type=int, default=1,
+                    help="workload 5 only: time an encoder of this many layers (lf_encoder_forward), each with "
+                         "its own seeded weights")
     return ap.parse_args()
 
 
@@ -195,12 +198,19 @@ def run_ours(args):
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
     layer = args.workload == 5
+    n_layers = 1
     if layer:
         wl, x_cpu, wts_cpu, lm_cpu, gm_cpu = inputs.layer_inputs(5)
         x = x_cpu.to(dev)
         wts = {n: v.to(dev) for n, v in wts_cpu.items()}
         ffn = wts["W_1"].shape[0]
-        ws = torch.empty(max(256, lf.lf_encoder_layer_workspace_bytes(wl.B, wl.H, wl.L, wl.w, ffn, x.dtype)),
+        n_layers = max(1, args.layers)
+        # further layers: the same architecture, weights ~ N(0, 0.02) drawn on the device from a seeded generator
+        gen = torch.Generator(device=dev).manual_seed(5000)
+        stack = [wts] + [{n: ((torch.randn(v.shape, generator=gen, device=dev) * 0.02).to(v.dtype)
+                               if n.startswith("W_") else v.clone()) for n, v in wts.items()}
+                         for _ in range(n_layers - 1)]
+        ws = torch.empty(max(256, lf.lf_encoder_workspace_bytes(n_layers, wl.B, wl.H, wl.L, wl.w, ffn, x.dtype)),
                          dtype=torch.uint8, device=dev)
         args_in = [x]
         t_cpu = None
@@ -216,7 +226,9 @@ def run_ours(args):
     flush = torch.empty(max(2 * l2, 256 << 20) // 4, dtype=torch.float32, device=dev)
 
     def compute(ins, lm_, gm_):
-        if layer:
+        if layer and n_layers > 1:
+            lf.lf_encoder_forward(ins[0], lm_, gm_, stack, wl.H, wl.w, out=out, workspace=ws)
+        elif layer:
             lf.lf_encoder_layer_forward(ins[0], lm_, gm_, wts, wl.H, wl.w, out=out, workspace=ws)
         else:
             lf.lf_attention_forward(*ins, lm_, gm_, wl.w, out=out)
@@ -296,8 +308,8 @@ def run_ours(args):
 
     pk, pk_kind = peaks()
     if layer:
-        F = metrics.layer_flops(wl.B, wl.H, wl.L, wl.w, wl.g, wl.pad, ffn)
-        wbytes = sum(v.numel() * v.element_size() for v in wts.values())
+        F = n_layers * metrics.layer_flops(wl.B, wl.H, wl.L, wl.w, wl.g, wl.pad, ffn)
+        wbytes = sum(v.numel() * v.element_size() for W in stack for v in W.values())
         By = float(wbytes + 2 * x.numel() * x.element_size() + 2 * wl.B * wl.L * 4)
     else:
         F = metrics.flops(wl.B, wl.H, wl.L, wl.w, wl.g, wl.pad)
@@ -329,7 +341,8 @@ def run_ours(args):
         "dtype": wl.dtype,
         "data": "synthetic (seeded inputs of the workload's shape%s)" %
                 (": x ~ N(0,1), weights ~ N(0, 0.02)" if layer else ", N(0,1)*0.5"),
-        "config": {"workload": wl.name, "B": wl.B, "H": wl.H, "L": wl.L, "w": wl.w, "g": wl.g,
+        "config": {"workload": wl.name + (" x %d layers" % n_layers if layer and n_layers > 1 else ""),
+                   "B": wl.B, "H": wl.H, "L": wl.L, "w": wl.w, "g": wl.g,
                    "pad": wl.pad, "head_dim": 64, "l2": "flushed before every timed step (2 x L2 write)",
                    "parallelism": "replica per GPU (weak)" if world > 1 else "single GPU"},
         "tflops": F / (total_ms * 1e-3 / K) / 1e12,
@@ -343,7 +356,7 @@ def run_ours(args):
         "roofline": roof,
         "e2e": {"value": job_throughput(world, tokens, 1, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": (1 + (8 if layer else 1)) * K,
+        "gpu_launches": (1 + (8 * n_layers if layer else 1)) * K,
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not layer:

@@ -194,6 +194,29 @@ lf_status lf_encoder_layer_forward(const void* x, const float* local_mask, const
                                    lf_stream_t stream, void* out);
 
 /*
+ * lf_encoder_forward -- the encoder: n_layers layers of lf_encoder_layer_forward
+ * applied in turn (FasterTransformer Longformer page, §Longformer Encoder
+ * 计算流程: preprocessing once, then the layer loop; the attention of every
+ * layer derives g_b from the global_mask prefix itself, so no separate
+ * preprocessing pass is needed).  layers is a HOST array of n_layers weight
+ * sets (each as for lf_encoder_layer_forward, all with the same ffn_dim).
+ * x and out are [B, L, D] of `dtype`; they must not alias.  `workspace` is
+ * caller-owned device memory of at least lf_encoder_workspace_bytes(...)
+ * bytes, 256-byte aligned: one layer's workspace plus, for n_layers > 1, two
+ * [B, L, D] activation buffers the layers alternate between.
+ * Errors: LF_ERR_BAD_DIM for n_layers <= 0 or differing ffn_dim; every
+ * layer's weights are checked (LF_ERR_NULL, LF_ERR_MISALIGNED) before the
+ * first layer is launched; otherwise as lf_encoder_layer_forward.
+ * Asynchronous on `stream`.
+ */
+size_t lf_encoder_workspace_bytes(int n_layers, int B, int H, int L, int w, int ffn_dim, lf_dtype dtype);
+lf_status lf_encoder_forward(const void* x, const float* local_mask, const float* global_mask,
+                             const lf_layer_weights* layers, int n_layers, int B, int H, int L, int w,
+                             float attn_scale, float ln_eps, lf_dtype dtype,
+                             void* workspace, size_t workspace_bytes,
+                             lf_stream_t stream, void* out);
+
+/*
  * lf_attention_forward_noalloc -- lf_attention_forward for callers that
  * cannot allocate device memory.  The pages describe no such entry point: it
  * exists for code that may not call cudaMalloc (for example code running

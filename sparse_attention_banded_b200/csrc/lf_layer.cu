@@ -36,6 +36,17 @@ Workspace layout(int B, int H, int L, int w, int F, int elem) {
     return s;
 }
 
+lf_status check_weights(const lf_layer_weights* wt) {
+    const void* wptrs[] = {wt->W_qkv_kgvg, wt->b_qkv_kgvg, wt->W_qg, wt->b_qg, wt->W_o, wt->b_o,
+                           wt->ln1_gamma, wt->ln1_beta, wt->W_1, wt->b_1, wt->W_2, wt->b_2,
+                           wt->ln2_gamma, wt->ln2_beta};
+    for (const void* p : wptrs) {
+        if (!p) return LF_ERR_NULL;
+        if (!aligned16(p)) return LF_ERR_MISALIGNED;
+    }
+    return LF_OK;
+}
+
 lf_status check_layer(int B, int H, int L, int w, int F, lf_dtype dtype) {
     lf_status st = check_shape(B, H, L, w);
     if (st != LF_OK) return st;
@@ -63,13 +74,7 @@ extern "C" lf_status lf_encoder_layer_forward(const void* x, const float* local_
     const int F = wt->ffn_dim;
     lf_status st = check_layer(B, H, L, w, F, dtype);
     if (st != LF_OK) return st;
-    const void* wptrs[] = {wt->W_qkv_kgvg, wt->b_qkv_kgvg, wt->W_qg, wt->b_qg, wt->W_o, wt->b_o,
-                           wt->ln1_gamma, wt->ln1_beta, wt->W_1, wt->b_1, wt->W_2, wt->b_2,
-                           wt->ln2_gamma, wt->ln2_beta};
-    for (const void* p : wptrs) {
-        if (!p) return LF_ERR_NULL;
-        if (!aligned16(p)) return LF_ERR_MISALIGNED;
-    }
+    if ((st = check_weights(wt)) != LF_OK) return st;
     const void* ptrs[] = {x, local_mask, global_mask, out};
     for (const void* p : ptrs)
         if (!aligned16(p)) return LF_ERR_MISALIGNED;
@@ -133,4 +138,47 @@ extern "C" lf_status lf_encoder_layer_forward(const void* x, const float* local_
     if ((st = launch_gemm_tc(f2, dtype, d->sm_count, s)) != LF_OK) return st;
     return launch_layernorm(reinterpret_cast<float*>(base + ws.z), wt->ln2_gamma, wt->ln2_beta, B * L, D, ln_eps,
                             dtype, out, s);
+}
+
+// ---------------------------------------------------------------- the stack
+
+extern "C" size_t lf_encoder_workspace_bytes(int n_layers, int B, int H, int L, int w, int ffn_dim, lf_dtype dtype) {
+    if (n_layers <= 0) return 0;
+    const size_t layer = lf_encoder_layer_workspace_bytes(B, H, L, w, ffn_dim, dtype);
+    if (layer == 0) return 0;
+    const size_t act = align256((size_t)B * L * H * 64 * 2);
+    return layer + (n_layers > 1 ? 2 * act : 0);
+}
+
+// The page's encoder (§Longformer Encoder 计算流程) runs its preprocessing
+// once per forward and then the layer loop; here every layer's attention
+// reads g_b from the mask prefix itself, so the loop is the whole forward.
+extern "C" lf_status lf_encoder_forward(const void* x, const float* local_mask, const float* global_mask,
+                                        const lf_layer_weights* layers, int n_layers, int B, int H, int L, int w,
+                                        float attn_scale, float ln_eps, lf_dtype dtype, void* workspace,
+                                        size_t workspace_bytes, lf_stream_t stream, void* out) {
+    if (!x || !local_mask || !global_mask || !layers || !out) return LF_ERR_NULL;
+    if (n_layers <= 0) return LF_ERR_BAD_DIM;
+    const int F = layers[0].ffn_dim;
+    lf_status st = check_layer(B, H, L, w, F, dtype);
+    if (st != LF_OK) return st;
+    // every layer is checked before the first one is launched
+    for (int i = 0; i < n_layers; ++i) {
+        if (layers[i].ffn_dim != F) return LF_ERR_BAD_DIM;
+        if ((st = check_weights(&layers[i])) != LF_OK) return st;
+    }
+    const size_t need = lf_encoder_workspace_bytes(n_layers, B, H, L, w, F, dtype);
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < need)
+        return LF_ERR_WORKSPACE;
+    const size_t layer_bytes = layout(B, H, L, w, F, 2).total;
+    uint8_t* act[2] = {reinterpret_cast<uint8_t*>(workspace) + layer_bytes, nullptr};
+    act[1] = act[0] + align256((size_t)B * L * H * 64 * 2);
+    for (int i = 0; i < n_layers; ++i) {
+        const void* in = i == 0 ? x : act[(i - 1) & 1];
+        void* o = i == n_layers - 1 ? out : act[i & 1];
+        st = lf_encoder_layer_forward(in, local_mask, global_mask, &layers[i], B, H, L, w, attn_scale, ln_eps, dtype,
+                                      workspace, layer_bytes, stream, o);
+        if (st != LF_OK) return st;
+    }
+    return LF_OK;
 }

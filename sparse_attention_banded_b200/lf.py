@@ -65,6 +65,11 @@ def lib():
         L.lf_encoder_layer_forward.argtypes = [vp, vp, vp, ctypes.POINTER(LayerWeights), i, i, i, i,
                                                ctypes.c_float, ctypes.c_float, i, vp, ctypes.c_size_t, vp, vp]
         L.lf_encoder_layer_forward.restype = st
+        L.lf_encoder_workspace_bytes.argtypes = [i, i, i, i, i, i, i]
+        L.lf_encoder_workspace_bytes.restype = ctypes.c_size_t
+        L.lf_encoder_forward.argtypes = [vp, vp, vp, ctypes.POINTER(LayerWeights), i, i, i, i, i,
+                                         ctypes.c_float, ctypes.c_float, i, vp, ctypes.c_size_t, vp, vp]
+        L.lf_encoder_forward.restype = st
         _lib = L
     return _lib
 
@@ -180,4 +185,33 @@ def lf_encoder_layer_forward(x, local_mask, global_mask, weights: dict, H: int, 
                                         w, attn_scale, ln_eps, DTYPE_CODE.get(x.dtype, 99), _ptr(workspace),
                                         workspace.numel(), _stream(stream), _ptr(out))
     _check(st, "lf_encoder_layer_forward")
+    return out
+
+
+def lf_encoder_workspace_bytes(n_layers: int, B: int, H: int, L: int, w: int, ffn_dim: int, dtype) -> int:
+    return lib().lf_encoder_workspace_bytes(n_layers, B, H, L, w, ffn_dim, DTYPE_CODE[dtype])
+
+
+def lf_encoder_forward(x, local_mask, global_mask, layers: list, H: int, w: int, attn_scale: float = 0.125,
+                       ln_eps: float = 1e-5, out=None, workspace=None, stream=None):
+    """The encoder: the layers in `layers` (each a weight dict as for
+    lf_encoder_layer_forward, same FFN width) applied in turn to x
+    [B, L, H*64].  Returns out [B, L, H*64]."""
+    B, L, D = x.shape
+    n = len(layers)
+    ffn = layers[0]["W_1"].shape[0] if n else 0
+    arr = (LayerWeights * max(n, 1))()
+    for j, weights in enumerate(layers):
+        for name in LAYER_FIELDS:
+            _ptr(weights[name])
+        arr[j] = LayerWeights(weights["W_1"].shape[0], *[weights[name].data_ptr() for name in LAYER_FIELDS])
+    if out is None:
+        out = torch.empty_like(x)
+    need = lf_encoder_workspace_bytes(n, B, H, L, w, ffn, x.dtype) if n else 0
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=x.device)
+    st = lib().lf_encoder_forward(_ptr(x), _ptr(local_mask), _ptr(global_mask), arr, n, B, H, L, w, attn_scale,
+                                  ln_eps, DTYPE_CODE.get(x.dtype, 99), _ptr(workspace), workspace.numel(),
+                                  _stream(stream), _ptr(out))
+    _check(st, "lf_encoder_forward")
     return out

@@ -118,3 +118,36 @@ def test_layer_workspace_bytes_host_only(L):
     assert n >= (5 + 1 + 1 + 2 + 1) * rows * D * 2 + rows * 4096 * 2
     assert lf.lf_encoder_layer_workspace_bytes(1, 1, 512, 64, 512, torch.float16) == 0   # hidden 64
     assert lf.lf_encoder_layer_workspace_bytes(1, 4, 512, 64, 512, torch.float32) == 0
+
+
+def _encoder(L, n=3, ffns=(512, 512, 512), bad_layer=None, ws_bytes=1 << 30, layers="ok"):
+    arr = (lf.LayerWeights * max(n, 1))()
+    for j in range(min(n, len(ffns))):
+        vals = [FAKE] * len(lf.LAYER_FIELDS)
+        if bad_layer == j:
+            vals[8] = 0  # W_1 of that layer
+        arr[j] = lf.LayerWeights(ffns[j], *vals)
+    lp = None if layers == "null" else arr
+    return L.lf_encoder_forward(ctypes.c_void_p(FAKE), ctypes.c_void_p(FAKE), ctypes.c_void_p(FAKE), lp, n,
+                                1, 4, 512, 64, 0.125, 1e-5, 1, ctypes.c_void_p(FAKE), ws_bytes, None,
+                                ctypes.c_void_p(FAKE + 256))
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(layers="null"), 1),
+    (dict(n=0), 2),
+    (dict(ffns=(512, 384, 512)), 2),  # the layers must share the FFN width
+    (dict(bad_layer=2), 1),           # the last layer's missing weight is caught before any launch
+    (dict(ws_bytes=1024), 12),
+])
+def test_encoder_host_validation(L, kw, status):
+    assert _encoder(L, **kw) == status
+
+
+def test_encoder_workspace_bytes_host_only(L):
+    import torch
+    one = lf.lf_encoder_layer_workspace_bytes(1, 4, 512, 64, 512, torch.float16)
+    assert lf.lf_encoder_workspace_bytes(1, 1, 4, 512, 64, 512, torch.float16) == one
+    act = 512 * 256 * 2  # one [B, L, D] buffer, D = 256
+    assert lf.lf_encoder_workspace_bytes(24, 1, 4, 512, 64, 512, torch.float16) == one + 2 * act
+    assert lf.lf_encoder_workspace_bytes(0, 1, 4, 512, 64, 512, torch.float16) == 0

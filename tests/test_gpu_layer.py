@@ -79,3 +79,52 @@ def test_layer_workspace_errors():
     with pytest.raises(lf.LFError) as e:
         lf.lf_encoder_layer_forward(x.cuda(), lm.cuda(), gm.cuda(), dev, 2, 64, workspace=small)
     assert e.value.status == 12
+
+
+# ---------------------------------------------------------------- the encoder stack
+
+def _stack_weights(n, H, ffn, dtype, seed):
+    return [inputs.layer_inputs(5, hidden=H * 64, ffn=ffn, B=1, L=512, dtype=dtype, g=[4], pad=[0],
+                                seed=seed + j, bias_scale=0.1, ln_scale=0.1)[2] for j in range(n)]
+
+
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+def test_encoder_stack_equals_chained_layers(dtype):
+    """lf_encoder_forward over three layers gives exactly the bits of three
+    chained lf_encoder_layer_forward calls."""
+    B, H, L, w, ffn = 2, 2, 640, 128, 256
+    wl, x, _, lm, gm = inputs.layer_inputs(5, hidden=H * 64, ffn=ffn, B=B, L=L, dtype=dtype, g=[5, 70], pad=[0, 41],
+                                           seed=91)
+    layers = [{k: v.cuda() for k, v in W.items()} for W in _stack_weights(3, H, ffn, dtype, 300)]
+    xd, lmd, gmd = x.cuda(), lm.cuda(), gm.cuda()
+    got = lf.lf_encoder_forward(xd, lmd, gmd, layers, H, w)
+    ref = xd
+    for W in layers:
+        ref = lf.lf_encoder_layer_forward(ref, lmd, gmd, W, H, w)
+    torch.cuda.synchronize()
+    assert lf.lf_device_status(reset=True) == 0
+    assert torch.equal(got, ref)
+
+
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+def test_encoder_stack_two_layer_parity(dtype):
+    """Two layers against the float64 oracle applied twice, the activation
+    between them rounded to the dtype as the kernels store it."""
+    B, H, L, w, ffn = 1, 2, 512, 64, 256
+    wl, x, _, lm, gm = inputs.layer_inputs(5, hidden=H * 64, ffn=ffn, B=B, L=L, dtype=dtype, g=[8], pad=[19], seed=92)
+    Ws = _stack_weights(2, H, ffn, dtype, 400)
+    out = lf.lf_encoder_forward(x.cuda(), lm.cuda(), gm.cuda(), [{k: v.cuda() for k, v in W.items()} for W in Ws],
+                                H, w)
+    torch.cuda.synchronize()
+    assert lf.lf_device_status(reset=True) == 0
+    got = out.float().cpu().numpy()
+    rnd = _round_to(TDT[dtype])
+    h = x
+    for W in Ws:
+        y = oracle.encoder_layer(h, lm, gm, _oracle_weights(W), H, w, 0.125, 1e-5,
+                                 round_attention_inputs=rnd, round_stored=rnd)
+        h = torch.from_numpy(np.ascontiguousarray(y)).to(TDT[dtype])
+    ref = h.double().numpy()
+    assert np.isfinite(got).all()
+    scaled = np.abs(got - ref) / np.maximum(1.0, np.abs(ref))
+    assert scaled.max() <= TOL[TDT[dtype]], "max scaled err %g" % scaled.max()
