@@ -12,7 +12,11 @@ Parity status per function:
   * global_partition   -- pinned (brute force + hand-written golden file).
   * attention          -- pinned (dense brute force with an explicit mask,
                           closed form at q = 0, library SDPA special cases,
-                          invariants).
+                          invariants); with any_pos (global tokens at any
+                          position) pinned by a hand-worked golden file,
+                          dense brute force, the q = 0 closed form,
+                          invariants and bit-equality with the prefix
+                          definition on prefix masks.
   * encoder_layer      -- pinned per step (numpy/scipy library routines,
                           LayerNorm moments, GELU closed values).
 """
@@ -42,12 +46,14 @@ def _load():
         lib.lfo_num_threads.restype = ctypes.c_int
         lib.lfo_check_shape.argtypes = [ctypes.c_int] * 4
         lib.lfo_check_shape.restype = ctypes.c_int
-        lib.lfo_global_partition.argtypes = [fp, ctypes.c_int, ctypes.c_int, ctypes.c_int, ip, ip]
-        lib.lfo_global_partition.restype = ctypes.c_int
-        lib.lfo_attention.argtypes = [dp] * 6 + [fp, fp] + [ctypes.c_int] * 4 + [ctypes.c_double, dp]
-        lib.lfo_attention.restype = ctypes.c_int
+        for fn in (lib.lfo_global_partition, lib.lfo_global_partition_any):
+            fn.argtypes = [fp, ctypes.c_int, ctypes.c_int, ctypes.c_int, ip, ip]
+            fn.restype = ctypes.c_int
+        for fn in (lib.lfo_attention, lib.lfo_attention_any):
+            fn.argtypes = [dp] * 6 + [fp, fp] + [ctypes.c_int] * 4 + [ctypes.c_double, dp]
+            fn.restype = ctypes.c_int
         lib.lfo_attention_rows.argtypes = ([dp] * 6 + [fp, fp] + [ctypes.c_int] * 4 +
-                                           [ctypes.c_double, ip, ctypes.c_longlong, dp])
+                                           [ctypes.c_double, ctypes.c_int, ip, ctypes.c_longlong, dp])
         lib.lfo_attention_rows.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -85,44 +91,52 @@ def check_shape(B: int, H: int, L: int, w: int) -> int:
     return _load().lfo_check_shape(B, H, L, w)
 
 
-def global_partition(global_mask, w: int):
+def global_partition(global_mask, w: int, any_pos: bool = False):
     """invokeInitLongformerIdx, FTL §计算流程 / 预处理.
 
     Returns (global_idx int32 [B, L], global_token_nums int32 [B], status):
     flagged (global_mask == 0.0) positions ascending at the front, the others
     descending at the back; status 5 if some g_b > w, 6 if the flagged
     positions of some sample are not the prefix 0..g_b-1 (FTL §使用前提 items
-    3-4)."""
+    3-4; with any_pos, global tokens may lie anywhere and only item 3 is
+    checked)."""
     gm = _f32(global_mask)
     B, L = gm.shape
     idx = np.zeros((B, L), dtype=np.int32)
     nums = np.zeros((B,), dtype=np.int32)
-    st = _load().lfo_global_partition(_ptr(gm, ctypes.c_float), B, L, w,
-                                      _ptr(idx, ctypes.c_int32), _ptr(nums, ctypes.c_int32))
+    fn = _load().lfo_global_partition_any if any_pos else _load().lfo_global_partition
+    st = fn(_ptr(gm, ctypes.c_float), B, L, w, _ptr(idx, ctypes.c_int32), _ptr(nums, ctypes.c_int32))
     return idx, nums, st
 
 
-def attention(q, k, v, qg, kg, vg, local_mask, global_mask, w: int, scale: float = SCALE):
+def attention(q, k, v, qg, kg, vg, local_mask, global_mask, w: int, scale: float = SCALE,
+              any_pos: bool = False):
     """The attention layer of FTL §计算流程 / 每个 Transformer 层 steps 3-5.
 
     Inputs q, k, v, qg, kg, vg are [B, H, L, 64] (their stored values are
     widened exactly to float64); masks are [B, L] float32.  Returns out
-    float64 [B, L, H, 64].  Raises OracleError on a constraint failure."""
+    float64 [B, L, H, 64].  Raises OracleError on a constraint failure.
+
+    any_pos: global tokens (global_mask == 0.0) may lie anywhere, the
+    HuggingFace arrangement that FTL §使用前提 item 4 sets apart from FT's
+    prefix rule; a non-global row then attends its window united with every
+    global token, each key once."""
     arrs = [_f64(t) for t in (q, k, v, qg, kg, vg)]
     B, H, L, d = arrs[0].shape
     assert d == D
     lm, gm = _f32(local_mask), _f32(global_mask)
     out = np.zeros((B, L, H, D), dtype=np.float64)
-    st = _load().lfo_attention(*[_ptr(a, ctypes.c_double) for a in arrs],
-                               _ptr(lm, ctypes.c_float), _ptr(gm, ctypes.c_float),
-                               B, H, L, w, float(scale), _ptr(out, ctypes.c_double))
+    fn = _load().lfo_attention_any if any_pos else _load().lfo_attention
+    st = fn(*[_ptr(a, ctypes.c_double) for a in arrs],
+            _ptr(lm, ctypes.c_float), _ptr(gm, ctypes.c_float),
+            B, H, L, w, float(scale), _ptr(out, ctypes.c_double))
     if st != 0:
         raise OracleError(st)
     return out
 
 
 def attention_rows(q, k, v, qg, kg, vg, local_mask, global_mask, w: int, rows,
-                   scale: float = SCALE):
+                   scale: float = SCALE, any_pos: bool = False):
     """Same as :func:`attention`, for the listed rows only.
 
     rows: int array [n, 3] of (b, h, i).  Returns float64 [n, 64] =
@@ -134,7 +148,7 @@ def attention_rows(q, k, v, qg, kg, vg, local_mask, global_mask, w: int, rows,
     out = np.zeros((rows.shape[0], D), dtype=np.float64)
     st = _load().lfo_attention_rows(*[_ptr(a, ctypes.c_double) for a in arrs],
                                     _ptr(lm, ctypes.c_float), _ptr(gm, ctypes.c_float),
-                                    B, H, L, w, float(scale),
+                                    B, H, L, w, float(scale), 1 if any_pos else 0,
                                     _ptr(rows, ctypes.c_int32), rows.shape[0],
                                     _ptr(out, ctypes.c_double))
     if st != 0:

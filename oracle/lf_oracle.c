@@ -38,6 +38,14 @@
  *   - The partition's output order is that of a stable flagged partition:
  *     selected indices ascending at the front, rejected ones in reverse
  *     order at the back.
+ *   - Global tokens at any position (the "_any" entry points): FTL
+ *     §使用前提 item 4 names placing global tokens anywhere as the
+ *     HuggingFace behaviour that FT does not support.  There the global set
+ *     is G_b = { j : global_mask[b, j] == 0.0 } wherever its members lie; a
+ *     row i in G_b is a global row (qg/kg/vg over the whole sequence), any
+ *     other row attends its window united with all of G_b, each key once.
+ *     Constraint 3 (g_b <= w) is kept.  With G_b a prefix this is exactly
+ *     the prefix definition above.
  *
  * Arithmetic: IEEE double throughout, no fast-math; exp() from libm.  The
  * bias is formed in float with fmaf exactly as the page writes it, then
@@ -83,15 +91,17 @@ int lfo_check_shape(int B, int H, int L, int w)
 }
 
 /* The set G_b of global positions of sample b is { j : global_mask == 0.0 }
- * (FTL input list).  Constraint 4 requires G_b == {0..g_b-1}, constraint 3
- * g_b <= w.  Returns the status and writes g_b. */
-static int global_count(const float* gm_row, int L, int w, int* g_out)
+ * (FTL input list).  Constraint 4 requires G_b == {0..g_b-1} (checked
+ * unless any_pos), constraint 3 g_b <= w.  Returns the status and writes
+ * g_b. */
+static int global_count(const float* gm_row, int L, int w, int any_pos, int* g_out)
 {
     int g = 0;
     for (int j = 0; j < L; ++j)
         if (gm_row[j] == 0.0f) ++g;
-    for (int j = 0; j < g; ++j)
-        if (gm_row[j] != 0.0f) return LFO_ERR_GLOBAL_NOT_PREFIX;
+    if (!any_pos)
+        for (int j = 0; j < g; ++j)
+            if (gm_row[j] != 0.0f) return LFO_ERR_GLOBAL_NOT_PREFIX;
     *g_out = g;
     if (g > w) return LFO_ERR_G_GT_W;
     return LFO_OK;
@@ -103,8 +113,8 @@ static int global_count(const float* gm_row, int L, int w, int* g_out)
  * global_idx[b, g_b..L-1] = unflagged positions in descending order;
  * global_token_nums[b] = g_b.  The outputs are written even when the
  * constraints fail; the first failing sample's status is returned. */
-int lfo_global_partition(const float* global_mask, int B, int L, int w,
-                         int32_t* global_idx, int32_t* global_token_nums)
+static int global_partition(const float* global_mask, int B, int L, int w, int any_pos,
+                            int32_t* global_idx, int32_t* global_token_nums)
 {
     int status = LFO_OK;
     for (int b = 0; b < B; ++b) {
@@ -117,10 +127,24 @@ int lfo_global_partition(const float* global_mask, int B, int L, int w,
         }
         global_token_nums[b] = front;
         int g;
-        int st = global_count(row, L, w, &g);
+        int st = global_count(row, L, w, any_pos, &g);
         if (st != LFO_OK && status == LFO_OK) status = st;
     }
     return status;
+}
+
+int lfo_global_partition(const float* global_mask, int B, int L, int w,
+                         int32_t* global_idx, int32_t* global_token_nums)
+{
+    return global_partition(global_mask, B, L, w, 0, global_idx, global_token_nums);
+}
+
+/* The same partition with the global tokens at any position (only g_b <= w
+ * is checked). */
+int lfo_global_partition_any(const float* global_mask, int B, int L, int w,
+                             int32_t* global_idx, int32_t* global_token_nums)
+{
+    return global_partition(global_mask, B, L, w, 1, global_idx, global_token_nums);
 }
 
 /* Shifted local mask, invokeLocalAttnMaskShift (FTL §计算流程 / 预处理). */
@@ -140,17 +164,20 @@ typedef struct {
     const double *q, *k, *v, *qg, *kg, *vg; /* [B,H,L,64] */
     const float *local_mask, *global_mask;  /* [B,L] */
     const int* g;                            /* per-sample global count */
+    const int* gpos;                         /* [B][L]: sample b's global positions, ascending */
     int B, H, L, w;
     double scale;
+    int any_pos;                             /* global tokens may lie anywhere */
 } lfo_ctx;
 
 /* One output row out[b, i, h, :] of the attention layer.
  *   e_j = scale * <q_i, k_j> + lb[j] (+ global_mask[j] on global columns)
  *   p_j = exp(e_j - max e) / sum exp(e - max e)   over the row's key set
  *   out = sum_j p_j * v_j
- * Key set: local row i >= g_b -> window [max(0,i-w), min(L-1,i+w)] united
- * with the global positions [0, g_b); global row i < g_b -> all of [0, L)
- * with qg/kg/vg.  A row with lb[i] != 0 is zero. */
+ * Key set: local row i (not in G_b) -> window [max(0,i-w), min(L-1,i+w)]
+ * united with the global positions G_b; global row i in G_b -> all of
+ * [0, L) with qg/kg/vg.  (G_b = [0, g_b) unless any_pos.)  A row with
+ * lb[i] != 0 is zero. */
 static void attention_row(const lfo_ctx* c, int b, int h, int i, double* o,
                           double* e /* scratch [L] */, int* keys /* scratch [L] */)
 {
@@ -162,7 +189,8 @@ static void attention_row(const lfo_ctx* c, int b, int h, int i, double* o,
     for (int d = 0; d < LFO_D; ++d) o[d] = 0.0;
     if (local_bias(lm[i]) != 0.0) return; /* padded query row: zero */
 
-    const int global_row = i < g;
+    const int* G = c->gpos + (size_t)b * L; /* G[0..g) */
+    const int global_row = gm[i] == 0.0f;
     const double* qi = (global_row ? c->qg : c->q) + head + (size_t)i * LFO_D;
     const double* K = (global_row ? c->kg : c->k) + head;
     const double* V = (global_row ? c->vg : c->v) + head;
@@ -174,15 +202,16 @@ static void attention_row(const lfo_ctx* c, int b, int h, int i, double* o,
     } else {
         int lo = i - w < 0 ? 0 : i - w;
         int hi = i + w > L - 1 ? L - 1 : i + w;
-        for (int j = 0; j < g; ++j) keys[n++] = j;             /* global tokens */
-        for (int j = (lo > g ? lo : g); j <= hi; ++j) keys[n++] = j; /* window minus globals */
+        for (int t = 0; t < g; ++t) keys[n++] = G[t];          /* global tokens */
+        for (int j = lo; j <= hi; ++j)                         /* window minus globals */
+            if (gm[j] != 0.0f) keys[n++] = j;
     }
 
     double m = -INFINITY;
     for (int t = 0; t < n; ++t) {
         int j = keys[t];
         double s = c->scale * dot64(qi, K + (size_t)j * LFO_D) + local_bias(lm[j]);
-        if (!global_row && j < g) s += (double)gm[j];
+        if (!global_row && t < g) s += (double)gm[j];          /* global column */
         e[t] = s;
         if (s > m) m = s;
     }
@@ -198,28 +227,35 @@ static void attention_row(const lfo_ctx* c, int b, int h, int i, double* o,
     }
 }
 
-static int prepare(lfo_ctx* c, int* g)
+/* Per-sample global counts and position lists (gpos: [B][L]). */
+static int prepare(lfo_ctx* c, int* g, int* gpos)
 {
     int st = lfo_check_shape(c->B, c->H, c->L, c->w);
     if (st != LFO_OK) return st;
     for (int b = 0; b < c->B; ++b) {
-        st = global_count(c->global_mask + (size_t)b * c->L, c->L, c->w, &g[b]);
+        const float* row = c->global_mask + (size_t)b * c->L;
+        st = global_count(row, c->L, c->w, c->any_pos, &g[b]);
         if (st != LFO_OK) return st;
+        int n = 0;
+        for (int j = 0; j < c->L; ++j)
+            if (row[j] == 0.0f) gpos[(size_t)b * c->L + n++] = j;
     }
     c->g = g;
+    c->gpos = gpos;
     return LFO_OK;
 }
 
 /* Full attention layer: out[B, L, H, 64] (the multi-head-to-single layout of
  * FTL step 5).  Returns a status; out is untouched on error. */
-int lfo_attention(const double* q, const double* k, const double* v,
-                  const double* qg, const double* kg, const double* vg,
-                  const float* local_mask, const float* global_mask,
-                  int B, int H, int L, int w, double scale, double* out)
+static int attention_all(const double* q, const double* k, const double* v,
+                         const double* qg, const double* kg, const double* vg,
+                         const float* local_mask, const float* global_mask,
+                         int B, int H, int L, int w, double scale, int any_pos, double* out)
 {
-    lfo_ctx c = {q, k, v, qg, kg, vg, local_mask, global_mask, NULL, B, H, L, w, scale};
+    lfo_ctx c = {q, k, v, qg, kg, vg, local_mask, global_mask, NULL, NULL, B, H, L, w, scale, any_pos};
     int* g = (int*)malloc(sizeof(int) * (size_t)(B > 0 ? B : 1));
-    int st = prepare(&c, g);
+    int* gpos = (int*)malloc(sizeof(int) * (size_t)(B > 0 ? B : 1) * (size_t)(L > 0 ? L : 1));
+    int st = prepare(&c, g, gpos);
     if (st == LFO_OK) {
         long long total = (long long)B * H * L;
 #pragma omp parallel
@@ -238,19 +274,38 @@ int lfo_attention(const double* q, const double* k, const double* v,
         }
     }
     free(g);
+    free(gpos);
     return st;
+}
+
+int lfo_attention(const double* q, const double* k, const double* v,
+                  const double* qg, const double* kg, const double* vg,
+                  const float* local_mask, const float* global_mask,
+                  int B, int H, int L, int w, double scale, double* out)
+{
+    return attention_all(q, k, v, qg, kg, vg, local_mask, global_mask, B, H, L, w, scale, 0, out);
+}
+
+/* Global tokens at any position. */
+int lfo_attention_any(const double* q, const double* k, const double* v,
+                      const double* qg, const double* kg, const double* vg,
+                      const float* local_mask, const float* global_mask,
+                      int B, int H, int L, int w, double scale, double* out)
+{
+    return attention_all(q, k, v, qg, kg, vg, local_mask, global_mask, B, H, L, w, scale, 1, out);
 }
 
 /* Selected rows only: rows[3*r .. 3*r+2] = (b, h, i); out_rows[r, 64]. */
 int lfo_attention_rows(const double* q, const double* k, const double* v,
                        const double* qg, const double* kg, const double* vg,
                        const float* local_mask, const float* global_mask,
-                       int B, int H, int L, int w, double scale,
+                       int B, int H, int L, int w, double scale, int any_pos,
                        const int32_t* rows, long long n_rows, double* out_rows)
 {
-    lfo_ctx c = {q, k, v, qg, kg, vg, local_mask, global_mask, NULL, B, H, L, w, scale};
+    lfo_ctx c = {q, k, v, qg, kg, vg, local_mask, global_mask, NULL, NULL, B, H, L, w, scale, any_pos};
     int* g = (int*)malloc(sizeof(int) * (size_t)(B > 0 ? B : 1));
-    int st = prepare(&c, g);
+    int* gpos = (int*)malloc(sizeof(int) * (size_t)(B > 0 ? B : 1) * (size_t)(L > 0 ? L : 1));
+    int st = prepare(&c, g, gpos);
     if (st == LFO_OK) {
 #pragma omp parallel
         {
@@ -265,5 +320,6 @@ int lfo_attention_rows(const double* q, const double* k, const double* v,
         }
     }
     free(g);
+    free(gpos);
     return st;
 }

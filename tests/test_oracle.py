@@ -154,7 +154,6 @@ def dense_reference(t, lm, gm, w, scale=0.125):
     out = np.zeros((B, L, H, 64))
     for b in range(B):
         is_global = (gm[b] == 0.0)
-        g = int(is_global.sum())
         lb = np.where(lm[b] == 1.0, 0.0, -10000.0)
         allowed = np.zeros((L, L), dtype=bool)
         for i in range(L):
@@ -167,7 +166,7 @@ def dense_reference(t, lm, gm, w, scale=0.125):
             o_loc = softmax(s_loc, axis=1) @ v[b, h]
             s_glb = scale * qg[b, h] @ kg[b, h].T + lb[None, :]
             o_glb = softmax(s_glb, axis=1) @ vg[b, h]
-            rows = np.where(np.arange(L)[:, None] < g, o_glb, o_loc)
+            rows = np.where(is_global[:, None], o_glb, o_loc)
             rows[lb != 0.0] = 0.0
             out[b, :, h, :] = rows
     return out
@@ -299,6 +298,161 @@ def test_oracle_rejects_bad_globals():
     with pytest.raises(oracle.OracleError) as e:
         oracle.attention(*[t[n] for n in inputs.NAMES], lm, gm, 4)
     assert e.value.status == 5
+
+
+# ------------------------------------------------- global tokens at any position
+
+def _scattered_masks(rng, B, L, w, pad_global=True):
+    """Masks with g_b <= w global tokens at random positions (the HuggingFace
+    arrangement of FTL §使用前提 item 4) and random padded positions, some of
+    them on global tokens."""
+    lm = np.ones((B, L), np.float32)
+    gm = np.full((B, L), -10000.0, np.float32)
+    for b in range(B):
+        g = int(rng.integers(0, w + 1))
+        gm[b, rng.choice(L, size=g, replace=False)] = 0.0
+        pad = int(rng.integers(0, L // 2))
+        if pad:
+            lm[b, L - pad:] = 0.0
+        if pad_global and rng.random() < 0.5:
+            lm[b, rng.integers(0, L)] = 0.0
+    return lm, gm
+
+
+def test_any_globals_golden():
+    g = _golden_kv("attention_any_globals.txt")
+    L, w = int(g["L"][0]), int(g["w"][0])
+    z = np.zeros((1, 1, L, 64))
+    v = np.zeros((1, 1, L, 64)); v[0, 0, :, 0] = np.arange(L) + 1
+    vg = np.zeros((1, 1, L, 64)); vg[0, 0, :, 0] = np.arange(L) + 101
+    for case in ("a", "b"):
+        lm = np.ones((1, L), np.float32)
+        gm = np.full((1, L), -10000.0, np.float32)
+        gm[0, [int(x) for x in g[case + "_globals"]]] = 0.0
+        lm[0, [int(x) for x in g[case + "_padded"]]] = 0.0
+        out = oracle.attention(z, z, v, z, z, vg, lm, gm, w, any_pos=True)
+        np.testing.assert_allclose(out[0, :, 0, 0], np.array(g[case + "_out0"]), rtol=0, atol=1e-12)
+        assert np.all(out[0, :, 0, 1:] == 0.0)
+
+
+@pytest.mark.parametrize("seed", range(30))
+def test_any_globals_match_dense_brute_force(seed):
+    rng = np.random.default_rng(700 + seed)
+    w = int(rng.choice([2, 4, 8, 16, 32]))
+    L = w * int(rng.integers(2, max(3, 64 // w) + 1))
+    B, H = int(rng.integers(1, 3)), int(rng.integers(1, 3))
+    lm, gm = _scattered_masks(rng, B, L, w)
+    t = inputs.attention_inputs(B, H, L, "f32", int(rng.integers(1 << 30)))
+    t = [t[n] for n in inputs.NAMES]
+    got = oracle.attention(*t, lm, gm, w, any_pos=True)
+    want = dense_reference(t, lm, gm, w)
+    np.testing.assert_allclose(got, want, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_any_globals_q_zero_closed_form(seed):
+    """q = qg = 0: an unpadded row is the mean of v (vg for a global row)
+    over its unpadded key set, the sets built here with Python set algebra."""
+    rng = np.random.default_rng(800 + seed)
+    w = int(rng.choice([4, 8, 16]))
+    L = w * int(rng.integers(2, 5))
+    B, H = 2, 2
+    lm, gm = _scattered_masks(rng, B, L, w)
+    t = inputs.attention_inputs(B, H, L, "f32", seed)
+    q, k, v, qg, kg, vg = [t[n].double().numpy() for n in inputs.NAMES]
+    q[:] = 0; qg[:] = 0
+    out = oracle.attention(q, k, v, qg, kg, vg, lm, gm, w, any_pos=True)
+    for b in range(B):
+        G = {j for j in range(L) if gm[b, j] == 0.0}
+        valid = {j for j in range(L) if lm[b, j] == 1.0}
+        for i in range(L):
+            if i not in valid:
+                assert np.all(out[b, i] == 0.0)
+                continue
+            if i in G:
+                keys, vals = set(range(L)), vg
+            else:
+                keys, vals = set(range(max(0, i - w), min(L - 1, i + w) + 1)) | G, v
+            keys = sorted(keys & valid)
+            for h in range(H):
+                np.testing.assert_allclose(out[b, i, h], vals[b, h, keys].mean(axis=0), atol=1e-12)
+
+
+@pytest.mark.parametrize("seed", range(5))
+def test_any_globals_prefix_case_is_the_prefix_oracle(seed):
+    """With the global tokens at the front both definitions are the same
+    computation, bit for bit."""
+    rng = np.random.default_rng(900 + seed)
+    t, lm, gm, w = _random_case(rng)
+    a = oracle.attention(*t, lm, gm, w)
+    b = oracle.attention(*t, lm, gm, w, any_pos=True)
+    assert np.array_equal(a, b)
+
+
+def test_any_globals_invariants_and_errors():
+    rng = np.random.default_rng(11)
+    B, H, L, w = 2, 2, 48, 8
+    lm, gm = _scattered_masks(rng, B, L, w)
+    t = inputs.attention_inputs(B, H, L, "f32", 3)
+    q, k, v, qg, kg, vg = [t[n].double().numpy() for n in inputs.NAMES]
+    ones = np.ones_like(v)
+    out = oracle.attention(q, k, ones, qg, kg, ones, lm, gm, w, any_pos=True)
+    for b in range(B):
+        for i in range(L):
+            if lm[b, i] == 1.0:
+                np.testing.assert_allclose(out[b, i], 1.0, atol=1e-12)
+            else:
+                assert np.all(out[b, i] == 0.0)
+    # keys outside a local row's set (outside the window and not global) do not matter
+    base = oracle.attention(q, k, v, qg, kg, vg, lm, gm, w, any_pos=True)
+    b, h = 0, 1
+    G = set(np.flatnonzero(gm[b] == 0.0).tolist())
+    i = next(i for i in range(L) if i not in G)
+    outside = [j for j in range(L) if abs(i - j) > w and j not in G]
+    k2, v2 = k.copy(), v.copy()
+    k2[b, h, outside] += rng.normal(size=(len(outside), 64))
+    v2[b, h, outside] += rng.normal(size=(len(outside), 64))
+    pert = oracle.attention(q, k2, v2, qg, kg, vg, lm, gm, w, any_pos=True)
+    assert np.array_equal(pert[b, i, h], base[b, i, h])
+    # more than w global tokens is still an error; scattered ones are not
+    gm2 = np.full((1, 16), -10000.0, np.float32); gm2[0, [3, 9, 14]] = 0.0
+    t1 = inputs.attention_inputs(1, 1, 16, "f32", 1)
+    args = [t1[n] for n in inputs.NAMES]
+    oracle.attention(*args, np.ones((1, 16), np.float32), gm2, 4, any_pos=True)
+    gm2[0, [1, 5]] = 0.0
+    with pytest.raises(oracle.OracleError) as e:
+        oracle.attention(*args, np.ones((1, 16), np.float32), gm2, 4, any_pos=True)
+    assert e.value.status == 5
+
+
+@pytest.mark.parametrize("seed", range(10))
+def test_any_globals_partition_brute_force(seed):
+    rng = np.random.default_rng(1000 + seed)
+    B, w = 3, int(rng.integers(1, 9))
+    L = w * int(rng.integers(2, 6))
+    gm = np.full((B, L), -10000.0, np.float32)
+    for b in range(B):
+        gm[b, rng.random(L) < rng.random() * 0.5] = 0.0
+    idx, nums, st = oracle.global_partition(gm, w, any_pos=True)
+    expect = 0
+    for b in range(B):
+        e_idx, e_num = _partition_brute(gm[b].tolist())
+        assert idx[b].tolist() == e_idx and nums[b] == e_num
+        if e_num > w and not expect:
+            expect = 5
+    assert st == expect
+
+
+def test_any_globals_rows_match_full():
+    rng = np.random.default_rng(12)
+    lm, gm = _scattered_masks(rng, 2, 32, 8)
+    t = inputs.attention_inputs(2, 2, 32, "f32", 4)
+    t = [t[n] for n in inputs.NAMES]
+    full = oracle.attention(*t, lm, gm, 8, any_pos=True)
+    rows = np.array([[b, h, i] for b in range(2) for h in range(2) for i in range(32)])
+    sub = oracle.attention_rows(*t, lm, gm, 8, rows, any_pos=True)
+    for r, (b, h, i) in enumerate(rows):
+        assert np.array_equal(sub[r], full[b, i, h])
 
 
 # ---------------------------------------------------------------- encoder layer
