@@ -14,7 +14,10 @@ Under torchrun each rank runs its own replica of the workload (weak scaling,
 no collective on the data path); timings are the max over ranks.
 --workload selects another of the synthetic configurations (1: fp32
 attention, 3: bf16 batched, 4: fp16 L=16384, 5: one fp16 encoder layer with
-its projections, LayerNorms and FFN); 2 is the default and the headline.
+its projections, LayerNorms and FFN, 6: workload 2 with its global tokens at
+random positions, through the entry point for global tokens anywhere, whose
+one call runs the partition, the gather of the global rows and the
+attention kernel); 2 is the default and the headline.
 """
 from __future__ import annotations
 
@@ -50,7 +53,7 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=50)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", type=int, default=WORKLOAD_ID, choices=[1, 2, 3, 4, 5])
+    ap.add_argument("--workload", type=int, default=WORKLOAD_ID, choices=[1, 2, 3, 4, 5, 6])
     ap.add_argument("--layers", type=int, default=1,
                     help="workload 5 only: time an encoder of this many layers (lf_encoder_forward), each with "
                          "its own seeded weights")
@@ -178,7 +181,7 @@ def cpu_baseline(wl, t, lm, gm, budget_s=10.0):
     lmn, gmn = lm.numpy(), gm.numpy()
     passes, t0 = 0, time.perf_counter()
     while True:
-        oracle.attention(*arrs, lmn, gmn, wl.w)
+        oracle.attention(*arrs, lmn, gmn, wl.w, any_pos=wl.scattered)
         passes += 1
         if time.perf_counter() - t0 >= budget_s:
             break
@@ -198,6 +201,7 @@ def run_ours(args):
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
     layer = args.workload == 5
+    anyg = args.workload == 6  # global tokens at any position: one call = partition + gather + attention
     n_layers = 1
     if layer:
         wl, x_cpu, wts_cpu, lm_cpu, gm_cpu = inputs.layer_inputs(5)
@@ -230,11 +234,14 @@ def run_ours(args):
             lf.lf_encoder_forward(ins[0], lm_, gm_, stack, wl.H, wl.w, out=out, workspace=ws)
         elif layer:
             lf.lf_encoder_layer_forward(ins[0], lm_, gm_, wts, wl.H, wl.w, out=out, workspace=ws)
+        elif anyg:
+            lf.lf_attention_forward_any_globals(*ins, lm_, gm_, wl.w, out=out)
         else:
             lf.lf_attention_forward(*ins, lm_, gm_, wl.w, out=out)
 
     def step(ev_a=None):
-        lf.lf_init_global_idx(gm, wl.w, gidx, gnum, sync=False)
+        if not anyg:
+            lf.lf_init_global_idx(gm, wl.w, gidx, gnum, sync=False)
         if ev_a is not None:
             ev_a.record()
         compute(args_in, lm, gm)
@@ -287,7 +294,8 @@ def run_ours(args):
     def e2e_step():
         for h, d in zip(h_in, d_in):
             d.copy_(h, non_blocking=True)
-        lf.lf_init_global_idx(d_in[n_t + 1], wl.w, gidx, gnum, sync=False)
+        if not anyg:
+            lf.lf_init_global_idx(d_in[n_t + 1], wl.w, gidx, gnum, sync=False)
         compute(d_in[:n_t], d_in[n_t], d_in[n_t + 1])
         h_out.copy_(out, non_blocking=True)
 
@@ -312,7 +320,8 @@ def run_ours(args):
         wbytes = sum(v.numel() * v.element_size() for W in stack for v in W.values())
         By = float(wbytes + 2 * x.numel() * x.element_size() + 2 * wl.B * wl.L * 4)
     else:
-        F = metrics.flops(wl.B, wl.H, wl.L, wl.w, wl.g, wl.pad)
+        F = (metrics.flops_masks(lm_cpu.numpy(), gm_cpu.numpy(), wl.H, wl.w) if anyg
+             else metrics.flops(wl.B, wl.H, wl.L, wl.w, wl.g, wl.pad))
         By = metrics.algorithmic_bytes(wl.B, wl.H, wl.L, wl.w, wl.g, wl.dtype)
     t_attn = attn_avg_ms * 1e-3
     tokens = wl.B * wl.L
@@ -351,12 +360,13 @@ def run_ours(args):
             "tflops": F / t_attn / 1e12,
             "tensor_peak_frac": F / t_attn / 1e12 / pk["bf16_tflops"] if tensor_path else None,
             "tensor_peak_tflops": pk["bf16_tflops"],
-            "note": "fp16 and bf16 dense tensor rates are equal; peak = measured bf16 burst (%s)" % pk_kind,
+            "note": "fp16 and bf16 dense tensor rates are equal; peak = measured bf16 burst (%s)" % pk_kind
+                    + ("; the timed call is partition + gather + attention (3 kernels)" if anyg else ""),
         },
         "roofline": roof,
         "e2e": {"value": job_throughput(world, tokens, 1, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": (1 + (8 * n_layers if layer else 1)) * K,
+        "gpu_launches": (3 if anyg else 1 + (8 * n_layers if layer else 1)) * K,
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not layer:

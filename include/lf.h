@@ -138,6 +138,39 @@ lf_status lf_attention_forward(const void* q, const void* k, const void* v,
 /* Bytes of scratch lf_attention_forward needs for this shape (0 if none). */
 size_t lf_attention_scratch_bytes(int B, int H, int L, int w, lf_dtype dtype);
 
+/*
+ * lf_attention_forward_any_globals -- lf_attention_forward with the global
+ * tokens at any positions of the sequence: the HuggingFace arrangement that
+ * FTL §使用前提 item 4 names as unsupported by FT, gathered through the
+ * global_idx of the partition (invokeInitLongformerIdx, FTL §计算流程 /
+ * 预处理) instead of being read as a prefix.
+ *
+ * Arguments, layouts, dtypes, shape checks and the scratch rules are those of
+ * lf_attention_forward.  With G_b = { j : global_mask[b,j] == 0.0 } and
+ * g_b = |G_b|:
+ *   row i with lb[i] != 0                -> out row = 0 (global rows too);
+ *   row i in G_b (global row)            -> softmax_j(s*qg_i.kg_j + lb[j]) over
+ *                                           all j, values vg;
+ *   any other row (local row)            -> softmax over the set
+ *                                           {|i-j| <= w} U G_b (each key once)
+ *                                           of s*q_i.k_j + lb[j], values v.
+ * qg is read only at the rows of G_b.  A sample with g_b > w records
+ * LF_ERR_G_GT_W and gets an all-zero output.  With G_b = {0..g_b-1} the
+ * result is that of lf_attention_forward.  The call runs the partition into
+ * its scratch (global_idx, global_token_nums and a per-position count of the
+ * global tokens before it), then for LF_F16 / LF_BF16 a gather of the global
+ * tokens' qg, k and v rows into per-head slot buffers, then the attention
+ * kernel; all three are asynchronous on `stream`.
+ */
+lf_status lf_attention_forward_any_globals(const void* q, const void* k, const void* v,
+                                           const void* qg, const void* kg, const void* vg,
+                                           const float* local_mask, const float* global_mask,
+                                           int B, int H, int L, int w, lf_dtype dtype,
+                                           lf_stream_t stream, void* out);
+
+/* Bytes of scratch lf_attention_forward_any_globals needs for this shape. */
+size_t lf_attention_any_globals_scratch_bytes(int B, int H, int L, int w, lf_dtype dtype);
+
 /* Free the library-owned scratch of the current device (synchronises it). */
 lf_status lf_release_scratch(void);
 

@@ -58,6 +58,7 @@ lf_status ensure_scratch(DeviceCtx* d, size_t bytes) {
         cudaFree(d->scratch);
         d->scratch = nullptr;
         d->scratch_bytes = 0;
+        d->scratch_clean = 0;
     }
     void* p = nullptr;
     if (cudaMalloc(&p, bytes) != cudaSuccess) return LF_ERR_CUDA;
@@ -67,7 +68,27 @@ lf_status ensure_scratch(DeviceCtx* d, size_t bytes) {
     }
     d->scratch = p;
     d->scratch_bytes = bytes;
+    d->scratch_clean = bytes;
     return LF_OK;
+}
+
+lf_status prepare_scratch_counters(DeviceCtx* d, size_t zero_bytes, cudaStream_t stream) {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if (zero_bytes > d->scratch_clean) {
+        // A call of another shape (whose partials reached into this range)
+        // or another use of the scratch left other bytes here.
+        if (cudaMemsetAsync(d->scratch, 0, zero_bytes, stream) != cudaSuccess) {
+            d->scratch_clean = 0;
+            return LF_ERR_CUDA;
+        }
+    }
+    d->scratch_clean = zero_bytes;
+    return LF_OK;
+}
+
+void scratch_dirty(DeviceCtx* d) {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    d->scratch_clean = 0;
 }
 
 lf_status check_shape(int B, int H, int L, int w) {
@@ -183,8 +204,62 @@ lf_status lf_attention_forward(const void* q, const void* k, const void* v, cons
                                          d->status, s);
     st = ensure_scratch(d, attention_tc_scratch_bytes(B, H, L, w));
     if (st != LF_OK) return st;
-    return launch_attention_tc(q, k, v, qg, kg, vg, local_mask, global_mask, B, H, L, w, scale, dtype,
-                               out, d->scratch, d->status, d->sm_count, s);
+    st = prepare_scratch_counters(d, attention_tc_scratch_zero_bytes(B, H, L, w), s);
+    if (st != LF_OK) return st;
+    st = launch_attention_tc(q, k, v, qg, kg, vg, local_mask, global_mask, B, H, L, w, scale, dtype, out,
+                             d->scratch, d->status, d->sm_count, s);
+    if (st != LF_OK) scratch_dirty(d);
+    return st;
+}
+
+size_t lf_attention_any_globals_scratch_bytes(int B, int H, int L, int w, lf_dtype dtype) {
+    if (check_shape(B, H, L, w) != LF_OK) return 0;
+    const bool tc = dtype == LF_F16 || dtype == LF_BF16;
+    return (tc ? attention_tc_scratch_bytes(B, H, L, w) : 0) + any_globals_bytes(B, H, L, w, tc);
+}
+
+lf_status lf_attention_forward_any_globals(const void* q, const void* k, const void* v, const void* qg,
+                                           const void* kg, const void* vg, const float* local_mask,
+                                           const float* global_mask, int B, int H, int L, int w,
+                                           lf_dtype dtype, lf_stream_t stream, void* out) {
+    if (!q || !k || !v || !qg || !kg || !vg || !local_mask || !global_mask || !out) return LF_ERR_NULL;
+    lf_status st = check_shape(B, H, L, w);
+    if (st != LF_OK) return st;
+    if (dtype != LF_F32 && dtype != LF_F16 && dtype != LF_BF16) return LF_ERR_DTYPE;
+    const void* ptrs[] = {q, k, v, qg, kg, vg, local_mask, global_mask, out};
+    for (const void* p : ptrs)
+        if (!aligned16(p)) return LF_ERR_MISALIGNED;
+    DeviceCtx* d = current_device(&st);
+    if (!d) return st;
+    const float scale = 0.125f;  // 1/sqrt(64)
+    cudaStream_t s = (cudaStream_t)stream;
+    const bool tc = dtype != LF_F32;
+    // scratch: [attention scratch (16-bit)][partition outputs + slot buffers]
+    const size_t att = tc ? attention_tc_scratch_bytes(B, H, L, w) : 0;
+    st = ensure_scratch(d, att + any_globals_bytes(B, H, L, w, tc));
+    if (st != LF_OK) return st;
+    const AnyGlobals a = any_globals_layout(static_cast<uint8_t*>(d->scratch) + att, B, H, L, w, tc);
+    if (tc) {
+        st = prepare_scratch_counters(d, attention_tc_scratch_zero_bytes(B, H, L, w), s);
+        if (st != LF_OK) return st;
+    } else {
+        scratch_dirty(d);  // the partition's outputs start at the scratch's first byte
+    }
+    st = launch_global_idx(global_mask, B, L, w, const_cast<int32_t*>(a.global_idx),
+                           const_cast<int32_t*>(a.global_token_nums), d->status, s,
+                           const_cast<int32_t*>(a.rank), false);
+    if (st != LF_OK) return st;
+    if (!tc)
+        return launch_attention_simt_f32((const float*)q, (const float*)k, (const float*)v,
+                                         (const float*)qg, (const float*)kg, (const float*)vg,
+                                         local_mask, global_mask, B, H, L, w, scale, (float*)out,
+                                         d->status, s, &a);
+    st = launch_gather_globals(qg, k, v, local_mask, a, B, H, L, w, s);
+    if (st == LF_OK)
+        st = launch_attention_tc(q, k, v, qg, kg, vg, local_mask, global_mask, B, H, L, w, scale, dtype, out,
+                                 d->scratch, d->status, d->sm_count, s, &a);
+    if (st != LF_OK) scratch_dirty(d);
+    return st;
 }
 
 lf_status lf_release_scratch(void) {
@@ -197,6 +272,7 @@ lf_status lf_release_scratch(void) {
         cudaFree(d->scratch);
         d->scratch = nullptr;
         d->scratch_bytes = 0;
+        d->scratch_clean = 0;
     }
     return LF_OK;
 }

@@ -11,6 +11,11 @@
 // Key set (local row i >= g_b): [0, g_b) then [max(i - w, g_b), min(i + w,
 // L - 1)], each key once; global row i < g_b: [0, L) with qg/kg/vg.  Score
 // = scale * <q_i, k_j> + lb[j], lb[j] = fmaf(local_mask[j], 1e4, -1e4).
+// Global tokens at any position (the HuggingFace arrangement that the page's
+// §使用前提 item 4 sets apart): a row is global iff global_mask[i] == 0.0; a
+// local row's list is the sample's global positions global_idx[b, 0..g_b)
+// then its window [max(i - w, 0), min(i + w, L - 1)], where window keys that
+// are global are skipped (each key once).
 #include "lf_internal.h"
 
 namespace lf {
@@ -46,13 +51,22 @@ struct RowState {
 };
 
 // Keys at list positions [pos0, pos0 + 32) of one row (lane = key): the
-// row's key list is [0, g_seg) followed by [lo, hi], each key once.
+// row's key list is [0, g_seg) followed by [lo, hi], each key once.  With
+// kAny (global tokens at any position) the first g_seg entries are
+// gl[0..g_seg), and for a local row (skip_g) window keys with gm_row[j] == 0
+// (global, already listed) are skipped; a global row keeps all of [0, L).
+template <bool kAny>
 __device__ __forceinline__ void process_chunk(RowState& st, const float* sq, const float* K, const float* V,
                                               const float* lm_row, int pos0, int g_seg, int lo, int n_keys,
-                                              float scale, int lane) {
+                                              float scale, int lane, const int32_t* gl, const float* gm_row,
+                                              bool skip_g) {
     const int pos = pos0 + lane;
-    const bool valid = pos < n_keys;
-    const int j = valid ? (pos < g_seg ? pos : lo + (pos - g_seg)) : 0;
+    bool valid = pos < n_keys;
+    int j = valid ? (pos < g_seg ? (kAny ? gl[pos] : pos) : lo + (pos - g_seg)) : 0;
+    if (kAny && skip_g && valid && pos >= g_seg && gm_row[j] == 0.0f) {
+        valid = false;
+        j = 0;
+    }
     float s = -INFINITY;
     if (valid) {
         const float4* kr = reinterpret_cast<const float4*>(K + (size_t)j * 64);
@@ -93,12 +107,14 @@ __device__ __forceinline__ void process_chunk(RowState& st, const float* sq, con
 // each with its own online softmax, and warp 0 merges the partial (m, l, o)
 // through shared memory.  Many short chains per SM instead of one long one
 // keep the L2 latency of the K/V rows hidden, global rows included.
+template <bool kAny>
 __global__ void __launch_bounds__(kWarps * 32, 4)
 attention_simt_kernel(const float* __restrict__ q, const float* __restrict__ k, const float* __restrict__ v,
                       const float* __restrict__ qg, const float* __restrict__ kg,
                       const float* __restrict__ vg, const float* __restrict__ local_mask,
                       const float* __restrict__ global_mask, int B, int H, int L, int w, float scale,
-                      float* __restrict__ out, int* status) {
+                      float* __restrict__ out, int* status, const int32_t* __restrict__ gidx,
+                      const int32_t* __restrict__ gnum) {
     __shared__ __align__(16) float sq[64];
     __shared__ float part_ml[kWarps][2];
     __shared__ float part_o[kWarps][64];
@@ -112,11 +128,13 @@ attention_simt_kernel(const float* __restrict__ q, const float* __restrict__ k, 
         const float* gm_row = global_mask + (size_t)b * L;
         float* o = out + (((size_t)b * L + i) * H + h) * 64;
 
-        const int g = leading_globals(gm_row, L, w, lane);  // same in every warp
+        // gidx: global tokens at any position, g from the partition
+        const int g = kAny ? gnum[b] : leading_globals(gm_row, L, w, lane);  // same in every warp
         const bool bad_sample = g > w;
+        const int32_t* gl = kAny ? gidx + (size_t)b * L : nullptr;
         if (wid == 0) {
             if (bad_sample && lane == 0 && h == 0 && i == 0) record_status(status, b, LF_ERR_G_GT_W);
-            if (!bad_sample && i >= g && gm_row[i] == 0.0f && lane == 0 && h == 0)
+            if (!kAny && !bad_sample && i >= g && gm_row[i] == 0.0f && lane == 0 && h == 0)
                 record_status(status, b, LF_ERR_GLOBAL_NOT_PREFIX);
         }
         if (bad_sample || fmaf(lm_row[i], 10000.0f, -10000.0f) != 0.0f) {
@@ -126,7 +144,7 @@ attention_simt_kernel(const float* __restrict__ q, const float* __restrict__ k, 
             }
             continue;  // uniform over the CTA
         }
-        const bool global_row = i < g;
+        const bool global_row = kAny ? gm_row[i] == 0.0f : i < g;
         const size_t head = ((size_t)b * H + h) * (size_t)L * 64;
         const float* Q = (global_row ? qg : q) + head;
         const float* K = (global_row ? kg : k) + head;
@@ -138,19 +156,21 @@ attention_simt_kernel(const float* __restrict__ q, const float* __restrict__ k, 
         __syncthreads();
 
         // key list: global row [0, L); local row [0, g) then [max(i - w, g), min(i + w, L - 1)]
+        // (any position: global_idx[b, 0..g) then [max(i - w, 0), min(i + w, L - 1)])
         int g_seg, lo, n_keys;
         if (global_row) {
             g_seg = 0;
             lo = 0;
             n_keys = L;
         } else {
-            lo = max(i - w, g);
+            lo = max(i - w, kAny ? 0 : g);
             g_seg = g;
             n_keys = g + (min(i + w, L - 1) - lo + 1);
         }
         RowState st{-INFINITY, 0.0f, 0.0f, 0.0f};
         for (int pos0 = wid * 32; pos0 < n_keys; pos0 += kWarps * 32)
-            process_chunk(st, sq, K, V, lm_row, pos0, g_seg, lo, n_keys, scale, lane);
+            process_chunk<kAny>(st, sq, K, V, lm_row, pos0, g_seg, lo, n_keys, scale, lane, gl, gm_row,
+                                !global_row);
         if (lane == 0) {
             part_ml[wid][0] = st.m;
             part_ml[wid][1] = st.l;
@@ -184,12 +204,17 @@ attention_simt_kernel(const float* __restrict__ q, const float* __restrict__ k, 
 lf_status launch_attention_simt_f32(const float* q, const float* k, const float* v, const float* qg,
                                     const float* kg, const float* vg, const float* local_mask,
                                     const float* global_mask, int B, int H, int L, int w, float scale,
-                                    float* out, int* status, cudaStream_t stream) {
+                                    float* out, int* status, cudaStream_t stream, const AnyGlobals* any) {
     const long long rows = (long long)B * H * L;
     long long blocks = rows;
     if (blocks > 148 * 64) blocks = 148 * 64;
-    attention_simt_kernel<<<(int)blocks, kWarps * 32, 0, stream>>>(q, k, v, qg, kg, vg, local_mask, global_mask,
-                                                                  B, H, L, w, scale, out, status);
+    if (any)
+        attention_simt_kernel<true><<<(int)blocks, kWarps * 32, 0, stream>>>(
+            q, k, v, qg, kg, vg, local_mask, global_mask, B, H, L, w, scale, out, status, any->global_idx,
+            any->global_token_nums);
+    else
+        attention_simt_kernel<false><<<(int)blocks, kWarps * 32, 0, stream>>>(
+            q, k, v, qg, kg, vg, local_mask, global_mask, B, H, L, w, scale, out, status, nullptr, nullptr);
     return cudaGetLastError() == cudaSuccess ? LF_OK : LF_ERR_CUDA;
 }
 

@@ -120,6 +120,16 @@ struct Params {
     int* sched;      // [0] next item, [1] finished CTAs
     int* status;
     int* trace;      // diagnostic builds only: [CTA][16 roles][4] wait sites, then [CTA][16 roles][16] cycle counts
+    // Global tokens at any position (kernel instance kAny): the partition's
+    // outputs and the slot buffers gathered from them.  Global row tiles
+    // then hold slots (the c-th global token of the sample) instead of
+    // positions, and a band tile's global key blocks are slot blocks read
+    // from the compact k / v maps.
+    const int* gnum;    // [B] global tokens per sample
+    const int* gidx;    // [B][L] slot -> position (first gnum[b] entries)
+    const int* grank;   // [B][L + 1] global tokens before each position
+    const float* lm_c;  // [B][gcap] local_mask of each slot (0 past gnum[b])
+    int gcap;           // slots per (b, h) in the compact buffers
 };
 
 // Diagnostic builds (-DLF_TRACE=1) record per CTA and role the cycles spent
@@ -190,6 +200,7 @@ struct Params {
 
 struct Maps {
     CUtensorMap q, k, v, qg, kg, vg;
+    CUtensorMap kc, vc;  // kAny: k / v rows of the global tokens by slot (qg then also by slot)
 };
 
 struct Tile {
@@ -232,10 +243,20 @@ __device__ int leading_globals(const Params& p, int b) {
     return cap;
 }
 
+// Global tokens of sample b: the leading 0.0 entries of global_mask
+// (capped at w + 1), or with kAny the partition's count.
+template <bool kAny>
+__device__ __forceinline__ int sample_globals(const Params& p, int b) {
+    if constexpr (kAny) return p.gnum[b];
+    else return leading_globals(p, b);
+}
+
 // Whole warp: for each of the two band tiles starting at r0[x], does it have
 // a row g <= i < L that is not padded (work), and padded rows in [g, L)?
-// The local_mask loads of both tiles are issued before the global count is
-// needed, so the first plan of a sample costs one round of loads.
+// (kAny: any row i < L; rows of global tokens are left out of the output
+// later.)  The local_mask loads of both tiles are issued before the global
+// count is needed, so the first plan of a sample costs one round of loads.
+template <bool kAny>
 __device__ void band_rows2(const Params& p, int b, const int (&r0)[2], int& cached_b, int& g, int (&work)[2],
                            int (&padded)[2]) {
     const int lane = threadIdx.x & 31;
@@ -249,7 +270,7 @@ __device__ void band_rows2(const Params& p, int b, const int (&r0)[2], int& cach
             v[x][k] = i < p.L ? lm[i] : 1.0f;
         }
     if (b != cached_b) {
-        g = leading_globals(p, b);
+        g = sample_globals<kAny>(p, b);
         cached_b = b;
     }
 #pragma unroll
@@ -258,7 +279,7 @@ __device__ void band_rows2(const Params& p, int b, const int (&r0)[2], int& cach
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
             const int i = r0[x] + lane + 32 * k;
-            if (i < p.L && i >= g) {
+            if (i < p.L && (kAny || i >= g)) {
                 const bool tok = v[x][k] == 1.0f;
                 w_ |= tok;
                 pd |= !tok;
@@ -270,6 +291,7 @@ __device__ void band_rows2(const Params& p, int b, const int (&r0)[2], int& cach
 }
 
 // Whole warp: the item's plan (identical in every role).
+template <bool kAny>
 __device__ Plan make_plan(const Params& p, int id, int& cached_b, int& g) {
     Plan pl;
     pl.id = id;
@@ -311,12 +333,12 @@ __device__ Plan make_plan(const Params& p, int id, int& cached_b, int& g) {
     int work[2] = {0, 0}, padded[2] = {0, 0};
     if (pl.global) {
         if (pl.b != cached_b) {
-            g = leading_globals(p, pl.b);
+            g = sample_globals<kAny>(p, pl.b);
             cached_b = pl.b;
         }
     } else {
         const int r0[2] = {pl.t[0].r0, pl.t[1].r0};
-        band_rows2(p, pl.b, r0, cached_b, g, work, padded);
+        band_rows2<kAny>(p, pl.b, r0, cached_b, g, work, padded);
     }
     pl.g = g;
     pl.nloads = 0;
@@ -358,19 +380,26 @@ __device__ Plan make_plan(const Params& p, int id, int& cached_b, int& g) {
         const int lo = t.r0 - p.w;
         t.lo = lo <= 0 ? 0 : lo / kBN;
         t.hi = min(p.NKB - 1, (t.r0 + kBM - 1 + p.w) / kBN);
-        t.glob_hi = min((g + kBN - 1) / kBN, t.lo);
+        // Global key blocks: the blocks of positions [0, g) that the band
+        // does not load anyway; kAny: the slot blocks of [0, g), all of them
+        // (global tokens inside a row's window are masked in the slot block).
+        t.glob_hi = kAny ? (g + kBN - 1) / kBN : min((g + kBN - 1) / kBN, t.lo);
         G = max(G, t.glob_hi);
         lo_min = min(lo_min, t.lo);
         hi_max = max(hi_max, t.hi);
     }
     if (hi_max < 0) return pl;
-    pl.e1 = min(G, lo_min);
+    pl.e1 = kAny ? G : min(G, lo_min);
     pl.lo_min = lo_min;
     pl.nloads = pl.e1 + (hi_max - lo_min + 1);
     return pl;
 }
 
-__device__ __forceinline__ void load_at(const Plan& pl, int q, int& kb, int& needA, int& needB) {
+// Load q of an item: key block kb (a slot block of the compact maps when
+// cmp is set) and which tiles use it.
+template <bool kAny>
+__device__ __forceinline__ void load_at(const Plan& pl, int q, int& kb, int& needA, int& needB, int& cmp) {
+    cmp = 0;
     if (pl.global) {
         const int nA = pl.t[0].present ? pl.t[0].hi - pl.t[0].lo + 1 : 0;
         const int nB = pl.t[1].present ? pl.t[1].hi - pl.t[1].lo + 1 : 0;
@@ -391,8 +420,14 @@ __device__ __forceinline__ void load_at(const Plan& pl, int q, int& kb, int& nee
     kb = q < pl.e1 ? q : pl.lo_min + (q - pl.e1);
     const Tile& A = pl.t[0];
     const Tile& Bt = pl.t[1];
-    needA = A.present && (kb < A.glob_hi || (kb >= A.lo && kb <= A.hi));
-    needB = Bt.present && (kb < Bt.glob_hi || (kb >= Bt.lo && kb <= Bt.hi));
+    if (kAny && q < pl.e1) {  // slot block q
+        cmp = 1;
+        needA = A.present && q < A.glob_hi;
+        needB = Bt.present && q < Bt.glob_hi;
+        return;
+    }
+    needA = A.present && ((!kAny && kb < A.glob_hi) || (kb >= A.lo && kb <= A.hi));
+    needB = Bt.present && ((!kAny && kb < Bt.glob_hi) || (kb >= Bt.lo && kb <= Bt.hi));
 }
 
 // Key blocks of one tile of an item.
@@ -554,7 +589,9 @@ __device__ __forceinline__ uint32_t range_bits(int lo, int hi) {
     return low_bits(hi + 1) & ~low_bits(lo);
 }
 
-template <typename T>
+// kAny: global tokens at any position (slot-indexed global rows and global
+// key blocks, see Params); otherwise the global tokens are positions 0..g-1.
+template <typename T, bool kAny>
 __global__ void __launch_bounds__(kThreads, 1)
 attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Params p) {
     extern __shared__ uint8_t smem_raw[];
@@ -623,6 +660,10 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
         prefetch_tensormap(&maps.qg);
         prefetch_tensormap(&maps.kg);
         prefetch_tensormap(&maps.vg);
+        if (kAny) {
+            prefetch_tensormap(&maps.kc);
+            prefetch_tensormap(&maps.vc);
+        }
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, kTmemCols);
@@ -686,17 +727,17 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
                 // Every load of the plan is issued (the MMA warp maps a tile's
                 // blocks to ring stages by load index).
                 for (int q = 0; q < pl.nloads && ok; ++q) {
-                    int kb, nA, nB;
-                    load_at(pl, q, kb, nA, nB);
+                    int kb, nA, nB, cmp;
+                    load_at<kAny>(pl, q, kb, nA, nB, cmp);
+                    const CUtensorMap* mk = pl.global ? &maps.kg : (cmp ? &maps.kc : &maps.k);
+                    const CUtensorMap* mv = pl.global ? &maps.vg : (cmp ? &maps.vc : &maps.v);
                     const uint32_t st = kv_cnt % kStages;
                     TRACE(0, 13, pl.id, q, kv_cnt);
                     TIMED(2, ok = mbar_wait(&kv_empty[st], ((kv_cnt / kStages) & 1) ^ 1, abort_flag));
                     if (!ok) break;
                     mbar_arrive_expect_tx(&kv_full[st], 2 * kTileBytes);
-                    tma_load_3d(smem + kOffK + st * kTileBytes, pl.global ? &maps.kg : &maps.k, &kv_full[st], 0,
-                                kb * kBN, pl.bh);
-                    tma_load_3d(smem + kOffV + st * kTileBytes, pl.global ? &maps.vg : &maps.v, &kv_full[st], 0,
-                                kb * kBN, pl.bh);
+                    tma_load_3d(smem + kOffK + st * kTileBytes, mk, &kv_full[st], 0, kb * kBN, pl.bh);
+                    tma_load_3d(smem + kOffV + st * kTileBytes, mv, &kv_full[st], 0, kb * kBN, pl.bh);
                     ++kv_cnt;
                 }
                 if (ok) mbar_arrive(tma_done);
@@ -741,7 +782,7 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
             id = __shfl_sync(0xffffffffu, id, 0);
             if (!ok) break;
             Plan pl;
-            if (id >= 0) pl = make_plan(p, id, cached_b, g);
+            if (id >= 0) pl = make_plan<kAny>(p, id, cached_b, g);
             else pl.id = -1;
             if (lane == 0) {
                 plans[slot] = pl;
@@ -818,6 +859,7 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
                 // load index of this tile's block j
                 auto load_idx = [&](int j) -> int {
                     if (glob) return j < m ? 2 * j + x : m + j;
+                    if (kAny) return j < gh ? j : e1 + (lo + (j - gh) - lo_min);  // slot blocks first
                     const int kb = j < gh ? j : lo + (j - gh);
                     return kb < e1 ? kb : e1 + (kb - lo_min);
                 };
@@ -825,8 +867,9 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
                 auto mine = [&](int q) -> bool {
                     if (nx == 0) return false;
                     if (glob) return q < 2 * m ? (q & 1) == x : nx > m;
+                    if (kAny && q < e1) return q < gh;
                     const int kb = q < e1 ? q : lo_min + (q - e1);
-                    return kb < gh || (kb >= lo && kb <= hi);
+                    return (!kAny && kb < gh) || (kb >= lo && kb <= hi);
                 };
                 int q_ready = -1;
                 // wait for loads up to q; loads this tile does not use are released at once
@@ -912,6 +955,8 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
             const int g = pl.g;
             const Tile& me = pl.t[x];
             const float* lm = p.local_mask + (size_t)pl.b * p.L;
+            // kAny: local_mask of the slots (global rows, slot key blocks)
+            const float* lmc = kAny ? p.lm_c + (size_t)pl.b * p.gcap : nullptr;
             const int i = me.r0 + r;
             // Only these few scalars stay live through the block loop.
             const int is_global = pl.global;
@@ -919,7 +964,24 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
 
             // Does this warp have rows whose output is kept?
             const int wr0 = me.r0 + sp * 32;
-            const bool row_kept = is_global ? (i < g && lm[i] == 1.0f) : (i < p.L && i >= g && lm[i] == 1.0f);
+            bool row_kept;
+            // kAny band rows: the slots [clo, chi) of the global tokens inside
+            // the row's window, which the band blocks already hold
+            int clo = 0, chi = 0;
+            if (is_global) {
+                row_kept = i < g && (kAny ? lmc[i] : lm[i]) == 1.0f;
+            } else if (kAny) {
+                row_kept = false;
+                if (i < p.L) {
+                    const int* rk = p.grank + (size_t)pl.b * (p.L + 1);
+                    const float lmi = lm[i], gmi = p.global_mask[(size_t)pl.b * p.L + i];
+                    clo = rk[max(0, i - p.w)];
+                    chi = rk[min(p.L, i + p.w + 1)];
+                    row_kept = lmi == 1.0f && gmi != 0.0f;
+                }
+            } else {
+                row_kept = i < p.L && i >= g && lm[i] == 1.0f;
+            }
             const bool warp_active = __any_sync(0xffffffffu, row_kept);
 
             float m_used = -INFINITY, l_run = 0.0f;
@@ -935,10 +997,12 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
                     for (int u = 0; u < 8; ++u) {
                         const int j = j0 + u;
                         const int c2 = (j < blk_gh ? j : blk_lo + (j - blk_gh)) * kBN;
+                        const bool cmp = kAny && !is_global && j < blk_gh;  // slot block
 #pragma unroll
                         for (int t = 0; t < 4; ++t) {
                             const int key = c2 + t * 32 + lane;
-                            v[u][t] = (j < nblk && key < p.L) ? lm[key] : 1.0f;
+                            if (kAny && cmp) v[u][t] = (j < nblk && key < g) ? lmc[key] : 1.0f;
+                            else v[u][t] = (j < nblk && key < p.L) ? lm[key] : 1.0f;
                         }
                     }
 #pragma unroll
@@ -954,14 +1018,17 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
 #endif
                 const bool first = n == 0;
                 const int kb = n < blk_gh ? n : blk_lo + (n - blk_gh);
-                const int c0 = kb * kBN;
+                const int c0 = kb * kBN;  // first key (kAny slot block: first slot)
+                const bool cmp = kAny && !is_global && n < blk_gh;
                 // Padding bias of the block's keys (keys >= L are masked instead).
                 const bool has_pad = warp_active && (n >= 32 || ((padbits >> n) & 1u));
                 if (has_pad) {
 #pragma unroll
                     for (int t = 0; t < 4; ++t) {
                         const int key = c0 + t * 32 + lane;
-                        const float mv = key < p.L ? lm[key] : 1.0f;
+                        float mv;
+                        if (kAny && cmp) mv = key < g ? lmc[key] : 1.0f;
+                        else mv = key < p.L ? lm[key] : 1.0f;
                         bias_w[t * 32 + lane] = fmaf(mv, 10000.0f, -10000.0f) * p.inv_scale;
                     }
                     __syncwarp();
@@ -975,13 +1042,15 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
                 for (int ch = 0; ch < 4; ++ch) {
                     const int cj0 = c0 + ch * 32;
                     int s;
-                    if (cj0 >= p.L) {
+                    if (kAny && cmp) {
+                        s = cj0 >= g ? kSkip : kPart;  // slots past g; window overlap per row
+                    } else if (cj0 >= p.L) {
                         s = kSkip;
                     } else if (is_global) {
                         s = (cj0 + 31 < p.L) ? kFull : kPart;
                     } else {
-                        const bool any_g = cj0 < g;
-                        const bool all_g = cj0 + 31 < g;
+                        const bool any_g = !kAny && cj0 < g;
+                        const bool all_g = !kAny && cj0 + 31 < g;
                         const bool overlap = cj0 <= wr0 + 31 + p.w && cj0 + 31 >= wr0 - p.w;
                         const bool inside = (wr0 + 31 - cj0 <= p.w) && (cj0 + 31 - wr0 <= p.w);
                         if (!any_g && !overlap) s = kSkip;
@@ -1038,8 +1107,13 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
                     const int lo_c = d0 - p.w, hi_c = d0 + p.w, gl_c = g - c0, lim_c = p.L - c0;
                     auto chunk_bits = [&](int ch) -> uint32_t {
                         const int b0 = ch * 32;
+                        if (kAny && cmp)  // slots < g outside the row's window
+                            return low_bits(gl_c - b0) & ~range_bits(clo - c0 - b0, chi - 1 - c0 - b0);
                         uint32_t bits = low_bits(lim_c - b0);
-                        if (!is_global) bits &= low_bits(gl_c - b0) | range_bits(lo_c - b0, hi_c - b0);
+                        if (!is_global) {
+                            if (kAny) bits &= range_bits(lo_c - b0, hi_c - b0);
+                            else bits &= low_bits(gl_c - b0) | range_bits(lo_c - b0, hi_c - b0);
+                        }
                         return bits;
                     };
                     // bias and mask of chunk ch, applied to raw scores in r
@@ -1214,9 +1288,20 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
                 // their latency is hidden; a global_mask 0.0 past the prefix
                 // is recorded at the end of the tile.
                 const bool in_row = me.r0 < p.L && i < p.L;
-                const float lmi = in_row ? lm[i] : 1.0f;
+                // kAny global tiles hold slots: their local_mask values and
+                // the positions their rows are written to
+                float lmi;
+                int pos = i;
+                if (kAny && pl.global) {
+                    lmi = i < p.gcap ? p.lm_c[(size_t)pl.b * p.gcap + i] : 0.0f;
+                    if (i < g && g <= p.w) pos = p.gidx[(size_t)pl.b * p.L + i];
+                } else {
+                    lmi = in_row ? lm[i] : 1.0f;
+                }
                 const float gmi = (in_row && !pl.global) ? p.global_mask[(size_t)pl.b * p.L + i] : 1.0f;
-                const bool not_prefix = !pl.global && g <= p.w && in_row && i >= g;
+                // band rows whose output this tile writes (not global tokens)
+                const bool local_row = kAny ? gmi != 0.0f : i >= g;
+                const bool not_prefix = !kAny && !pl.global && g <= p.w && in_row && i >= g;
                 if (!pl.global) {
                     if (g > p.w) {  // invalid sample: zero output, record once
                         if (in_row) store_zero_row(p.out, ((size_t)(pl.b * p.L + i) * p.H + pl.h) * kHD, sizeof(T));
@@ -1224,7 +1309,7 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
                         continue;
                     }
                     if (pl.zero_only[x]) {
-                        if (in_row && i >= g && lmi != 1.0f)
+                        if (in_row && local_row && lmi != 1.0f)
                             store_zero_row(p.out, ((size_t)(pl.b * p.L + i) * p.H + pl.h) * kHD, sizeof(T));
                         if (not_prefix && gmi == 0.0f) record_status(p.status, pl.b, LF_ERR_GLOBAL_NOT_PREFIX);
                         continue;
@@ -1273,7 +1358,7 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
 #endif
 
                 if (!pl.global) {
-                    if (in_row && i >= g) {
+                    if (in_row && local_row) {
                         const size_t off = ((size_t)(pl.b * p.L + i) * p.H + pl.h) * kHD;
                         if (lmi != 1.0f) store_zero_row(p.out, off, sizeof(T));
                         else store_row<T>(p.out, off, o, fast_rcp(ml.y));
@@ -1309,7 +1394,7 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
                     if (last) {
                         __threadfence();
                         if (i < g) {
-                            const size_t off = ((size_t)(pl.b * p.L + i) * p.H + pl.h) * kHD;
+                            const size_t off = ((size_t)(pl.b * p.L + pos) * p.H + pl.h) * kHD;
                             if (lmi != 1.0f) {
                                 store_zero_row(p.out, off, sizeof(T));
                             } else {
@@ -1557,6 +1642,16 @@ int current_sm_count() {
     return sms[dev];
 }
 
+template <typename T, bool kAny>
+void launch_instance(int grid, const Maps& maps, const Params& p, cudaStream_t stream) {
+    static bool attr = false;  // the shared-memory opt-in, once per instance
+    if (!attr) {
+        cudaFuncSetAttribute(attention_tc_kernel<T, kAny>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+        attr = true;
+    }
+    attention_tc_kernel<T, kAny><<<grid, kThreads, kSmemBytes, stream>>>(maps, p);
+}
+
 struct Geometry {
     int NKB, NT, RT, NS, NSP, NTP, chunk;
     size_t sched_bytes, counters_bytes, part_o_bytes, part_ml_bytes;
@@ -1594,13 +1689,22 @@ size_t attention_tc_scratch_zero_bytes(int B, int H, int L, int w) {
 lf_status launch_attention_tc(const void* q, const void* k, const void* v, const void* qg, const void* kg,
                               const void* vg, const float* local_mask, const float* global_mask, int B, int H,
                               int L, int w, float scale, lf_dtype dtype, void* out, void* scratch, int* status,
-                              int sm_count, cudaStream_t stream) {
+                              int sm_count, cudaStream_t stream, const AnyGlobals* any) {
     const Geometry geo = geometry(B, H, L, w, sm_count);
     Maps maps;
     const int BH = B * H;
     if (!make_map(&maps.q, q, BH, L) || !make_map(&maps.k, k, BH, L) || !make_map(&maps.v, v, BH, L) ||
-        !make_map(&maps.qg, qg, BH, L) || !make_map(&maps.kg, kg, BH, L) || !make_map(&maps.vg, vg, BH, L))
+        !make_map(&maps.kg, kg, BH, L) || !make_map(&maps.vg, vg, BH, L))
         return LF_ERR_CUDA;
+    if (any) {  // global rows and global key blocks by slot
+        if (!make_map(&maps.qg, any->qg_c, BH, any->gcap) || !make_map(&maps.kc, any->k_c, BH, any->gcap) ||
+            !make_map(&maps.vc, any->v_c, BH, any->gcap))
+            return LF_ERR_CUDA;
+    } else {
+        if (!make_map(&maps.qg, qg, BH, L)) return LF_ERR_CUDA;
+        maps.kc = maps.k;
+        maps.vc = maps.v;
+    }
     Params p;
     p.B = B;
     p.H = H;
@@ -1628,26 +1732,22 @@ lf_status launch_attention_tc(const void* q, const void* k, const void* v, const
     p.part_ml = reinterpret_cast<float*>(s + geo.sched_bytes + geo.counters_bytes + geo.part_o_bytes);
     p.status = status;
     p.trace = nullptr;
+    p.gnum = any ? any->global_token_nums : nullptr;
+    p.gidx = any ? any->global_idx : nullptr;
+    p.grank = any ? any->rank : nullptr;
+    p.lm_c = any ? any->lm_c : nullptr;
+    p.gcap = any ? any->gcap : 0;
 #if LF_TRACE
     if (const char* a = getenv("LF_TRACE_ADDR")) p.trace = reinterpret_cast<int*>(strtoull(a, nullptr, 10));
 #endif
 
     const int grid = p.n_items < sm_count ? p.n_items : sm_count;
     if (dtype == LF_F16) {
-        static bool attr = false;
-        if (!attr) {
-            cudaFuncSetAttribute(attention_tc_kernel<__half>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-            attr = true;
-        }
-        attention_tc_kernel<__half><<<grid, kThreads, kSmemBytes, stream>>>(maps, p);
+        if (any) launch_instance<__half, true>(grid, maps, p, stream);
+        else launch_instance<__half, false>(grid, maps, p, stream);
     } else {
-        static bool attr = false;
-        if (!attr) {
-            cudaFuncSetAttribute(attention_tc_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 kSmemBytes);
-            attr = true;
-        }
-        attention_tc_kernel<__nv_bfloat16><<<grid, kThreads, kSmemBytes, stream>>>(maps, p);
+        if (any) launch_instance<__nv_bfloat16, true>(grid, maps, p, stream);
+        else launch_instance<__nv_bfloat16, false>(grid, maps, p, stream);
     }
     return cudaGetLastError() == cudaSuccess ? LF_OK : LF_ERR_CUDA;
 }

@@ -8,7 +8,12 @@
 // (descending), which is the output order of a stable flagged partition that
 // writes rejected items from the end.  The CTA also checks the page's
 // constraints 3 and 4 (§使用前提): the flagged positions must be exactly
-// 0..g-1 and g <= w.
+// 0..g-1 (unless global tokens may lie anywhere) and g <= w.
+//
+// For global tokens at any position the same scan also gives the rank table
+// rank[b, j] = flagged positions before j (j = 0..L, rank[b, L] = g), from
+// which a row's window [i - w, i + w] maps to the range [rank[i - w],
+// rank[i + w + 1]) of global-token slots it covers.
 //
 // The work is one pass over the mask: L * 4 bytes read, L * 4 bytes written
 // per sample -- HBM-bound and tiny next to the attention kernel.
@@ -22,10 +27,12 @@ constexpr int kItems = 4;
 
 __global__ void __launch_bounds__(kThreads)
 global_idx_kernel(const float* __restrict__ global_mask, int L, int w, int32_t* __restrict__ global_idx,
-                  int32_t* __restrict__ global_token_nums, int* status) {
+                  int32_t* __restrict__ global_token_nums, int32_t* __restrict__ rank, int require_prefix,
+                  int* status) {
     const int b = blockIdx.x;
     const float* row = global_mask + (size_t)b * L;
     int32_t* idx = global_idx + (size_t)b * L;
+    int32_t* rk = rank ? rank + (size_t)b * (L + 1) : nullptr;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
     __shared__ int warp_tot[kThreads / 32 + 1];
@@ -80,6 +87,7 @@ global_idx_kernel(const float* __restrict__ global_mask, int L, int w, int32_t* 
         for (int t = 0; t < kItems; ++t) {
             const int j = j0 + t;
             if (j < L) {
+                if (rk) rk[j] = sel;
                 if (f[t]) {
                     idx[sel] = j;
                     ++sel;
@@ -93,7 +101,8 @@ global_idx_kernel(const float* __restrict__ global_mask, int L, int w, int32_t* 
     }
     if (tid == 0) {
         global_token_nums[b] = base;
-        if (first_unflagged < base) record_status(status, b, LF_ERR_GLOBAL_NOT_PREFIX);
+        if (rk) rk[L] = base;
+        if (require_prefix && first_unflagged < base) record_status(status, b, LF_ERR_GLOBAL_NOT_PREFIX);
         else if (base > w) record_status(status, b, LF_ERR_G_GT_W);
     }
 }
@@ -101,8 +110,104 @@ global_idx_kernel(const float* __restrict__ global_mask, int L, int w, int32_t* 
 }  // namespace
 
 lf_status launch_global_idx(const float* global_mask, int B, int L, int w, int32_t* global_idx,
-                            int32_t* global_token_nums, int* status, cudaStream_t stream) {
-    global_idx_kernel<<<B, kThreads, 0, stream>>>(global_mask, L, w, global_idx, global_token_nums, status);
+                            int32_t* global_token_nums, int* status, cudaStream_t stream, int32_t* rank,
+                            bool require_prefix) {
+    global_idx_kernel<<<B, kThreads, 0, stream>>>(global_mask, L, w, global_idx, global_token_nums, rank,
+                                                  require_prefix ? 1 : 0, status);
+    return cudaGetLastError() == cudaSuccess ? LF_OK : LF_ERR_CUDA;
+}
+
+}  // namespace lf
+
+// ---------------------------------------------------------------- global tokens at any position
+//
+// The tensor-core attention kernel reads the global tokens' rows through
+// compact per-head buffers: slot c of sample b holds the row of position
+// global_idx[b, c] (the c-th global token), so that the global rows form
+// whole 128-row query tiles and the global keys whole 128-key blocks, each
+// one TMA box, wherever the tokens lie in the sequence.
+
+namespace lf {
+namespace {
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// One CTA of 256 threads per 32 slots of one (b, h): thread t copies the
+// 16-byte column part t % 8 of slot c0 + t / 8 for qg, k and v; slots past
+// g are zero (finite rows for the masked tail of a block).  The h == 0 CTAs
+// also write the slots' local_mask values.
+__global__ void __launch_bounds__(256)
+gather_globals_kernel(const uint4* __restrict__ qg, const uint4* __restrict__ k, const uint4* __restrict__ v,
+                      const float* __restrict__ local_mask, const int32_t* __restrict__ gidx,
+                      const int32_t* __restrict__ gnum, int H, int L, int gcap, uint4* __restrict__ qg_c,
+                      uint4* __restrict__ k_c, uint4* __restrict__ v_c, float* __restrict__ lm_c) {
+    const int per = gcap / 32;  // CTAs per (b, h)
+    const int bh = blockIdx.x / per, b = bh / H, h = bh % H;
+    const int c0 = (blockIdx.x % per) * 32;
+    const int c = c0 + (threadIdx.x >> 3), part = threadIdx.x & 7;
+    // a sample with g > w is rejected by the attention kernel; min() keeps
+    // the slots in range (c < g <= L also keeps the index read in range)
+    const int g = min(gnum[b], gcap);
+    const size_t dst = ((size_t)bh * gcap + c) * 8 + part;
+    if (c < g) {
+        const int j = gidx[(size_t)b * L + c];
+        const size_t src = ((size_t)bh * L + j) * 8 + part;
+        const uint4 a = qg[src], kk = k[src], vv = v[src];
+        qg_c[dst] = a;
+        k_c[dst] = kk;
+        v_c[dst] = vv;
+    } else {
+        const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+        qg_c[dst] = z;
+        k_c[dst] = z;
+        v_c[dst] = z;
+    }
+    if (h == 0 && threadIdx.x < 32) {
+        const int cc = c0 + threadIdx.x;
+        lm_c[(size_t)b * gcap + cc] = cc < g ? local_mask[(size_t)b * L + gidx[(size_t)b * L + cc]] : 0.0f;
+    }
+}
+
+}  // namespace
+
+size_t any_globals_bytes(int B, int H, int L, int w, bool compact) {
+    size_t n = align256((size_t)B * L * 4) + align256((size_t)B * 4) + align256((size_t)B * (L + 1) * 4);
+    if (compact) {
+        const size_t gcap = (size_t)any_globals_gcap(w);
+        n += 3 * align256((size_t)B * H * gcap * 64 * 2) + align256((size_t)B * gcap * 4);
+    }
+    return n;
+}
+
+AnyGlobals any_globals_layout(void* base, int B, int H, int L, int w, bool compact) {
+    AnyGlobals a{};
+    uint8_t* s = reinterpret_cast<uint8_t*>(base);
+    a.global_idx = reinterpret_cast<int32_t*>(s);
+    s += align256((size_t)B * L * 4);
+    a.global_token_nums = reinterpret_cast<int32_t*>(s);
+    s += align256((size_t)B * 4);
+    a.rank = reinterpret_cast<int32_t*>(s);
+    s += align256((size_t)B * (L + 1) * 4);
+    a.gcap = any_globals_gcap(w);
+    if (compact) {
+        const size_t tb = align256((size_t)B * H * a.gcap * 64 * 2);
+        a.qg_c = s;
+        a.k_c = s + tb;
+        a.v_c = s + 2 * tb;
+        a.lm_c = reinterpret_cast<float*>(s + 3 * tb);
+    }
+    return a;
+}
+
+lf_status launch_gather_globals(const void* qg, const void* k, const void* v, const float* local_mask,
+                                const AnyGlobals& a, int B, int H, int L, int w, cudaStream_t stream) {
+    (void)w;
+    const long long blocks = (long long)B * H * (a.gcap / 32);
+    if (blocks >= (1LL << 31)) return LF_ERR_TOO_LARGE;
+    gather_globals_kernel<<<(unsigned)blocks, 256, 0, stream>>>(
+        reinterpret_cast<const uint4*>(qg), reinterpret_cast<const uint4*>(k), reinterpret_cast<const uint4*>(v),
+        local_mask, a.global_idx, a.global_token_nums, H, L, a.gcap, reinterpret_cast<uint4*>(a.qg_c),
+        reinterpret_cast<uint4*>(a.k_c), reinterpret_cast<uint4*>(a.v_c), a.lm_c);
     return cudaGetLastError() == cudaSuccess ? LF_OK : LF_ERR_CUDA;
 }
 

@@ -26,6 +26,9 @@ struct DeviceCtx {
     int* status = nullptr;  // device word, see LF_STATUS_CLEAR
     void* scratch = nullptr;
     size_t scratch_bytes = 0;
+    // Leading bytes of the scratch known to be zero when the next call
+    // starts (the attention kernel's scheduler and split counters must be).
+    size_t scratch_clean = 0;
     // encoder layer: a second stream (and its fork/join events) on which a
     // small GEMM runs beside a large one
     cudaStream_t side = nullptr;
@@ -37,19 +40,56 @@ DeviceCtx* current_device(lf_status* st);
 // Make sure the current device's library scratch holds `bytes` (grows by
 // cudaMalloc; the new region is zeroed).
 lf_status ensure_scratch(DeviceCtx* dev, size_t bytes);
+// Before an attention launch on the library scratch: clears its first
+// `zero_bytes` on `stream` unless they are known to be zero already, and
+// records that after the launch only they are (the kernel re-zeroes its
+// counters; what follows them is written).
+lf_status prepare_scratch_counters(DeviceCtx* dev, size_t zero_bytes, cudaStream_t stream);
+// Records that a call wrote the scratch from its start (nothing is known
+// to be zero any more).
+void scratch_dirty(DeviceCtx* dev);
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 lf_status check_shape(int B, int H, int L, int w);
 
 // ---- launchers (return LF_OK or LF_ERR_CUDA) ----
+// rank (may be NULL): [B][L + 1] global tokens before each position.
+// require_prefix: record LF_ERR_GLOBAL_NOT_PREFIX for global tokens that are
+// not positions 0..g-1.
 lf_status launch_global_idx(const float* global_mask, int B, int L, int w, int32_t* global_idx,
-                            int32_t* global_token_nums, int* status, cudaStream_t stream);
+                            int32_t* global_token_nums, int* status, cudaStream_t stream,
+                            int32_t* rank = nullptr, bool require_prefix = true);
 
+// Global tokens at any position: the partition's outputs and the rows of
+// the global tokens gathered from them into compact per-head buffers (slot
+// c = the c-th global token of the sample, slots g..gcap-1 zero).
+struct AnyGlobals {
+    const int32_t* global_idx;         // [B][L]
+    const int32_t* global_token_nums;  // [B]
+    const int32_t* rank;               // [B][L + 1]
+    void* qg_c;                        // [B*H][gcap][64] dtype
+    void* k_c;                         // [B*H][gcap][64] dtype
+    void* v_c;                         // [B*H][gcap][64] dtype
+    float* lm_c;                       // [B][gcap]: local_mask of each slot (0 past g)
+    int gcap;                          // w rounded up to a multiple of 128
+};
+inline int any_globals_gcap(int w) { return (w + 127) / 128 * 128; }
+// Bytes of the partition outputs and compact buffers (each part 256-aligned).
+size_t any_globals_bytes(int B, int H, int L, int w, bool compact);
+// Carves an AnyGlobals out of `base` (any_globals_bytes(..) bytes).
+AnyGlobals any_globals_layout(void* base, int B, int H, int L, int w, bool compact);
+// 16-bit dtypes: fills qg_c, k_c, v_c and lm_c from the partition's outputs.
+lf_status launch_gather_globals(const void* qg, const void* k, const void* v, const float* local_mask,
+                                const AnyGlobals& a, int B, int H, int L, int w, cudaStream_t stream);
+
+// any (may be NULL): global tokens at any position (global_idx and
+// global_token_nums are used).
 lf_status launch_attention_simt_f32(const float* q, const float* k, const float* v, const float* qg,
                                     const float* kg, const float* vg, const float* local_mask,
                                     const float* global_mask, int B, int H, int L, int w,
-                                    float scale, float* out, int* status, cudaStream_t stream);
+                                    float scale, float* out, int* status, cudaStream_t stream,
+                                    const AnyGlobals* any = nullptr);
 
 // Tensor-core path (fp16 / bf16).  `scratch` must hold
 // attention_tc_scratch_bytes(B, H, L, w) bytes whose counter region is zero
@@ -58,11 +98,13 @@ size_t attention_tc_scratch_bytes(int B, int H, int L, int w);
 // Leading part of that scratch (scheduler and split counters) that must be
 // zero when a launch starts.
 size_t attention_tc_scratch_zero_bytes(int B, int H, int L, int w);
+// any (may be NULL): global tokens at any position, with the compact
+// buffers filled by launch_gather_globals.
 lf_status launch_attention_tc(const void* q, const void* k, const void* v, const void* qg,
                               const void* kg, const void* vg, const float* local_mask,
                               const float* global_mask, int B, int H, int L, int w, float scale,
                               lf_dtype dtype, void* out, void* scratch, int* status,
-                              int sm_count, cudaStream_t stream);
+                              int sm_count, cudaStream_t stream, const AnyGlobals* any = nullptr);
 
 // ---- dense GEMM with fused epilogues (encoder layer) ----
 enum { kEpiHeads = 0, kEpiGelu = 1, kEpiResid = 2 };

@@ -13,6 +13,9 @@ Workloads (all head_dim 64; values ~ N(0, 1) * 0.5 rounded to the dtype):
   5  fp16  one encoder layer: B=1 L=4096 hidden 1024 (16 x 64) FFN 4096,
            w=256 g=64; x ~ N(0,1), weights ~ N(0, 0.02), biases 0,
            LayerNorm gamma 1 beta 0.
+  6  fp16  workload 2 with its 64 global tokens at seeded random positions
+           among the unpadded ones (the HuggingFace arrangement), for the
+           entry point that takes global tokens at any position.
 Mask conventions follow the FasterTransformer Longformer page's input list:
 local_mask 1.0 = token / 0.0 = padding; global_mask 0.0 = global /
 -10000.0 = not global.
@@ -40,6 +43,7 @@ class Workload:
     g: List[int] = field(default_factory=list)
     pad: List[int] = field(default_factory=list)
     seed: int = 0
+    scattered: bool = False  # global tokens at random positions (masks_scattered)
 
 
 def workload(cid: int) -> Workload:
@@ -62,6 +66,9 @@ def workload(cid: int) -> Workload:
     if cid == 5:
         return Workload(5, "fp16 encoder layer B1 L4096 hidden1024 H16 w256 g64 ffn4096", "f16",
                         1, 16, 4096, 256, [64], [0], 1005)
+    if cid == 6:
+        return Workload(6, "fp16 B1 H16 L4096 w256 64 globals at random positions pad300", "f16",
+                        1, 16, 4096, 256, [64], [300], 1006, scattered=True)
     raise ValueError("unknown workload %r" % cid)
 
 
@@ -74,6 +81,22 @@ def masks(B: int, L: int, g: List[int], pad: List[int]):
         if pad[b] > 0:
             local[b, L - pad[b]:] = 0.0
         glob[b, :g[b]] = 0.0
+    return local, glob
+
+
+def masks_scattered(B: int, L: int, g: List[int], pad: List[int], seed: int, padded_globals: int = 0):
+    """local_mask / global_mask [B, L] float32 with g[b] global tokens at
+    positions drawn without replacement from the unpadded ones [0, L -
+    pad[b]) (torch.Generator(seed), sample by sample), a padding tail of
+    pad[b] positions, and padded_globals of each sample's global tokens also
+    marked as padding."""
+    gen = torch.Generator().manual_seed(seed)
+    local, glob = masks(B, L, [0] * B, pad)
+    for b in range(B):
+        pos = torch.randperm(L - pad[b], generator=gen)[:g[b]]
+        glob[b, pos] = 0.0
+        if padded_globals:
+            local[b, pos[:padded_globals]] = 0.0
     return local, glob
 
 
@@ -92,7 +115,10 @@ def workload_inputs(cid: int, device: str = "cpu"):
     """(Workload, tensors dict, local_mask, global_mask) for workload cid."""
     wl = workload(cid)
     t = attention_inputs(wl.B, wl.H, wl.L, wl.dtype, wl.seed, device=device)
-    lm, gm = masks(wl.B, wl.L, wl.g, wl.pad)
+    if wl.scattered:
+        lm, gm = masks_scattered(wl.B, wl.L, wl.g, wl.pad, wl.seed + 1)
+    else:
+        lm, gm = masks(wl.B, wl.L, wl.g, wl.pad)
     return wl, t, lm.to(device), gm.to(device)
 
 

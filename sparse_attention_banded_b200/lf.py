@@ -57,6 +57,10 @@ def lib():
         L.lf_attention_forward.restype = st
         L.lf_attention_scratch_bytes.argtypes = [i, i, i, i, i]
         L.lf_attention_scratch_bytes.restype = ctypes.c_size_t
+        L.lf_attention_forward_any_globals.argtypes = [vp] * 8 + [i, i, i, i, i, vp, vp]
+        L.lf_attention_forward_any_globals.restype = st
+        L.lf_attention_any_globals_scratch_bytes.argtypes = [i, i, i, i, i]
+        L.lf_attention_any_globals_scratch_bytes.restype = ctypes.c_size_t
         L.lf_release_scratch.restype = st
         L.lf_attention_forward_noalloc.argtypes = [vp] * 8 + [i, i, i, i, i, vp, vp]
         L.lf_attention_forward_noalloc.restype = st
@@ -142,6 +146,25 @@ def lf_attention_forward(q, k, v, qg, kg, vg, local_mask, global_mask, w: int, o
 
 def lf_attention_scratch_bytes(B: int, H: int, L: int, w: int, dtype) -> int:
     return lib().lf_attention_scratch_bytes(B, H, L, w, DTYPE_CODE[dtype])
+
+
+def lf_attention_forward_any_globals(q, k, v, qg, kg, vg, local_mask, global_mask, w: int, out=None,
+                                     stream=None):
+    """Same as :func:`lf_attention_forward` with the global tokens
+    (global_mask == 0.0) at any positions of the sequence."""
+    B, H, L, _ = q.shape
+    if out is None:
+        out = torch.empty(B, L, H * 64, dtype=q.dtype, device=q.device)
+    code = DTYPE_CODE.get(q.dtype, 99)
+    st = lib().lf_attention_forward_any_globals(_ptr(q), _ptr(k), _ptr(v), _ptr(qg), _ptr(kg), _ptr(vg),
+                                                _ptr(local_mask), _ptr(global_mask), B, H, L, w, code,
+                                                _stream(stream), _ptr(out))
+    _check(st, "lf_attention_forward_any_globals")
+    return out
+
+
+def lf_attention_any_globals_scratch_bytes(B: int, H: int, L: int, w: int, dtype) -> int:
+    return lib().lf_attention_any_globals_scratch_bytes(B, H, L, w, DTYPE_CODE[dtype])
 
 
 def lf_release_scratch():

@@ -37,6 +37,26 @@ def flops(B: int, H: int, L: int, w: int, g_list, pad_list) -> float:
     return 4.0 * 64 * H * total
 
 
+def flops_masks(local_mask, global_mask, H: int, w: int) -> float:
+    """F for any masks, global tokens at any position: G_b = {j : global_mask
+    == 0.0}; a local row's key set is its window united with G_b (each key
+    once), a global row's is all L keys; unpadded query rows only."""
+    lm = np.asarray(local_mask, dtype=np.float32)
+    gm = np.asarray(global_mask, dtype=np.float32)
+    B, L = lm.shape
+    i = np.arange(L)
+    lo = np.maximum(0, i - w)
+    hi = np.minimum(L - 1, i + w)
+    total = 0
+    for b in range(B):
+        G = gm[b] == 0.0
+        before = np.concatenate([[0], np.cumsum(G)])  # global tokens before each position
+        in_window = before[hi + 1] - before[lo]
+        sizes = (hi - lo + 1) + int(G.sum()) - in_window
+        total += int(np.where(G, L, sizes)[lm[b] == 1.0].sum())
+    return 4.0 * 64 * H * total
+
+
 def algorithmic_bytes(B: int, H: int, L: int, w: int, g_list, dtype: str) -> float:
     e = ELEM[dtype]
     full = 5 * B * H * L * 64 * e

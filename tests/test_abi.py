@@ -55,6 +55,44 @@ def test_attention_host_validation(L, kw, status):
     assert _attn(L, **kw) == status
 
 
+def _attn_any(L, B=1, H=1, Ln=512, w=64, dtype=1, ptrs=None, out=FAKE):
+    p = ptrs or [FAKE] * 8
+    return L.lf_attention_forward_any_globals(*[ctypes.c_void_p(x) for x in p], B, H, Ln, w, dtype, None,
+                                              ctypes.c_void_p(out))
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(ptrs=[FAKE] * 7 + [0]), 1),
+    (dict(ptrs=[0] + [FAKE] * 7), 1),
+    (dict(out=0), 1),
+    (dict(B=0), 2), (dict(H=-1), 2), (dict(w=0), 2), (dict(Ln=0), 2),
+    (dict(Ln=500, w=64), 3),
+    (dict(Ln=64, w=64), 4),
+    (dict(dtype=7), 7),
+    (dict(ptrs=[FAKE] * 6 + [FAKE + 4, FAKE]), 8),
+    (dict(out=FAKE + 2), 8),
+    (dict(B=1, H=1 << 16, Ln=1 << 16, w=64), 13),
+])
+def test_attention_any_globals_host_validation(L, kw, status):
+    """The entry point for global tokens at any position rejects bad
+    arguments on the host, before any device call."""
+    assert _attn_any(L, **kw) == status
+
+
+def test_any_globals_scratch_bytes_host_only(L):
+    import torch
+    B, H, Ln, w = 2, 16, 4096, 256
+    tc = lf.lf_attention_scratch_bytes(B, H, Ln, w, torch.float16)
+    anyb = lf.lf_attention_any_globals_scratch_bytes(B, H, Ln, w, torch.float16)
+    # partition outputs (idx, counts, rank) plus qg/k/v slot buffers and slot masks
+    slots = 3 * B * H * 256 * 64 * 2 + B * 256 * 4
+    assert anyb >= tc + B * Ln * 4 + B * 4 + B * (Ln + 1) * 4 + slots
+    assert anyb < tc + B * Ln * 4 + B * (Ln + 1) * 4 + slots + 8 * 256
+    f32 = lf.lf_attention_any_globals_scratch_bytes(B, H, Ln, w, torch.float32)
+    assert B * Ln * 4 < f32 < B * Ln * 4 + B * (Ln + 1) * 4 + 4 * 256
+    assert lf.lf_attention_any_globals_scratch_bytes(1, 2, 500, 64, torch.float16) == 0
+
+
 @pytest.mark.parametrize("args,status", [
     ((0, 1, 512, 64, FAKE, FAKE), 1),
     ((FAKE, 0, 512, 64, FAKE, FAKE), 2),

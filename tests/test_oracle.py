@@ -515,3 +515,39 @@ def test_workload_draws_are_stable():
     assert len(wl.g) == 4 and all(1 <= g <= 128 for g in wl.g)
     assert all(0 <= p <= 1024 for p in wl.pad)
     assert inputs.workload(3).g == wl.g
+
+
+# ---------------------------------------------------------------- work counts (host side)
+
+@pytest.mark.parametrize("seed", range(4))
+def test_flops_from_masks_brute_force(seed):
+    """The benchmark's FLOP count for any masks equals 4*64*H times the sizes
+    of the key sets built with Python set algebra, and the prefix formula on
+    prefix masks."""
+    from sparse_attention_banded_b200 import metrics
+    rng = np.random.default_rng(1200 + seed)
+    B, H, w = 2, 3, int(rng.choice([4, 8, 16]))
+    L = w * int(rng.integers(2, 6))
+    lm, gm = _scattered_masks(rng, B, L, w)
+    total = 0
+    for b in range(B):
+        G = {j for j in range(L) if gm[b, j] == 0.0}
+        for i in range(L):
+            if lm[b, i] != 1.0:
+                continue
+            total += L if i in G else len(set(range(max(0, i - w), min(L - 1, i + w) + 1)) | G)
+    assert metrics.flops_masks(lm, gm, H, w) == 4.0 * 64 * H * total
+    g = [int(rng.integers(0, w + 1)) for _ in range(B)]
+    pad = [int(rng.integers(0, L)) for _ in range(B)]
+    lm2, gm2 = inputs.masks(B, L, g, pad)
+    assert metrics.flops_masks(lm2.numpy(), gm2.numpy(), H, w) == metrics.flops(B, H, L, w, g, pad)
+
+
+def test_scattered_masks_generator():
+    lm, gm = inputs.masks_scattered(3, 256, [0, 10, 64], [0, 50, 100], seed=5, padded_globals=2)
+    for b, (g, pad) in enumerate([(0, 0), (10, 50), (64, 100)]):
+        G = np.flatnonzero(gm[b].numpy() == 0.0)
+        assert len(G) == g and (G < 256 - pad).all()
+        assert set(np.unique(gm[b].numpy())) <= {0.0, -10000.0}
+        assert (lm[b, 256 - pad:] == 0.0).all()
+        assert int((lm[b, :256 - pad] == 0.0).sum()) == min(2, g)
