@@ -54,6 +54,9 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=50)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--workload", type=int, default=WORKLOAD_ID, choices=[1, 2, 3, 4, 5, 6])
+    ap.add_argument("--any-globals", action="store_true",
+                    help="workload 5 only: its 64 global tokens at random positions, through the entry points for "
+                         "global tokens anywhere")
     ap.add_argument("--layers", type=int, default=1,
                     help="workload 5 only: time an encoder of this many layers (lf_encoder_forward), each with "
                          "its own seeded weights")
@@ -203,8 +206,11 @@ def run_ours(args):
     layer = args.workload == 5
     anyg = args.workload == 6  # global tokens at any position: one call = partition + gather + attention
     n_layers = 1
+    any_layer = layer and args.any_globals
     if layer:
         wl, x_cpu, wts_cpu, lm_cpu, gm_cpu = inputs.layer_inputs(5)
+        if any_layer:
+            lm_cpu, gm_cpu = inputs.masks_scattered(wl.B, wl.L, wl.g, wl.pad, seed=1105)
         x = x_cpu.to(dev)
         wts = {n: v.to(dev) for n, v in wts_cpu.items()}
         ffn = wts["W_1"].shape[0]
@@ -214,7 +220,8 @@ def run_ours(args):
         stack = [wts] + [{n: ((torch.randn(v.shape, generator=gen, device=dev) * 0.02).to(v.dtype)
                                if n.startswith("W_") else v.clone()) for n, v in wts.items()}
                          for _ in range(n_layers - 1)]
-        ws = torch.empty(max(256, lf.lf_encoder_workspace_bytes(n_layers, wl.B, wl.H, wl.L, wl.w, ffn, x.dtype)),
+        ws_fn = lf.lf_encoder_any_globals_workspace_bytes if any_layer else lf.lf_encoder_workspace_bytes
+        ws = torch.empty(max(256, ws_fn(n_layers, wl.B, wl.H, wl.L, wl.w, ffn, x.dtype)),
                          dtype=torch.uint8, device=dev)
         args_in = [x]
         t_cpu = None
@@ -230,7 +237,11 @@ def run_ours(args):
     flush = torch.empty(max(2 * l2, 256 << 20) // 4, dtype=torch.float32, device=dev)
 
     def compute(ins, lm_, gm_):
-        if layer and n_layers > 1:
+        if any_layer and n_layers > 1:
+            lf.lf_encoder_forward_any_globals(ins[0], lm_, gm_, stack, wl.H, wl.w, out=out, workspace=ws)
+        elif any_layer:
+            lf.lf_encoder_layer_forward_any_globals(ins[0], lm_, gm_, wts, wl.H, wl.w, out=out, workspace=ws)
+        elif layer and n_layers > 1:
             lf.lf_encoder_forward(ins[0], lm_, gm_, stack, wl.H, wl.w, out=out, workspace=ws)
         elif layer:
             lf.lf_encoder_layer_forward(ins[0], lm_, gm_, wts, wl.H, wl.w, out=out, workspace=ws)
@@ -240,7 +251,7 @@ def run_ours(args):
             lf.lf_attention_forward(*ins, lm_, gm_, wl.w, out=out)
 
     def step(ev_a=None):
-        if not anyg:
+        if not anyg and not any_layer:
             lf.lf_init_global_idx(gm, wl.w, gidx, gnum, sync=False)
         if ev_a is not None:
             ev_a.record()
@@ -294,7 +305,7 @@ def run_ours(args):
     def e2e_step():
         for h, d in zip(h_in, d_in):
             d.copy_(h, non_blocking=True)
-        if not anyg:
+        if not anyg and not any_layer:
             lf.lf_init_global_idx(d_in[n_t + 1], wl.w, gidx, gnum, sync=False)
         compute(d_in[:n_t], d_in[n_t], d_in[n_t + 1])
         h_out.copy_(out, non_blocking=True)
@@ -317,6 +328,9 @@ def run_ours(args):
     pk, pk_kind = peaks()
     if layer:
         F = n_layers * metrics.layer_flops(wl.B, wl.H, wl.L, wl.w, wl.g, wl.pad, ffn)
+        if any_layer:  # the attention part over the scattered key sets
+            F += n_layers * (metrics.flops_masks(lm_cpu.numpy(), gm_cpu.numpy(), wl.H, wl.w)
+                             - metrics.flops(wl.B, wl.H, wl.L, wl.w, wl.g, wl.pad))
         wbytes = sum(v.numel() * v.element_size() for W in stack for v in W.values())
         By = float(wbytes + 2 * x.numel() * x.element_size() + 2 * wl.B * wl.L * 4)
     else:
@@ -350,7 +364,8 @@ def run_ours(args):
         "dtype": wl.dtype,
         "data": "synthetic (seeded inputs of the workload's shape%s)" %
                 (": x ~ N(0,1), weights ~ N(0, 0.02)" if layer else ", N(0,1)*0.5"),
-        "config": {"workload": wl.name + (" x %d layers" % n_layers if layer and n_layers > 1 else ""),
+        "config": {"workload": wl.name + (", globals at random positions" if any_layer else "")
+                   + (" x %d layers" % n_layers if layer and n_layers > 1 else ""),
                    "B": wl.B, "H": wl.H, "L": wl.L, "w": wl.w, "g": wl.g,
                    "pad": wl.pad, "head_dim": 64, "l2": "flushed before every timed step (2 x L2 write)",
                    "parallelism": "replica per GPU (weak)" if world > 1 else "single GPU"},
@@ -366,7 +381,8 @@ def run_ours(args):
         "roofline": roof,
         "e2e": {"value": job_throughput(world, tokens, 1, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": (3 if anyg else 1 + (8 * n_layers if layer else 1)) * K,
+        "gpu_launches": (3 if anyg else (1 + 10 * n_layers) if any_layer
+                         else 1 + (8 * n_layers if layer else 1)) * K,
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not layer:

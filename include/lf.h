@@ -250,6 +250,34 @@ lf_status lf_encoder_forward(const void* x, const float* local_mask, const float
                              lf_stream_t stream, void* out);
 
 /*
+ * lf_encoder_layer_forward_any_globals, lf_encoder_forward_any_globals -- the
+ * layer and the encoder with the global tokens at any positions (the
+ * attention as in lf_attention_forward_any_globals: global rows are the
+ * positions with global_mask == 0.0, a local row attends its window and
+ * every global token).  Arguments, layouts, validation and errors as for
+ * lf_encoder_layer_forward / lf_encoder_forward, with the workspace sizes
+ * below.  The partition of global_mask (with a count of the global tokens
+ * before each position) runs once per call, before the first layer; each
+ * layer projects qg only for the global tokens' rows of its input, gathered
+ * through global_idx, and gathers their k / v rows after its projections.
+ * A sample with more than w global tokens records LF_ERR_G_GT_W and gets a
+ * zero attention output in every layer.  Asynchronous on `stream`.
+ */
+size_t lf_encoder_layer_any_globals_workspace_bytes(int B, int H, int L, int w, int ffn_dim, lf_dtype dtype);
+lf_status lf_encoder_layer_forward_any_globals(const void* x, const float* local_mask, const float* global_mask,
+                                               const lf_layer_weights* wts, int B, int H, int L, int w,
+                                               float attn_scale, float ln_eps, lf_dtype dtype,
+                                               void* workspace, size_t workspace_bytes,
+                                               lf_stream_t stream, void* out);
+size_t lf_encoder_any_globals_workspace_bytes(int n_layers, int B, int H, int L, int w, int ffn_dim,
+                                              lf_dtype dtype);
+lf_status lf_encoder_forward_any_globals(const void* x, const float* local_mask, const float* global_mask,
+                                         const lf_layer_weights* layers, int n_layers, int B, int H, int L,
+                                         int w, float attn_scale, float ln_eps, lf_dtype dtype,
+                                         void* workspace, size_t workspace_bytes,
+                                         lf_stream_t stream, void* out);
+
+/*
  * lf_attention_forward_noalloc -- lf_attention_forward for callers that
  * cannot allocate device memory.  The pages describe no such entry point: it
  * exists for code that may not call cudaMalloc (for example code running

@@ -183,7 +183,8 @@ def to_heads(y, H):
 
 
 def encoder_layer(x, local_mask, global_mask, weights: dict, H: int, w: int,
-                  scale: float, eps: float, round_attention_inputs=None, round_stored=None):
+                  scale: float, eps: float, round_attention_inputs=None, round_stored=None,
+                  any_pos: bool = False):
     """x: [B, L, H*64]; weights: float64 arrays with keys
     W_qkv_kgvg [5, D, D], b_qkv_kgvg [5, D], W_qg [D, D], b_qg [D],
     W_o [D, D], b_o [D], ln1_gamma, ln1_beta [D], W_1 [D, F], b_1 [F],
@@ -194,7 +195,8 @@ def encoder_layer(x, local_mask, global_mask, weights: dict, H: int, w: int,
     applied to the attention output, to h and to the FFN intermediate.  The
     page's LongformerEncoder<T> keeps every intermediate buffer in T (FTL
     §Longformer Encoder 计算流程), so the comparison rounds where values are
-    stored; all arithmetic stays float64.  Returns float64 [B, L, D]."""
+    stored; all arithmetic stays float64.  any_pos: global tokens at any
+    position (as in :func:`attention`).  Returns float64 [B, L, D]."""
     x = _f64(x)
     W = {k: _f64(v) for k, v in weights.items()}
     rnd = round_attention_inputs or (lambda a: a)
@@ -202,7 +204,7 @@ def encoder_layer(x, local_mask, global_mask, weights: dict, H: int, w: int,
     proj = [to_heads(x @ W["W_qkv_kgvg"][n] + W["b_qkv_kgvg"][n], H) for n in range(5)]
     q, k, v, kg, vg = [rnd(p) for p in proj]
     qg = rnd(to_heads(x @ W["W_qg"] + W["b_qg"], H))
-    att = attention(q, k, v, qg, kg, vg, local_mask, global_mask, w, scale)
+    att = attention(q, k, v, qg, kg, vg, local_mask, global_mask, w, scale, any_pos=any_pos)
     B, L = x.shape[:2]
     att = keep(att.reshape(B, L, H * D))
     h = keep(layer_norm(att @ W["W_o"] + W["b_o"] + x, W["ln1_gamma"], W["ln1_beta"], eps))

@@ -133,7 +133,8 @@ namespace {
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 // One CTA of 256 threads per 32 slots of one (b, h): thread t copies the
-// 16-byte column part t % 8 of slot c0 + t / 8 for qg, k and v; slots past
+// 16-byte column part t % 8 of slot c0 + t / 8 for qg (unless qg is NULL:
+// the encoder layer projects the slots' qg rows itself), k and v; slots past
 // g are zero (finite rows for the masked tail of a block).  The h == 0 CTAs
 // also write the slots' local_mask values.
 __global__ void __launch_bounds__(256)
@@ -152,13 +153,13 @@ gather_globals_kernel(const uint4* __restrict__ qg, const uint4* __restrict__ k,
     if (c < g) {
         const int j = gidx[(size_t)b * L + c];
         const size_t src = ((size_t)bh * L + j) * 8 + part;
-        const uint4 a = qg[src], kk = k[src], vv = v[src];
-        qg_c[dst] = a;
+        const uint4 kk = k[src], vv = v[src];
+        if (qg) qg_c[dst] = qg[src];
         k_c[dst] = kk;
         v_c[dst] = vv;
     } else {
         const uint4 z = make_uint4(0u, 0u, 0u, 0u);
-        qg_c[dst] = z;
+        if (qg) qg_c[dst] = z;
         k_c[dst] = z;
         v_c[dst] = z;
     }
@@ -168,7 +169,34 @@ gather_globals_kernel(const uint4* __restrict__ qg, const uint4* __restrict__ k,
     }
 }
 
+// Rows of a [B][L][D] 16-bit matrix at the global tokens' positions into
+// [B][gcap][D] (slot c = position global_idx[b, c]; slots past g zero).  One
+// CTA of 128 threads per slot, 16 bytes per thread and step.
+__global__ void __launch_bounds__(128)
+gather_rows_kernel(const uint4* __restrict__ src, const int32_t* __restrict__ gidx,
+                   const int32_t* __restrict__ gnum, int L, int gcap, int parts, uint4* __restrict__ dst) {
+    const int b = blockIdx.x / gcap, c = blockIdx.x % gcap;
+    const int g = min(gnum[b], gcap);
+    uint4* d = dst + ((size_t)b * gcap + c) * parts;
+    if (c < g) {
+        const uint4* s = src + ((size_t)b * L + gidx[(size_t)b * L + c]) * parts;
+        for (int t = threadIdx.x; t < parts; t += 128) d[t] = s[t];
+    } else {
+        for (int t = threadIdx.x; t < parts; t += 128) d[t] = make_uint4(0u, 0u, 0u, 0u);
+    }
+}
+
 }  // namespace
+
+lf_status launch_gather_rows(const void* src, const AnyGlobals& a, int B, int L, int D, void* dst,
+                             cudaStream_t stream) {
+    const long long blocks = (long long)B * a.gcap;
+    if (blocks >= (1LL << 31)) return LF_ERR_TOO_LARGE;
+    gather_rows_kernel<<<(unsigned)blocks, 128, 0, stream>>>(reinterpret_cast<const uint4*>(src), a.global_idx,
+                                                             a.global_token_nums, L, a.gcap, D * 2 / 16,
+                                                             reinterpret_cast<uint4*>(dst));
+    return cudaGetLastError() == cudaSuccess ? LF_OK : LF_ERR_CUDA;
+}
 
 size_t any_globals_bytes(int B, int H, int L, int w, bool compact) {
     size_t n = align256((size_t)B * L * 4) + align256((size_t)B * 4) + align256((size_t)B * (L + 1) * 4);
@@ -206,6 +234,7 @@ lf_status launch_gather_globals(const void* qg, const void* k, const void* v, co
     if (blocks >= (1LL << 31)) return LF_ERR_TOO_LARGE;
     gather_globals_kernel<<<(unsigned)blocks, 256, 0, stream>>>(
         reinterpret_cast<const uint4*>(qg), reinterpret_cast<const uint4*>(k), reinterpret_cast<const uint4*>(v),
+        // (qg may be NULL: qg_c is then left to the caller)
         local_mask, a.global_idx, a.global_token_nums, H, L, a.gcap, reinterpret_cast<uint4*>(a.qg_c),
         reinterpret_cast<uint4*>(a.k_c), reinterpret_cast<uint4*>(a.v_c), a.lm_c);
     return cudaGetLastError() == cudaSuccess ? LF_OK : LF_ERR_CUDA;

@@ -79,9 +79,14 @@ inline int any_globals_gcap(int w) { return (w + 127) / 128 * 128; }
 size_t any_globals_bytes(int B, int H, int L, int w, bool compact);
 // Carves an AnyGlobals out of `base` (any_globals_bytes(..) bytes).
 AnyGlobals any_globals_layout(void* base, int B, int H, int L, int w, bool compact);
-// 16-bit dtypes: fills qg_c, k_c, v_c and lm_c from the partition's outputs.
+// 16-bit dtypes: fills qg_c, k_c, v_c and lm_c from the partition's outputs
+// (qg NULL: qg_c is not written).
 lf_status launch_gather_globals(const void* qg, const void* k, const void* v, const float* local_mask,
                                 const AnyGlobals& a, int B, int H, int L, int w, cudaStream_t stream);
+// Rows of a [B][L][D] 16-bit matrix at the global tokens' positions into
+// [B][gcap][D] (slots past g zero).  D % 8 == 0.
+lf_status launch_gather_rows(const void* src, const AnyGlobals& a, int B, int L, int D, void* dst,
+                             cudaStream_t stream);
 
 // any (may be NULL): global tokens at any position (global_idx and
 // global_token_nums are used).

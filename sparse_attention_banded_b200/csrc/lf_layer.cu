@@ -10,28 +10,40 @@
 //   banded + global attention -> a [B, L, D]
 //   GEMM(a, W_o) + b_o + x -> z (fp32);  LayerNorm -> h
 //   GEMM(h, W_1) + b_1, GELU -> f;  GEMM(f, W_2) + b_2 + h -> z;  LayerNorm -> out
+// With the global tokens at any position (the _any_globals entry points) the
+// partition (with its rank table) runs once per forward, the qg projection
+// multiplies only the global tokens' rows of x, gathered through global_idx,
+// and writes them straight into the slot buffer of the attention kernel, and
+// the k / v rows of the global tokens are gathered after the projections.
 #include "lf_internal.h"
 
 namespace lf {
 namespace {
 
 struct Workspace {
-    size_t qkv, qg, att, z, h, f, scratch, total;
+    size_t qkv, qg, att, z, h, f, scratch, any, xg, total;
 };
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-Workspace layout(int B, int H, int L, int w, int F, int elem) {
+// any: global tokens at any position (partition outputs and slot buffers,
+// and the gathered rows of x; no position-indexed qg buffer).
+Workspace layout(int B, int H, int L, int w, int F, int elem, bool any) {
     const size_t D = (size_t)H * 64, rows = (size_t)B * L;
     Workspace s;
     size_t o = 0;
     s.qkv = o; o += align256(5 * rows * D * elem);
-    s.qg = o; o += align256(rows * D * elem);
+    s.qg = o; if (!any) o += align256(rows * D * elem);
     s.att = o; o += align256(rows * D * elem);
     s.z = o; o += align256(rows * D * 4);
     s.h = o; o += align256(rows * D * elem);
     s.f = o; o += align256(rows * (size_t)F * elem);
     s.scratch = o; o += align256(attention_tc_scratch_bytes(B, H, L, w));
+    s.any = s.xg = o;
+    if (any) {
+        o += align256(any_globals_bytes(B, H, L, w, true));
+        s.xg = o; o += align256((size_t)B * any_globals_gcap(w) * D * elem);
+    }
     s.total = o;
     return s;
 }
@@ -61,34 +73,29 @@ lf_status check_layer(int B, int H, int L, int w, int F, lf_dtype dtype) {
 
 using namespace lf;
 
-extern "C" size_t lf_encoder_layer_workspace_bytes(int B, int H, int L, int w, int ffn_dim, lf_dtype dtype) {
-    if (check_layer(B, H, L, w, ffn_dim, dtype) != LF_OK) return 0;
-    return layout(B, H, L, w, ffn_dim, 2).total;
-}
+namespace lf {
+namespace {
 
-extern "C" lf_status lf_encoder_layer_forward(const void* x, const float* local_mask, const float* global_mask,
-                                              const lf_layer_weights* wt, int B, int H, int L, int w,
-                                              float attn_scale, float ln_eps, lf_dtype dtype, void* workspace,
-                                              size_t workspace_bytes, lf_stream_t stream, void* out) {
-    if (!x || !local_mask || !global_mask || !wt || !out) return LF_ERR_NULL;
-    const int F = wt->ffn_dim;
-    lf_status st = check_layer(B, H, L, w, F, dtype);
-    if (st != LF_OK) return st;
-    if ((st = check_weights(wt)) != LF_OK) return st;
-    const void* ptrs[] = {x, local_mask, global_mask, out};
-    for (const void* p : ptrs)
-        if (!aligned16(p)) return LF_ERR_MISALIGNED;
-    const Workspace ws = layout(B, H, L, w, F, 2);
-    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < ws.total)
-        return LF_ERR_WORKSPACE;
-    DeviceCtx* d = current_device(&st);
-    if (!d) return st;
-    cudaStream_t s = (cudaStream_t)stream;
-    uint8_t* base = reinterpret_cast<uint8_t*>(workspace);
-    const int D = H * 64;
+// One layer on the workspace `base` (layout ws).  any: global tokens at any
+// position; run_partition: run the partition here (the stack runs it once
+// before its first layer).  Arguments are validated by the callers.
+lf_status layer_forward(const void* x, const float* local_mask, const float* global_mask, const lf_layer_weights* wt,
+                        int B, int H, int L, int w, float attn_scale, float ln_eps, lf_dtype dtype, uint8_t* base,
+                        const Workspace& ws, bool any, bool run_partition, DeviceCtx* d, cudaStream_t s, void* out) {
+    lf_status st;
+    const int D = H * 64, F = wt->ffn_dim;
     const size_t head_elems = (size_t)B * H * L * 64;
     uint8_t* qkv = base + ws.qkv;  // [5][B][H][L][64]
     auto slot = [&](int i) { return qkv + (size_t)i * head_elems * 2; };
+    AnyGlobals a{};
+    if (any) {
+        a = any_globals_layout(base + ws.any, B, H, L, w, true);
+        if (run_partition &&
+            (st = launch_global_idx(global_mask, B, L, w, const_cast<int32_t*>(a.global_idx),
+                                    const_cast<int32_t*>(a.global_token_nums), d->status, s,
+                                    const_cast<int32_t*>(a.rank), false)) != LF_OK)
+            return st;
+    }
 
     if (!d->side) {
         if (cudaStreamCreateWithFlags(&d->side, cudaStreamNonBlocking) != cudaSuccess ||
@@ -104,18 +111,29 @@ extern "C" lf_status lf_encoder_layer_forward(const void* x, const float* local_
     if (cudaEventRecord(d->ev_fork, s) != cudaSuccess || cudaStreamWaitEvent(d->side, d->ev_fork, 0) != cudaSuccess)
         return LF_ERR_CUDA;
     if ((st = launch_gemm_tc(g, dtype, d->sm_count, s)) != LF_OK) return st;
-    // Qg over the rows that can be global tokens (g_b <= w), beside the above
-    const int qrows = ((w + 127) / 128) * 128 < L ? ((w + 127) / 128) * 128 : L;
-    g.rows = qrows; g.W = wt->W_qg; g.N = D; g.bias = wt->b_qg; g.out = base + ws.qg;
+    if (any) {
+        // Qg of the global tokens only: their rows of x, gathered, into the
+        // slot buffer (slot layout [B][H][gcap][64]), beside the above
+        if ((st = launch_gather_rows(x, a, B, L, D, base + ws.xg, d->side)) != LF_OK) return st;
+        g.A = base + ws.xg; g.rows = a.gcap; g.batch_stride = a.gcap; g.heads_L = a.gcap;
+        g.W = wt->W_qg; g.N = D; g.bias = wt->b_qg; g.out = a.qg_c;
+    } else {
+        // Qg over the rows that can be global tokens (g_b <= w), beside the above
+        const int qrows = ((w + 127) / 128) * 128 < L ? ((w + 127) / 128) * 128 : L;
+        g.rows = qrows; g.W = wt->W_qg; g.N = D; g.bias = wt->b_qg; g.out = base + ws.qg;
+    }
     if ((st = launch_gemm_tc(g, dtype, d->sm_count, d->side)) != LF_OK) return st;
     if (cudaEventRecord(d->ev_join, d->side) != cudaSuccess || cudaStreamWaitEvent(s, d->ev_join, 0) != cudaSuccess)
         return LF_ERR_CUDA;
+    // the global tokens' k / v rows and local_mask values into their slots
+    if (any && (st = launch_gather_globals(nullptr, slot(1), slot(2), local_mask, a, B, H, L, w, s)) != LF_OK)
+        return st;
     // steps 3-5: attention (its split counters must start at zero)
     if (cudaMemsetAsync(base + ws.scratch, 0, attention_tc_scratch_zero_bytes(B, H, L, w), s) != cudaSuccess)
         return LF_ERR_CUDA;
-    if ((st = launch_attention_tc(slot(0), slot(1), slot(2), base + ws.qg, slot(3), slot(4), local_mask, global_mask,
-                                  B, H, L, w, attn_scale, dtype, base + ws.att, base + ws.scratch, d->status,
-                                  d->sm_count, s)) != LF_OK)
+    if ((st = launch_attention_tc(slot(0), slot(1), slot(2), any ? a.qg_c : base + ws.qg, slot(3), slot(4),
+                                  local_mask, global_mask, B, H, L, w, attn_scale, dtype, base + ws.att,
+                                  base + ws.scratch, d->status, d->sm_count, s, any ? &a : nullptr)) != LF_OK)
         return st;
     // step 5: output projection + bias + residual, LayerNorm
     GemmArgs o{};
@@ -140,23 +158,82 @@ extern "C" lf_status lf_encoder_layer_forward(const void* x, const float* local_
                             dtype, out, s);
 }
 
+size_t layer_workspace_bytes(int B, int H, int L, int w, int ffn_dim, lf_dtype dtype, bool any) {
+    if (check_layer(B, H, L, w, ffn_dim, dtype) != LF_OK) return 0;
+    return layout(B, H, L, w, ffn_dim, 2, any).total;
+}
+
+lf_status layer_entry(const void* x, const float* local_mask, const float* global_mask, const lf_layer_weights* wt,
+                      int B, int H, int L, int w, float attn_scale, float ln_eps, lf_dtype dtype, void* workspace,
+                      size_t workspace_bytes, lf_stream_t stream, void* out, bool any) {
+    if (!x || !local_mask || !global_mask || !wt || !out) return LF_ERR_NULL;
+    const int F = wt->ffn_dim;
+    lf_status st = check_layer(B, H, L, w, F, dtype);
+    if (st != LF_OK) return st;
+    if ((st = check_weights(wt)) != LF_OK) return st;
+    const void* ptrs[] = {x, local_mask, global_mask, out};
+    for (const void* p : ptrs)
+        if (!aligned16(p)) return LF_ERR_MISALIGNED;
+    const Workspace ws = layout(B, H, L, w, F, 2, any);
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < ws.total)
+        return LF_ERR_WORKSPACE;
+    DeviceCtx* d = current_device(&st);
+    if (!d) return st;
+    return layer_forward(x, local_mask, global_mask, wt, B, H, L, w, attn_scale, ln_eps, dtype,
+                         reinterpret_cast<uint8_t*>(workspace), ws, any, true, d, (cudaStream_t)stream, out);
+}
+
+}  // namespace
+}  // namespace lf
+
+extern "C" size_t lf_encoder_layer_workspace_bytes(int B, int H, int L, int w, int ffn_dim, lf_dtype dtype) {
+    return layer_workspace_bytes(B, H, L, w, ffn_dim, dtype, false);
+}
+
+extern "C" lf_status lf_encoder_layer_forward(const void* x, const float* local_mask, const float* global_mask,
+                                              const lf_layer_weights* wt, int B, int H, int L, int w,
+                                              float attn_scale, float ln_eps, lf_dtype dtype, void* workspace,
+                                              size_t workspace_bytes, lf_stream_t stream, void* out) {
+    return layer_entry(x, local_mask, global_mask, wt, B, H, L, w, attn_scale, ln_eps, dtype, workspace,
+                       workspace_bytes, stream, out, false);
+}
+
+extern "C" size_t lf_encoder_layer_any_globals_workspace_bytes(int B, int H, int L, int w, int ffn_dim,
+                                                               lf_dtype dtype) {
+    return layer_workspace_bytes(B, H, L, w, ffn_dim, dtype, true);
+}
+
+extern "C" lf_status lf_encoder_layer_forward_any_globals(const void* x, const float* local_mask,
+                                                          const float* global_mask, const lf_layer_weights* wt,
+                                                          int B, int H, int L, int w, float attn_scale, float ln_eps,
+                                                          lf_dtype dtype, void* workspace, size_t workspace_bytes,
+                                                          lf_stream_t stream, void* out) {
+    return layer_entry(x, local_mask, global_mask, wt, B, H, L, w, attn_scale, ln_eps, dtype, workspace,
+                       workspace_bytes, stream, out, true);
+}
+
 // ---------------------------------------------------------------- the stack
 
-extern "C" size_t lf_encoder_workspace_bytes(int n_layers, int B, int H, int L, int w, int ffn_dim, lf_dtype dtype) {
+namespace lf {
+namespace {
+
+size_t encoder_workspace_bytes(int n_layers, int B, int H, int L, int w, int ffn_dim, lf_dtype dtype, bool any) {
     if (n_layers <= 0) return 0;
-    const size_t layer = lf_encoder_layer_workspace_bytes(B, H, L, w, ffn_dim, dtype);
+    const size_t layer = layer_workspace_bytes(B, H, L, w, ffn_dim, dtype, any);
     if (layer == 0) return 0;
     const size_t act = align256((size_t)B * L * H * 64 * 2);
     return layer + (n_layers > 1 ? 2 * act : 0);
 }
 
 // The page's encoder (§Longformer Encoder 计算流程) runs its preprocessing
-// once per forward and then the layer loop; here every layer's attention
-// reads g_b from the mask prefix itself, so the loop is the whole forward.
-extern "C" lf_status lf_encoder_forward(const void* x, const float* local_mask, const float* global_mask,
-                                        const lf_layer_weights* layers, int n_layers, int B, int H, int L, int w,
-                                        float attn_scale, float ln_eps, lf_dtype dtype, void* workspace,
-                                        size_t workspace_bytes, lf_stream_t stream, void* out) {
+// once per forward and then the layer loop.  With prefix global tokens every
+// layer's attention reads g_b from the mask prefix itself, so the loop is
+// the whole forward; with global tokens at any position the partition runs
+// once, before the first layer, and every layer reuses its outputs.
+lf_status encoder_entry(const void* x, const float* local_mask, const float* global_mask,
+                        const lf_layer_weights* layers, int n_layers, int B, int H, int L, int w, float attn_scale,
+                        float ln_eps, lf_dtype dtype, void* workspace, size_t workspace_bytes, lf_stream_t stream,
+                        void* out, bool any) {
     if (!x || !local_mask || !global_mask || !layers || !out) return LF_ERR_NULL;
     if (n_layers <= 0) return LF_ERR_BAD_DIM;
     const int F = layers[0].ffn_dim;
@@ -167,18 +244,53 @@ extern "C" lf_status lf_encoder_forward(const void* x, const float* local_mask, 
         if (layers[i].ffn_dim != F) return LF_ERR_BAD_DIM;
         if ((st = check_weights(&layers[i])) != LF_OK) return st;
     }
-    const size_t need = lf_encoder_workspace_bytes(n_layers, B, H, L, w, F, dtype);
+    const void* ptrs[] = {x, local_mask, global_mask, out};
+    for (const void* p : ptrs)
+        if (!aligned16(p)) return LF_ERR_MISALIGNED;
+    const size_t need = encoder_workspace_bytes(n_layers, B, H, L, w, F, dtype, any);
     if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < need)
         return LF_ERR_WORKSPACE;
-    const size_t layer_bytes = layout(B, H, L, w, F, 2).total;
-    uint8_t* act[2] = {reinterpret_cast<uint8_t*>(workspace) + layer_bytes, nullptr};
+    DeviceCtx* d = current_device(&st);
+    if (!d) return st;
+    const Workspace ws = layout(B, H, L, w, F, 2, any);
+    uint8_t* base = reinterpret_cast<uint8_t*>(workspace);
+    uint8_t* act[2] = {base + ws.total, nullptr};
     act[1] = act[0] + align256((size_t)B * L * H * 64 * 2);
     for (int i = 0; i < n_layers; ++i) {
         const void* in = i == 0 ? x : act[(i - 1) & 1];
         void* o = i == n_layers - 1 ? out : act[i & 1];
-        st = lf_encoder_layer_forward(in, local_mask, global_mask, &layers[i], B, H, L, w, attn_scale, ln_eps, dtype,
-                                      workspace, layer_bytes, stream, o);
+        st = layer_forward(in, local_mask, global_mask, &layers[i], B, H, L, w, attn_scale, ln_eps, dtype, base, ws,
+                           any, i == 0, d, (cudaStream_t)stream, o);
         if (st != LF_OK) return st;
     }
     return LF_OK;
+}
+
+}  // namespace
+}  // namespace lf
+
+extern "C" size_t lf_encoder_workspace_bytes(int n_layers, int B, int H, int L, int w, int ffn_dim, lf_dtype dtype) {
+    return encoder_workspace_bytes(n_layers, B, H, L, w, ffn_dim, dtype, false);
+}
+
+extern "C" lf_status lf_encoder_forward(const void* x, const float* local_mask, const float* global_mask,
+                                        const lf_layer_weights* layers, int n_layers, int B, int H, int L, int w,
+                                        float attn_scale, float ln_eps, lf_dtype dtype, void* workspace,
+                                        size_t workspace_bytes, lf_stream_t stream, void* out) {
+    return encoder_entry(x, local_mask, global_mask, layers, n_layers, B, H, L, w, attn_scale, ln_eps, dtype,
+                         workspace, workspace_bytes, stream, out, false);
+}
+
+extern "C" size_t lf_encoder_any_globals_workspace_bytes(int n_layers, int B, int H, int L, int w, int ffn_dim,
+                                                         lf_dtype dtype) {
+    return encoder_workspace_bytes(n_layers, B, H, L, w, ffn_dim, dtype, true);
+}
+
+extern "C" lf_status lf_encoder_forward_any_globals(const void* x, const float* local_mask, const float* global_mask,
+                                                    const lf_layer_weights* layers, int n_layers, int B, int H, int L,
+                                                    int w, float attn_scale, float ln_eps, lf_dtype dtype,
+                                                    void* workspace, size_t workspace_bytes, lf_stream_t stream,
+                                                    void* out) {
+    return encoder_entry(x, local_mask, global_mask, layers, n_layers, B, H, L, w, attn_scale, ln_eps, dtype,
+                         workspace, workspace_bytes, stream, out, true);
 }

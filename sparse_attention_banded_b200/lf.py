@@ -73,6 +73,14 @@ def lib():
         L.lf_encoder_workspace_bytes.restype = ctypes.c_size_t
         L.lf_encoder_forward.argtypes = [vp, vp, vp, ctypes.POINTER(LayerWeights), i, i, i, i, i,
                                          ctypes.c_float, ctypes.c_float, i, vp, ctypes.c_size_t, vp, vp]
+        L.lf_encoder_layer_any_globals_workspace_bytes.argtypes = [i, i, i, i, i, i]
+        L.lf_encoder_layer_any_globals_workspace_bytes.restype = ctypes.c_size_t
+        L.lf_encoder_layer_forward_any_globals.argtypes = L.lf_encoder_layer_forward.argtypes
+        L.lf_encoder_layer_forward_any_globals.restype = st
+        L.lf_encoder_any_globals_workspace_bytes.argtypes = [i, i, i, i, i, i, i]
+        L.lf_encoder_any_globals_workspace_bytes.restype = ctypes.c_size_t
+        L.lf_encoder_forward_any_globals.argtypes = L.lf_encoder_forward.argtypes
+        L.lf_encoder_forward_any_globals.restype = st
         L.lf_encoder_forward.restype = st
         _lib = L
     return _lib
@@ -189,11 +197,7 @@ def lf_encoder_layer_workspace_bytes(B: int, H: int, L: int, w: int, ffn_dim: in
     return lib().lf_encoder_layer_workspace_bytes(B, H, L, w, ffn_dim, DTYPE_CODE[dtype])
 
 
-def lf_encoder_layer_forward(x, local_mask, global_mask, weights: dict, H: int, w: int, attn_scale: float = 0.125,
-                             ln_eps: float = 1e-5, out=None, workspace=None, stream=None):
-    """One encoder layer; x [B, L, H*64]; weights: tensors named as the
-    fields of lf_layer_weights (nn.Linear layout [out, in]), LayerNorm
-    parameters fp32.  Returns out [B, L, H*64]."""
+def _layer(name, size_fn, x, local_mask, global_mask, weights, H, w, attn_scale, ln_eps, out, workspace, stream):
     B, L, D = x.shape
     ffn = weights["W_1"].shape[0]
     wt = LayerWeights(ffn, *[weights[n].data_ptr() for n in LAYER_FIELDS])
@@ -201,14 +205,36 @@ def lf_encoder_layer_forward(x, local_mask, global_mask, weights: dict, H: int, 
         _ptr(weights[n])
     if out is None:
         out = torch.empty_like(x)
-    need = lf_encoder_layer_workspace_bytes(B, H, L, w, ffn, x.dtype)
+    need = size_fn(B, H, L, w, ffn, x.dtype)
     if workspace is None:
         workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=x.device)
-    st = lib().lf_encoder_layer_forward(_ptr(x), _ptr(local_mask), _ptr(global_mask), ctypes.byref(wt), B, H, L,
-                                        w, attn_scale, ln_eps, DTYPE_CODE.get(x.dtype, 99), _ptr(workspace),
-                                        workspace.numel(), _stream(stream), _ptr(out))
-    _check(st, "lf_encoder_layer_forward")
+    st = getattr(lib(), name)(_ptr(x), _ptr(local_mask), _ptr(global_mask), ctypes.byref(wt), B, H, L,
+                              w, attn_scale, ln_eps, DTYPE_CODE.get(x.dtype, 99), _ptr(workspace),
+                              workspace.numel(), _stream(stream), _ptr(out))
+    _check(st, name)
     return out
+
+
+def lf_encoder_layer_forward(x, local_mask, global_mask, weights: dict, H: int, w: int, attn_scale: float = 0.125,
+                             ln_eps: float = 1e-5, out=None, workspace=None, stream=None):
+    """One encoder layer; x [B, L, H*64]; weights: tensors named as the
+    fields of lf_layer_weights (nn.Linear layout [out, in]), LayerNorm
+    parameters fp32.  Returns out [B, L, H*64]."""
+    return _layer("lf_encoder_layer_forward", lf_encoder_layer_workspace_bytes, x, local_mask, global_mask,
+                  weights, H, w, attn_scale, ln_eps, out, workspace, stream)
+
+
+def lf_encoder_layer_any_globals_workspace_bytes(B: int, H: int, L: int, w: int, ffn_dim: int, dtype) -> int:
+    return lib().lf_encoder_layer_any_globals_workspace_bytes(B, H, L, w, ffn_dim, DTYPE_CODE[dtype])
+
+
+def lf_encoder_layer_forward_any_globals(x, local_mask, global_mask, weights: dict, H: int, w: int,
+                                         attn_scale: float = 0.125, ln_eps: float = 1e-5, out=None, workspace=None,
+                                         stream=None):
+    """Same as :func:`lf_encoder_layer_forward` with the global tokens
+    (global_mask == 0.0) at any positions."""
+    return _layer("lf_encoder_layer_forward_any_globals", lf_encoder_layer_any_globals_workspace_bytes, x,
+                  local_mask, global_mask, weights, H, w, attn_scale, ln_eps, out, workspace, stream)
 
 
 def lf_encoder_workspace_bytes(n_layers: int, B: int, H: int, L: int, w: int, ffn_dim: int, dtype) -> int:
@@ -220,6 +246,25 @@ def lf_encoder_forward(x, local_mask, global_mask, layers: list, H: int, w: int,
     """The encoder: the layers in `layers` (each a weight dict as for
     lf_encoder_layer_forward, same FFN width) applied in turn to x
     [B, L, H*64].  Returns out [B, L, H*64]."""
+    return _encoder("lf_encoder_forward", lf_encoder_workspace_bytes, x, local_mask, global_mask, layers, H, w,
+                    attn_scale, ln_eps, out, workspace, stream)
+
+
+def lf_encoder_any_globals_workspace_bytes(n_layers: int, B: int, H: int, L: int, w: int, ffn_dim: int,
+                                           dtype) -> int:
+    return lib().lf_encoder_any_globals_workspace_bytes(n_layers, B, H, L, w, ffn_dim, DTYPE_CODE[dtype])
+
+
+def lf_encoder_forward_any_globals(x, local_mask, global_mask, layers: list, H: int, w: int,
+                                   attn_scale: float = 0.125, ln_eps: float = 1e-5, out=None, workspace=None,
+                                   stream=None):
+    """Same as :func:`lf_encoder_forward` with the global tokens
+    (global_mask == 0.0) at any positions."""
+    return _encoder("lf_encoder_forward_any_globals", lf_encoder_any_globals_workspace_bytes, x, local_mask,
+                    global_mask, layers, H, w, attn_scale, ln_eps, out, workspace, stream)
+
+
+def _encoder(fn_name, size_fn, x, local_mask, global_mask, layers, H, w, attn_scale, ln_eps, out, workspace, stream):
     B, L, D = x.shape
     n = len(layers)
     ffn = layers[0]["W_1"].shape[0] if n else 0
@@ -230,11 +275,11 @@ def lf_encoder_forward(x, local_mask, global_mask, layers: list, H: int, w: int,
         arr[j] = LayerWeights(weights["W_1"].shape[0], *[weights[name].data_ptr() for name in LAYER_FIELDS])
     if out is None:
         out = torch.empty_like(x)
-    need = lf_encoder_workspace_bytes(n, B, H, L, w, ffn, x.dtype) if n else 0
+    need = size_fn(n, B, H, L, w, ffn, x.dtype) if n else 0
     if workspace is None:
         workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=x.device)
-    st = lib().lf_encoder_forward(_ptr(x), _ptr(local_mask), _ptr(global_mask), arr, n, B, H, L, w, attn_scale,
-                                  ln_eps, DTYPE_CODE.get(x.dtype, 99), _ptr(workspace), workspace.numel(),
-                                  _stream(stream), _ptr(out))
-    _check(st, "lf_encoder_forward")
+    st = getattr(lib(), fn_name)(_ptr(x), _ptr(local_mask), _ptr(global_mask), arr, n, B, H, L, w, attn_scale,
+                                 ln_eps, DTYPE_CODE.get(x.dtype, 99), _ptr(workspace), workspace.numel(),
+                                 _stream(stream), _ptr(out))
+    _check(st, fn_name)
     return out

@@ -114,7 +114,8 @@ def test_scratch_bytes_host_only(L):
     assert lf.lf_attention_scratch_bytes(1, 2, 500, 64, torch.float16) == 0
 
 
-def _layer(L, B=1, H=4, Ln=512, w=64, ffn=512, dtype=1, ws_bytes=1 << 30, weights="ok", x=FAKE, ws=FAKE):
+def _layer(L, B=1, H=4, Ln=512, w=64, ffn=512, dtype=1, ws_bytes=1 << 30, weights="ok", x=FAKE, ws=FAKE,
+           fn="lf_encoder_layer_forward"):
     if weights == "null":
         wp = None
     else:
@@ -124,9 +125,9 @@ def _layer(L, B=1, H=4, Ln=512, w=64, ffn=512, dtype=1, ws_bytes=1 << 30, weight
         if weights == "misaligned":
             vals[2] = FAKE + 2
         wp = ctypes.byref(lf.LayerWeights(ffn, *vals))
-    return L.lf_encoder_layer_forward(ctypes.c_void_p(x), ctypes.c_void_p(FAKE), ctypes.c_void_p(FAKE), wp,
-                                      B, H, Ln, w, 0.125, 1e-5, dtype, ctypes.c_void_p(ws), ws_bytes, None,
-                                      ctypes.c_void_p(FAKE))
+    return getattr(L, fn)(ctypes.c_void_p(x), ctypes.c_void_p(FAKE), ctypes.c_void_p(FAKE), wp,
+                          B, H, Ln, w, 0.125, 1e-5, dtype, ctypes.c_void_p(ws), ws_bytes, None,
+                          ctypes.c_void_p(FAKE))
 
 
 @pytest.mark.parametrize("kw,status", [
@@ -144,8 +145,9 @@ def _layer(L, B=1, H=4, Ln=512, w=64, ffn=512, dtype=1, ws_bytes=1 << 30, weight
     (dict(ws_bytes=1024), 12),  # workspace smaller than lf_encoder_layer_workspace_bytes
     (dict(ws=FAKE + 16), 12),   # workspace not 256-byte aligned
 ])
-def test_layer_host_validation(L, kw, status):
-    assert _layer(L, **kw) == status
+@pytest.mark.parametrize("fn", ["lf_encoder_layer_forward", "lf_encoder_layer_forward_any_globals"])
+def test_layer_host_validation(L, kw, status, fn):
+    assert _layer(L, fn=fn, **kw) == status
 
 
 def test_layer_workspace_bytes_host_only(L):
@@ -158,7 +160,7 @@ def test_layer_workspace_bytes_host_only(L):
     assert lf.lf_encoder_layer_workspace_bytes(1, 4, 512, 64, 512, torch.float32) == 0
 
 
-def _encoder(L, n=3, ffns=(512, 512, 512), bad_layer=None, ws_bytes=1 << 30, layers="ok"):
+def _encoder(L, n=3, ffns=(512, 512, 512), bad_layer=None, ws_bytes=1 << 30, layers="ok", fn="lf_encoder_forward"):
     arr = (lf.LayerWeights * max(n, 1))()
     for j in range(min(n, len(ffns))):
         vals = [FAKE] * len(lf.LAYER_FIELDS)
@@ -166,9 +168,9 @@ def _encoder(L, n=3, ffns=(512, 512, 512), bad_layer=None, ws_bytes=1 << 30, lay
             vals[8] = 0  # W_1 of that layer
         arr[j] = lf.LayerWeights(ffns[j], *vals)
     lp = None if layers == "null" else arr
-    return L.lf_encoder_forward(ctypes.c_void_p(FAKE), ctypes.c_void_p(FAKE), ctypes.c_void_p(FAKE), lp, n,
-                                1, 4, 512, 64, 0.125, 1e-5, 1, ctypes.c_void_p(FAKE), ws_bytes, None,
-                                ctypes.c_void_p(FAKE + 256))
+    return getattr(L, fn)(ctypes.c_void_p(FAKE), ctypes.c_void_p(FAKE), ctypes.c_void_p(FAKE), lp, n,
+                          1, 4, 512, 64, 0.125, 1e-5, 1, ctypes.c_void_p(FAKE), ws_bytes, None,
+                          ctypes.c_void_p(FAKE + 256))
 
 
 @pytest.mark.parametrize("kw,status", [
@@ -178,8 +180,9 @@ def _encoder(L, n=3, ffns=(512, 512, 512), bad_layer=None, ws_bytes=1 << 30, lay
     (dict(bad_layer=2), 1),           # the last layer's missing weight is caught before any launch
     (dict(ws_bytes=1024), 12),
 ])
-def test_encoder_host_validation(L, kw, status):
-    assert _encoder(L, **kw) == status
+@pytest.mark.parametrize("fn", ["lf_encoder_forward", "lf_encoder_forward_any_globals"])
+def test_encoder_host_validation(L, kw, status, fn):
+    assert _encoder(L, fn=fn, **kw) == status
 
 
 def test_encoder_workspace_bytes_host_only(L):
@@ -189,3 +192,18 @@ def test_encoder_workspace_bytes_host_only(L):
     act = 512 * 256 * 2  # one [B, L, D] buffer, D = 256
     assert lf.lf_encoder_workspace_bytes(24, 1, 4, 512, 64, 512, torch.float16) == one + 2 * act
     assert lf.lf_encoder_workspace_bytes(0, 1, 4, 512, 64, 512, torch.float16) == 0
+
+
+def test_any_globals_layer_workspace_bytes_host_only(L):
+    import torch
+    B, H, Ln, w, F = 1, 16, 4096, 256, 4096
+    pre = lf.lf_encoder_layer_workspace_bytes(B, H, Ln, w, F, torch.float16)
+    anyb = lf.lf_encoder_layer_any_globals_workspace_bytes(B, H, Ln, w, F, torch.float16)
+    D, gcap = H * 64, 256
+    # no position-indexed qg buffer; the partition, rank table, slot buffers
+    # and the gathered rows of x instead
+    extra = (Ln * 4 + Ln * 4 + 3 * B * H * gcap * 64 * 2 + B * gcap * 4 + B * gcap * D * 2)
+    assert anyb == pytest.approx(pre - B * Ln * D * 2 + extra, abs=16 * 256)
+    act = B * Ln * D * 2
+    assert lf.lf_encoder_any_globals_workspace_bytes(3, B, H, Ln, w, F, torch.float16) == anyb + 2 * act
+    assert lf.lf_encoder_layer_any_globals_workspace_bytes(1, 4, 512, 64, 512, torch.float32) == 0

@@ -36,14 +36,16 @@ def _round_to(dtype):
     return rnd
 
 
-def _run_and_compare(x, W, lm, gm, H, w, dtype, rows=None):
+def _run_and_compare(x, W, lm, gm, H, w, dtype, rows=None, any_pos=False):
     dev = {k: v.cuda() for k, v in W.items()}
-    out = lf.lf_encoder_layer_forward(x.cuda(), lm.cuda(), gm.cuda(), dev, H, w, 0.125, 1e-5)
+    fn = lf.lf_encoder_layer_forward_any_globals if any_pos else lf.lf_encoder_layer_forward
+    out = fn(x.cuda(), lm.cuda(), gm.cuda(), dev, H, w, 0.125, 1e-5)
     torch.cuda.synchronize()
     assert lf.lf_device_status(reset=True) == 0
     got = out.float().cpu().numpy()
     ref = oracle.encoder_layer(x, lm, gm, _oracle_weights(W), H, w, 0.125, 1e-5,
-                               round_attention_inputs=_round_to(dtype), round_stored=_round_to(dtype))
+                               round_attention_inputs=_round_to(dtype), round_stored=_round_to(dtype),
+                               any_pos=any_pos)
     # The stated bounds (1e-2 fp16, 2e-2 bf16) are for unit-scale outputs; the
     # layer's LayerNorm outputs reach |y| ~ 5, where one bf16 ulp is 0.0156.
     # Bound: |got - ref| <= tol * max(1, |ref|) per element (~5 bf16 or ~10
@@ -128,3 +130,68 @@ def test_encoder_stack_two_layer_parity(dtype):
     assert np.isfinite(got).all()
     scaled = np.abs(got - ref) / np.maximum(1.0, np.abs(ref))
     assert scaled.max() <= TOL[TDT[dtype]], "max scaled err %g" % scaled.max()
+
+
+# ---------------------------------------------------------------- global tokens at any position
+
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+@pytest.mark.parametrize("B,H,L,w,ffn,g,pad,pg", [
+    (1, 2, 512, 64, 256, [8], [0], 0),
+    (2, 2, 640, 128, 384, [5, 100], [0, 33], 1),   # ragged last M tile, padded global tokens
+    (1, 4, 1024, 256, 512, [200], [17], 3),        # two slot blocks
+])
+def test_layer_any_globals_small_parity(dtype, B, H, L, w, ffn, g, pad, pg):
+    """lf_encoder_layer_forward_any_globals: qg projected from the gathered
+    rows of x, global rows and keys through the slots, against the layer
+    oracle with any_pos."""
+    wl, x, W, _, _ = inputs.layer_inputs(5, hidden=H * 64, ffn=ffn, B=B, L=L, dtype=dtype, g=[0] * B, pad=pad,
+                                         seed=177 + L, bias_scale=0.1, ln_scale=0.1)
+    lm, gm = inputs.masks_scattered(B, L, g, pad, seed=L + 3, padded_globals=pg)
+    _run_and_compare(x, W, lm, gm, H, w, TDT[dtype], any_pos=True)
+
+
+def test_workload5_any_globals_full_parity():
+    """Workload 5's layer with its 64 global tokens at random positions."""
+    wl, x, W, _, _ = inputs.layer_inputs(5)
+    lm, gm = inputs.masks_scattered(wl.B, wl.L, wl.g, wl.pad, seed=1105)
+    _run_and_compare(x, W, lm, gm, wl.H, wl.w, TDT[wl.dtype], any_pos=True)
+
+
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+def test_encoder_any_globals_stack_equals_chained_layers(dtype):
+    """lf_encoder_forward_any_globals (one partition for all layers) gives
+    exactly the bits of chained lf_encoder_layer_forward_any_globals calls."""
+    B, H, L, w, ffn = 2, 2, 640, 128, 256
+    wl, x, _, _, _ = inputs.layer_inputs(5, hidden=H * 64, ffn=ffn, B=B, L=L, dtype=dtype, g=[0, 0], pad=[0, 41],
+                                         seed=191)
+    lm, gm = inputs.masks_scattered(B, L, [5, 70], [0, 41], seed=192, padded_globals=1)
+    layers = [{k: v.cuda() for k, v in W.items()} for W in _stack_weights(3, H, ffn, dtype, 500)]
+    xd, lmd, gmd = x.cuda(), lm.cuda(), gm.cuda()
+    got = lf.lf_encoder_forward_any_globals(xd, lmd, gmd, layers, H, w)
+    ref = xd
+    for W in layers:
+        ref = lf.lf_encoder_layer_forward_any_globals(ref, lmd, gmd, W, H, w)
+    torch.cuda.synchronize()
+    assert lf.lf_device_status(reset=True) == 0
+    assert torch.equal(got, ref)
+
+
+def test_layer_any_globals_too_many_globals():
+    """More than w global tokens: LF_ERR_G_GT_W in the status word, and the
+    other sample's layer output still matches the oracle."""
+    B, H, L, w, ffn = 2, 2, 512, 64, 256
+    wl, x, W, _, _ = inputs.layer_inputs(5, hidden=H * 64, ffn=ffn, B=B, L=L, dtype="f16", g=[0, 0], pad=[0, 0],
+                                         seed=93)
+    lm, gm = inputs.masks_scattered(B, L, [6, 0], [0, 0], seed=94)
+    gm[1, ::5] = 0.0  # 103 > w global tokens in sample 1
+    dev = {k: v.cuda() for k, v in W.items()}
+    lf.lf_device_status(reset=True)
+    out = lf.lf_encoder_layer_forward_any_globals(x.cuda(), lm.cuda(), gm.cuda(), dev, H, w)
+    torch.cuda.synchronize()
+    assert lf.lf_device_status(reset=True) == 5
+    got = out[:1].float().cpu().numpy()
+    ref = oracle.encoder_layer(x[:1], lm[:1], gm[:1], _oracle_weights(W), H, w, 0.125, 1e-5,
+                               round_attention_inputs=_round_to(torch.float16),
+                               round_stored=_round_to(torch.float16), any_pos=True)
+    scaled = np.abs(got - ref) / np.maximum(1.0, np.abs(ref))
+    assert scaled.max() <= TOL[torch.float16]
