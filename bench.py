@@ -16,8 +16,8 @@ no collective on the data path); timings are the max over ranks.
 attention, 3: bf16 batched, 4: fp16 L=16384, 5: one fp16 encoder layer with
 its projections, LayerNorms and FFN, 6: workload 2 with its global tokens at
 random positions, through the entry point for global tokens anywhere, whose
-one call runs the partition, the gather of the global rows and the
-attention kernel); 2 is the default and the headline.
+one call runs the partition fused with the gather of the global rows, and
+the attention kernel); 2 is the default and the headline.
 """
 from __future__ import annotations
 
@@ -376,12 +376,13 @@ def run_ours(args):
             "tensor_peak_frac": F / t_attn / 1e12 / pk["bf16_tflops"] if tensor_path else None,
             "tensor_peak_tflops": pk["bf16_tflops"],
             "note": "fp16 and bf16 dense tensor rates are equal; peak = measured bf16 burst (%s)" % pk_kind
-                    + ("; the timed call is partition + gather + attention (3 kernels)" if anyg else ""),
+                    + ("; the timed call is the fused partition + gather kernel and the attention kernel"
+                       if anyg else ""),
         },
         "roofline": roof,
         "e2e": {"value": job_throughput(world, tokens, 1, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": (3 if anyg else (1 + 10 * n_layers) if any_layer
+        "gpu_launches": (2 if anyg else (1 + 10 * n_layers) if any_layer
                          else 1 + (8 * n_layers if layer else 1)) * K,
         "clocks": clocks,
     }

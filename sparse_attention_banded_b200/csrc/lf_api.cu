@@ -245,16 +245,18 @@ lf_status lf_attention_forward_any_globals(const void* q, const void* k, const v
     } else {
         scratch_dirty(d);  // the partition's outputs start at the scratch's first byte
     }
-    st = launch_global_idx(global_mask, B, L, w, const_cast<int32_t*>(a.global_idx),
-                           const_cast<int32_t*>(a.global_token_nums), d->status, s,
-                           const_cast<int32_t*>(a.rank), false);
-    if (st != LF_OK) return st;
-    if (!tc)
+    if (!tc) {
+        st = launch_global_idx(global_mask, B, L, w, const_cast<int32_t*>(a.global_idx),
+                               const_cast<int32_t*>(a.global_token_nums), d->status, s,
+                               const_cast<int32_t*>(a.rank), false);
+        if (st != LF_OK) return st;
         return launch_attention_simt_f32((const float*)q, (const float*)k, (const float*)v,
                                          (const float*)qg, (const float*)kg, (const float*)vg,
                                          local_mask, global_mask, B, H, L, w, scale, (float*)out,
                                          d->status, s, &a);
-    st = launch_gather_globals(qg, k, v, local_mask, a, B, H, L, w, s);
+    }
+    // partition + gather of the global tokens' rows in one launch
+    st = launch_partition_gather(global_mask, local_mask, qg, k, v, a, B, H, L, w, d->status, s);
     if (st == LF_OK)
         st = launch_attention_tc(q, k, v, qg, kg, vg, local_mask, global_mask, B, H, L, w, scale, dtype, out,
                                  d->scratch, d->status, d->sm_count, s, &a);

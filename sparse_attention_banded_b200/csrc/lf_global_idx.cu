@@ -135,8 +135,9 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 // One CTA of 256 threads per 32 slots of one (b, h): thread t copies the
 // 16-byte column part t % 8 of slot c0 + t / 8 for qg (unless qg is NULL:
 // the encoder layer projects the slots' qg rows itself), k and v; slots past
-// g are zero (finite rows for the masked tail of a block).  The h == 0 CTAs
-// also write the slots' local_mask values.
+// g up to the end of their 128-slot block are zero (finite rows for the
+// masked tail of a block).  The h == 0 CTAs also write the slots' local_mask
+// values.
 __global__ void __launch_bounds__(256)
 gather_globals_kernel(const uint4* __restrict__ qg, const uint4* __restrict__ k, const uint4* __restrict__ v,
                       const float* __restrict__ local_mask, const int32_t* __restrict__ gidx,
@@ -149,6 +150,12 @@ gather_globals_kernel(const uint4* __restrict__ qg, const uint4* __restrict__ k,
     // a sample with g > w is rejected by the attention kernel; min() keeps
     // the slots in range (c < g <= L also keeps the index read in range)
     const int g = min(gnum[b], gcap);
+    if (h == 0 && threadIdx.x < 32) {
+        const int cc = c0 + threadIdx.x;
+        lm_c[(size_t)b * gcap + cc] = cc < g ? local_mask[(size_t)b * L + gidx[(size_t)b * L + cc]] : 0.0f;
+    }
+    // the attention kernel reads the slot blocks that hold slots < g
+    if (c >= (g + 127) / 128 * 128) return;
     const size_t dst = ((size_t)bh * gcap + c) * 8 + part;
     if (c < g) {
         const int j = gidx[(size_t)b * L + c];
@@ -163,9 +170,110 @@ gather_globals_kernel(const uint4* __restrict__ qg, const uint4* __restrict__ k,
         k_c[dst] = z;
         v_c[dst] = z;
     }
-    if (h == 0 && threadIdx.x < 32) {
-        const int cc = c0 + threadIdx.x;
-        lm_c[(size_t)b * gcap + cc] = cc < g ? local_mask[(size_t)b * L + gidx[(size_t)b * L + cc]] : 0.0f;
+}
+
+// The partition and the gather in one launch, for the attention call: one
+// CTA of 1024 threads per (b, h).  Every CTA scans sample b's mask as the
+// partition kernel does and keeps the positions of its first gcap global
+// tokens in shared memory; the h == 0 CTA also writes global_idx,
+// global_token_nums, the rank table and the slots' local_mask values.  Then
+// each CTA copies its head's qg, k and v rows into the slots (zero from g to
+// the end of the last slot block read).
+__global__ void __launch_bounds__(kThreads)
+partition_gather_kernel(const float* __restrict__ global_mask, const float* __restrict__ local_mask, int H, int L,
+                        int w, int gcap, const uint4* __restrict__ qg, const uint4* __restrict__ k,
+                        const uint4* __restrict__ v, int32_t* __restrict__ global_idx,
+                        int32_t* __restrict__ global_token_nums, int32_t* __restrict__ rank, uint4* __restrict__ qg_c,
+                        uint4* __restrict__ k_c, uint4* __restrict__ v_c, float* __restrict__ lm_c, int* status) {
+    extern __shared__ int slot_pos[];  // [gcap]
+    const int bh = blockIdx.x, b = bh / H, h = bh % H;
+    const bool lead = h == 0;  // writes the partition's outputs
+    const float* row = global_mask + (size_t)b * L;
+    int32_t* idx = global_idx + (size_t)b * L;
+    int32_t* rk = rank + (size_t)b * (L + 1);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    __shared__ int warp_tot[kThreads / 32 + 1];
+
+    int base = 0;
+    for (int c0 = 0; c0 < L; c0 += kThreads * kItems) {
+        const int j0 = c0 + tid * kItems;
+        bool f[kItems];
+        int cnt = 0;
+        if (j0 + kItems <= L && (L & 3) == 0) {
+            float4 m4 = *reinterpret_cast<const float4*>(row + j0);
+            f[0] = m4.x == 0.0f; f[1] = m4.y == 0.0f; f[2] = m4.z == 0.0f; f[3] = m4.w == 0.0f;
+        } else {
+#pragma unroll
+            for (int t = 0; t < kItems; ++t) f[t] = (j0 + t < L) && row[j0 + t] == 0.0f;
+        }
+#pragma unroll
+        for (int t = 0; t < kItems; ++t) cnt += f[t];
+        int incl = cnt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            int y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        if (lane == 31) warp_tot[warp] = incl;
+        __syncthreads();
+        if (warp == 0) {
+            const int t = warp_tot[lane];
+            int x = t;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, x, o);
+                if (lane >= o) x += y;
+            }
+            warp_tot[lane] = x - t;
+            if (lane == 31) warp_tot[32] = x;
+        }
+        __syncthreads();
+        int sel = base + warp_tot[warp] + incl - cnt;
+        const int chunk_tot = warp_tot[32];
+#pragma unroll
+        for (int t = 0; t < kItems; ++t) {
+            const int j = j0 + t;
+            if (j < L) {
+                if (lead) rk[j] = sel;
+                if (f[t]) {
+                    if (lead) idx[sel] = j;
+                    if (sel < gcap) slot_pos[sel] = j;
+                    ++sel;
+                } else if (lead) {
+                    idx[L - 1 - (j - sel)] = j;
+                }
+            }
+        }
+        base += chunk_tot;
+        __syncthreads();
+    }
+    const int g = min(base, gcap);
+    if (lead) {
+        if (tid == 0) {
+            global_token_nums[b] = base;
+            rk[L] = base;
+            if (base > w) record_status(status, b, LF_ERR_G_GT_W);
+        }
+        for (int c = tid; c < gcap; c += kThreads)
+            lm_c[(size_t)b * gcap + c] = c < g ? local_mask[(size_t)b * L + slot_pos[c]] : 0.0f;
+    }
+    // this head's rows: 8 threads of 16 bytes per row, 128 rows per pass
+    const int end = (g + 127) / 128 * 128;
+    const int part = tid & 7;
+    for (int c = tid >> 3; c < end; c += kThreads / 8) {
+        const size_t dst = ((size_t)bh * gcap + c) * 8 + part;
+        if (c < g) {
+            const size_t src = ((size_t)bh * L + slot_pos[c]) * 8 + part;
+            const uint4 a = qg[src], kk = k[src], vv = v[src];
+            qg_c[dst] = a;
+            k_c[dst] = kk;
+            v_c[dst] = vv;
+        } else {
+            const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+            qg_c[dst] = z;
+            k_c[dst] = z;
+            v_c[dst] = z;
+        }
     }
 }
 
@@ -195,6 +303,26 @@ lf_status launch_gather_rows(const void* src, const AnyGlobals& a, int B, int L,
     gather_rows_kernel<<<(unsigned)blocks, 128, 0, stream>>>(reinterpret_cast<const uint4*>(src), a.global_idx,
                                                              a.global_token_nums, L, a.gcap, D * 2 / 16,
                                                              reinterpret_cast<uint4*>(dst));
+    return cudaGetLastError() == cudaSuccess ? LF_OK : LF_ERR_CUDA;
+}
+
+lf_status launch_partition_gather(const float* global_mask, const float* local_mask, const void* qg, const void* k,
+                                  const void* v, const AnyGlobals& a, int B, int H, int L, int w, int* status,
+                                  cudaStream_t stream) {
+    const size_t smem = (size_t)a.gcap * sizeof(int);
+    if (smem > 200 * 1024) return LF_ERR_TOO_LARGE;
+    static bool attr = false;
+    if (!attr && smem > 48 * 1024) {
+        if (cudaFuncSetAttribute(partition_gather_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024) !=
+            cudaSuccess)
+            return LF_ERR_CUDA;
+        attr = true;
+    }
+    partition_gather_kernel<<<B * H, kThreads, smem, stream>>>(
+        global_mask, local_mask, H, L, w, a.gcap, reinterpret_cast<const uint4*>(qg),
+        reinterpret_cast<const uint4*>(k), reinterpret_cast<const uint4*>(v), const_cast<int32_t*>(a.global_idx),
+        const_cast<int32_t*>(a.global_token_nums), const_cast<int32_t*>(a.rank), reinterpret_cast<uint4*>(a.qg_c),
+        reinterpret_cast<uint4*>(a.k_c), reinterpret_cast<uint4*>(a.v_c), a.lm_c, status);
     return cudaGetLastError() == cudaSuccess ? LF_OK : LF_ERR_CUDA;
 }
 

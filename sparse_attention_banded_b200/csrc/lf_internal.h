@@ -83,6 +83,11 @@ AnyGlobals any_globals_layout(void* base, int B, int H, int L, int w, bool compa
 // (qg NULL: qg_c is not written).
 lf_status launch_gather_globals(const void* qg, const void* k, const void* v, const float* local_mask,
                                 const AnyGlobals& a, int B, int H, int L, int w, cudaStream_t stream);
+// The partition (with the rank table, no prefix check) and the gather of
+// qg, k, v and local_mask in one launch of B*H CTAs (16-bit dtypes).
+lf_status launch_partition_gather(const float* global_mask, const float* local_mask, const void* qg, const void* k,
+                                  const void* v, const AnyGlobals& a, int B, int H, int L, int w, int* status,
+                                  cudaStream_t stream);
 // Rows of a [B][L][D] 16-bit matrix at the global tokens' positions into
 // [B][gcap][D] (slots past g zero).  D % 8 == 0.
 lf_status launch_gather_rows(const void* src, const AnyGlobals& a, int B, int L, int D, void* dst,

@@ -203,3 +203,46 @@ def test_scratch_reuse_across_shapes_and_dtypes():
     call(anyf, *small[:6], "f32", 34, True)
     assert torch.equal(call(pre, *big, False), ref_pre)
     assert lf.lf_device_status(reset=True) == 0
+
+
+def _sampled(wl_shape, g, pad, dtype, seed, pg=0):
+    B, H, L, w = wl_shape
+    t = inputs.attention_inputs(B, H, L, dtype, seed=seed)
+    lm, gm = inputs.masks_scattered(B, L, g, pad, seed=seed + 1, padded_globals=pg)
+    out = _run(t, lm, gm, w).float().cpu().numpy().reshape(B, L, H, 64)
+    rng = np.random.default_rng(seed)
+    rows = set()
+    for b in range(B):
+        G = np.flatnonzero(gm[b].numpy() == 0.0)
+        rows |= {(b, h, int(i)) for h in (0, H - 1) for i in G}
+        rows |= {(b, int(rng.integers(H)), i) for i in list(range(0, L, 128)) + list(range(127, L, 128))
+                 if rng.random() < 0.3}
+        rows |= {(b, 0, i) for i in (L - pad[b] - 1, L - pad[b], L - 1) if 0 <= i < L}
+    rows |= {(int(rng.integers(B)), int(rng.integers(H)), int(rng.integers(L))) for _ in range(300)}
+    rows = np.array(sorted(rows), dtype=np.int32)
+    ref = oracle.attention_rows(*[t[n] for n in inputs.NAMES], lm, gm, w, rows, any_pos=True)
+    got = out[rows[:, 0], rows[:, 2], rows[:, 1]]
+    err = np.abs(got - ref).max()
+    assert err <= TOL[TDT[dtype]], "max abs err %g" % err
+    assert np.all(out[lm.numpy() != 1.0] == 0.0)
+    assert np.isfinite(out).all()
+
+
+def test_any_globals_batched_bf16_sampled():
+    """Workload 3's shape (bf16, four samples) with each sample's global
+    tokens at random positions, some of them padded."""
+    wl = inputs.workload(3)
+    _sampled((wl.B, wl.H, wl.L, wl.w), wl.g, wl.pad, "bf16", seed=3003, pg=2)
+
+
+def test_any_globals_long_sequence_sampled():
+    """Workload 4's shape (16384 tokens) with 32 global tokens at random positions."""
+    wl = inputs.workload(4)
+    _sampled((wl.B, wl.H, wl.L, wl.w), wl.g, wl.pad, "f16", seed=3004)
+
+
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+def test_any_globals_g_equals_w_odd_band(dtype):
+    """g = w = 192 (a band that is not a multiple of 128, two slot blocks,
+    two global row tiles, the second one partial) at 3072 tokens."""
+    _sampled((1, 4, 3072, 192), [192], [77], dtype, seed=3005, pg=4)
