@@ -126,8 +126,14 @@ lf_status lf_init_global_idx(const float* global_mask, int B, int L, int w,
  * position g_b records LF_ERR_GLOBAL_NOT_PREFIX (output computed with g_b).
  * Scratch: the call uses a library-owned per-device scratch buffer, allocated
  * (cudaMalloc) on the first call on a device and regrown when a call needs
- * more; make that first call before any stream capture.  Calls that overlap
- * on the GPU (different streams) share the scratch and must not overlap.
+ * more.  Make the largest call before any stream capture: regrowing frees
+ * the old buffer, which graphs captured earlier still reference.  The
+ * scratch's counters must be zero when the kernel starts: a call clears
+ * them (a cudaMemsetAsync on `stream`) when a call of another shape or dtype
+ * may have left other data there, and always while `stream` is capturing,
+ * so that a captured call stays correct whatever runs between replays.
+ * Calls that overlap on the GPU (different streams) share the scratch and
+ * must not overlap.
  */
 lf_status lf_attention_forward(const void* q, const void* k, const void* v,
                                const void* qg, const void* kg, const void* vg,

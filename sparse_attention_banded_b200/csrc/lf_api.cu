@@ -73,8 +73,15 @@ lf_status ensure_scratch(DeviceCtx* d, size_t bytes) {
 }
 
 lf_status prepare_scratch_counters(DeviceCtx* d, size_t zero_bytes, cudaStream_t stream) {
+    // Under stream capture the clear is always recorded: the graph may be
+    // replayed after calls of other shapes have written the scratch.
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(stream, &cs) != cudaSuccess) {
+        cudaGetLastError();  // not a launch error of this call
+        cs = cudaStreamCaptureStatusNone;
+    }
     std::lock_guard<std::mutex> lock(g_mutex);
-    if (zero_bytes > d->scratch_clean) {
+    if (zero_bytes > d->scratch_clean || cs == cudaStreamCaptureStatusActive) {
         // A call of another shape (whose partials reached into this range)
         // or another use of the scratch left other bytes here.
         if (cudaMemsetAsync(d->scratch, 0, zero_bytes, stream) != cudaSuccess) {
