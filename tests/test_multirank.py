@@ -69,3 +69,11 @@ def test_reference_arm_prints_on_rank_zero_only(monkeypatch):
     with redirect_stdout(buf):
         bench.run_reference(ns)
     assert buf.getvalue() == ""
+
+
+def test_percentiles_nearest_rank():
+    import bench
+    q = bench.percentiles([5.0, 1.0, 3.0, 2.0, 4.0, 6.0, 7.0, 8.0, 9.0, 10.0, 11.0])
+    assert q == {"p10": 2.0, "median": 6.0, "p90": 10.0}
+    assert bench.percentiles([2.5]) == {"p10": 2.5, "median": 2.5, "p90": 2.5}
+    assert bench.percentiles([]) == {"p10": None, "median": None, "p90": None}
