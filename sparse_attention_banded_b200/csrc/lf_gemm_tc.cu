@@ -30,6 +30,7 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "lf_internal.h"
@@ -347,10 +348,15 @@ lf_status launch_t(const GemmArgs& g, int sm_count, cudaStream_t stream) {
     p.heads_H = g.heads_H;
     p.heads_L = g.heads_L;
     p.status = g.status;
-    static bool attr = false;
-    if (!attr) {
-        cudaFuncSetAttribute(gemm_tc_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-        attr = true;
+    // the shared-memory opt-in is a per-device function attribute
+    static std::atomic<bool> attr[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return LF_ERR_CUDA;
+    if (!attr[dev].load()) {
+        if (cudaFuncSetAttribute(gemm_tc_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) !=
+            cudaSuccess)
+            return LF_ERR_CUDA;
+        attr[dev].store(true);
     }
     const int grid = p.tiles < sm_count ? p.tiles : sm_count;
     gemm_tc_kernel<T><<<grid, kThreads, kSmemBytes, stream>>>(ma, mw, p);

@@ -17,6 +17,8 @@
 //
 // The work is one pass over the mask: L * 4 bytes read, L * 4 bytes written
 // per sample -- HBM-bound and tiny next to the attention kernel.
+#include <atomic>
+
 #include "lf_internal.h"
 
 namespace lf {
@@ -311,12 +313,17 @@ lf_status launch_partition_gather(const float* global_mask, const float* local_m
                                   cudaStream_t stream) {
     const size_t smem = (size_t)a.gcap * sizeof(int);
     if (smem > 200 * 1024) return LF_ERR_TOO_LARGE;
-    static bool attr = false;
-    if (!attr && smem > 48 * 1024) {
-        if (cudaFuncSetAttribute(partition_gather_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024) !=
-            cudaSuccess)
-            return LF_ERR_CUDA;
-        attr = true;
+    if (smem > 48 * 1024) {
+        // the shared-memory opt-in is a per-device function attribute
+        static std::atomic<bool> attr[64];
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return LF_ERR_CUDA;
+        if (!attr[dev].load()) {
+            if (cudaFuncSetAttribute(partition_gather_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     200 * 1024) != cudaSuccess)
+                return LF_ERR_CUDA;
+            attr[dev].store(true);
+        }
     }
     partition_gather_kernel<<<B * H, kThreads, smem, stream>>>(
         global_mask, local_mask, H, L, w, a.gcap, reinterpret_cast<const uint4*>(qg),
