@@ -134,7 +134,7 @@ const char* lf_status_string(int s) {
     }
 }
 
-int lf_version(void) { return 100; }
+int lf_version(void) { return 101; }  // 1.1: the _any_globals entry points
 
 lf_status lf_device_status(lf_stream_t stream, int reset) {
     lf_status st;

@@ -207,3 +207,8 @@ def test_any_globals_layer_workspace_bytes_host_only(L):
     act = B * Ln * D * 2
     assert lf.lf_encoder_any_globals_workspace_bytes(3, B, H, Ln, w, F, torch.float16) == anyb + 2 * act
     assert lf.lf_encoder_layer_any_globals_workspace_bytes(1, 4, 512, 64, 512, torch.float32) == 0
+
+
+def test_version(L):
+    """1.1: the entry points for global tokens at any position."""
+    assert L.lf_version() == 101
