@@ -510,6 +510,38 @@ def test_encoder_layer_matches_torch_composition():
     np.testing.assert_allclose(got, y.numpy(), atol=1e-10)
 
 
+def test_encoder_layer_any_pos_wiring():
+    """The layer oracle with global tokens at any position: on prefix masks
+    the same bits as the prefix definition, and on scattered masks the same
+    composition around oracle.attention(any_pos=True)."""
+    rng = np.random.default_rng(2)
+    B, H, L, w, D, F = 1, 2, 32, 8, 128, 256
+    x = rng.normal(size=(B, L, D))
+    W = {"W_qkv_kgvg": rng.normal(size=(5, D, D)) * 0.05, "b_qkv_kgvg": rng.normal(size=(5, D)) * 0.1,
+         "W_qg": rng.normal(size=(D, D)) * 0.05, "b_qg": rng.normal(size=D) * 0.1,
+         "W_o": rng.normal(size=(D, D)) * 0.05, "b_o": rng.normal(size=D) * 0.1,
+         "ln1_gamma": np.ones(D), "ln1_beta": np.zeros(D),
+         "W_1": rng.normal(size=(D, F)) * 0.05, "b_1": rng.normal(size=F) * 0.1,
+         "W_2": rng.normal(size=(F, D)) * 0.05, "b_2": rng.normal(size=D) * 0.1,
+         "ln2_gamma": np.ones(D), "ln2_beta": np.zeros(D)}
+    lm, gm = inputs.masks(B, L, [3], [4])
+    a = oracle.encoder_layer(x, lm, gm, W, H, w, 0.125, 1e-5)
+    b = oracle.encoder_layer(x, lm, gm, W, H, w, 0.125, 1e-5, any_pos=True)
+    assert np.array_equal(a, b)
+    lm2, gm2 = inputs.masks_scattered(B, L, [5], [4], seed=9, padded_globals=1)
+    got = oracle.encoder_layer(x, lm2, gm2, W, H, w, 0.125, 1e-5, any_pos=True)
+    proj = [oracle.to_heads(x @ W["W_qkv_kgvg"][n] + W["b_qkv_kgvg"][n], H) for n in range(5)]
+    qg = oracle.to_heads(x @ W["W_qg"] + W["b_qg"], H)
+    att = oracle.attention(proj[0], proj[1], proj[2], qg, proj[3], proj[4], lm2, gm2, w, any_pos=True)
+    h = oracle.layer_norm(att.reshape(B, L, D) @ W["W_o"] + W["b_o"] + x, W["ln1_gamma"], W["ln1_beta"], 1e-5)
+    y = oracle.layer_norm(oracle.gelu(h @ W["W_1"] + W["b_1"]) @ W["W_2"] + W["b_2"] + h,
+                          W["ln2_gamma"], W["ln2_beta"], 1e-5)
+    np.testing.assert_allclose(got, y, atol=1e-12)
+    # and it differs from treating the same mask as a prefix would (that is an error there)
+    with pytest.raises(oracle.OracleError):
+        oracle.encoder_layer(x, lm2, gm2, W, H, w, 0.125, 1e-5)
+
+
 def test_workload_draws_are_stable():
     wl = inputs.workload(3)
     assert len(wl.g) == 4 and all(1 <= g <= 128 for g in wl.g)
