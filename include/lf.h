@@ -294,22 +294,46 @@ lf_status lf_encoder_forward_any_globals(const void* x, const float* local_mask,
  * LF_BF16 only (LF_F32 needs no scratch: use lf_attention_forward).  The
  * caller still provides every input and the output.  This call allocates
  * nothing: its scratch is a fixed 32 MiB array in the library's device image,
- * held on every device that has run it until the process exits.  A shape
- * whose scratch (lf_attention_scratch_bytes) exceeds 32 MiB returns
- * LF_ERR_SCRATCH_LIMIT before anything is launched.  The first call on a
- * device looks up the array's device address (cudaGetSymbolAddress); make
- * that first call before any stream capture.  Each call clears the array's
- * counter region on `stream` (cudaMemsetAsync) before its kernel.  All calls
- * share the one array: calls that overlap on the GPU (different streams)
- * race and must not overlap.  Content errors (g_b > w, globals not a prefix)
- * are recorded in a device word of this entry point that the library does
- * not expose; validate masks beforehand when that matters.
+ * reserved on every device where the library's module is loaded (any device
+ * that has made any lf call) until the process exits.  A shape whose scratch
+ * (lf_attention_scratch_bytes) exceeds 32 MiB returns LF_ERR_SCRATCH_LIMIT
+ * before anything is launched.  The first call on a device looks up the
+ * array's device address (cudaGetSymbolAddress); make that first call before
+ * any stream capture.  Each call clears the array's counter region on
+ * `stream` (cudaMemsetAsync) before its kernel.  All calls share the one
+ * array: calls that overlap on the GPU (different streams) race and must not
+ * overlap.  Content errors (g_b > w, globals not a prefix) and expired
+ * device waits are recorded in a status word of this entry point, separate
+ * from the library's, read by lf_noalloc_device_status.
  */
 lf_status lf_attention_forward_noalloc(const void* q, const void* k, const void* v,
                                        const void* qg, const void* kg, const void* vg,
                                        const float* local_mask, const float* global_mask,
                                        int B, int H, int L, int w, lf_dtype dtype,
                                        lf_stream_t stream, void* out);
+
+/*
+ * lf_noalloc_device_status -- as lf_device_status, for the status word of
+ * lf_attention_forward_noalloc (no counterpart on the pages): synchronise
+ * `stream`, return the first error recorded by that entry point's kernel on
+ * the current device since the last reset (LF_OK if none; LF_ERR_G_GT_W,
+ * LF_ERR_GLOBAL_NOT_PREFIX or LF_ERR_DEVICE_TIMEOUT otherwise); reset != 0
+ * clears the word.  Allocates nothing.
+ */
+lf_status lf_noalloc_device_status(lf_stream_t stream, int reset);
+
+/*
+ * lf_selftest_bounded_wait -- a check of the library's failure detection
+ * (no counterpart on the pages).  Every device-side wait of the kernels is
+ * bounded; when one gives up, the kernel records LF_ERR_DEVICE_TIMEOUT in the
+ * device status word and returns instead of hanging.  This call launches one
+ * CTA that waits, with that same bounded routine, on an mbarrier phase that
+ * nothing completes, giving up after limit_ns nanoseconds; it then records
+ * LF_ERR_DEVICE_TIMEOUT (read by lf_device_status) and returns.  limit_ns
+ * must lie in [1000, 100000000] (LF_ERR_BAD_DIM otherwise).  Asynchronous on
+ * `stream`; nothing else is in flight in that CTA when the wait gives up.
+ */
+lf_status lf_selftest_bounded_wait(unsigned long long limit_ns, lf_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -134,7 +134,7 @@ const char* lf_status_string(int s) {
     }
 }
 
-int lf_version(void) { return 101; }  // 1.1: the _any_globals entry points
+int lf_version(void) { return 102; }  // 1.2: lf_noalloc_device_status, lf_selftest_bounded_wait
 
 lf_status lf_device_status(lf_stream_t stream, int reset) {
     lf_status st;

@@ -45,6 +45,7 @@
 #include <stdlib.h>
 
 #include <algorithm>
+#include <atomic>
 #include <functional>
 #include <mutex>
 #include <vector>
@@ -1643,13 +1644,20 @@ int current_sm_count() {
 }
 
 template <typename T, bool kAny>
-void launch_instance(int grid, const Maps& maps, const Params& p, cudaStream_t stream) {
-    static bool attr = false;  // the shared-memory opt-in, once per instance
-    if (!attr) {
-        cudaFuncSetAttribute(attention_tc_kernel<T, kAny>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-        attr = true;
+lf_status launch_instance(int grid, const Maps& maps, const Params& p, cudaStream_t stream) {
+    // The shared-memory opt-in is a per-device function attribute: set once
+    // per device and instance, with the device current.
+    static std::atomic<bool> attr[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return LF_ERR_CUDA;
+    if (!attr[dev].load()) {
+        if (cudaFuncSetAttribute(attention_tc_kernel<T, kAny>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kSmemBytes) != cudaSuccess)
+            return LF_ERR_CUDA;
+        attr[dev].store(true);
     }
     attention_tc_kernel<T, kAny><<<grid, kThreads, kSmemBytes, stream>>>(maps, p);
+    return LF_OK;
 }
 
 struct Geometry {
@@ -1742,13 +1750,12 @@ lf_status launch_attention_tc(const void* q, const void* k, const void* v, const
 #endif
 
     const int grid = p.n_items < sm_count ? p.n_items : sm_count;
-    if (dtype == LF_F16) {
-        if (any) launch_instance<__half, true>(grid, maps, p, stream);
-        else launch_instance<__half, false>(grid, maps, p, stream);
-    } else {
-        if (any) launch_instance<__nv_bfloat16, true>(grid, maps, p, stream);
-        else launch_instance<__nv_bfloat16, false>(grid, maps, p, stream);
-    }
+    lf_status st;
+    if (dtype == LF_F16) st = any ? launch_instance<__half, true>(grid, maps, p, stream)
+                                  : launch_instance<__half, false>(grid, maps, p, stream);
+    else st = any ? launch_instance<__nv_bfloat16, true>(grid, maps, p, stream)
+                  : launch_instance<__nv_bfloat16, false>(grid, maps, p, stream);
+    if (st != LF_OK) return st;
     return cudaGetLastError() == cudaSuccess ? LF_OK : LF_ERR_CUDA;
 }
 

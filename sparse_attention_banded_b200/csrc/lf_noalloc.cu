@@ -88,3 +88,17 @@ extern "C" lf_status lf_attention_forward_noalloc(const void* q, const void* k, 
     return launch_attention_tc(q, k, v, qg, kg, vg, local_mask, global_mask, B, H, L, w, 0.125f, dtype, out,
                                d->scratch, d->status, d->sm_count, s);
 }
+
+extern "C" lf_status lf_noalloc_device_status(lf_stream_t stream, int reset) {
+    NoAllocDevice* d = nullptr;
+    lf_status st = noalloc_device(&d);
+    if (st != LF_OK) return st;
+    if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return LF_ERR_CUDA;
+    int word = LF_STATUS_CLEAR;
+    if (cudaMemcpy(&word, d->status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return LF_ERR_CUDA;
+    if (reset) {
+        const int clear = LF_STATUS_CLEAR;
+        if (cudaMemcpy(d->status, &clear, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return LF_ERR_CUDA;
+    }
+    return word == LF_STATUS_CLEAR ? LF_OK : (lf_status)(word & 0xff);
+}

@@ -64,6 +64,10 @@ def lib():
         L.lf_release_scratch.restype = st
         L.lf_attention_forward_noalloc.argtypes = [vp] * 8 + [i, i, i, i, i, vp, vp]
         L.lf_attention_forward_noalloc.restype = st
+        L.lf_noalloc_device_status.argtypes = [vp, i]
+        L.lf_noalloc_device_status.restype = st
+        L.lf_selftest_bounded_wait.argtypes = [ctypes.c_ulonglong, vp]
+        L.lf_selftest_bounded_wait.restype = st
         L.lf_encoder_layer_workspace_bytes.argtypes = [i, i, i, i, i, i]
         L.lf_encoder_layer_workspace_bytes.restype = ctypes.c_size_t
         L.lf_encoder_layer_forward.argtypes = [vp, vp, vp, ctypes.POINTER(LayerWeights), i, i, i, i,
@@ -191,6 +195,18 @@ def lf_attention_forward_noalloc(q, k, v, qg, kg, vg, local_mask, global_mask, w
                                             _stream(stream), _ptr(out))
     _check(st, "lf_attention_forward_noalloc")
     return out
+
+
+def lf_noalloc_device_status(reset: bool = False, stream=None) -> int:
+    """Synchronise and return the status word of the no-allocation entry
+    point (see lf.h)."""
+    return lib().lf_noalloc_device_status(_stream(stream), 1 if reset else 0)
+
+
+def lf_selftest_bounded_wait(limit_ns: int, stream=None):
+    """Launch the one-CTA kernel whose bounded wait runs out after limit_ns
+    (see lf.h); the result is read with :func:`lf_device_status`."""
+    _check(lib().lf_selftest_bounded_wait(int(limit_ns), _stream(stream)), "lf_selftest_bounded_wait")
 
 
 def lf_encoder_layer_workspace_bytes(B: int, H: int, L: int, w: int, ffn_dim: int, dtype) -> int:

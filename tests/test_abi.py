@@ -210,5 +210,13 @@ def test_any_globals_layer_workspace_bytes_host_only(L):
 
 
 def test_version(L):
-    """1.1: the entry points for global tokens at any position."""
-    assert L.lf_version() == 101
+    """1.2: the no-allocation path's status reader and the bounded-wait self-test."""
+    assert L.lf_version() == 102
+
+
+def test_selftest_wait_limits_checked_on_host(L):
+    """Wait limits outside [1 us, 100 ms] are rejected before anything is
+    launched (no GPU needed)."""
+    import ctypes
+    for bad in (0, 999, 100000001):
+        assert L.lf_selftest_bounded_wait(ctypes.c_ulonglong(bad), None) == 2

@@ -148,25 +148,16 @@ def test_any_globals_repeated_calls_identical():
         assert torch.equal(a, b)
 
 
-def test_any_globals_workload_sampled_parity():
-    """Workload 6 at full size: every global row of two heads, tile edges,
-    the padding boundary and random rows against the oracle."""
+def test_any_globals_workload_full_parity():
+    """Workload 6 at full size (workload 2 with its 64 global tokens at random
+    positions): every element against the oracle."""
     wl, t, lm, gm = inputs.workload_inputs(6)
     out = _run(t, lm, gm, wl.w).float().cpu().numpy().reshape(wl.B, wl.L, wl.H, 64)
-    rng = np.random.default_rng(6)
-    G = np.flatnonzero(gm[0].numpy() == 0.0)
-    rows = {(0, h, int(i)) for h in (0, wl.H - 1) for i in G}
-    rows |= {(0, int(rng.integers(wl.H)), i) for i in list(range(0, wl.L, 128)) + list(range(127, wl.L, 128))}
-    rows |= {(0, int(rng.integers(wl.H)), int(rng.integers(wl.L))) for _ in range(400)}
-    rows |= {(0, 0, wl.L - wl.pad[0] - 1), (0, 0, wl.L - wl.pad[0])}
-    rows = np.array(sorted(rows), dtype=np.int32)
-    ref = oracle.attention_rows(*[t[n] for n in inputs.NAMES], lm, gm, wl.w, rows, any_pos=True)
-    got = out[rows[:, 0], rows[:, 2], rows[:, 1]]
-    err = np.abs(got - ref).max()
+    ref = oracle.attention(*[t[n] for n in inputs.NAMES], lm, gm, wl.w, any_pos=True)
+    err = float(np.abs(out - ref).max())
+    print("workload 6: max abs err %.3e over %d elements" % (err, out.size))
     assert err <= TOL[torch.float16], "max abs err %g" % err
-    pad = lm.numpy() != 1.0
-    assert np.all(out[pad] == 0.0)
-    assert np.isfinite(out).all()
+    assert np.all(out[lm.numpy() != 1.0] == 0.0)
 
 
 def test_scratch_reuse_across_shapes_and_dtypes():
@@ -205,44 +196,35 @@ def test_scratch_reuse_across_shapes_and_dtypes():
     assert lf.lf_device_status(reset=True) == 0
 
 
-def _sampled(wl_shape, g, pad, dtype, seed, pg=0):
+def _full(wl_shape, g, pad, dtype, seed, pg=0):
+    """Global tokens at random positions (pg of them padded per sample) on a
+    full-size shape: every element against the oracle."""
     B, H, L, w = wl_shape
     t = inputs.attention_inputs(B, H, L, dtype, seed=seed)
     lm, gm = inputs.masks_scattered(B, L, g, pad, seed=seed + 1, padded_globals=pg)
     out = _run(t, lm, gm, w).float().cpu().numpy().reshape(B, L, H, 64)
-    rng = np.random.default_rng(seed)
-    rows = set()
-    for b in range(B):
-        G = np.flatnonzero(gm[b].numpy() == 0.0)
-        rows |= {(b, h, int(i)) for h in (0, H - 1) for i in G}
-        rows |= {(b, int(rng.integers(H)), i) for i in list(range(0, L, 128)) + list(range(127, L, 128))
-                 if rng.random() < 0.3}
-        rows |= {(b, 0, i) for i in (L - pad[b] - 1, L - pad[b], L - 1) if 0 <= i < L}
-    rows |= {(int(rng.integers(B)), int(rng.integers(H)), int(rng.integers(L))) for _ in range(300)}
-    rows = np.array(sorted(rows), dtype=np.int32)
-    ref = oracle.attention_rows(*[t[n] for n in inputs.NAMES], lm, gm, w, rows, any_pos=True)
-    got = out[rows[:, 0], rows[:, 2], rows[:, 1]]
-    err = np.abs(got - ref).max()
+    ref = oracle.attention(*[t[n] for n in inputs.NAMES], lm, gm, w, any_pos=True)
+    err = float(np.abs(out - ref).max())
+    print("B%d H%d L%d w%d %s: max abs err %.3e over %d elements" % (B, H, L, w, dtype, err, out.size))
     assert err <= TOL[TDT[dtype]], "max abs err %g" % err
     assert np.all(out[lm.numpy() != 1.0] == 0.0)
-    assert np.isfinite(out).all()
 
 
-def test_any_globals_batched_bf16_sampled():
+def test_any_globals_batched_bf16_full():
     """Workload 3's shape (bf16, four samples) with each sample's global
     tokens at random positions, some of them padded."""
     wl = inputs.workload(3)
-    _sampled((wl.B, wl.H, wl.L, wl.w), wl.g, wl.pad, "bf16", seed=3003, pg=2)
+    _full((wl.B, wl.H, wl.L, wl.w), wl.g, wl.pad, "bf16", seed=3003, pg=2)
 
 
-def test_any_globals_long_sequence_sampled():
+def test_any_globals_long_sequence_full():
     """Workload 4's shape (16384 tokens) with 32 global tokens at random positions."""
     wl = inputs.workload(4)
-    _sampled((wl.B, wl.H, wl.L, wl.w), wl.g, wl.pad, "f16", seed=3004)
+    _full((wl.B, wl.H, wl.L, wl.w), wl.g, wl.pad, "f16", seed=3004)
 
 
 @pytest.mark.parametrize("dtype", ["f16", "bf16"])
 def test_any_globals_g_equals_w_odd_band(dtype):
     """g = w = 192 (a band that is not a multiple of 128, two slot blocks,
     two global row tiles, the second one partial) at 3072 tokens."""
-    _sampled((1, 4, 3072, 192), [192], [77], dtype, seed=3005, pg=4)
+    _full((1, 4, 3072, 192), [192], [77], dtype, seed=3005, pg=4)

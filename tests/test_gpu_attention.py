@@ -9,7 +9,7 @@ import torch
 
 import oracle
 from sparse_attention_banded_b200 import build, inputs, lf
-from tests._util import TOL, sample_rows
+from tests._util import TOL
 
 pytestmark = pytest.mark.gpu
 
@@ -203,15 +203,16 @@ def test_workload1_full_parity():
 
 
 @pytest.mark.parametrize("cid", [2, 3, 4])
-def test_workload_sampled_parity(cid):
+def test_workload_full_parity(cid):
+    """Workloads 2 (fp16, 4096 tokens, 300 padded), 3 (bf16, four samples
+    with their own g and padding) and 4 (fp16, 16384 tokens) at full size:
+    every element of the output against the oracle, in the launch
+    configuration the benchmark times."""
     wl, t, lm, gm = inputs.workload_inputs(cid)
     out = _run(t, lm, gm, wl.w).float().cpu().numpy().reshape(wl.B, wl.L, wl.H, 64)
-    rows = sample_rows(wl.B, wl.H, wl.L, wl.g, wl.pad, seed=cid)
-    ref = oracle.attention_rows(*[t[n] for n in inputs.NAMES], lm, gm, wl.w, rows)
-    got = out[rows[:, 0], rows[:, 2], rows[:, 1]]
-    err = np.abs(got - ref).max()
+    ref = oracle.attention(*[t[n] for n in inputs.NAMES], lm, gm, wl.w)
+    err = float(np.abs(out - ref).max())
+    print("workload %d: max abs err %.3e over %d elements" % (cid, err, out.size))
     assert err <= TOL[TDT[wl.dtype]], "max abs err %g" % err
-    # properties over every row at full size
     pad = lm.numpy() != 1.0
     assert np.all(out[pad] == 0.0)
-    assert np.isfinite(out).all()
