@@ -683,18 +683,21 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
     }
 #endif
 
-    // Every role but the planner reads the item plans from the ring in order.
-    auto next_plan = [&](uint32_t k, Plan& pl) -> bool {
+    // Every role but the planner reads the item plans in order, in place in
+    // the shared-memory ring: the slot of item k - 1 is handed back when the
+    // role asks for item k (so no role keeps a copy of a plan).
+    auto next_plan = [&](uint32_t k) -> const Plan* {
+        if (k > 0) {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&item_empty[(k - 1) % kRing]);
+        }
         const uint32_t slot = k % kRing;
         bool ok = true;
         if (lane == 0) ok = mbar_wait(&item_full[slot], (k / kRing) & 1, abort_flag);
         ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-        if (!ok) return false;
-        __syncwarp();       // lane 0's acquire orders the reads below
-        pl = plans[slot];   // published by the planner before item_full
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&item_empty[slot]);
-        return true;
+        if (!ok) return nullptr;
+        __syncwarp();  // lane 0's acquire orders the other lanes' reads of the plan
+        return &plans[slot];
     };
 
     if (warp < kSoftmaxWarp0) {
@@ -705,9 +708,11 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
         uint32_t kv_cnt = 0, item_cnt = 0;
         bool ok = true;
         for (uint32_t k = 0; ok; ++k) {
-            Plan pl;
-            TIMED(0, ok = next_plan(k, pl));
+            const Plan* plp = nullptr;
+            TIMED(0, plp = next_plan(k));
+            ok = plp != nullptr;
             if (!ok) break;
+            const Plan& pl = *plp;
             if (pl.id < 0) break;
             if (pl.nloads == 0) {
                 if (lane == 0) mbar_arrive(tma_done);
@@ -845,9 +850,11 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
         };
         bool ok = true;
         for (uint32_t k = 0; ok; ++k) {
-            Plan pl;
-            TIMED(0, ok = next_plan(k, pl));
+            const Plan* plp = nullptr;
+            TIMED(0, plp = next_plan(k));
+            ok = plp != nullptr;
             if (!ok) break;
+            const Plan& pl = *plp;
             if (pl.id < 0) break;
             if (pl.nloads == 0) continue;
             if (lane == 0) {
@@ -945,9 +952,11 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
         TDECL;
         bool ok = true;
         for (uint32_t k = 0; ok; ++k) {
-            Plan pl;
-            TIMED(0, ok = next_plan(k, pl));
+            const Plan* plp = nullptr;
+            TIMED(0, plp = next_plan(k));
+            ok = plp != nullptr;
             if (!ok) break;
+            const Plan& pl = *plp;
             if (pl.id < 0) break;
             if (pl.nloads == 0) continue;
             const int nA = tile_blocks(pl.t[0]), nB = tile_blocks(pl.t[1]);
@@ -1270,9 +1279,11 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
         const unsigned long long tent_ = globaltimer();
 #endif
         for (uint32_t k = 0; ok; ++k) {
-            Plan pl;
-            TIMED(0, ok = next_plan(k, pl));
+            const Plan* plp = nullptr;
+            TIMED(0, plp = next_plan(k));
+            ok = plp != nullptr;
             if (!ok) break;
+            const Plan& pl = *plp;
             if (pl.id < 0) break;
 #if LF_TRACE
             if (k < 3) tacc[11 + k] = (long long)(globaltimer() - tent_);
