@@ -1509,6 +1509,10 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
+    // Launched with programmatic stream serialization, this grid may have
+    // started while the kernel before it was still running; it completes only
+    // after that kernel has, so work queued after it sees both.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 #if LF_TRACE
     if (threadIdx.x == 32 && p.trace) {  // exit time (after the TMEM release)
         volatile int* d_ = p.trace + gridDim.x * 16 * 4 + (blockIdx.x * 16 + 15) * 16;
@@ -1667,7 +1671,22 @@ lf_status launch_instance(int grid, const Maps& maps, const Params& p, cudaStrea
             return LF_ERR_CUDA;
         attr[dev].store(true);
     }
-    attention_tc_kernel<T, kAny><<<grid, kThreads, kSmemBytes, stream>>>(maps, p);
+    // The prefix instance reads nothing that the kernel before it may still
+    // be writing when that kernel is this library's partition kernel (the
+    // only kernel here that lets a dependent start early), so it is launched
+    // with programmatic stream serialization and overlaps it.  Any other
+    // preceding work completes first, as usual.
+    cudaLaunchAttribute attr_pdl[1];
+    attr_pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr_pdl[0].val.programmaticStreamSerializationAllowed = kAny ? 0 : 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kSmemBytes;
+    cfg.stream = stream;
+    cfg.attrs = attr_pdl;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, attention_tc_kernel<T, kAny>, maps, p) != cudaSuccess) return LF_ERR_CUDA;
     return LF_OK;
 }
 
