@@ -53,7 +53,13 @@ def _run_and_compare(x, W, lm, gm, H, w, dtype, rows=None, any_pos=False):
     assert np.isfinite(got).all()
     scaled = np.abs(got - ref) / np.maximum(1.0, np.abs(ref))
     err = scaled.max()
-    assert err <= TOL[dtype], "max scaled err %g (max abs %g)" % (err, np.abs(got - ref).max())
+    abs_err = float(np.abs(got - ref).max())
+    print("layer %s: max abs err %.3e, max scaled err %.3e, max |ref| %.2f" % (dtype, abs_err, err, np.abs(ref).max()))
+    assert err <= TOL[dtype], "max scaled err %g (max abs %g)" % (err, abs_err)
+    if dtype == torch.float16:
+        # fp16 also meets the absolute bound (measured ~2.5e-3); bf16 does not
+        # always (~2.1e-2 at |y| ~ 5, under one bf16 ulp there, 0.031)
+        assert abs_err <= TOL[dtype], "max abs err %g" % abs_err
     return err
 
 
