@@ -188,7 +188,7 @@ def traffic_from_profile(kernel_src_hash: str):
 
 def kernel_source_hash():
     h = hashlib.sha256()
-    for name in ("lf_attn_tc.cu", "sm100.cuh"):
+    for name in ("lf_attn_tc.cu", "lf_pair_math.cuh", "sm100.cuh"):
         with open(os.path.join(ROOT, "sparse_attention_banded_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
