@@ -652,11 +652,9 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
             if (lane == 0) mbar_arrive(&item_empty[(k - 1) % kRing]);
         }
         const uint32_t slot = k % kRing;
-        bool ok = true;
-        if (lane == 0) ok = mbar_wait(&item_full[slot], (k / kRing) & 1, abort_flag);
-        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        // every lane waits (and so acquires the planner's writes of the plan)
+        const bool ok = __all_sync(0xffffffffu, mbar_wait(&item_full[slot], (k / kRing) & 1, abort_flag));
         if (!ok) return nullptr;
-        __syncwarp();  // lane 0's acquire orders the other lanes' reads of the plan
         return &plans[slot];
     };
 
@@ -664,9 +662,13 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
     regs_dec<kRegsProducer>();
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
+        // The whole warp runs the control flow; lane 0 issues the copies.
         TDECL;
         uint32_t kv_cnt = 0, item_cnt = 0;
         bool ok = true;
+        auto wait_all = [&](uint64_t* bar, uint32_t parity) -> bool {
+            return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
+        };
         for (uint32_t k = 0; ok; ++k) {
             const Plan* plp = nullptr;
             TIMED(0, plp = next_plan(k));
@@ -678,38 +680,38 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
                 if (lane == 0) mbar_arrive(tma_done);
                 continue;
             }
-            if (lane == 0) {
-                const uint32_t qb = item_cnt & 1;
-                TRACE(0, 12, pl.id, item_cnt, 0);
-                TIMED(1, ok = mbar_wait(&q_empty[qb], ((item_cnt >> 1) & 1) ^ 1, abort_flag));
-                if (ok) {
-                    const int nq = pl.t[0].present + pl.t[1].present;
-                    mbar_arrive_expect_tx(&q_full[qb], nq * kTileBytes);
-                    for (int x = 0; x < 2; ++x)
-                        if (pl.t[x].present)
-                            tma_load_3d(smem + kOffQ + (qb * 2 + x) * kTileBytes, pl.global ? &maps.qg : &maps.q,
-                                        &q_full[qb], 0, pl.t[x].r0, pl.bh);
-                }
-                // Every load of the plan is issued (the MMA warp maps a tile's
-                // blocks to ring stages by load index).
-                for (int q = 0; q < pl.nloads && ok; ++q) {
-                    int kb, nA, nB, cmp;
-                    load_at<kAny>(pl, q, kb, nA, nB, cmp);
+            const uint32_t qb = item_cnt & 1;
+            if (lane == 0) TRACE(0, 12, pl.id, item_cnt, 0);
+            TIMED(1, ok = wait_all(&q_empty[qb], ((item_cnt >> 1) & 1) ^ 1));
+            if (ok && lane == 0) {
+                const int nq = pl.t[0].present + pl.t[1].present;
+                mbar_arrive_expect_tx(&q_full[qb], nq * kTileBytes);
+                for (int x = 0; x < 2; ++x)
+                    if (pl.t[x].present)
+                        tma_load_3d(smem + kOffQ + (qb * 2 + x) * kTileBytes, pl.global ? &maps.qg : &maps.q,
+                                    &q_full[qb], 0, pl.t[x].r0, pl.bh);
+            }
+            // Every load of the plan is issued (the MMA warp maps a tile's
+            // blocks to ring stages by load index).
+            for (int q = 0; q < pl.nloads && ok; ++q) {
+                int kb, nA, nB, cmp;
+                load_at<kAny>(pl, q, kb, nA, nB, cmp);
+                const uint32_t st = kv_cnt % kStages;
+                if (lane == 0) TRACE(0, 13, pl.id, q, kv_cnt);
+                TIMED(2, ok = wait_all(&kv_empty[st], ((kv_cnt / kStages) & 1) ^ 1));
+                if (!ok) break;
+                if (lane == 0) {
                     const CUtensorMap* mk = pl.global ? &maps.kg : (cmp ? &maps.kc : &maps.k);
                     const CUtensorMap* mv = pl.global ? &maps.vg : (cmp ? &maps.vc : &maps.v);
-                    const uint32_t st = kv_cnt % kStages;
-                    TRACE(0, 13, pl.id, q, kv_cnt);
-                    TIMED(2, ok = mbar_wait(&kv_empty[st], ((kv_cnt / kStages) & 1) ^ 1, abort_flag));
-                    if (!ok) break;
                     mbar_arrive_expect_tx(&kv_full[st], 2 * kTileBytes);
                     tma_load_3d(smem + kOffK + st * kTileBytes, mk, &kv_full[st], 0, kb * kBN, pl.bh);
                     tma_load_3d(smem + kOffV + st * kTileBytes, mv, &kv_full[st], 0, kb * kBN, pl.bh);
-                    ++kv_cnt;
                 }
-                if (ok) mbar_arrive(tma_done);
+                ++kv_cnt;
             }
+            if (ok && lane == 0) mbar_arrive(tma_done);
+            __syncwarp();
             ++item_cnt;
-            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
         }
         if (lane == 0) TRACE(0, 19, ok ? 1 : 0, item_cnt, kv_cnt);
         if (lane == 0) TDUMP(0);
@@ -729,24 +731,21 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
         for (uint32_t k = 0; ok; ++k) {
             const uint32_t slot = k % kRing;
             int id = -1;
-            if (lane == 0) {
-                // Take item k only once the TMA warp has issued every load of
-                // item k-1: a CTA holds at most one item in reserve, taken a
-                // few K/V stages before it is needed, so items are not hoarded
-                // by early CTAs while others idle.
-                if (k > 0) ok = mbar_wait(tma_done, (k - 1) & 1, abort_flag);
-                if (ok) ok = mbar_wait(&item_empty[slot], ((k / kRing) & 1) ^ 1, abort_flag);
-                if (ok) {
-                    // The first item of CTA c is item c (no atomic on the
-                    // critical path of the start); later ones come from the
-                    // counter, which counts past the first gridDim.x items.
-                    id = k == 0 ? (int)blockIdx.x : (int)gridDim.x + atomicAdd(p.sched, 1);
-                    if (id >= p.n_items) id = -1;
-                }
-            }
-            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-            id = __shfl_sync(0xffffffffu, id, 0);
+            // Take item k only once the TMA warp has issued every load of
+            // item k-1: a CTA holds at most one item in reserve, taken a few
+            // K/V stages before it is needed, so items are not hoarded by
+            // early CTAs while others idle.  (The whole warp waits.)
+            if (k > 0) ok = __all_sync(0xffffffffu, mbar_wait(tma_done, (k - 1) & 1, abort_flag));
+            if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&item_empty[slot], ((k / kRing) & 1) ^ 1, abort_flag));
             if (!ok) break;
+            if (lane == 0) {
+                // The first item of CTA c is item c (no atomic on the critical
+                // path of the start); later ones come from the counter, which
+                // counts past the first gridDim.x items.
+                id = k == 0 ? (int)blockIdx.x : (int)gridDim.x + atomicAdd(p.sched, 1);
+                if (id >= p.n_items) id = -1;
+            }
+            id = __shfl_sync(0xffffffffu, id, 0);
             Plan pl;
             if (id >= 0) pl = make_plan<kAny>(p, id, cached_b, g);
             else pl.id = -1;
@@ -780,32 +779,42 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
         uint32_t s_use = 0;  // S products issued (s_free phases)
         uint32_t p_use = 0;  // P blocks consumed (p_full phases)
         uint32_t o_use = 0;  // items with blocks (o_free phases)
+        // The whole warp runs the control flow together (a single lane running
+        // it while the other 31 wait at a warp barrier made every step of it
+        // take microseconds); only the tensor-core instructions, commits and
+        // arrivals are issued by lane 0.
+        auto wait_all = [&](uint64_t* bar, uint32_t parity) -> bool {
+            return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
+        };
         // O (+)= P V for the tile's block j read from stage st; the stage is
         // released when the product is done.
         auto issue_pv = [&](int j, uint32_t st) -> bool {
             bool w_ok;
-            TIMED(3, w_ok = mbar_wait(&p_full[x], p_use & 1u, abort_flag));
+            TIMED(3, w_ok = wait_all(&p_full[x], p_use & 1u));
             if (!w_ok) return false;
             ++p_use;
             TCOUNT(5);
             if (j == 0) {
-                TIMED(4, w_ok = mbar_wait(&o_free[x], (o_use & 1u) ^ 1u, abort_flag));
+                TIMED(4, w_ok = wait_all(&o_free[x], (o_use & 1u) ^ 1u));
                 if (!w_ok) return false;
                 ++o_use;
             }
             tc_fence_after();
-            const uint64_t dv = dv0 + st * kTileStep;
+            if (lane == 0) {
+                const uint64_t dv = dv0 + st * kTileStep;
 #if LF_TRACE
-            const long long tp0_ = clock64();
+                const long long tp0_ = clock64();
 #endif
 #pragma unroll
-            for (int kk = 0; kk < kBN / 16; ++kk)
-                mma_f16_ts(t_o, t_p + kk * 8, dv + kk * (2048 >> 4), idesc_pv, (j == 0 && kk == 0) ? 0u : 1u);
-            tc_commit(&pv_done[x]);
-            tc_commit(&kv_empty[st]);
+                for (int kk = 0; kk < kBN / 16; ++kk)
+                    mma_f16_ts(t_o, t_p + kk * 8, dv + kk * (2048 >> 4), idesc_pv, (j == 0 && kk == 0) ? 0u : 1u);
+                tc_commit(&pv_done[x]);
+                tc_commit(&kv_empty[st]);
 #if LF_TRACE
-            tacc[8] += clock64() - tp0_;
+                tacc[8] += clock64() - tp0_;
 #endif
+            }
+            __syncwarp();
             return true;
         };
         bool ok = true;
@@ -817,54 +826,54 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
             const Plan& pl = *plp;
             if (pl.id < 0) break;
             if (pl.nloads == 0) continue;
-            if (lane == 0) {
-                const uint32_t qb = item_cnt & 1;
-                const int nA = tile_blocks(pl.t[0]), nB = tile_blocks(pl.t[1]);
-                const int nx = x ? nB : nA;
-                const int glob = pl.global, e1 = pl.e1, lo_min = pl.lo_min;
-                const int gh = pl.t[x].glob_hi, lo = pl.t[x].lo, hi = pl.t[x].hi;
-                const int m = min(nA, nB);
-                // load index of this tile's block j
-                auto load_idx = [&](int j) -> int {
-                    if (glob) return j < m ? 2 * j + x : m + j;
-                    if (kAny) return j < gh ? j : e1 + (lo + (j - gh) - lo_min);  // slot blocks first
-                    const int kb = j < gh ? j : lo + (j - gh);
-                    return kb < e1 ? kb : e1 + (kb - lo_min);
-                };
-                // is load q one of this tile's blocks?
-                auto mine = [&](int q) -> bool {
-                    if (nx == 0) return false;
-                    if (glob) return q < 2 * m ? (q & 1) == x : nx > m;
-                    if (kAny && q < e1) return q < gh;
-                    const int kb = q < e1 ? q : lo_min + (q - e1);
-                    return (!kAny && kb < gh) || (kb >= lo && kb <= hi);
-                };
-                int q_ready = -1;
-                // wait for loads up to q; loads this tile does not use are released at once
-                auto take_loads = [&](int q) -> bool {
-                    while (q_ready < q) {
-                        ++q_ready;
-                        const uint32_t c = kv_cnt + q_ready, st = c % kStages;
-                        bool w_ok;
-                        TIMED(2, w_ok = mbar_wait(&kv_full[st], (c / kStages) & 1, abort_flag));
-                        if (!w_ok) return false;
-                        if (!mine(q_ready)) mbar_arrive(&kv_empty[st]);
-                    }
-                    return true;
-                };
-                if (nx > 0) TIMED(1, ok = mbar_wait(&q_full[qb], (item_cnt >> 1) & 1, abort_flag));
-                const uint64_t dqx = dq0 + (qb * 2 + x) * kTileStep;
-                uint32_t st_prev = 0;
-                for (int j = 0; j < nx && ok; ++j) {
-                    const int q = load_idx(j);
-                    ok = take_loads(q);
-                    if (!ok) break;
-                    // the softmax warps have read the previous S
-                    TIMED(6, ok = mbar_wait(&s_free[x], (s_use & 1u) ^ 1u, abort_flag));
-                    if (!ok) break;
-                    ++s_use;
-                    tc_fence_after();
-                    const uint32_t st = (kv_cnt + q) % kStages;
+            const uint32_t qb = item_cnt & 1;
+            const int nA = tile_blocks(pl.t[0]), nB = tile_blocks(pl.t[1]);
+            const int nx = x ? nB : nA;
+            const int glob = pl.global, e1 = pl.e1, lo_min = pl.lo_min;
+            const int gh = pl.t[x].glob_hi, lo = pl.t[x].lo, hi = pl.t[x].hi;
+            const int m = min(nA, nB);
+            // load index of this tile's block j
+            auto load_idx = [&](int j) -> int {
+                if (glob) return j < m ? 2 * j + x : m + j;
+                if (kAny) return j < gh ? j : e1 + (lo + (j - gh) - lo_min);  // slot blocks first
+                const int kb = j < gh ? j : lo + (j - gh);
+                return kb < e1 ? kb : e1 + (kb - lo_min);
+            };
+            // is load q one of this tile's blocks?
+            auto mine = [&](int q) -> bool {
+                if (nx == 0) return false;
+                if (glob) return q < 2 * m ? (q & 1) == x : nx > m;
+                if (kAny && q < e1) return q < gh;
+                const int kb = q < e1 ? q : lo_min + (q - e1);
+                return (!kAny && kb < gh) || (kb >= lo && kb <= hi);
+            };
+            int q_ready = -1;
+            // wait for loads up to q; loads this tile does not use are released at once
+            auto take_loads = [&](int q) -> bool {
+                while (q_ready < q) {
+                    ++q_ready;
+                    const uint32_t c = kv_cnt + q_ready, st = c % kStages;
+                    bool w_ok;
+                    TIMED(2, w_ok = wait_all(&kv_full[st], (c / kStages) & 1));
+                    if (!w_ok) return false;
+                    if (!mine(q_ready) && lane == 0) mbar_arrive(&kv_empty[st]);
+                }
+                return true;
+            };
+            if (nx > 0) TIMED(1, ok = wait_all(&q_full[qb], (item_cnt >> 1) & 1));
+            const uint64_t dqx = dq0 + (qb * 2 + x) * kTileStep;
+            uint32_t st_prev = 0;
+            for (int j = 0; j < nx && ok; ++j) {
+                const int q = load_idx(j);
+                ok = take_loads(q);
+                if (!ok) break;
+                // the softmax warps have read the previous S
+                TIMED(6, ok = wait_all(&s_free[x], (s_use & 1u) ^ 1u));
+                if (!ok) break;
+                ++s_use;
+                tc_fence_after();
+                const uint32_t st = (kv_cnt + q) % kStages;
+                if (lane == 0) {
                     const uint64_t dk = dk0 + st * kTileStep;
 #if LF_TRACE
                     const long long tq0_ = clock64();
@@ -876,19 +885,20 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
 #if LF_TRACE
                     tacc[7] += clock64() - tq0_;
 #endif
-                    if (j > 0) ok = issue_pv(j - 1, st_prev);
-                    st_prev = st;
                 }
-                if (ok && nx > 0) ok = issue_pv(nx - 1, st_prev);
-                if (ok) ok = take_loads(pl.nloads - 1);
-                if (ok) {
-                    if (nx > 0) tc_commit(&q_empty[qb]);
-                    else mbar_arrive(&q_empty[qb]);
-                }
+                __syncwarp();
+                if (j > 0) ok = issue_pv(j - 1, st_prev);
+                st_prev = st;
             }
+            if (ok && nx > 0) ok = issue_pv(nx - 1, st_prev);
+            if (ok) ok = take_loads(pl.nloads - 1);
+            if (ok && lane == 0) {
+                if (nx > 0) tc_commit(&q_empty[qb]);
+                else mbar_arrive(&q_empty[qb]);
+            }
+            __syncwarp();
             ++item_cnt;
             kv_cnt += pl.nloads;
-            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
         }
         if (lane == 0) TDUMP(1 + 2 * x);
         if (lane == 0 && !ok) {  // wind-down: wait for the MMAs already issued
