@@ -146,45 +146,53 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
+    // The TMA and MMA warps run their loops with all 32 lanes (lane 0 issues
+    // the copies, tensor-core instructions and commits): a lone lane running
+    // the loop while the other 31 wait at a warp barrier is several times
+    // slower at every hand-off.
+    auto wait_all = [&](uint64_t* bar, uint32_t parity) -> bool {
+        return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
+    };
     if (warp == 0) {
-        if (lane == 0) {
-            uint32_t kc = 0;
-            bool ok = true;
-            for (int t = blockIdx.x; t < p.tiles && ok; t += gridDim.x) {
-                const int nt = t % p.ntiles;
-                const int bm = t / p.ntiles;
-                const int mt = bm % p.mtiles, b = bm / p.mtiles;
-                for (int kt = 0; kt < p.ktiles && ok; ++kt, ++kc) {
-                    const uint32_t st = kc % kStages;
-                    ok = mbar_wait(&empty[st], ((kc / kStages) & 1) ^ 1, abort_flag);
-                    if (!ok) break;
+        uint32_t kc = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < p.tiles && ok; t += gridDim.x) {
+            const int nt = t % p.ntiles;
+            const int bm = t / p.ntiles;
+            const int mt = bm % p.mtiles, b = bm / p.mtiles;
+            for (int kt = 0; kt < p.ktiles && ok; ++kt, ++kc) {
+                const uint32_t st = kc % kStages;
+                ok = wait_all(&empty[st], ((kc / kStages) & 1) ^ 1);
+                if (!ok) break;
+                if (lane == 0) {
                     mbar_arrive_expect_tx(&full[st], kABytes + kBBytes);
                     tma_load_3d(smem + kOffA + st * kABytes, &map_a, &full[st], kt * kTK, mt * kTM, b);
                     tma_load_2d(smem + kOffB + st * kBBytes, &map_w, &full[st], kt * kTK, nt * kTN);
                 }
+                __syncwarp();
             }
-            if (!ok) {  // wind-down: let issued copies land
-                for (uint32_t c = (kc > kStages ? kc - kStages : 0); c < kc; ++c) {
-                    volatile int never = 0;
-                    mbar_wait(&full[c % kStages], (c / kStages) & 1, &never, 200000000ull);
-                }
+        }
+        if (!ok && lane == 0) {  // wind-down: let issued copies land
+            for (uint32_t c = (kc > kStages ? kc - kStages : 0); c < kc; ++c) {
+                volatile int never = 0;
+                mbar_wait(&full[c % kStages], (c / kStages) & 1, &never, 200000000ull);
             }
         }
     } else if (warp == 1) {
-        if (lane == 0) {
-            constexpr uint32_t idesc = idesc_f16(Cvt<T>::fmt, kTM, kTN, 0, 0);
-            uint32_t kc = 0, tc = 0;
-            bool ok = true;
-            for (int t = blockIdx.x; t < p.tiles && ok; t += gridDim.x, ++tc) {
-                const uint32_t ab = tc & 1;
-                ok = mbar_wait(&acc_empty[ab], ((tc >> 1) & 1) ^ 1, abort_flag);
+        constexpr uint32_t idesc = idesc_f16(Cvt<T>::fmt, kTM, kTN, 0, 0);
+        uint32_t kc = 0, tc = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < p.tiles && ok; t += gridDim.x, ++tc) {
+            const uint32_t ab = tc & 1;
+            ok = wait_all(&acc_empty[ab], ((tc >> 1) & 1) ^ 1);
+            if (!ok) break;
+            tc_fence_after();
+            for (int kt = 0; kt < p.ktiles && ok; ++kt, ++kc) {
+                const uint32_t st = kc % kStages;
+                ok = wait_all(&full[st], (kc / kStages) & 1);
                 if (!ok) break;
                 tc_fence_after();
-                for (int kt = 0; kt < p.ktiles && ok; ++kt, ++kc) {
-                    const uint32_t st = kc % kStages;
-                    ok = mbar_wait(&full[st], (kc / kStages) & 1, abort_flag);
-                    if (!ok) break;
-                    tc_fence_after();
+                if (lane == 0) {
                     const uint32_t a_addr = smem_u32(smem + kOffA + st * kABytes);
                     const uint32_t b_addr = smem_u32(smem + kOffB + st * kBBytes);
 #pragma unroll
@@ -193,13 +201,15 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
                                    (kt > 0 || kk > 0) ? 1u : 0u);
                     tc_commit(&empty[st]);
                 }
-                if (ok) tc_commit(&acc_full[ab]);
+                __syncwarp();
             }
-            if (!ok) {
-                tc_commit(drain);
-                volatile int never = 0;
-                mbar_wait(drain, 0, &never, 200000000ull);
-            }
+            if (ok && lane == 0) tc_commit(&acc_full[ab]);
+            __syncwarp();
+        }
+        if (!ok && lane == 0) {
+            tc_commit(drain);
+            volatile int never = 0;
+            mbar_wait(drain, 0, &never, 200000000ull);
         }
     } else if (warp >= 4) {
         const int sp = warp & 3;               // TMEM lane quarter
