@@ -176,6 +176,19 @@ def layer_norm(z, gamma, beta, eps):
     return gamma * (z - mu) / np.sqrt(var + eps) + beta
 
 
+def gelu_ffn(h, W_1, b_1, W_2, b_2, round_stored=None):
+    """Step 6 of the layer before its LayerNorm (FTL §Longformer Encoder
+    计算流程 / 每个 Transformer 层 step 6, GeluFfnLayer; the FastFFN page's
+    linear -> GELU -> linear): h + b_2 + GELU(h W_1 + b_1) W_2, with the
+    oracle's x @ W convention (W_1 [D, F], W_2 [F, D]).  round_stored:
+    optional function applied to the F-wide intermediate, which the page's
+    layer stores in T.  Float64 throughout."""
+    keep = round_stored or (lambda a: a)
+    h = _f64(h)
+    f = keep(gelu(h @ _f64(W_1) + _f64(b_1)))
+    return f @ _f64(W_2) + _f64(b_2) + h
+
+
 def to_heads(y, H):
     """[B, L, H*64] -> [B, H, L, 64] (AddBiasTransposeToMultiHead layout, step 2)."""
     B, L, _ = y.shape
@@ -208,5 +221,5 @@ def encoder_layer(x, local_mask, global_mask, weights: dict, H: int, w: int,
     B, L = x.shape[:2]
     att = keep(att.reshape(B, L, H * D))
     h = keep(layer_norm(att @ W["W_o"] + W["b_o"] + x, W["ln1_gamma"], W["ln1_beta"], eps))
-    f = keep(gelu(h @ W["W_1"] + W["b_1"]))
-    return layer_norm(f @ W["W_2"] + W["b_2"] + h, W["ln2_gamma"], W["ln2_beta"], eps)
+    z = gelu_ffn(h, W["W_1"], W["b_1"], W["W_2"], W["b_2"], round_stored=keep)
+    return layer_norm(z, W["ln2_gamma"], W["ln2_beta"], eps)

@@ -510,6 +510,30 @@ def test_encoder_layer_matches_torch_composition():
     np.testing.assert_allclose(got, y.numpy(), atol=1e-10)
 
 
+def test_gelu_ffn_matches_torch_and_rounds_only_the_intermediate():
+    """The FFN oracle (step 6 before LN) against torch float64 library ops
+    (linear, gelu with its own erf), and its rounding hook: applied to the
+    intermediate only (rounding to fp16 changes the result, and equals
+    rounding that intermediate by hand)."""
+    rng = np.random.default_rng(5)
+    M, D, F = 37, 128, 384
+    h = rng.normal(size=(M, D))
+    W1, b1 = rng.normal(size=(D, F)) * 0.05, rng.normal(size=F) * 0.1
+    W2, b2 = rng.normal(size=(F, D)) * 0.05, rng.normal(size=D) * 0.1
+    got = oracle.gelu_ffn(h, W1, b1, W2, b2)
+    F_ = torch.nn.functional
+    T = [torch.from_numpy(a) for a in (h, W1, b1, W2, b2)]
+    ref = F_.linear(F_.gelu(F_.linear(T[0], T[1].T, T[2]), approximate="none"), T[3].T, T[4]) + T[0]
+    np.testing.assert_allclose(got, ref.numpy(), atol=1e-12)
+
+    def r16(a):
+        return torch.from_numpy(np.ascontiguousarray(a)).half().double().numpy()
+    rounded = oracle.gelu_ffn(h, W1, b1, W2, b2, round_stored=r16)
+    f = r16(oracle.gelu(h @ W1 + b1))
+    np.testing.assert_allclose(rounded, f @ W2 + b2 + h, atol=1e-12)
+    assert np.abs(rounded - got).max() > 1e-6
+
+
 def test_encoder_layer_any_pos_wiring():
     """The layer oracle with global tokens at any position: on prefix masks
     the same bits as the prefix definition, and on scattered masks the same
