@@ -64,6 +64,9 @@ def parse():
     ap.add_argument("--layers", type=int, default=1,
                     help="workload 5 only: time an encoder of this many layers (lf_encoder_forward), each with "
                          "its own seeded weights")
+    ap.add_argument("--ffn-path", default="auto", choices=["auto", "unfused", "fused"],
+                    help="workload 5 only: the FFN path of the layer (two GEMMs, or the fused kernel that keeps "
+                         "the intermediate on chip; auto picks the faster for the shape)")
     return ap.parse_args()
 
 
@@ -237,6 +240,7 @@ def run_ours(args):
         stack = [wts] + [{n: ((torch.randn(v.shape, generator=gen, device=dev) * 0.02).to(v.dtype)
                                if n.startswith("W_") else v.clone()) for n, v in wts.items()}
                          for _ in range(n_layers - 1)]
+        lf.lf_set_ffn_path(args.ffn_path)
         ws_fn = lf.lf_encoder_any_globals_workspace_bytes if any_layer else lf.lf_encoder_workspace_bytes
         ws = torch.empty(max(256, ws_fn(n_layers, wl.B, wl.H, wl.L, wl.w, ffn, x.dtype)),
                          dtype=torch.uint8, device=dev)
@@ -408,6 +412,7 @@ def run_ours(args):
                    + (" x %d layers" % n_layers if layer and n_layers > 1 else ""),
                    "B": wl.B, "H": wl.H, "L": wl.L, "w": wl.w, "g": wl.g,
                    "pad": wl.pad, "head_dim": 64, "l2": "flushed before every timed step (2 x L2 write)",
+                   **({"ffn_path": args.ffn_path} if layer else {}),
                    "parallelism": "replica per GPU (weak)" if world > 1 else "single GPU"},
         "tflops": F / (total_ms * 1e-3 / K) / 1e12,
         "step_us": {k: (v * 1e3 if v is not None else None) for k, v in step_q.items()},

@@ -284,6 +284,59 @@ lf_status lf_encoder_forward_any_globals(const void* x, const float* local_mask,
                                          lf_stream_t stream, void* out);
 
 /*
+ * The GELU feed-forward network of the layer (FTL §Longformer Encoder
+ * 计算流程 / 每个 Transformer 层 step 6, GeluFfnLayer) before its LayerNorm:
+ *   z[r, :] = h[r, :] + b_2 + GELU(h[r, :] W_1^T + b_1) W_2^T
+ * GELU in the erf form; the F-wide intermediate is rounded to `dtype`
+ * (where the page's layer stores it).  Two paths compute it:
+ *   LF_FFN_UNFUSED  two GEMMs with fused epilogues; the intermediate
+ *                   [rows, F] goes through `workspace`
+ *   LF_FFN_FUSED    one kernel (the fused linear -> GELU -> linear of the
+ *                   PaddleNLP FastFFN page, §FastFFN融合计算): clusters of
+ *                   CTAs keep the intermediate on chip in 128-wide chunks
+ *                   (needs F a multiple of 128 * c, c = 1, 2, 4 for D <= 256,
+ *                   <= 512, <= 1024); no workspace
+ *   LF_FFN_AUTO     the path measured faster on B200: fused for d_model
+ *                   <= 256 (one CTA holds a row tile's whole output), the
+ *                   two GEMMs above that
+ * Both sum over D and over F in the same order and give the same result bit
+ * for bit.
+ */
+typedef enum { LF_FFN_AUTO = 0, LF_FFN_UNFUSED = 1, LF_FFN_FUSED = 2 } lf_ffn_path;
+
+/* Bytes of workspace lf_gelu_ffn_forward needs for `path` (0 when it needs
+ * none or the sizes are invalid). */
+size_t lf_gelu_ffn_workspace_bytes(int rows, int d_model, int ffn_dim, lf_dtype dtype, int path);
+
+/*
+ * lf_gelu_ffn_forward -- the FFN above.
+ *   h     [rows, d_model] of dtype (LF_F16 or LF_BF16); also the residual
+ *   W_1   [ffn_dim, d_model], b_1 [ffn_dim]; W_2 [d_model, ffn_dim],
+ *         b_2 [d_model] (nn.Linear layout, dtype)
+ *   z     [rows, d_model] float32, written
+ *   workspace: device memory of lf_gelu_ffn_workspace_bytes(...) bytes,
+ *         256-byte aligned (may be NULL when that is 0)
+ * Shape rules: rows > 0; d_model a multiple of 128, <= 1024; ffn_dim a
+ * multiple of 128.  Errors: LF_ERR_NULL, LF_ERR_MISALIGNED, LF_ERR_DTYPE,
+ * LF_ERR_BAD_DIM (shape rules, unknown path, or LF_FFN_FUSED for a shape it
+ * does not take), LF_ERR_WORKSPACE, LF_ERR_CUDA; a device-side wait that
+ * expires records LF_ERR_DEVICE_TIMEOUT (lf_device_status).  Asynchronous.
+ */
+lf_status lf_gelu_ffn_forward(const void* h, const void* W_1, const void* b_1, const void* W_2, const void* b_2,
+                              int rows, int d_model, int ffn_dim, lf_dtype dtype, int path,
+                              void* workspace, size_t workspace_bytes, lf_stream_t stream, float* z);
+
+/*
+ * lf_set_ffn_path -- the FFN path (lf_ffn_path) the encoder-layer and
+ * encoder entry points use from now on, in this process (default
+ * LF_FFN_AUTO; a shape the fused path does not take always runs unfused).
+ * The layer workspace sizes do not depend on it.  Returns LF_ERR_BAD_DIM for
+ * an unknown value.  lf_get_ffn_path returns the current setting.
+ */
+lf_status lf_set_ffn_path(int path);
+int lf_get_ffn_path(void);
+
+/*
  * lf_attention_forward_noalloc -- lf_attention_forward for callers that
  * cannot allocate device memory.  The pages describe no such entry point: it
  * exists for code that may not call cudaMalloc (for example code running

@@ -134,7 +134,7 @@ const char* lf_status_string(int s) {
     }
 }
 
-int lf_version(void) { return 102; }  // 1.2: lf_noalloc_device_status, lf_selftest_bounded_wait
+int lf_version(void) { return 103; }  // 1.3: lf_gelu_ffn_forward, lf_set_ffn_path (fused FFN)
 
 lf_status lf_device_status(lf_stream_t stream, int reset) {
     lf_status st;

@@ -133,6 +133,22 @@ struct GemmArgs {
 // N % 128 == 0, K % 64 == 0; fp16 / bf16.
 lf_status launch_gemm_tc(const GemmArgs& g, lf_dtype dtype, int sm_count, cudaStream_t stream);
 
+// ---- fused GELU FFN: out = h + b2 + GELU(h W1^T + b1) W2^T (fp32) ----
+struct FfnArgs {
+    const void* h;    // [M][D] (also the residual)
+    const void* W1;   // [F][D]
+    const void* b1;   // [F]
+    const void* W2;   // [D][F]
+    const void* b2;   // [D]
+    int M, D, F;
+    float* out;       // [M][D]
+    int* status;
+};
+// CTAs per cluster of the fused kernel for model width D (0: unsupported).
+int ffn_fused_cluster(int D);
+bool ffn_fused_supported(int M, int D, int F);
+lf_status launch_ffn_fused(const FfnArgs& a, lf_dtype dtype, cudaStream_t stream);
+
 // LayerNorm over rows of an fp32 [rows][N] matrix into dtype (N % 32 == 0, N <= 1024).
 lf_status launch_layernorm(const float* z, const float* gamma, const float* beta, int rows, int N, float eps,
                            lf_dtype dtype, void* out, cudaStream_t stream);

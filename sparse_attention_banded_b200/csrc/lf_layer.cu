@@ -10,11 +10,14 @@
 //   banded + global attention -> a [B, L, D]
 //   GEMM(a, W_o) + b_o + x -> z (fp32);  LayerNorm -> h
 //   GEMM(h, W_1) + b_1, GELU -> f;  GEMM(f, W_2) + b_2 + h -> z;  LayerNorm -> out
+//     (or the fused FFN kernel for the first line, which keeps f on chip)
 // With the global tokens at any position (the _any_globals entry points) the
 // partition (with its rank table) runs once per forward, the qg projection
 // multiplies only the global tokens' rows of x, gathered through global_idx,
 // and writes them straight into the slot buffer of the attention kernel, and
 // the k / v rows of the global tokens are gathered after the projections.
+#include <atomic>
+
 #include "lf_internal.h"
 
 namespace lf {
@@ -75,6 +78,41 @@ using namespace lf;
 
 namespace lf {
 namespace {
+
+std::atomic<int> g_ffn_path{LF_FFN_AUTO};
+
+// The path a call with FFN path setting `path` takes for this shape.  AUTO
+// takes the fused kernel where it measured faster on B200: when one CTA
+// holds a row tile's whole output (D <= 256).  With clusters of 2 or 4 CTAs
+// both paths stream the same operand bytes per flop from L2, and the fused
+// kernel has less shared memory for its TMA ring and fills 128 of the 148
+// SMs at 4096 rows; there the two GEMMs are faster.
+int ffn_path_for(int M, int D, int F, int path) {
+    if (path == LF_FFN_UNFUSED || !ffn_fused_supported(M, D, F)) return LF_FFN_UNFUSED;
+    if (path == LF_FFN_AUTO && ffn_fused_cluster(D) != 1) return LF_FFN_UNFUSED;
+    return LF_FFN_FUSED;
+}
+
+// Step 6 before its LayerNorm: z = h + b_2 + GELU(h W_1^T + b_1) W_2^T,
+// fused or as two GEMMs through f ([M][F] of dtype).
+lf_status gelu_ffn(const void* h, const void* W1, const void* b1, const void* W2, const void* b2, int M, int D, int F,
+                   lf_dtype dtype, int path, void* f, float* z, DeviceCtx* d, cudaStream_t s) {
+    if (path == LF_FFN_FUSED) {
+        FfnArgs a{};
+        a.h = h; a.W1 = W1; a.b1 = b1; a.W2 = W2; a.b2 = b2;
+        a.M = M; a.D = D; a.F = F; a.out = z; a.status = d->status;
+        return launch_ffn_fused(a, dtype, s);
+    }
+    lf_status st;
+    GemmArgs f1{};
+    f1.A = h; f1.batches = 1; f1.rows = M; f1.batch_stride = M; f1.K = D;
+    f1.W = W1; f1.N = F; f1.bias = b1; f1.mode = kEpiGelu; f1.out = f; f1.status = d->status;
+    if ((st = launch_gemm_tc(f1, dtype, d->sm_count, s)) != LF_OK) return st;
+    GemmArgs f2{};
+    f2.A = f; f2.batches = 1; f2.rows = M; f2.batch_stride = M; f2.K = F;
+    f2.W = W2; f2.N = D; f2.bias = b2; f2.mode = kEpiResid; f2.resid = h; f2.out = z; f2.status = d->status;
+    return launch_gemm_tc(f2, dtype, d->sm_count, s);
+}
 
 // One layer on the workspace `base` (layout ws).  any: global tokens at any
 // position; run_partition: run the partition here (the stack runs it once
@@ -145,15 +183,10 @@ lf_status layer_forward(const void* x, const float* local_mask, const float* glo
                                dtype, base + ws.h, s)) != LF_OK)
         return st;
     // step 6: GELU FFN + bias + residual, LayerNorm
-    GemmArgs f1{};
-    f1.A = base + ws.h; f1.batches = B; f1.rows = L; f1.batch_stride = L; f1.K = D;
-    f1.W = wt->W_1; f1.N = F; f1.bias = wt->b_1; f1.mode = kEpiGelu; f1.out = base + ws.f; f1.status = d->status;
-    if ((st = launch_gemm_tc(f1, dtype, d->sm_count, s)) != LF_OK) return st;
-    GemmArgs f2{};
-    f2.A = base + ws.f; f2.batches = B; f2.rows = L; f2.batch_stride = L; f2.K = F;
-    f2.W = wt->W_2; f2.N = D; f2.bias = wt->b_2; f2.mode = kEpiResid; f2.resid = base + ws.h; f2.out = base + ws.z;
-    f2.status = d->status;
-    if ((st = launch_gemm_tc(f2, dtype, d->sm_count, s)) != LF_OK) return st;
+    if ((st = gelu_ffn(base + ws.h, wt->W_1, wt->b_1, wt->W_2, wt->b_2, B * L, D, F, dtype,
+                       ffn_path_for(B * L, D, F, g_ffn_path.load()), base + ws.f,
+                       reinterpret_cast<float*>(base + ws.z), d, s)) != LF_OK)
+        return st;
     return launch_layernorm(reinterpret_cast<float*>(base + ws.z), wt->ln2_gamma, wt->ln2_beta, B * L, D, ln_eps,
                             dtype, out, s);
 }
@@ -211,6 +244,51 @@ extern "C" lf_status lf_encoder_layer_forward_any_globals(const void* x, const f
     return layer_entry(x, local_mask, global_mask, wt, B, H, L, w, attn_scale, ln_eps, dtype, workspace,
                        workspace_bytes, stream, out, true);
 }
+
+// ---------------------------------------------------------------- the FFN alone
+
+extern "C" size_t lf_gelu_ffn_workspace_bytes(int rows, int d_model, int ffn_dim, lf_dtype dtype, int path) {
+    if (rows <= 0 || d_model <= 0 || d_model % 128 != 0 || d_model > 1024 || ffn_dim <= 0 || ffn_dim % 128 != 0)
+        return 0;
+    if (dtype != LF_F16 && dtype != LF_BF16) return 0;
+    if (path < LF_FFN_AUTO || path > LF_FFN_FUSED) return 0;
+    if (path == LF_FFN_FUSED && !ffn_fused_supported(rows, d_model, ffn_dim)) return 0;  // rejected by the call
+    if (ffn_path_for(rows, d_model, ffn_dim, path) == LF_FFN_FUSED) return 0;
+    return (size_t)rows * ffn_dim * 2;
+}
+
+extern "C" lf_status lf_gelu_ffn_forward(const void* h, const void* W_1, const void* b_1, const void* W_2,
+                                         const void* b_2, int rows, int d_model, int ffn_dim, lf_dtype dtype,
+                                         int path, void* workspace, size_t workspace_bytes, lf_stream_t stream,
+                                         float* z) {
+    const void* ptrs[] = {h, W_1, b_1, W_2, b_2, z};
+    for (const void* p : ptrs)
+        if (!p) return LF_ERR_NULL;
+    for (const void* p : ptrs)
+        if (!aligned16(p)) return LF_ERR_MISALIGNED;
+    if (dtype != LF_F16 && dtype != LF_BF16) return LF_ERR_DTYPE;
+    if (rows <= 0 || d_model <= 0 || d_model % 128 != 0 || d_model > 1024 || ffn_dim <= 0 || ffn_dim % 128 != 0)
+        return LF_ERR_BAD_DIM;
+    if (path < LF_FFN_AUTO || path > LF_FFN_FUSED) return LF_ERR_BAD_DIM;
+    if (path == LF_FFN_FUSED && !ffn_fused_supported(rows, d_model, ffn_dim)) return LF_ERR_BAD_DIM;
+    const int use = ffn_path_for(rows, d_model, ffn_dim, path);
+    if (use == LF_FFN_UNFUSED &&
+        (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
+         workspace_bytes < (size_t)rows * ffn_dim * 2))
+        return LF_ERR_WORKSPACE;
+    lf_status st;
+    DeviceCtx* d = current_device(&st);
+    if (!d) return st;
+    return gelu_ffn(h, W_1, b_1, W_2, b_2, rows, d_model, ffn_dim, dtype, use, workspace, z, d, (cudaStream_t)stream);
+}
+
+extern "C" lf_status lf_set_ffn_path(int path) {
+    if (path < LF_FFN_AUTO || path > LF_FFN_FUSED) return LF_ERR_BAD_DIM;
+    g_ffn_path.store(path);
+    return LF_OK;
+}
+
+extern "C" int lf_get_ffn_path(void) { return g_ffn_path.load(); }
 
 // ---------------------------------------------------------------- the stack
 

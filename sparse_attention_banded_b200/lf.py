@@ -86,6 +86,14 @@ def lib():
         L.lf_encoder_forward_any_globals.argtypes = L.lf_encoder_forward.argtypes
         L.lf_encoder_forward_any_globals.restype = st
         L.lf_encoder_forward.restype = st
+        L.lf_gelu_ffn_workspace_bytes.argtypes = [i, i, i, i, i]
+        L.lf_gelu_ffn_workspace_bytes.restype = ctypes.c_size_t
+        L.lf_gelu_ffn_forward.argtypes = [vp] * 5 + [i, i, i, i, i, vp, ctypes.c_size_t, vp, vp]
+        L.lf_gelu_ffn_forward.restype = st
+        L.lf_set_ffn_path.argtypes = [i]
+        L.lf_set_ffn_path.restype = st
+        L.lf_get_ffn_path.argtypes = []
+        L.lf_get_ffn_path.restype = i
         _lib = L
     return _lib
 
@@ -207,6 +215,41 @@ def lf_selftest_bounded_wait(limit_ns: int, stream=None):
     """Launch the one-CTA kernel whose bounded wait runs out after limit_ns
     (see lf.h); the result is read with :func:`lf_device_status`."""
     _check(lib().lf_selftest_bounded_wait(int(limit_ns), _stream(stream)), "lf_selftest_bounded_wait")
+
+
+FFN_PATH = {"auto": 0, "unfused": 1, "fused": 2}
+
+
+def lf_gelu_ffn_workspace_bytes(rows: int, d_model: int, ffn_dim: int, dtype, path: str = "auto") -> int:
+    return lib().lf_gelu_ffn_workspace_bytes(rows, d_model, ffn_dim, DTYPE_CODE[dtype], FFN_PATH[path])
+
+
+def lf_gelu_ffn_forward(h, W_1, b_1, W_2, b_2, path: str = "auto", out=None, workspace=None, stream=None):
+    """z = h + b_2 + GELU(h W_1^T + b_1) W_2^T (fp32) for h [rows, D];
+    path "unfused" (two GEMMs), "fused" (one kernel, the intermediate kept
+    on chip) or "auto" (see lf.h)."""
+    rows, D = h.shape
+    F = W_1.shape[0]
+    if out is None:
+        out = torch.empty(rows, D, dtype=torch.float32, device=h.device)
+    need = lf_gelu_ffn_workspace_bytes(rows, D, F, h.dtype, path) if h.dtype in DTYPE_CODE else 0
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=h.device)
+    st = lib().lf_gelu_ffn_forward(_ptr(h), _ptr(W_1), _ptr(b_1), _ptr(W_2), _ptr(b_2), rows, D, F,
+                                   DTYPE_CODE.get(h.dtype, 99), FFN_PATH[path], _ptr(workspace),
+                                   0 if workspace is None else workspace.numel(), _stream(stream), _ptr(out))
+    _check(st, "lf_gelu_ffn_forward")
+    return out
+
+
+def lf_set_ffn_path(path: str):
+    """The FFN path of the layer and encoder calls in this process."""
+    _check(lib().lf_set_ffn_path(FFN_PATH[path]), "lf_set_ffn_path")
+
+
+def lf_get_ffn_path() -> str:
+    code = lib().lf_get_ffn_path()
+    return {v: k for k, v in FFN_PATH.items()}[code]
 
 
 def lf_encoder_layer_workspace_bytes(B: int, H: int, L: int, w: int, ffn_dim: int, dtype) -> int:

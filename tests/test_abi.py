@@ -210,8 +210,8 @@ def test_any_globals_layer_workspace_bytes_host_only(L):
 
 
 def test_version(L):
-    """1.2: the no-allocation path's status reader and the bounded-wait self-test."""
-    assert L.lf_version() == 102
+    """1.3: the GELU FFN entry point and the FFN path setting."""
+    assert L.lf_version() == 103
 
 
 def test_selftest_wait_limits_checked_on_host(L):
@@ -220,3 +220,47 @@ def test_selftest_wait_limits_checked_on_host(L):
     import ctypes
     for bad in (0, 999, 100000001):
         assert L.lf_selftest_bounded_wait(ctypes.c_ulonglong(bad), None) == 2
+
+
+def _ffn(L, rows=256, D=1024, F=4096, dtype=1, path=0, ws=FAKE, ws_bytes=1 << 30, h=FAKE, z=FAKE, w1=FAKE):
+    return L.lf_gelu_ffn_forward(ctypes.c_void_p(h), ctypes.c_void_p(w1), ctypes.c_void_p(FAKE),
+                                 ctypes.c_void_p(FAKE), ctypes.c_void_p(FAKE), rows, D, F, dtype, path,
+                                 ctypes.c_void_p(ws), ws_bytes, None, ctypes.c_void_p(z))
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(h=0), 1),
+    (dict(z=0), 1),
+    (dict(w1=FAKE + 4), 8),
+    (dict(dtype=0), 7),
+    (dict(rows=0), 2),
+    (dict(D=64), 2),            # not a multiple of 128
+    (dict(D=2048), 2),          # > 1024
+    (dict(F=200), 2),           # not a multiple of 128
+    (dict(path=3), 2),          # unknown path
+    (dict(F=640, path=2), 2),   # the fused path needs F a multiple of 4 * 128 at D = 1024
+    (dict(F=640, path=1, ws_bytes=1024), 12),
+    (dict(F=640, path=0, ws=FAKE + 16), 12),  # auto runs F = 640 unfused: workspace misaligned
+])
+def test_ffn_host_validation(L, kw, status):
+    assert _ffn(L, **kw) == status
+
+
+def test_ffn_workspace_bytes_and_path_setting(L):
+    import torch
+    f16 = torch.float16
+    assert lf.lf_gelu_ffn_workspace_bytes(4096, 1024, 4096, f16, "unfused") == 4096 * 4096 * 2
+    assert lf.lf_gelu_ffn_workspace_bytes(4096, 1024, 4096, f16, "fused") == 0
+    assert lf.lf_gelu_ffn_workspace_bytes(4096, 1024, 640, f16, "fused") == 0      # not taken: invalid
+    assert lf.lf_gelu_ffn_workspace_bytes(4096, 1024, 640, f16, "auto") == 4096 * 640 * 2
+    assert lf.lf_gelu_ffn_workspace_bytes(4096, 1024, 4096, torch.float32, "auto") == 0
+    # auto: fused (no workspace) where one CTA holds a row tile's output, else the two GEMMs
+    assert lf.lf_gelu_ffn_workspace_bytes(4096, 256, 1024, f16, "auto") == 0
+    assert lf.lf_gelu_ffn_workspace_bytes(4096, 512, 2048, f16, "auto") == 4096 * 2048 * 2
+    assert lf.lf_gelu_ffn_workspace_bytes(4096, 1024, 4096, f16, "auto") == 4096 * 4096 * 2
+    assert L.lf_set_ffn_path(7) == 2
+    before = lf.lf_get_ffn_path()
+    for p in ("unfused", "fused", "auto"):
+        lf.lf_set_ffn_path(p)
+        assert lf.lf_get_ffn_path() == p
+    lf.lf_set_ffn_path(before)
