@@ -323,6 +323,11 @@ ffn_fused_kernel(const __grid_constant__ CUtensorMap map_h, const __grid_constan
         for (int t = 0; t < R; ++t) {
             const int c = t * CS + (int)rank;
             const uint32_t hb = t & 1;
+            // this chunk's 64 biases, fetched before the wait (off the critical path)
+            uint4 bq[8];
+            const uint4* bb = reinterpret_cast<const uint4*>(b1 + c * kChunk + half * 64);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) bq[q] = bb[q];
             bool fail = !__all_sync(0xffffffffu, mbar_wait(&chunk_full[hb], (t >> 1) & 1, abort_flag));
             float v[2][32];
             if (!fail) {
@@ -335,10 +340,9 @@ ffn_fused_kernel(const __grid_constant__ CUtensorMap map_h, const __grid_constan
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&chunk_empty[hb]);
-                const uint4* bb = reinterpret_cast<const uint4*>(b1 + c * kChunk + half * 64);
 #pragma unroll
                 for (int q = 0; q < 8; ++q) {
-                    const uint4 u = bb[q];
+                    const uint4 u = bq[q];
                     const T* e = reinterpret_cast<const T*>(&u);
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
