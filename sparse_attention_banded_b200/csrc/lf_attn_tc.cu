@@ -580,6 +580,10 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // The next kernel in the stream may be scheduled now: its CTAs take the
+    // SMs this grid's tail leaves idle and set themselves up there (a kernel
+    // of this library launched after it waits for it before touching memory).
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 #if LF_TRACE
     if (threadIdx.x == 0 && p.trace) {  // kernel entry time
         volatile int* d_ = p.trace + gridDim.x * 16 * 4 + (blockIdx.x * 16 + 15) * 16;

@@ -146,6 +146,9 @@ ffn_fused_kernel(const __grid_constant__ CUtensorMap map_h, const __grid_constan
     const int m0 = (int)(CS > 1 ? cluster_id_x() : blockIdx.x) * kTM;
     const int NQ = p.NQ;
     const int R = p.rounds;
+    // The next kernel in the stream may be scheduled now (it waits for this
+    // one before touching memory).
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
@@ -181,6 +184,9 @@ ffn_fused_kernel(const __grid_constant__ CUtensorMap map_h, const __grid_constan
     // every CTA's barriers are initialised before any peer arrives on them
     if (CS > 1) cluster_sync();
     const uint32_t tmem = *tmem_slot;
+    // Launched as a programmatic dependent: no global memory is read or
+    // written before the kernel before this one has completed.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 
     auto wait_all = [&](uint64_t* bar, uint32_t parity) -> bool {
         return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
@@ -512,18 +518,20 @@ lf_status launch_fused_t(const FfnArgs& a, cudaStream_t stream) {
         attr[dev].store(true);
     }
     const int mtiles = (a.M + kTM - 1) / kTM;
-    cudaLaunchAttribute at[1];
-    at[0].id = cudaLaunchAttributeClusterDimension;
-    at[0].val.clusterDim.x = CS;
-    at[0].val.clusterDim.y = 1;
-    at[0].val.clusterDim.z = 1;
+    cudaLaunchAttribute at[2];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    at[1].id = cudaLaunchAttributeClusterDimension;
+    at[1].val.clusterDim.x = CS;
+    at[1].val.clusterDim.y = 1;
+    at[1].val.clusterDim.z = 1;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(mtiles * CS));
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = C::kSmemBytes;
     cfg.stream = stream;
     cfg.attrs = at;
-    cfg.numAttrs = CS > 1 ? 1 : 0;
+    cfg.numAttrs = CS > 1 ? 2 : 1;
     if (cudaLaunchKernelEx(&cfg, ffn_fused_kernel<T, CS>, mh, m1, m2, p) != cudaSuccess) return LF_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? LF_OK : LF_ERR_CUDA;
 }

@@ -119,6 +119,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // The next kernel in the stream may be scheduled now: its CTAs take the
+    // SMs this grid leaves idle in its last wave and set themselves up there.
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
@@ -145,6 +148,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    // Launched as a programmatic dependent, this grid may have started while
+    // the kernel before it still runs: no global memory is read or written
+    // before that kernel has completed.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 
     // The TMA and MMA warps run their loops with all 32 lanes (lane 0 issues
     // the copies, tensor-core instructions and commits): a lone lane running
@@ -369,7 +376,17 @@ lf_status launch_t(const GemmArgs& g, int sm_count, cudaStream_t stream) {
         attr[dev].store(true);
     }
     const int grid = p.tiles < sm_count ? p.tiles : sm_count;
-    gemm_tc_kernel<T><<<grid, kThreads, kSmemBytes, stream>>>(ma, mw, p);
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kSmemBytes;
+    cfg.stream = stream;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, gemm_tc_kernel<T>, ma, mw, p) != cudaSuccess) return LF_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? LF_OK : LF_ERR_CUDA;
 }
 

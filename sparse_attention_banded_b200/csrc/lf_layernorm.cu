@@ -39,6 +39,10 @@ template <typename T, int VPL>
 __global__ void __launch_bounds__(256) layernorm_kernel(const float* __restrict__ z, const float* __restrict__ gamma,
                                                         const float* __restrict__ beta, int rows, int N, float eps,
                                                         T* __restrict__ out) {
+    // Let the next kernel in the stream be scheduled; wait for the one before
+    // (launched as a programmatic dependent) before touching memory.
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const int lane = threadIdx.x & 31;
     const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
     if (row >= rows) return;
@@ -81,17 +85,28 @@ lf_status launch_t(const float* z, const float* gamma, const float* beta, int ro
                    cudaStream_t stream) {
     const int blocks = (rows + 7) / 8;
     T* o = reinterpret_cast<T*>(out);
+    void (*kern)(const float*, const float*, const float*, int, int, float, T*);
     switch (N / 128) {
-        case 1: layernorm_kernel<T, 1><<<blocks, 256, 0, stream>>>(z, gamma, beta, rows, N, eps, o); break;
-        case 2: layernorm_kernel<T, 2><<<blocks, 256, 0, stream>>>(z, gamma, beta, rows, N, eps, o); break;
-        case 3: layernorm_kernel<T, 3><<<blocks, 256, 0, stream>>>(z, gamma, beta, rows, N, eps, o); break;
-        case 4: layernorm_kernel<T, 4><<<blocks, 256, 0, stream>>>(z, gamma, beta, rows, N, eps, o); break;
-        case 5: layernorm_kernel<T, 5><<<blocks, 256, 0, stream>>>(z, gamma, beta, rows, N, eps, o); break;
-        case 6: layernorm_kernel<T, 6><<<blocks, 256, 0, stream>>>(z, gamma, beta, rows, N, eps, o); break;
-        case 7: layernorm_kernel<T, 7><<<blocks, 256, 0, stream>>>(z, gamma, beta, rows, N, eps, o); break;
-        case 8: layernorm_kernel<T, 8><<<blocks, 256, 0, stream>>>(z, gamma, beta, rows, N, eps, o); break;
+        case 1: kern = layernorm_kernel<T, 1>; break;
+        case 2: kern = layernorm_kernel<T, 2>; break;
+        case 3: kern = layernorm_kernel<T, 3>; break;
+        case 4: kern = layernorm_kernel<T, 4>; break;
+        case 5: kern = layernorm_kernel<T, 5>; break;
+        case 6: kern = layernorm_kernel<T, 6>; break;
+        case 7: kern = layernorm_kernel<T, 7>; break;
+        case 8: kern = layernorm_kernel<T, 8>; break;
         default: return LF_ERR_BAD_DIM;
     }
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)blocks);
+    cfg.blockDim = dim3(256);
+    cfg.stream = stream;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kern, z, gamma, beta, rows, N, eps, o) != cudaSuccess) return LF_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? LF_OK : LF_ERR_CUDA;
 }
 
