@@ -145,6 +145,25 @@ lf_status lf_attention_forward(const void* q, const void* k, const void* v,
 size_t lf_attention_scratch_bytes(int B, int H, int L, int w, lf_dtype dtype);
 
 /*
+ * lf_attention_forward_idx -- lf_init_global_idx (asynchronous mode) and
+ * lf_attention_forward in one call: FTL §Longformer Encoder 计算流程 /
+ * 预处理 followed by steps 3-5.  For fp16 / bf16 it is ONE kernel launch:
+ * the attention kernel's epilogue warps of CTA b compute the partition of
+ * sample b while the first scores are computed.  Arguments as
+ * lf_attention_forward, plus global_idx [B, L] and global_token_nums [B]
+ * (int32, device, written exactly as lf_init_global_idx writes them, with
+ * its content check recorded in the device status word).  Errors: as
+ * lf_attention_forward; LF_ERR_NULL / LF_ERR_MISALIGNED also for the two
+ * partition outputs.  Asynchronous on `stream`.
+ */
+lf_status lf_attention_forward_idx(const void* q, const void* k, const void* v,
+                                   const void* qg, const void* kg, const void* vg,
+                                   const float* local_mask, const float* global_mask,
+                                   int B, int H, int L, int w, lf_dtype dtype,
+                                   lf_stream_t stream, void* out,
+                                   int32_t* global_idx, int32_t* global_token_nums);
+
+/*
  * lf_attention_forward_any_globals -- lf_attention_forward with the global
  * tokens at any positions of the sequence: the HuggingFace arrangement that
  * FTL §使用前提 item 4 names as unsupported by FT, gathered through the

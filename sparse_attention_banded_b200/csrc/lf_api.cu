@@ -109,6 +109,46 @@ lf_status check_shape(int B, int H, int L, int w) {
 
 }  // namespace lf
 
+namespace lf {
+namespace {
+
+// lf_attention_forward, and with gidx / gnum also the partition of
+// lf_init_global_idx (for fp16 / bf16 inside the attention kernel's launch).
+lf_status attention_entry(const void* q, const void* k, const void* v, const void* qg, const void* kg,
+                          const void* vg, const float* local_mask, const float* global_mask, int B, int H, int L,
+                          int w, lf_dtype dtype, lf_stream_t stream, void* out, int32_t* gidx, int32_t* gnum) {
+    if (!q || !k || !v || !qg || !kg || !vg || !local_mask || !global_mask || !out) return LF_ERR_NULL;
+    lf_status st = check_shape(B, H, L, w);
+    if (st != LF_OK) return st;
+    if (dtype != LF_F32 && dtype != LF_F16 && dtype != LF_BF16) return LF_ERR_DTYPE;
+    const void* ptrs[] = {q, k, v, qg, kg, vg, local_mask, global_mask, out};
+    for (const void* p : ptrs)
+        if (!aligned16(p)) return LF_ERR_MISALIGNED;
+    if (gidx && (!aligned16(gidx) || !aligned16(gnum))) return LF_ERR_MISALIGNED;
+    DeviceCtx* d = current_device(&st);
+    if (!d) return st;
+    const float scale = 0.125f;  // 1/sqrt(64)
+    cudaStream_t s = (cudaStream_t)stream;
+    if (dtype == LF_F32) {
+        if (gidx && (st = launch_global_idx(global_mask, B, L, w, gidx, gnum, d->status, s)) != LF_OK) return st;
+        return launch_attention_simt_f32((const float*)q, (const float*)k, (const float*)v,
+                                         (const float*)qg, (const float*)kg, (const float*)vg,
+                                         local_mask, global_mask, B, H, L, w, scale, (float*)out,
+                                         d->status, s);
+    }
+    st = ensure_scratch(d, attention_tc_scratch_bytes(B, H, L, w));
+    if (st != LF_OK) return st;
+    st = prepare_scratch_counters(d, attention_tc_scratch_zero_bytes(B, H, L, w), s);
+    if (st != LF_OK) return st;
+    st = launch_attention_tc(q, k, v, qg, kg, vg, local_mask, global_mask, B, H, L, w, scale, dtype, out,
+                             d->scratch, d->status, d->sm_count, s, nullptr, gidx, gnum);
+    if (st != LF_OK) scratch_dirty(d);
+    return st;
+}
+
+}  // namespace
+}  // namespace lf
+
 using namespace lf;
 
 extern "C" {
@@ -134,7 +174,7 @@ const char* lf_status_string(int s) {
     }
 }
 
-int lf_version(void) { return 103; }  // 1.3: lf_gelu_ffn_forward, lf_set_ffn_path (fused FFN)
+int lf_version(void) { return 104; }  // 1.4: lf_attention_forward_idx
 
 lf_status lf_device_status(lf_stream_t stream, int reset) {
     lf_status st;
@@ -193,30 +233,18 @@ lf_status lf_attention_forward(const void* q, const void* k, const void* v, cons
                                const void* kg, const void* vg, const float* local_mask,
                                const float* global_mask, int B, int H, int L, int w, lf_dtype dtype,
                                lf_stream_t stream, void* out) {
-    if (!q || !k || !v || !qg || !kg || !vg || !local_mask || !global_mask || !out) return LF_ERR_NULL;
-    lf_status st = check_shape(B, H, L, w);
-    if (st != LF_OK) return st;
-    if (dtype != LF_F32 && dtype != LF_F16 && dtype != LF_BF16) return LF_ERR_DTYPE;
-    const void* ptrs[] = {q, k, v, qg, kg, vg, local_mask, global_mask, out};
-    for (const void* p : ptrs)
-        if (!aligned16(p)) return LF_ERR_MISALIGNED;
-    DeviceCtx* d = current_device(&st);
-    if (!d) return st;
-    const float scale = 0.125f;  // 1/sqrt(64)
-    cudaStream_t s = (cudaStream_t)stream;
-    if (dtype == LF_F32)
-        return launch_attention_simt_f32((const float*)q, (const float*)k, (const float*)v,
-                                         (const float*)qg, (const float*)kg, (const float*)vg,
-                                         local_mask, global_mask, B, H, L, w, scale, (float*)out,
-                                         d->status, s);
-    st = ensure_scratch(d, attention_tc_scratch_bytes(B, H, L, w));
-    if (st != LF_OK) return st;
-    st = prepare_scratch_counters(d, attention_tc_scratch_zero_bytes(B, H, L, w), s);
-    if (st != LF_OK) return st;
-    st = launch_attention_tc(q, k, v, qg, kg, vg, local_mask, global_mask, B, H, L, w, scale, dtype, out,
-                             d->scratch, d->status, d->sm_count, s);
-    if (st != LF_OK) scratch_dirty(d);
-    return st;
+    return attention_entry(q, k, v, qg, kg, vg, local_mask, global_mask, B, H, L, w, dtype, stream, out, nullptr,
+                           nullptr);
+}
+
+lf_status lf_attention_forward_idx(const void* q, const void* k, const void* v, const void* qg,
+                                   const void* kg, const void* vg, const float* local_mask,
+                                   const float* global_mask, int B, int H, int L, int w, lf_dtype dtype,
+                                   lf_stream_t stream, void* out, int32_t* global_idx,
+                                   int32_t* global_token_nums) {
+    if (!global_idx || !global_token_nums) return LF_ERR_NULL;
+    return attention_entry(q, k, v, qg, kg, vg, local_mask, global_mask, B, H, L, w, dtype, stream, out,
+                           global_idx, global_token_nums);
 }
 
 size_t lf_attention_any_globals_scratch_bytes(int B, int H, int L, int w, lf_dtype dtype) {

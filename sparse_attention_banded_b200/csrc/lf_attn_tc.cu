@@ -132,6 +132,11 @@ struct Params {
     const int* grank;   // [B][L + 1] global tokens before each position
     const float* lm_c;  // [B][gcap] local_mask of each slot (0 past gnum[b])
     int gcap;           // slots per (b, h) in the compact buffers
+    // Prefix instance, optional: the global-index partition of global_mask
+    // (as lf_init_global_idx writes it), computed by the epilogue warps of
+    // CTA b while the first items' scores are being computed.
+    int32_t* gidx_out;  // [B][L] or NULL
+    int32_t* gnum_out;  // [B]
 };
 
 // Diagnostic builds (-DLF_TRACE=1) record per CTA and role the cycles spent
@@ -290,6 +295,75 @@ __device__ void band_rows2(const Params& p, int b, const int (&r0)[2], int& cach
         work[x] = __any_sync(0xffffffffu, w_);
         padded[x] = __any_sync(0xffffffffu, pd);
     }
+}
+
+// The 128 epilogue threads (te = 0..127, warp ew = 0..3 of them): the
+// global-index partition of sample b (FTL §Longformer Encoder 计算流程 /
+// 预处理): the positions with global_mask == 0.0 in ascending order, then
+// the others in descending order (the order of a stable flagged partition
+// that writes rejected items from the back), their count, and the content
+// check of the prefix rule.  sm: 5 ints of shared memory; named barrier 1.
+__device__ void partition_sample(const Params& p, int b, int te, int ew, int lane, int* sm) {
+    constexpr int kN = 128, kIt = 4;
+    const int L = p.L;
+    const float* row = p.global_mask + (size_t)b * L;
+    int32_t* idx = p.gidx_out + (size_t)b * L;
+    if (te == 0) sm[4] = L;  // first position that is not global
+    named_bar_sync(1, kN);
+    int base = 0;  // global positions before this chunk
+    for (int c0 = 0; c0 < L; c0 += kN * kIt) {
+        const int j0 = c0 + te * kIt;
+        bool f[kIt];
+        if (j0 + kIt <= L && (L & 3) == 0) {
+            const float4 m4 = *reinterpret_cast<const float4*>(row + j0);
+            f[0] = m4.x == 0.0f;
+            f[1] = m4.y == 0.0f;
+            f[2] = m4.z == 0.0f;
+            f[3] = m4.w == 0.0f;
+        } else {
+#pragma unroll
+            for (int t = 0; t < kIt; ++t) f[t] = (j0 + t < L) && row[j0 + t] == 0.0f;
+        }
+        int cnt = 0, my_first = L;
+#pragma unroll
+        for (int t = 0; t < kIt; ++t) {
+            cnt += f[t];
+            if (!f[t] && j0 + t < L && my_first == L) my_first = j0 + t;
+        }
+        if (my_first < L) atomicMin(&sm[4], my_first);
+        int incl = cnt;  // inclusive scan of the counts within the warp
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        if (lane == 31) sm[ew] = incl;
+        named_bar_sync(1, kN);
+        int wbase = 0;
+        for (int u = 0; u < ew; ++u) wbase += sm[u];
+        const int tot = sm[0] + sm[1] + sm[2] + sm[3];
+        int sel = base + wbase + incl - cnt;  // global positions before j0
+#pragma unroll
+        for (int t = 0; t < kIt; ++t) {
+            const int j = j0 + t;
+            if (j < L) {
+                if (f[t]) {
+                    idx[sel] = j;
+                    ++sel;
+                } else {
+                    idx[L - 1 - (j - sel)] = j;  // j - sel: other positions before j
+                }
+            }
+        }
+        base += tot;
+        named_bar_sync(1, kN);  // sm[0..3] are rewritten by the next chunk
+    }
+    if (te == 0) {
+        p.gnum_out[b] = base;
+        if (sm[4] < base) record_status(p.status, b, LF_ERR_GLOBAL_NOT_PREFIX);
+        else if (base > p.w) record_status(p.status, b, LF_ERR_G_GT_W);
+    }
+    named_bar_sync(1, kN);  // sm[4] is reset for the next sample only after it was read
 }
 
 // Whole warp: the item's plan (identical in every role).
@@ -638,6 +712,10 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    // Launched as a programmatic dependent, this grid may have started while
+    // the kernel before it still runs (and may still be writing this
+    // kernel's inputs): no global memory is touched before it has completed.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 #if LF_TRACE
     if (threadIdx.x == 0 && p.trace) {
         volatile int* d_ = p.trace + gridDim.x * 16 * 4 + (blockIdx.x * 16 + 14) * 16;
@@ -1249,6 +1327,14 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
         uint32_t npv[2] = {0, 0}, st_cnt[2] = {0, 0};
         TDECL;
         bool ok = true;
+        if constexpr (!kAny) {
+            // the partition, while this CTA's first scores are computed
+            if (p.gidx_out) {
+                int* sm_i = reinterpret_cast<int*>(smem + kOffMisc + 16);
+                for (int b = blockIdx.x; b < p.B; b += gridDim.x)
+                    partition_sample(p, b, r, sp, lane, sm_i);
+            }
+        }
 #if LF_TRACE
         const unsigned long long tent_ = globaltimer();
 #endif
@@ -1483,10 +1569,6 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
-    // Launched with programmatic stream serialization, this grid may have
-    // started while the kernel before it was still running; it completes only
-    // after that kernel has, so work queued after it sees both.
-    asm volatile("griddepcontrol.wait;" ::: "memory");
 #if LF_TRACE
     if (threadIdx.x == 32 && p.trace) {  // exit time (after the TMEM release)
         volatile int* d_ = p.trace + gridDim.x * 16 * 4 + (blockIdx.x * 16 + 15) * 16;
@@ -1701,7 +1783,8 @@ size_t attention_tc_scratch_zero_bytes(int B, int H, int L, int w) {
 lf_status launch_attention_tc(const void* q, const void* k, const void* v, const void* qg, const void* kg,
                               const void* vg, const float* local_mask, const float* global_mask, int B, int H,
                               int L, int w, float scale, lf_dtype dtype, void* out, void* scratch, int* status,
-                              int sm_count, cudaStream_t stream, const AnyGlobals* any) {
+                              int sm_count, cudaStream_t stream, const AnyGlobals* any, int32_t* gidx_out,
+                              int32_t* gnum_out) {
     const Geometry geo = geometry(B, H, L, w, sm_count);
     Maps maps;
     const int BH = B * H;
@@ -1749,6 +1832,8 @@ lf_status launch_attention_tc(const void* q, const void* k, const void* v, const
     p.grank = any ? any->rank : nullptr;
     p.lm_c = any ? any->lm_c : nullptr;
     p.gcap = any ? any->gcap : 0;
+    p.gidx_out = any ? nullptr : gidx_out;
+    p.gnum_out = any ? nullptr : gnum_out;
 #if LF_TRACE
     if (const char* a = getenv("LF_TRACE_ADDR")) p.trace = reinterpret_cast<int*>(strtoull(a, nullptr, 10));
 #endif

@@ -56,18 +56,41 @@ constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
 constexpr uint32_t kSmemBytes = kOffMisc + 64 + 1024;
 constexpr uint32_t kTmemCols = 512;  // two 256-column fp32 accumulators
 
-struct GemmParams {
-    int batches, rows, K, N;  // per batch: rows x N outputs
-    int mtiles, ntiles, ktiles, tiles;
-    int mode;
+// One GEMM problem of a launch: per batch, rows x N outputs.
+struct GemmProb {
+    int rows, N;
+    int mtiles, ntiles, tiles;
     const void* bias;    // [N] of T
-    const void* resid;   // kEpiResid: [batches*rows][N] of T
     void* out;
+    int heads_L;         // kEpiHeads: rows of the head-layout tensors
+};
+
+// A launch runs one problem, or two sharing batches, K and the epilogue
+// mode (the second one's tiles follow the first's).
+struct GemmParams {
+    int batches, K, ktiles, tiles;
+    GemmProb pr[2];
+    int mode;
+    const void* resid;   // kEpiResid: [batches*rows][N] of T
     int heads_D;         // kEpiHeads: columns per output tensor (H*64)
     int heads_H;
-    int heads_L;         // rows of the head-layout tensors (L)
     int* status;
 };
+
+struct TileAt {
+    int pi, nt, mt, b;
+};
+__device__ __forceinline__ TileAt tile_at(const GemmParams& p, int t) {
+    TileAt a;
+    a.pi = t >= p.pr[0].tiles ? 1 : 0;
+    if (a.pi) t -= p.pr[0].tiles;
+    const GemmProb& q = p.pr[a.pi];
+    a.nt = t % q.ntiles;
+    const int bm = t / q.ntiles;
+    a.mt = bm % q.mtiles;
+    a.b = bm / q.mtiles;
+    return a;
+}
 
 template <typename T>
 struct Cvt;
@@ -107,6 +130,7 @@ __device__ __forceinline__ float gelu_erf(float x) { return 0.5f * x * (1.0f + e
 template <typename T>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_w,
+               const __grid_constant__ CUtensorMap map_a2, const __grid_constant__ CUtensorMap map_w2,
                const __grid_constant__ GemmParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -139,6 +163,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
     if (warp == 0 && lane == 0) {
         prefetch_tensormap(&map_a);
         prefetch_tensormap(&map_w);
+        if (p.pr[1].tiles > 0) {
+            prefetch_tensormap(&map_a2);
+            prefetch_tensormap(&map_w2);
+        }
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, kTmemCols);
@@ -164,17 +192,17 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
         uint32_t kc = 0;
         bool ok = true;
         for (int t = blockIdx.x; t < p.tiles && ok; t += gridDim.x) {
-            const int nt = t % p.ntiles;
-            const int bm = t / p.ntiles;
-            const int mt = bm % p.mtiles, b = bm / p.mtiles;
+            const TileAt at = tile_at(p, t);
+            const CUtensorMap* ma = at.pi ? &map_a2 : &map_a;
+            const CUtensorMap* mw = at.pi ? &map_w2 : &map_w;
             for (int kt = 0; kt < p.ktiles && ok; ++kt, ++kc) {
                 const uint32_t st = kc % kStages;
                 ok = wait_all(&empty[st], ((kc / kStages) & 1) ^ 1);
                 if (!ok) break;
                 if (lane == 0) {
                     mbar_arrive_expect_tx(&full[st], kABytes + kBBytes);
-                    tma_load_3d(smem + kOffA + st * kABytes, &map_a, &full[st], kt * kTK, mt * kTM, b);
-                    tma_load_2d(smem + kOffB + st * kBBytes, &map_w, &full[st], kt * kTK, nt * kTN);
+                    tma_load_3d(smem + kOffA + st * kABytes, ma, &full[st], kt * kTK, at.mt * kTM, at.b);
+                    tma_load_2d(smem + kOffB + st * kBBytes, mw, &full[st], kt * kTK, at.nt * kTN);
                 }
                 __syncwarp();
             }
@@ -224,15 +252,15 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
         const int r = sp * 32 + lane;
         const uint32_t lane_off = (uint32_t)(sp * 32) << 16;
         float* bias_w = reinterpret_cast<float*>(smem + kOffBias) + (warp - 4) * (kTN / 2);
-        const T* bias = reinterpret_cast<const T*>(p.bias);
         uint32_t tc = 0;
         bool ok = true;
         for (int t = blockIdx.x; t < p.tiles && ok; t += gridDim.x, ++tc) {
-            const int nt = t % p.ntiles;
-            const int bm = t / p.ntiles;
-            const int mt = bm % p.mtiles, b = bm / p.mtiles;
-            const int n0 = nt * kTN + half * (kTN / 2);  // this warp's columns
-            int ncols = p.N - n0 < kTN / 2 ? p.N - n0 : kTN / 2;  // a multiple of 32, maybe <= 0
+            const TileAt at = tile_at(p, t);
+            const GemmProb& q = p.pr[at.pi];
+            const int mt = at.mt, b = at.b;
+            const T* bias = reinterpret_cast<const T*>(q.bias);
+            const int n0 = at.nt * kTN + half * (kTN / 2);  // this warp's columns
+            int ncols = q.N - n0 < kTN / 2 ? q.N - n0 : kTN / 2;  // a multiple of 32, maybe <= 0
             if (ncols < 0) ncols = 0;
             // this warp's copy of its columns' bias
 #pragma unroll
@@ -244,8 +272,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
             if (!ok) break;
             tc_fence_after();
             const int m = mt * kTM + r;  // row within the batch
-            const bool row_ok = m < p.rows;
-            const size_t grow = (size_t)b * p.rows + m;  // global row (row-major outputs)
+            const bool row_ok = m < q.rows;
+            const size_t grow = (size_t)b * q.rows + m;  // global row (row-major outputs)
 #pragma unroll 1
             for (int c0 = 0; c0 < ncols; c0 += 32) {
                 float acc[32];
@@ -262,7 +290,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
                 }
                 if (!row_ok) {
                 } else if (p.mode == kEpiResid) {
-                    const uint4* rs = reinterpret_cast<const uint4*>(reinterpret_cast<const T*>(p.resid) + grow * p.N + n);
+                    const uint4* rs = reinterpret_cast<const uint4*>(reinterpret_cast<const T*>(p.resid) + grow * q.N + n);
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
                         uint4 u = rs[q];
@@ -270,7 +298,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
 #pragma unroll
                         for (int j = 0; j < 8; ++j) acc[q * 8 + j] += Cvt<T>::to_f(e[j]);
                     }
-                    float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) + grow * p.N + n);
+                    float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(q.out) + grow * q.N + n);
 #pragma unroll
                     for (int q = 0; q < 8; ++q)
                         dst[q] = make_float4(acc[4 * q], acc[4 * q + 1], acc[4 * q + 2], acc[4 * q + 3]);
@@ -279,10 +307,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
                     if (p.mode == kEpiHeads) {
                         const int which = n / p.heads_D;
                         const int h = (n % p.heads_D) / 64, d = n % 64;
-                        dst = reinterpret_cast<T*>(p.out) +
-                              ((((size_t)which * p.batches + b) * p.heads_H + h) * p.heads_L + m) * 64 + d;
+                        dst = reinterpret_cast<T*>(q.out) +
+                              ((((size_t)which * p.batches + b) * p.heads_H + h) * q.heads_L + m) * 64 + d;
                     } else {
-                        dst = reinterpret_cast<T*>(p.out) + grow * p.N + n;
+                        dst = reinterpret_cast<T*>(q.out) + grow * q.N + n;
                     }
                     uint4* d4 = reinterpret_cast<uint4*>(dst);
 #pragma unroll
@@ -327,43 +355,65 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
+// A [batches][batch_stride rows][K] (tiles over the first `rows` of each
+// batch) and W [N][K], both K-major.
+bool encode_ab(EncodeTiledFn enc, CUtensorMap* ma, CUtensorMap* mw, const void* A, int batches, int rows,
+               int batch_stride, int K, const void* W, int N) {
+    cuuint64_t adims[3] = {(cuuint64_t)K, (cuuint64_t)rows, (cuuint64_t)batches};
+    cuuint64_t astr[2] = {(cuuint64_t)K * 2, (cuuint64_t)batch_stride * K * 2};
+    cuuint32_t abox[3] = {(cuuint32_t)kTK, (cuuint32_t)kTM, 1};
+    cuuint32_t e3[3] = {1, 1, 1};
+    if (enc(ma, CU_TENSOR_MAP_DATA_TYPE_UINT16, 3, const_cast<void*>(A), adims, astr, abox, e3,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return false;
+    cuuint64_t wdims[2] = {(cuuint64_t)K, (cuuint64_t)N};
+    cuuint64_t wstr[1] = {(cuuint64_t)K * 2};
+    cuuint32_t wbox[2] = {(cuuint32_t)kTK, (cuuint32_t)kTN};
+    return enc(mw, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void*>(W), wdims, wstr, wbox, e3,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+GemmProb make_prob(int batches, int rows, int N, const void* bias, void* out, int heads_L) {
+    GemmProb q;
+    q.rows = rows;
+    q.N = N;
+    q.mtiles = (rows + kTM - 1) / kTM;
+    q.ntiles = (N + kTN - 1) / kTN;
+    q.tiles = batches * q.mtiles * q.ntiles;
+    q.bias = bias;
+    q.out = out;
+    q.heads_L = heads_L;
+    return q;
+}
+
 template <typename T>
 lf_status launch_t(const GemmArgs& g, int sm_count, cudaStream_t stream) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return LF_ERR_CUDA;
-    CUtensorMap ma, mw;
-    // A: [batches][batch_stride rows][K], tiles over the first `rows` of each batch
-    cuuint64_t adims[3] = {(cuuint64_t)g.K, (cuuint64_t)g.rows, (cuuint64_t)g.batches};
-    cuuint64_t astr[2] = {(cuuint64_t)g.K * 2, (cuuint64_t)g.batch_stride * g.K * 2};
-    cuuint32_t abox[3] = {(cuuint32_t)kTK, (cuuint32_t)kTM, 1};
-    cuuint32_t e3[3] = {1, 1, 1};
-    if (enc(&ma, CU_TENSOR_MAP_DATA_TYPE_UINT16, 3, const_cast<void*>(g.A), adims, astr, abox, e3,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-        return LF_ERR_CUDA;
-    cuuint64_t wdims[2] = {(cuuint64_t)g.K, (cuuint64_t)g.N};
-    cuuint64_t wstr[1] = {(cuuint64_t)g.K * 2};
-    cuuint32_t wbox[2] = {(cuuint32_t)kTK, (cuuint32_t)kTN};
-    if (enc(&mw, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void*>(g.W), wdims, wstr, wbox, e3,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-        return LF_ERR_CUDA;
+    CUtensorMap ma, mw, ma2, mw2;
+    if (!encode_ab(enc, &ma, &mw, g.A, g.batches, g.rows, g.batch_stride, g.K, g.W, g.N)) return LF_ERR_CUDA;
     GemmParams p;
     p.batches = g.batches;
-    p.rows = g.rows;
     p.K = g.K;
-    p.N = g.N;
-    p.mtiles = (g.rows + kTM - 1) / kTM;
-    p.ntiles = (g.N + kTN - 1) / kTN;
     p.ktiles = g.K / kTK;
-    p.tiles = g.batches * p.mtiles * p.ntiles;
+    p.pr[0] = make_prob(g.batches, g.rows, g.N, g.bias, g.out, g.heads_L);
+    p.pr[1] = make_prob(g.batches, 0, 128, nullptr, nullptr, 0);
+    p.pr[1].tiles = 0;
+    if (g.rows2 > 0) {
+        if (!encode_ab(enc, &ma2, &mw2, g.A2, g.batches, g.rows2, g.batch_stride2, g.K, g.W2, g.N2))
+            return LF_ERR_CUDA;
+        p.pr[1] = make_prob(g.batches, g.rows2, g.N2, g.bias2, g.out2, g.heads_L2);
+    } else {
+        ma2 = ma;
+        mw2 = mw;
+    }
+    p.tiles = p.pr[0].tiles + p.pr[1].tiles;
     p.mode = g.mode;
-    p.bias = g.bias;
     p.resid = g.resid;
-    p.out = g.out;
     p.heads_D = g.heads_D;
     p.heads_H = g.heads_H;
-    p.heads_L = g.heads_L;
     p.status = g.status;
     // the shared-memory opt-in is a per-device function attribute
     static std::atomic<bool> attr[64];
@@ -386,7 +436,7 @@ lf_status launch_t(const GemmArgs& g, int sm_count, cudaStream_t stream) {
     cfg.stream = stream;
     cfg.attrs = at;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, gemm_tc_kernel<T>, ma, mw, p) != cudaSuccess) return LF_ERR_CUDA;
+    if (cudaLaunchKernelEx(&cfg, gemm_tc_kernel<T>, ma, mw, ma2, mw2, p) != cudaSuccess) return LF_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? LF_OK : LF_ERR_CUDA;
 }
 
@@ -394,6 +444,7 @@ lf_status launch_t(const GemmArgs& g, int sm_count, cudaStream_t stream) {
 
 lf_status launch_gemm_tc(const GemmArgs& g, lf_dtype dtype, int sm_count, cudaStream_t stream) {
     if (g.N % 128 != 0 || g.K % kTK != 0 || g.rows <= 0 || g.batches <= 0) return LF_ERR_BAD_DIM;
+    if (g.rows2 > 0 && (g.N2 % 128 != 0 || g.N2 <= 0 || g.mode != kEpiHeads)) return LF_ERR_BAD_DIM;
     if (dtype == LF_F16) return launch_t<__half>(g, sm_count, stream);
     if (dtype == LF_BF16) return launch_t<__nv_bfloat16>(g, sm_count, stream);
     return LF_ERR_DTYPE;

@@ -31,9 +31,8 @@ __global__ void __launch_bounds__(kThreads)
 global_idx_kernel(const float* __restrict__ global_mask, int L, int w, int32_t* __restrict__ global_idx,
                   int32_t* __restrict__ global_token_nums, int32_t* __restrict__ rank, int require_prefix,
                   int* status) {
-    // A kernel launched after this one with programmatic stream
-    // serialization (the prefix attention kernel, which does not read what
-    // this kernel writes) may start right away.
+    // A kernel launched after this one as a programmatic dependent may be
+    // scheduled right away (it waits for this one before touching memory).
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int b = blockIdx.x;
     const float* row = global_mask + (size_t)b * L;

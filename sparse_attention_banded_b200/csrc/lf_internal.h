@@ -29,10 +29,6 @@ struct DeviceCtx {
     // Leading bytes of the scratch known to be zero when the next call
     // starts (the attention kernel's scheduler and split counters must be).
     size_t scratch_clean = 0;
-    // encoder layer: a second stream (and its fork/join events) on which a
-    // small GEMM runs beside a large one
-    cudaStream_t side = nullptr;
-    cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
 };
 
 // Current device's context (initialised on first use; NULL + status on error).
@@ -109,12 +105,15 @@ size_t attention_tc_scratch_bytes(int B, int H, int L, int w);
 // zero when a launch starts.
 size_t attention_tc_scratch_zero_bytes(int B, int H, int L, int w);
 // any (may be NULL): global tokens at any position, with the compact
-// buffers filled by launch_gather_globals.
+// buffers filled by launch_gather_globals.  gidx_out / gnum_out (prefix
+// path, may be NULL): the kernel also writes the global-index partition
+// (as launch_global_idx with the prefix check) into them.
 lf_status launch_attention_tc(const void* q, const void* k, const void* v, const void* qg,
                               const void* kg, const void* vg, const float* local_mask,
                               const float* global_mask, int B, int H, int L, int w, float scale,
                               lf_dtype dtype, void* out, void* scratch, int* status,
-                              int sm_count, cudaStream_t stream, const AnyGlobals* any = nullptr);
+                              int sm_count, cudaStream_t stream, const AnyGlobals* any = nullptr,
+                              int32_t* gidx_out = nullptr, int32_t* gnum_out = nullptr);
 
 // ---- dense GEMM with fused epilogues (encoder layer) ----
 enum { kEpiHeads = 0, kEpiGelu = 1, kEpiResid = 2 };
@@ -129,6 +128,16 @@ struct GemmArgs {
     void* out;
     int heads_D, heads_H, heads_L;  // kEpiHeads
     int* status;
+    // Optional second problem of the same launch (kEpiHeads only; rows2 > 0
+    // enables it): same batches, K, heads_D and heads_H; its tiles run after
+    // the first problem's, on the SMs its last wave leaves free.
+    const void* A2;    // [batches][batch_stride2][K]
+    int rows2, batch_stride2;
+    const void* W2;    // [N2][K]
+    int N2;
+    const void* bias2; // [N2]
+    void* out2;
+    int heads_L2;
 };
 // N % 128 == 0, K % 64 == 0; fp16 / bf16.
 lf_status launch_gemm_tc(const GemmArgs& g, lf_dtype dtype, int sm_count, cudaStream_t stream);

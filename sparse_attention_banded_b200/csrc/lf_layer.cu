@@ -2,11 +2,10 @@
 // FasterTransformer Longformer page, §Longformer Encoder 计算流程 / 每个
 // Transformer 层 steps 1-6, as a sequence of this library's kernels on one
 // stream (no host synchronisation):
-//   GEMM(x, W_qkv_kgvg) + bias -> q, k, v, kg, vg in head layout
-//   GEMM(x rows < ceil(w/128)*128, W_qg) + bias -> qg in head layout, on a
-//     second stream (forked from and joined back into the caller's stream)
-//     so that its few tiles run on the SMs the large GEMM's last wave leaves
-//     free
+//   GEMM(x, W_qkv_kgvg) + bias -> q, k, v, kg, vg in head layout, and in the
+//     same launch GEMM(x rows < ceil(w/128)*128, W_qg) + bias -> qg in head
+//     layout, whose few tiles run on the SMs the large one's last wave
+//     leaves free
 //   banded + global attention -> a [B, L, D]
 //   GEMM(a, W_o) + b_o + x -> z (fp32);  LayerNorm -> h
 //   GEMM(h, W_1) + b_1, GELU -> f;  GEMM(f, W_2) + b_2 + h -> z;  LayerNorm -> out
@@ -115,60 +114,55 @@ lf_status gelu_ffn(const void* h, const void* W1, const void* b1, const void* W2
 }
 
 // One layer on the workspace `base` (layout ws).  any: global tokens at any
-// position; run_partition: run the partition here (the stack runs it once
-// before its first layer).  Arguments are validated by the callers.
+// position; first: the first layer of the call, which runs the partition
+// (any) and clears the attention kernel's scheduler and split counters in
+// the workspace (every attention launch leaves them zero for the next
+// layer).  Arguments are validated by the callers.
 lf_status layer_forward(const void* x, const float* local_mask, const float* global_mask, const lf_layer_weights* wt,
                         int B, int H, int L, int w, float attn_scale, float ln_eps, lf_dtype dtype, uint8_t* base,
-                        const Workspace& ws, bool any, bool run_partition, DeviceCtx* d, cudaStream_t s, void* out) {
+                        const Workspace& ws, bool any, bool first, DeviceCtx* d, cudaStream_t s, void* out) {
     lf_status st;
     const int D = H * 64, F = wt->ffn_dim;
+    if (first &&
+        cudaMemsetAsync(base + ws.scratch, 0, attention_tc_scratch_zero_bytes(B, H, L, w), s) != cudaSuccess)
+        return LF_ERR_CUDA;
     const size_t head_elems = (size_t)B * H * L * 64;
     uint8_t* qkv = base + ws.qkv;  // [5][B][H][L][64]
     auto slot = [&](int i) { return qkv + (size_t)i * head_elems * 2; };
     AnyGlobals a{};
     if (any) {
         a = any_globals_layout(base + ws.any, B, H, L, w, true);
-        if (run_partition &&
+        if (first &&
             (st = launch_global_idx(global_mask, B, L, w, const_cast<int32_t*>(a.global_idx),
                                     const_cast<int32_t*>(a.global_token_nums), d->status, s,
                                     const_cast<int32_t*>(a.rank), false)) != LF_OK)
             return st;
     }
 
-    if (!d->side) {
-        if (cudaStreamCreateWithFlags(&d->side, cudaStreamNonBlocking) != cudaSuccess ||
-            cudaEventCreateWithFlags(&d->ev_fork, cudaEventDisableTiming) != cudaSuccess ||
-            cudaEventCreateWithFlags(&d->ev_join, cudaEventDisableTiming) != cudaSuccess)
-            return LF_ERR_CUDA;
-    }
-    // steps 1-2: the five projections with bias, scattered to head layout
+    // steps 1-2: the five projections with bias, scattered to head layout,
+    // and the Qg projection as a second problem of the same launch (its
+    // tiles run on the SMs the five projections' last wave leaves free)
     GemmArgs g{};
     g.A = x; g.batches = B; g.rows = L; g.batch_stride = L; g.K = D;
     g.W = wt->W_qkv_kgvg; g.N = 5 * D; g.bias = wt->b_qkv_kgvg; g.mode = kEpiHeads;
     g.out = qkv; g.heads_D = D; g.heads_H = H; g.heads_L = L; g.status = d->status;
-    if (cudaEventRecord(d->ev_fork, s) != cudaSuccess || cudaStreamWaitEvent(d->side, d->ev_fork, 0) != cudaSuccess)
-        return LF_ERR_CUDA;
-    if ((st = launch_gemm_tc(g, dtype, d->sm_count, s)) != LF_OK) return st;
+    g.W2 = wt->W_qg; g.N2 = D; g.bias2 = wt->b_qg;
     if (any) {
         // Qg of the global tokens only: their rows of x, gathered, into the
-        // slot buffer (slot layout [B][H][gcap][64]), beside the above
-        if ((st = launch_gather_rows(x, a, B, L, D, base + ws.xg, d->side)) != LF_OK) return st;
-        g.A = base + ws.xg; g.rows = a.gcap; g.batch_stride = a.gcap; g.heads_L = a.gcap;
-        g.W = wt->W_qg; g.N = D; g.bias = wt->b_qg; g.out = a.qg_c;
+        // slot buffer (slot layout [B][H][gcap][64])
+        if ((st = launch_gather_rows(x, a, B, L, D, base + ws.xg, s)) != LF_OK) return st;
+        g.A2 = base + ws.xg; g.rows2 = a.gcap; g.batch_stride2 = a.gcap; g.heads_L2 = a.gcap; g.out2 = a.qg_c;
     } else {
-        // Qg over the rows that can be global tokens (g_b <= w), beside the above
+        // Qg over the rows that can be global tokens (g_b <= w)
         const int qrows = ((w + 127) / 128) * 128 < L ? ((w + 127) / 128) * 128 : L;
-        g.rows = qrows; g.W = wt->W_qg; g.N = D; g.bias = wt->b_qg; g.out = base + ws.qg;
+        g.A2 = x; g.rows2 = qrows; g.batch_stride2 = L; g.heads_L2 = L; g.out2 = base + ws.qg;
     }
-    if ((st = launch_gemm_tc(g, dtype, d->sm_count, d->side)) != LF_OK) return st;
-    if (cudaEventRecord(d->ev_join, d->side) != cudaSuccess || cudaStreamWaitEvent(s, d->ev_join, 0) != cudaSuccess)
-        return LF_ERR_CUDA;
+    if ((st = launch_gemm_tc(g, dtype, d->sm_count, s)) != LF_OK) return st;
     // the global tokens' k / v rows and local_mask values into their slots
     if (any && (st = launch_gather_globals(nullptr, slot(1), slot(2), local_mask, a, B, H, L, w, s)) != LF_OK)
         return st;
-    // steps 3-5: attention (its split counters must start at zero)
-    if (cudaMemsetAsync(base + ws.scratch, 0, attention_tc_scratch_zero_bytes(B, H, L, w), s) != cudaSuccess)
-        return LF_ERR_CUDA;
+    // steps 3-5: attention (launched right after the projections, it waits
+    // for them on the device; its counters are zero, see above)
     if ((st = launch_attention_tc(slot(0), slot(1), slot(2), any ? a.qg_c : base + ws.qg, slot(3), slot(4),
                                   local_mask, global_mask, B, H, L, w, attn_scale, dtype, base + ws.att,
                                   base + ws.scratch, d->status, d->sm_count, s, any ? &a : nullptr)) != LF_OK)

@@ -54,6 +54,8 @@ def lib():
         L.lf_init_global_idx.argtypes = [vp, i, i, i, vp, vp, ctypes.POINTER(ctypes.c_int), vp]
         L.lf_init_global_idx.restype = st
         L.lf_attention_forward.argtypes = [vp] * 8 + [i, i, i, i, i, vp, vp]
+        L.lf_attention_forward_idx.argtypes = [vp] * 8 + [i, i, i, i, i, vp, vp, vp, vp]
+        L.lf_attention_forward_idx.restype = st
         L.lf_attention_forward.restype = st
         L.lf_attention_scratch_bytes.argtypes = [i, i, i, i, i]
         L.lf_attention_scratch_bytes.restype = ctypes.c_size_t
@@ -162,6 +164,26 @@ def lf_attention_forward(q, k, v, qg, kg, vg, local_mask, global_mask, w: int, o
                                     _stream(stream), _ptr(out))
     _check(st, "lf_attention_forward")
     return out
+
+
+def lf_attention_forward_idx(q, k, v, qg, kg, vg, local_mask, global_mask, w: int, out=None, global_idx=None,
+                             global_token_nums=None, stream=None):
+    """The partition of lf_init_global_idx and the attention in one call
+    (one kernel launch for fp16 / bf16).  Returns (out, global_idx,
+    global_token_nums)."""
+    B, H, L, _ = q.shape
+    if out is None:
+        out = torch.empty(B, L, H * 64, dtype=q.dtype, device=q.device)
+    if global_idx is None:
+        global_idx = torch.empty(B, L, dtype=torch.int32, device=q.device)
+    if global_token_nums is None:
+        global_token_nums = torch.empty(B, dtype=torch.int32, device=q.device)
+    code = DTYPE_CODE.get(q.dtype, 99)
+    st = lib().lf_attention_forward_idx(_ptr(q), _ptr(k), _ptr(v), _ptr(qg), _ptr(kg), _ptr(vg),
+                                        _ptr(local_mask), _ptr(global_mask), B, H, L, w, code,
+                                        _stream(stream), _ptr(out), _ptr(global_idx), _ptr(global_token_nums))
+    _check(st, "lf_attention_forward_idx")
+    return out, global_idx, global_token_nums
 
 
 def lf_attention_scratch_bytes(B: int, H: int, L: int, w: int, dtype) -> int:

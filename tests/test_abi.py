@@ -55,6 +55,29 @@ def test_attention_host_validation(L, kw, status):
     assert _attn(L, **kw) == status
 
 
+def _attn_idx(L, B=1, H=1, Ln=512, w=64, dtype=1, ptrs=None, out=FAKE, gidx=FAKE, gnum=FAKE):
+    p = ptrs or [FAKE] * 8
+    return L.lf_attention_forward_idx(*[ctypes.c_void_p(x) for x in p], B, H, Ln, w, dtype, None,
+                                      ctypes.c_void_p(out), ctypes.c_void_p(gidx), ctypes.c_void_p(gnum))
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(ptrs=[FAKE] * 7 + [0]), 1),
+    (dict(gidx=0), 1),
+    (dict(gnum=0), 1),
+    (dict(B=0), 2),
+    (dict(Ln=500, w=64), 3),
+    (dict(Ln=64, w=64), 4),
+    (dict(dtype=7), 7),
+    (dict(out=FAKE + 2), 8),
+    (dict(gidx=FAKE + 4), 8),
+    (dict(gnum=FAKE + 4), 8),
+    (dict(gidx=FAKE + 4, Ln=500), 3),   # shape errors come before alignment
+])
+def test_attention_idx_host_validation(L, kw, status):
+    assert _attn_idx(L, **kw) == status
+
+
 def _attn_any(L, B=1, H=1, Ln=512, w=64, dtype=1, ptrs=None, out=FAKE):
     p = ptrs or [FAKE] * 8
     return L.lf_attention_forward_any_globals(*[ctypes.c_void_p(x) for x in p], B, H, Ln, w, dtype, None,
@@ -210,8 +233,8 @@ def test_any_globals_layer_workspace_bytes_host_only(L):
 
 
 def test_version(L):
-    """1.3: the GELU FFN entry point and the FFN path setting."""
-    assert L.lf_version() == 103
+    """1.4: the partition and the attention in one call."""
+    assert L.lf_version() == 104
 
 
 def test_selftest_wait_limits_checked_on_host(L):

@@ -195,6 +195,96 @@ def test_attention_repeated_calls_identical():
         assert torch.equal(a, b)
 
 
+# ---------------------------------------------------------------- partition and attention in one call
+
+def _run_idx(t, lm, gm, w):
+    dev = {n: t[n].cuda() for n in inputs.NAMES}
+    out, idx, nums = lf.lf_attention_forward_idx(*[dev[n] for n in inputs.NAMES], lm.cuda(), gm.cuda(), w)
+    torch.cuda.synchronize()
+    return out, idx, nums
+
+
+@pytest.mark.parametrize("dtype", ["f32", "f16", "bf16"])
+@pytest.mark.parametrize("shape", SMALL, ids=lambda s: "B%dH%dL%dw%d" % s[:4])
+def test_attention_idx_small(dtype, shape):
+    """lf_attention_forward_idx: the same output bits as lf_attention_forward
+    and the partition bit-exact against the oracle (for fp16 / bf16 the
+    partition is computed inside the attention kernel's launch)."""
+    B, H, L, w, g, pad = shape
+    t = inputs.attention_inputs(B, H, L, dtype, seed=31 + L)
+    lm, gm = inputs.masks(B, L, g, pad)
+    lf.lf_device_status(reset=True)
+    out, idx, nums = _run_idx(t, lm, gm, w)
+    assert lf.lf_device_status(reset=True) == 0
+    assert torch.equal(out, _run(t, lm, gm, w))
+    e_idx, e_nums, st = oracle.global_partition(gm.numpy(), w)
+    assert st == 0
+    assert np.array_equal(idx.cpu().numpy(), e_idx)
+    assert np.array_equal(nums.cpu().numpy(), e_nums)
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_attention_idx_partition_bit_exact(seed):
+    """Random prefix lengths (0..w), batch sizes and window widths, among them
+    L not a multiple of 4: the in-kernel partition against the oracle."""
+    rng = np.random.default_rng(100 + seed)
+    B, w = int(rng.integers(1, 6)), int(rng.choice([3, 64, 256]))
+    L = w * int(rng.integers(2, 12))
+    gm = np.full((B, L), -10000.0, np.float32)
+    for b in range(B):
+        gm[b, : int(rng.integers(0, w + 1))] = 0.0
+    t = inputs.attention_inputs(B, 1, L, "f16", seed=seed)
+    lm = torch.ones(B, L, dtype=torch.float32)
+    lf.lf_device_status(reset=True)
+    _, idx, nums = _run_idx(t, lm, torch.from_numpy(gm), w)
+    assert lf.lf_device_status(reset=True) == 0
+    e_idx, e_nums, st = oracle.global_partition(gm, w)
+    assert np.array_equal(idx.cpu().numpy(), e_idx)
+    assert np.array_equal(nums.cpu().numpy(), e_nums)
+
+
+@pytest.mark.parametrize("case", ["not_prefix", "too_many", "scatter"])
+def test_attention_idx_content_errors(case):
+    """Masks that break the prefix rules: the combined call records the same
+    status as lf_init_global_idx followed by lf_attention_forward, writes the
+    oracle's partition and the same output."""
+    B, H, L, w = 3, 2, 1024, 128
+    gm = np.full((B, L), -10000.0, np.float32)
+    gm[0, :5] = 0.0
+    if case == "not_prefix":
+        gm[1, 700] = 0.0
+    elif case == "too_many":
+        gm[1, :w + 1] = 0.0
+    else:
+        gm[2, ::7] = 0.0
+    t = inputs.attention_inputs(B, H, L, "bf16", seed=8)
+    lm = torch.ones(B, L, dtype=torch.float32)
+    g = torch.from_numpy(gm)
+    lf.lf_device_status(reset=True)
+    lf.lf_init_global_idx(g.cuda(), w, sync=False)
+    ref_out = _run(t, lm, g, w)
+    st_sep = lf.lf_device_status(reset=True)
+    out, idx, nums = _run_idx(t, lm, g, w)
+    st = lf.lf_device_status(reset=True)
+    e_idx, e_nums, e_st = oracle.global_partition(gm, w)
+    assert st == st_sep and st != 0
+    assert np.array_equal(idx.cpu().numpy(), e_idx)
+    assert np.array_equal(nums.cpu().numpy(), e_nums)
+    assert torch.equal(out, ref_out)
+
+
+def test_attention_idx_workload2():
+    """The benchmark's step (workload 2): one launch gives the attention
+    output of lf_attention_forward bit for bit and the oracle's partition."""
+    wl, t, lm, gm = inputs.workload_inputs(2)
+    out, idx, nums = _run_idx(t, lm, gm, wl.w)
+    assert lf.lf_device_status(reset=True) == 0
+    assert torch.equal(out, _run(t, lm, gm, wl.w))
+    e_idx, e_nums, _ = oracle.global_partition(gm.numpy(), wl.w)
+    assert np.array_equal(idx.cpu().numpy(), e_idx)
+    assert np.array_equal(nums.cpu().numpy(), e_nums)
+
+
 # ---------------------------------------------------------------- the five workloads
 
 def test_workload1_full_parity():
