@@ -508,8 +508,6 @@ __device__ __forceinline__ void load_at(const Plan& pl, int q, int& kb, int& nee
 
 // Key blocks of one tile of an item.
 __device__ __forceinline__ int tile_blocks(const Tile& t) { return t.present ? t.glob_hi + (t.hi - t.lo + 1) : 0; }
-// Key block of a tile's j-th block: [0, glob_hi) then lo, lo + 1, ...
-__device__ __forceinline__ int block_kb(const Tile& t, int j) { return j < t.glob_hi ? j : t.lo + (j - t.glob_hi); }
 template <typename T>
 struct Pack;
 template <>
