@@ -69,6 +69,10 @@ struct GemmProb {
 // mode (the second one's tiles follow the first's).
 struct GemmParams {
     int batches, K, ktiles, tiles;
+    // The last n_split of the t_full + n_split full-width tiles are run as
+    // two 128-column halves each (tiles t_full .. t_full + 2 n_split - 1),
+    // so that the launch's last round fills the SMs.
+    int t_full, n_split;
     GemmProb pr[2];
     int mode;
     const void* resid;   // kEpiResid: [batches*rows][N] of T
@@ -79,9 +83,16 @@ struct GemmParams {
 
 struct TileAt {
     int pi, nt, mt, b;
+    int col0, width;  // output columns [col0, col0 + width) of problem pi
 };
 __device__ __forceinline__ TileAt tile_at(const GemmParams& p, int t) {
     TileAt a;
+    int part = -1;  // half tiles: which half
+    if (t >= p.t_full) {
+        const int h = t - p.t_full;
+        part = h & 1;
+        t = p.t_full + (h >> 1);
+    }
     a.pi = t >= p.pr[0].tiles ? 1 : 0;
     if (a.pi) t -= p.pr[0].tiles;
     const GemmProb& q = p.pr[a.pi];
@@ -89,6 +100,8 @@ __device__ __forceinline__ TileAt tile_at(const GemmParams& p, int t) {
     const int bm = t / q.ntiles;
     a.mt = bm % q.mtiles;
     a.b = bm / q.mtiles;
+    a.col0 = a.nt * kTN + (part > 0 ? kTN / 2 : 0);
+    a.width = part < 0 ? kTN : kTN / 2;
     return a;
 }
 
@@ -131,6 +144,7 @@ template <typename T>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_w,
                const __grid_constant__ CUtensorMap map_a2, const __grid_constant__ CUtensorMap map_w2,
+               const __grid_constant__ CUtensorMap map_wh, const __grid_constant__ CUtensorMap map_w2h,
                const __grid_constant__ GemmParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -167,6 +181,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
             prefetch_tensormap(&map_a2);
             prefetch_tensormap(&map_w2);
         }
+        if (p.n_split > 0) {
+            prefetch_tensormap(&map_wh);
+            if (p.pr[1].tiles > 0) prefetch_tensormap(&map_w2h);
+        }
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, kTmemCols);
@@ -194,15 +212,16 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
         for (int t = blockIdx.x; t < p.tiles && ok; t += gridDim.x) {
             const TileAt at = tile_at(p, t);
             const CUtensorMap* ma = at.pi ? &map_a2 : &map_a;
-            const CUtensorMap* mw = at.pi ? &map_w2 : &map_w;
+            const CUtensorMap* mw = at.width == kTN ? (at.pi ? &map_w2 : &map_w) : (at.pi ? &map_w2h : &map_wh);
+            const uint32_t bytes = kABytes + (at.width == kTN ? kBBytes : kBBytes / 2);
             for (int kt = 0; kt < p.ktiles && ok; ++kt, ++kc) {
                 const uint32_t st = kc % kStages;
                 ok = wait_all(&empty[st], ((kc / kStages) & 1) ^ 1);
                 if (!ok) break;
                 if (lane == 0) {
-                    mbar_arrive_expect_tx(&full[st], kABytes + kBBytes);
+                    mbar_arrive_expect_tx(&full[st], bytes);
                     tma_load_3d(smem + kOffA + st * kABytes, ma, &full[st], kt * kTK, at.mt * kTM, at.b);
-                    tma_load_2d(smem + kOffB + st * kBBytes, mw, &full[st], kt * kTK, at.nt * kTN);
+                    tma_load_2d(smem + kOffB + st * kBBytes, mw, &full[st], kt * kTK, at.col0);
                 }
                 __syncwarp();
             }
@@ -214,10 +233,12 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
             }
         }
     } else if (warp == 1) {
-        constexpr uint32_t idesc = idesc_f16(Cvt<T>::fmt, kTM, kTN, 0, 0);
+        constexpr uint32_t idesc_full = idesc_f16(Cvt<T>::fmt, kTM, kTN, 0, 0);
+        constexpr uint32_t idesc_half = idesc_f16(Cvt<T>::fmt, kTM, kTN / 2, 0, 0);
         uint32_t kc = 0, tc = 0;
         bool ok = true;
         for (int t = blockIdx.x; t < p.tiles && ok; t += gridDim.x, ++tc) {
+            const uint32_t idesc = t < p.t_full ? idesc_full : idesc_half;
             const uint32_t ab = tc & 1;
             ok = wait_all(&acc_empty[ab], ((tc >> 1) & 1) ^ 1);
             if (!ok) break;
@@ -259,8 +280,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
             const GemmProb& q = p.pr[at.pi];
             const int mt = at.mt, b = at.b;
             const T* bias = reinterpret_cast<const T*>(q.bias);
-            const int n0 = at.nt * kTN + half * (kTN / 2);  // this warp's columns
-            int ncols = q.N - n0 < kTN / 2 ? q.N - n0 : kTN / 2;  // a multiple of 32, maybe <= 0
+            const int wcols = at.width / 2;                // columns of each of the two warps
+            const int n0 = at.col0 + half * wcols;         // this warp's columns
+            int ncols = q.N - n0 < wcols ? q.N - n0 : wcols;  // a multiple of 32, maybe <= 0
             if (ncols < 0) ncols = 0;
             // this warp's copy of its columns' bias
 #pragma unroll
@@ -278,7 +300,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
             for (int c0 = 0; c0 < ncols; c0 += 32) {
                 float acc[32];
                 __syncwarp();  // tcgen05.ld is .sync.aligned: whole warp, converged
-                tmem_ld32v(tmem + lane_off + ab * kTN + half * (kTN / 2) + c0, acc);
+                tmem_ld32v(tmem + lane_off + ab * kTN + half * wcols + c0, acc);
                 tmem_ld_wait();
                 regs_ready<32>(acc);
 #pragma unroll
@@ -357,6 +379,16 @@ EncodeTiledFn encode_fn() {
 
 // A [batches][batch_stride rows][K] (tiles over the first `rows` of each
 // batch) and W [N][K], both K-major.
+bool encode_w(EncodeTiledFn enc, CUtensorMap* mw, const void* W, int N, int K, int box_rows) {
+    cuuint64_t wdims[2] = {(cuuint64_t)K, (cuuint64_t)N};
+    cuuint64_t wstr[1] = {(cuuint64_t)K * 2};
+    cuuint32_t wbox[2] = {(cuuint32_t)kTK, (cuuint32_t)box_rows};
+    cuuint32_t e2[2] = {1, 1};
+    return enc(mw, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void*>(W), wdims, wstr, wbox, e2,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool encode_ab(EncodeTiledFn enc, CUtensorMap* ma, CUtensorMap* mw, const void* A, int batches, int rows,
                int batch_stride, int K, const void* W, int N) {
     cuuint64_t adims[3] = {(cuuint64_t)K, (cuuint64_t)rows, (cuuint64_t)batches};
@@ -367,12 +399,7 @@ bool encode_ab(EncodeTiledFn enc, CUtensorMap* ma, CUtensorMap* mw, const void* 
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return false;
-    cuuint64_t wdims[2] = {(cuuint64_t)K, (cuuint64_t)N};
-    cuuint64_t wstr[1] = {(cuuint64_t)K * 2};
-    cuuint32_t wbox[2] = {(cuuint32_t)kTK, (cuuint32_t)kTN};
-    return enc(mw, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void*>(W), wdims, wstr, wbox, e3,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    return encode_w(enc, mw, W, N, K, kTN);
 }
 
 GemmProb make_prob(int batches, int rows, int N, const void* bias, void* out, int heads_L) {
@@ -392,8 +419,10 @@ template <typename T>
 lf_status launch_t(const GemmArgs& g, int sm_count, cudaStream_t stream) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return LF_ERR_CUDA;
-    CUtensorMap ma, mw, ma2, mw2;
-    if (!encode_ab(enc, &ma, &mw, g.A, g.batches, g.rows, g.batch_stride, g.K, g.W, g.N)) return LF_ERR_CUDA;
+    CUtensorMap ma, mw, ma2, mw2, mwh, mw2h;
+    if (!encode_ab(enc, &ma, &mw, g.A, g.batches, g.rows, g.batch_stride, g.K, g.W, g.N) ||
+        !encode_w(enc, &mwh, g.W, g.N, g.K, kTN / 2))
+        return LF_ERR_CUDA;
     GemmParams p;
     p.batches = g.batches;
     p.K = g.K;
@@ -402,14 +431,24 @@ lf_status launch_t(const GemmArgs& g, int sm_count, cudaStream_t stream) {
     p.pr[1] = make_prob(g.batches, 0, 128, nullptr, nullptr, 0);
     p.pr[1].tiles = 0;
     if (g.rows2 > 0) {
-        if (!encode_ab(enc, &ma2, &mw2, g.A2, g.batches, g.rows2, g.batch_stride2, g.K, g.W2, g.N2))
+        if (!encode_ab(enc, &ma2, &mw2, g.A2, g.batches, g.rows2, g.batch_stride2, g.K, g.W2, g.N2) ||
+            !encode_w(enc, &mw2h, g.W2, g.N2, g.K, kTN / 2))
             return LF_ERR_CUDA;
         p.pr[1] = make_prob(g.batches, g.rows2, g.N2, g.bias2, g.out2, g.heads_L2);
     } else {
         ma2 = ma;
         mw2 = mw;
+        mw2h = mwh;
     }
-    p.tiles = p.pr[0].tiles + p.pr[1].tiles;
+    // Whole rounds of full tiles, then the remaining R tiles as 2R halves
+    // when they fit in one round (R <= grid / 2): that round then takes half
+    // a tile's time on up to every SM instead of a whole one on R of them.
+    const int nt = p.pr[0].tiles + p.pr[1].tiles;
+    const int G = nt < sm_count ? nt : sm_count;
+    const int R = nt % G;
+    p.n_split = (nt > G && R > 0 && 2 * R <= G) ? R : 0;
+    p.t_full = nt - p.n_split;
+    p.tiles = nt + p.n_split;
     p.mode = g.mode;
     p.resid = g.resid;
     p.heads_D = g.heads_D;
@@ -425,7 +464,7 @@ lf_status launch_t(const GemmArgs& g, int sm_count, cudaStream_t stream) {
             return LF_ERR_CUDA;
         attr[dev].store(true);
     }
-    const int grid = p.tiles < sm_count ? p.tiles : sm_count;
+    const int grid = G;
     cudaLaunchAttribute at[1];
     at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     at[0].val.programmaticStreamSerializationAllowed = 1;
@@ -436,7 +475,7 @@ lf_status launch_t(const GemmArgs& g, int sm_count, cudaStream_t stream) {
     cfg.stream = stream;
     cfg.attrs = at;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, gemm_tc_kernel<T>, ma, mw, ma2, mw2, p) != cudaSuccess) return LF_ERR_CUDA;
+    if (cudaLaunchKernelEx(&cfg, gemm_tc_kernel<T>, ma, mw, ma2, mw2, mwh, mw2h, p) != cudaSuccess) return LF_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? LF_OK : LF_ERR_CUDA;
 }
 
