@@ -62,7 +62,7 @@ using namespace sm100;
 constexpr int kBM = 128;          // query rows per tile
 constexpr int kBN = 128;          // keys per block
 constexpr int kHD = 64;           // head dim
-constexpr int kStages = 4;        // K/V ring depth
+constexpr int kStages = 5;        // K/V ring depth
 constexpr int kMinChunk = 4;      // key blocks per global-row split: chosen per
 constexpr int kMaxChunk = 16;     // shape in [kMinChunk, kMaxChunk] on the host
 constexpr int kRing = 4;          // item-id ring depth
@@ -80,14 +80,17 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;
 
 // Shared memory map (offsets from a 1024-byte aligned base).
-constexpr uint32_t kOffQ = 0;                                 // [2 parity][2 tile] x 16 KB
-constexpr uint32_t kOffK = kOffQ + 4 * kTileBytes;            // kStages x 16 KB
+// Q of the current item's two tiles: the next item's Q is loaded once the
+// current item's last S products are done, which frees the shared memory
+// of a fifth K/V stage (the next item's first blocks load a block earlier).
+constexpr uint32_t kOffQ = 0;                                 // [2 tile] x 16 KB
+constexpr uint32_t kOffK = kOffQ + 2 * kTileBytes;            // kStages x 16 KB
 constexpr uint32_t kOffV = kOffK + kStages * kTileBytes;      // kStages x 16 KB
 constexpr uint32_t kOffBias = kOffV + kStages * kTileBytes;   // 8 warps x 128 floats
 constexpr uint32_t kOffStats = kOffBias + 8 * kBN * 4;        // [2 tiles][128 rows] (m, l)
 constexpr uint32_t kOffPlans = kOffStats + 2 * kBM * 8;       // kRing plans
 constexpr uint32_t kOffBar = kOffPlans + kRing * 128;
-constexpr uint32_t kNumBars = 2 + 2 + 2 * kStages + 2 * 7 + 2 * kRing + 2 + 1;
+constexpr uint32_t kNumBars = 1 + 1 + 2 * kStages + 2 * 7 + 2 * kRing + 2 + 1;
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
 constexpr uint32_t kSmemBytes = kOffMisc + 64 + 1024;  // + alignment slack
 
@@ -630,9 +633,9 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
-    uint64_t* q_full = bars + 0;
-    uint64_t* q_empty = bars + 2;
-    uint64_t* kv_full = bars + 4;
+    uint64_t* q_full = bars + 0;   // Q of the current item loaded (one phase per item)
+    uint64_t* q_empty = bars + 1;  // ... and read by both tiles' last S products
+    uint64_t* kv_full = bars + 2;
     uint64_t* kv_empty = kv_full + kStages;
     uint64_t* s_full = kv_empty + kStages;  // [tile]: S of the tile's next block computed
     uint64_t* s_free = s_full + 2;          // [tile]: its 4 softmax warps have read S
@@ -645,7 +648,7 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
     uint64_t* item_empty = item_full + kRing;
     uint64_t* drain = item_empty + kRing;   // [tile]: wind-down of an MMA warp
     uint64_t* tma_done = drain + 2;         // the TMA warp finished issuing an item's loads
-    static_assert(2 + 2 + 2 * kStages + 2 * 7 + 2 * kRing + 2 + 1 == kNumBars, "barriers");
+    static_assert(1 + 1 + 2 * kStages + 2 * 7 + 2 * kRing + 2 + 1 == kNumBars, "barriers");
     Plan* plans = reinterpret_cast<Plan*>(smem + kOffPlans);
     static_assert(sizeof(Plan) <= 128, "plan slot");
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
@@ -666,9 +669,9 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
 #endif
 
     if (threadIdx.x == 0) {
+        mbar_init(q_full, 1);
+        mbar_init(q_empty, 2);  // one commit per MMA warp
         for (int i = 0; i < 2; ++i) {
-            mbar_init(&q_full[i], 1);
-            mbar_init(&q_empty[i], 2);  // one arrival per MMA warp
             mbar_init(&s_full[i], 1);
             mbar_init(&s_free[i], 4);
             mbar_init(&p_full[i], 4);
@@ -760,16 +763,16 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
                 if (lane == 0) mbar_arrive(tma_done);
                 continue;
             }
-            const uint32_t qb = item_cnt & 1;
             if (lane == 0) TRACE(0, 12, pl.id, item_cnt, 0);
-            TIMED(1, ok = wait_all(&q_empty[qb], ((item_cnt >> 1) & 1) ^ 1));
+            // the previous item's last S products have read Q
+            TIMED(1, ok = wait_all(q_empty, (item_cnt & 1) ^ 1));
             if (ok && lane == 0) {
                 const int nq = pl.t[0].present + pl.t[1].present;
-                mbar_arrive_expect_tx(&q_full[qb], nq * kTileBytes);
+                mbar_arrive_expect_tx(q_full, nq * kTileBytes);
                 for (int x = 0; x < 2; ++x)
                     if (pl.t[x].present)
-                        tma_load_3d(smem + kOffQ + (qb * 2 + x) * kTileBytes, pl.global ? &maps.qg : &maps.q,
-                                    &q_full[qb], 0, pl.t[x].r0, pl.bh);
+                        tma_load_3d(smem + kOffQ + x * kTileBytes, pl.global ? &maps.qg : &maps.q, q_full, 0,
+                                    pl.t[x].r0, pl.bh);
             }
             // Every load of the plan is issued (the MMA warp maps a tile's
             // blocks to ring stages by load index).
@@ -906,7 +909,7 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
             const Plan& pl = *plp;
             if (pl.id < 0) break;
             if (pl.nloads == 0) continue;
-            const uint32_t qb = item_cnt & 1;
+
             const int nA = tile_blocks(pl.t[0]), nB = tile_blocks(pl.t[1]);
             const int nx = x ? nB : nA;
             const int glob = pl.global, e1 = pl.e1, lo_min = pl.lo_min;
@@ -940,8 +943,8 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
                 }
                 return true;
             };
-            if (nx > 0) TIMED(1, ok = wait_all(&q_full[qb], (item_cnt >> 1) & 1));
-            const uint64_t dqx = dq0 + (qb * 2 + x) * kTileStep;
+            if (nx > 0) TIMED(1, ok = wait_all(q_full, item_cnt & 1));
+            const uint64_t dqx = dq0 + x * kTileStep;
             uint32_t st_prev = 0;
             for (int j = 0; j < nx && ok; ++j) {
                 const int q = load_idx(j);
@@ -962,6 +965,7 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
                     for (int kk = 0; kk < kHD / 16; ++kk)
                         mma_f16_ss(t_s, dqx + kk * 2, dk + kk * 2, idesc_qk, kk > 0);
                     tc_commit(&s_full[x]);
+                    if (j == nx - 1) tc_commit(q_empty);  // the item's last S: Q is free once it is done
 #if LF_TRACE
                     tacc[7] += clock64() - tq0_;
 #endif
@@ -972,10 +976,7 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
             }
             if (ok && nx > 0) ok = issue_pv(nx - 1, st_prev);
             if (ok) ok = take_loads(pl.nloads - 1);
-            if (ok && lane == 0) {
-                if (nx > 0) tc_commit(&q_empty[qb]);
-                else mbar_arrive(&q_empty[qb]);
-            }
+            if (ok && lane == 0 && nx == 0) mbar_arrive(q_empty);
             __syncwarp();
             ++item_cnt;
             kv_cnt += pl.nloads;
