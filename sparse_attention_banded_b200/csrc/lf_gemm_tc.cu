@@ -79,6 +79,9 @@ struct GemmParams {
     int heads_D;         // kEpiHeads: columns per output tensor (H*64)
     int heads_H;
     int* status;
+    // The weights are not written by the kernel before this one: the TMA
+    // warp loads the first stages' W tiles before waiting for that kernel.
+    int w_early;
 };
 
 struct TileAt {
@@ -196,8 +199,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
     const uint32_t tmem = *tmem_slot;
     // Launched as a programmatic dependent, this grid may have started while
     // the kernel before it still runs: no global memory is read or written
-    // before that kernel has completed.
-    asm volatile("griddepcontrol.wait;" ::: "memory");
+    // before that kernel has completed (the TMA warp waits after its early
+    // weight loads, see below).
+    if (warp != 0) asm volatile("griddepcontrol.wait;" ::: "memory");
 
     // The TMA and MMA warps run their loops with all 32 lanes (lane 0 issues
     // the copies, tensor-core instructions and commits): a lone lane running
@@ -209,6 +213,22 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
     if (warp == 0) {
         uint32_t kc = 0;
         bool ok = true;
+        // W tiles of the first stages, issued before the wait when the
+        // weights do not come from the kernel before this one
+        uint32_t pre = 0;
+        if (p.w_early && (int)blockIdx.x < p.tiles) {
+            const TileAt at = tile_at(p, blockIdx.x);
+            const CUtensorMap* mw = at.width == kTN ? (at.pi ? &map_w2 : &map_w) : (at.pi ? &map_w2h : &map_wh);
+            const uint32_t bytes = kABytes + (at.width == kTN ? kBBytes : kBBytes / 2);
+            pre = p.ktiles < kStages ? (uint32_t)p.ktiles : (uint32_t)kStages;
+            if (lane == 0)
+                for (uint32_t st = 0; st < pre; ++st) {
+                    mbar_arrive_expect_tx(&full[st], bytes);
+                    tma_load_2d(smem + kOffB + st * kBBytes, mw, &full[st], (int)st * kTK, at.col0);
+                }
+            __syncwarp();
+        }
+        asm volatile("griddepcontrol.wait;" ::: "memory");
         for (int t = blockIdx.x; t < p.tiles && ok; t += gridDim.x) {
             const TileAt at = tile_at(p, t);
             const CUtensorMap* ma = at.pi ? &map_a2 : &map_a;
@@ -216,6 +236,12 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
             const uint32_t bytes = kABytes + (at.width == kTN ? kBBytes : kBBytes / 2);
             for (int kt = 0; kt < p.ktiles && ok; ++kt, ++kc) {
                 const uint32_t st = kc % kStages;
+                if (kc < pre) {  // fresh stage, its W tile already on the way
+                    if (lane == 0)
+                        tma_load_3d(smem + kOffA + st * kABytes, ma, &full[st], kt * kTK, at.mt * kTM, at.b);
+                    __syncwarp();
+                    continue;
+                }
                 ok = wait_all(&empty[st], ((kc / kStages) & 1) ^ 1);
                 if (!ok) break;
                 if (lane == 0) {
@@ -450,6 +476,7 @@ lf_status launch_t(const GemmArgs& g, int sm_count, cudaStream_t stream) {
     p.t_full = nt - p.n_split;
     p.tiles = nt + p.n_split;
     p.mode = g.mode;
+    p.w_early = g.w_early ? 1 : 0;
     p.resid = g.resid;
     p.heads_D = g.heads_D;
     p.heads_H = g.heads_H;

@@ -138,6 +138,10 @@ struct GemmArgs {
     const void* bias2; // [N2]
     void* out2;
     int heads_L2;
+    // The weights are not written by the work queued right before this
+    // launch (a kernel that may let it start early): their first tiles are
+    // loaded before the wait for that work.
+    bool w_early;
 };
 // N % 128 == 0, K % 64 == 0; fp16 / bf16.
 lf_status launch_gemm_tc(const GemmArgs& g, lf_dtype dtype, int sm_count, cudaStream_t stream);

@@ -93,9 +93,10 @@ int ffn_path_for(int M, int D, int F, int path) {
 }
 
 // Step 6 before its LayerNorm: z = h + b_2 + GELU(h W_1^T + b_1) W_2^T,
-// fused or as two GEMMs through f ([M][F] of dtype).
+// fused or as two GEMMs through f ([M][F] of dtype).  w_early: the work
+// queued before does not write the weights (inside a layer call).
 lf_status gelu_ffn(const void* h, const void* W1, const void* b1, const void* W2, const void* b2, int M, int D, int F,
-                   lf_dtype dtype, int path, void* f, float* z, DeviceCtx* d, cudaStream_t s) {
+                   lf_dtype dtype, int path, void* f, float* z, DeviceCtx* d, cudaStream_t s, bool w_early = false) {
     if (path == LF_FFN_FUSED) {
         FfnArgs a{};
         a.h = h; a.W1 = W1; a.b1 = b1; a.W2 = W2; a.b2 = b2;
@@ -106,10 +107,12 @@ lf_status gelu_ffn(const void* h, const void* W1, const void* b1, const void* W2
     GemmArgs f1{};
     f1.A = h; f1.batches = 1; f1.rows = M; f1.batch_stride = M; f1.K = D;
     f1.W = W1; f1.N = F; f1.bias = b1; f1.mode = kEpiGelu; f1.out = f; f1.status = d->status;
+    f1.w_early = w_early;
     if ((st = launch_gemm_tc(f1, dtype, d->sm_count, s)) != LF_OK) return st;
     GemmArgs f2{};
     f2.A = f; f2.batches = 1; f2.rows = M; f2.batch_stride = M; f2.K = F;
     f2.W = W2; f2.N = D; f2.bias = b2; f2.mode = kEpiResid; f2.resid = h; f2.out = z; f2.status = d->status;
+    f2.w_early = true;  // W_2 is not written by the FFN1 GEMM before it
     return launch_gemm_tc(f2, dtype, d->sm_count, s);
 }
 
@@ -147,6 +150,7 @@ lf_status layer_forward(const void* x, const float* local_mask, const float* glo
     g.W = wt->W_qkv_kgvg; g.N = 5 * D; g.bias = wt->b_qkv_kgvg; g.mode = kEpiHeads;
     g.out = qkv; g.heads_D = D; g.heads_H = H; g.heads_L = L; g.status = d->status;
     g.W2 = wt->W_qg; g.N2 = D; g.bias2 = wt->b_qg;
+    g.w_early = true;  // inside a layer call no kernel writes the weights
     if (any) {
         // Qg of the global tokens only: their rows of x, gathered, into the
         // slot buffer (slot layout [B][H][gcap][64])
@@ -171,7 +175,7 @@ lf_status layer_forward(const void* x, const float* local_mask, const float* glo
     GemmArgs o{};
     o.A = base + ws.att; o.batches = B; o.rows = L; o.batch_stride = L; o.K = D;
     o.W = wt->W_o; o.N = D; o.bias = wt->b_o; o.mode = kEpiResid; o.resid = x; o.out = base + ws.z;
-    o.status = d->status;
+    o.status = d->status; o.w_early = true;
     if ((st = launch_gemm_tc(o, dtype, d->sm_count, s)) != LF_OK) return st;
     if ((st = launch_layernorm(reinterpret_cast<float*>(base + ws.z), wt->ln1_gamma, wt->ln1_beta, B * L, D, ln_eps,
                                dtype, base + ws.h, s)) != LF_OK)
@@ -179,7 +183,7 @@ lf_status layer_forward(const void* x, const float* local_mask, const float* glo
     // step 6: GELU FFN + bias + residual, LayerNorm
     if ((st = gelu_ffn(base + ws.h, wt->W_1, wt->b_1, wt->W_2, wt->b_2, B * L, D, F, dtype,
                        ffn_path_for(B * L, D, F, g_ffn_path.load()), base + ws.f,
-                       reinterpret_cast<float*>(base + ws.z), d, s)) != LF_OK)
+                       reinterpret_cast<float*>(base + ws.z), d, s, true)) != LF_OK)
         return st;
     return launch_layernorm(reinterpret_cast<float*>(base + ws.z), wt->ln2_gamma, wt->ln2_beta, B * L, D, ln_eps,
                             dtype, out, s);
