@@ -50,7 +50,8 @@ def _oracle(h, W1, b1, W2, b2, dtype):
 
 
 # (rows, D, F): clusters of 1 (D <= 256), 2 (D <= 512) and 4 CTAs, output
-# quarters of 160 / 192 / 224 / 256 columns, ragged last row tiles
+# quarters of 160 / 192 / 224 / 256 columns, ragged last row tiles, and a
+# two-GEMM launch whose last partial round of tiles is split in halves
 SHAPES = [
     (300, 128, 256),
     (200, 256, 512),
@@ -60,6 +61,7 @@ SHAPES = [
     (260, 768, 1024),
     (129, 896, 512),
     (513, 1024, 2048),
+    (8192, 640, 512),   # the second GEMM's 192 tiles: its last 44 run as 128-wide halves, ragged last N tile among them
 ]
 
 
