@@ -26,6 +26,11 @@
 //   kEpiGelu   : + bias, GELU (erf form), round, row-major out[b*rows + m][n]
 //   kEpiResid  : + bias + residual (same dtype, row-major [.., N]), fp32
 //                row-major out (the LayerNorm kernel reads it)
+//   kEpiResidLN: + bias + residual, then LayerNorm over the row (step 5's
+//                AddBiasResidualLayerNorm and step 6's), rounded, row-major
+//                out: the N / 256 CTAs of a row tile form a cluster and
+//                exchange per-row sums through distributed shared memory
+//                (the mean, then the centred second moment)
 // Roofline: tensor-bound (2*M*N*K flops over (M*K + N*K)*2 + out bytes).
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -34,7 +39,7 @@
 #include <mutex>
 
 #include "lf_internal.h"
-#include "sm100.cuh"
+#include "sm100_cluster.cuh"
 
 namespace lf {
 namespace {
@@ -50,8 +55,11 @@ constexpr uint32_t kBBytes = kTN * kTK * 2;  // 32 KB
 constexpr uint32_t kOffA = 0;
 constexpr uint32_t kOffB = kOffA + kStages * kABytes;
 constexpr uint32_t kOffBias = kOffB + kStages * kBBytes;        // epilogue warps x kTN / 2 floats
-constexpr uint32_t kOffBar = kOffBias + kEpiWarps * (kTN / 2) * 4;
-constexpr uint32_t kNumBars = 2 * kStages + 4 + 1;
+constexpr uint32_t kOffRed = kOffBias + kEpiWarps * (kTN / 2) * 4;  // kEpiResidLN: [2 halves][kTM] row sums
+constexpr int kMaxLnCtas = 4;                                          // N <= 1024
+constexpr uint32_t kOffXch = kOffRed + 2 * kTM * 4;                    // [2 sums][kMaxLnCtas][kTM] from each CTA
+constexpr uint32_t kOffBar = kOffXch + 2 * kMaxLnCtas * kTM * 4;
+constexpr uint32_t kNumBars = 2 * kStages + 4 + 1 + 2;
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
 constexpr uint32_t kSmemBytes = kOffMisc + 64 + 1024;
 constexpr uint32_t kTmemCols = 512;  // two 256-column fp32 accumulators
@@ -82,6 +90,12 @@ struct GemmParams {
     // The weights are not written by the kernel before this one: the TMA
     // warp loads the first stages' W tiles before waiting for that kernel.
     int w_early;
+    // kEpiResidLN: LayerNorm parameters; ln_ctas = CTAs per cluster (one
+    // per 256-column tile of the row tile)
+    const float* ln_gamma;
+    const float* ln_beta;
+    float ln_eps;
+    int ln_ctas;
 };
 
 struct TileAt {
@@ -141,6 +155,19 @@ __device__ __forceinline__ void tmem_ld32v(uint32_t taddr, float (&r)[32]) {
         : "r"(taddr));
 }
 
+__device__ __forceinline__ void tmem_st32v(uint32_t taddr, const float (&r)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+        "f"(r[0]), "f"(r[1]), "f"(r[2]), "f"(r[3]), "f"(r[4]), "f"(r[5]), "f"(r[6]), "f"(r[7]), "f"(r[8]),
+        "f"(r[9]), "f"(r[10]), "f"(r[11]), "f"(r[12]), "f"(r[13]), "f"(r[14]), "f"(r[15]), "f"(r[16]), "f"(r[17]),
+        "f"(r[18]), "f"(r[19]), "f"(r[20]), "f"(r[21]), "f"(r[22]), "f"(r[23]), "f"(r[24]), "f"(r[25]), "f"(r[26]),
+        "f"(r[27]), "f"(r[28]), "f"(r[29]), "f"(r[30]), "f"(r[31])
+        : "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
 __device__ __forceinline__ float gelu_erf(float x) { return 0.5f * x * (1.0f + erff(x * 0.70710678118654752f)); }
 
 template <typename T>
@@ -157,6 +184,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
     uint64_t* acc_full = bars + 2 * kStages;
     uint64_t* acc_empty = acc_full + 2;
     uint64_t* drain = acc_empty + 2;
+    uint64_t* xbar = drain + 1;  // [2] kEpiResidLN: every CTA of the cluster has delivered its row sums
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -174,6 +202,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
             mbar_init(&acc_empty[i], kEpiWarps);
         }
         mbar_init(drain, 1);
+        mbar_init(&xbar[0], p.ln_ctas);
+        mbar_init(&xbar[1], p.ln_ctas);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -196,6 +226,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    // every CTA's barriers are initialised before a peer arrives on them
+    if (p.mode == kEpiResidLN) cluster_sync();
     const uint32_t tmem = *tmem_slot;
     // Launched as a programmatic dependent, this grid may have started while
     // the kernel before it still runs: no global memory is read or written
@@ -299,6 +331,126 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
         const int r = sp * 32 + lane;
         const uint32_t lane_off = (uint32_t)(sp * 32) << 16;
         float* bias_w = reinterpret_cast<float*>(smem + kOffBias) + (warp - 4) * (kTN / 2);
+        // kEpiResidLN: the sum over the cluster's columns of v (this
+        // thread's partial for row r): both warps' halves through shared
+        // memory, then every CTA's sum into every CTA's exchange slot, added
+        // in CTA order (so all CTAs of the cluster get the same bits).
+        // Returns false on a failure of any epilogue warp (taken together).
+        float* red = reinterpret_cast<float*>(smem + kOffRed);
+        float* xch = reinterpret_cast<float*>(smem + kOffXch);
+        const uint32_t rank = p.mode == kEpiResidLN ? cluster_ctarank() : 0;
+        auto cluster_row_sum = [&](float v, int e, uint32_t parity, bool fail, float& total) -> bool {
+            red[half * kTM + r] = v;
+            if (named_bar_any(1, kEpiWarps * 32, fail)) return false;
+            if (half == 0) {
+                const float part = red[r] + red[kTM + r];
+                const uint32_t slot = smem_u32(xch + (e * kMaxLnCtas + rank) * kTM + r);
+                for (int q = 0; q < p.ln_ctas; ++q) st_cluster_f32(mapa_shared(slot, (uint32_t)q), part);
+                fence_acq_rel_cluster();
+            }
+            named_bar_sync(1, kEpiWarps * 32);
+            if (warp == 4 && lane == 0)
+                for (int q = 0; q < p.ln_ctas; ++q) mbar_arrive_cluster(mapa_shared(smem_u32(&xbar[e]), (uint32_t)q));
+            const bool got = __all_sync(0xffffffffu, mbar_wait_cluster(&xbar[e], parity, abort_flag));
+            if (named_bar_any(1, kEpiWarps * 32, !got)) return false;
+            float t = 0.0f;
+            for (int q = 0; q < p.ln_ctas; ++q) t += xch[(e * kMaxLnCtas + q) * kTM + r];
+            total = t;
+            return true;
+        };
+        // kEpiResidLN, one tile: z = acc + bias + resid kept in TMEM, mean,
+        // centred second moment, then (z - mean) * rsqrt(var + eps) * gamma
+        // + beta rounded and stored.  False on a failure (all warps alike).
+        uint32_t ln_cnt = 0;
+        auto ln_tile = [&](const TileAt& at, const GemmProb& q, uint32_t ab, uint32_t tcn, int n0, int ncols,
+                           int wcols) -> bool {
+            bool fail = !__all_sync(0xffffffffu, mbar_wait(&acc_full[ab], (tcn >> 1) & 1, abort_flag));
+            const int m = at.mt * kTM + r;
+            const bool row_ok = m < q.rows;
+            const size_t grow = (size_t)at.b * q.rows + m;
+            const uint32_t tz = tmem + lane_off + ab * kTN + half * wcols;
+            float s1 = 0.0f;
+            if (!fail) {
+                tc_fence_after();
+#pragma unroll 1
+                for (int c0 = 0; c0 < ncols; c0 += 32) {
+                    float z[32];
+                    __syncwarp();
+                    tmem_ld32v(tz + c0, z);
+                    tmem_ld_wait();
+                    regs_ready<32>(z);
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) z[c] += bias_w[c0 + c];
+                    if (row_ok) {
+                        const uint4* rs =
+                            reinterpret_cast<const uint4*>(reinterpret_cast<const T*>(p.resid) + grow * q.N + n0 + c0);
+#pragma unroll
+                        for (int u4 = 0; u4 < 4; ++u4) {
+                            uint4 u = rs[u4];
+                            const T* e = reinterpret_cast<const T*>(&u);
+#pragma unroll
+                            for (int j = 0; j < 8; ++j) z[u4 * 8 + j] += Cvt<T>::to_f(e[j]);
+                        }
+                    }
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) s1 += z[c];
+                    tmem_st32v(tz + c0, z);
+                }
+                tmem_st_wait();
+            }
+            const uint32_t parity = ln_cnt & 1;
+            ++ln_cnt;
+            float sum = 0.0f, sq = 0.0f;
+            if (!cluster_row_sum(s1, 0, parity, fail, sum)) return false;
+            const float mean = sum / (float)q.N;
+            float s2 = 0.0f;
+#pragma unroll 1
+            for (int c0 = 0; c0 < ncols; c0 += 32) {
+                float z[32];
+                __syncwarp();
+                tmem_ld32v(tz + c0, z);
+                tmem_ld_wait();
+                regs_ready<32>(z);
+#pragma unroll
+                for (int c = 0; c < 32; ++c) {
+                    const float d = z[c] - mean;
+                    s2 = fmaf(d, d, s2);
+                }
+            }
+            if (!cluster_row_sum(s2, 1, parity, false, sq)) return false;
+            const float inv = rsqrtf(sq / (float)q.N + p.ln_eps);
+#pragma unroll 1
+            for (int c0 = 0; c0 < ncols; c0 += 32) {
+                float z[32];
+                __syncwarp();
+                tmem_ld32v(tz + c0, z);
+                tmem_ld_wait();
+                regs_ready<32>(z);
+                if (row_ok) {
+                    const int n = n0 + c0;
+                    uint4* d4 = reinterpret_cast<uint4*>(reinterpret_cast<T*>(q.out) + grow * q.N + n);
+#pragma unroll
+                    for (int u4 = 0; u4 < 4; ++u4) {
+                        float y[8];
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            const int c = u4 * 8 + j;
+                            y[j] = fmaf((z[c] - mean) * inv, __ldg(p.ln_gamma + n + c), __ldg(p.ln_beta + n + c));
+                        }
+                        uint4 u;
+                        u.x = Cvt<T>::two(y[0], y[1]);
+                        u.y = Cvt<T>::two(y[2], y[3]);
+                        u.z = Cvt<T>::two(y[4], y[5]);
+                        u.w = Cvt<T>::two(y[6], y[7]);
+                        d4[u4] = u;
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[ab]);
+            return true;
+        };
         uint32_t tc = 0;
         bool ok = true;
         for (int t = blockIdx.x; t < p.tiles && ok; t += gridDim.x, ++tc) {
@@ -316,6 +468,13 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
                 if (c * 32 < ncols) bias_w[c * 32 + lane] = Cvt<T>::to_f(bias[n0 + c * 32 + lane]);
             __syncwarp();
             const uint32_t ab = tc & 1;
+            if (p.mode == kEpiResidLN) {
+                if (!ln_tile(at, q, ab, tc, n0, ncols, wcols)) {
+                    ok = false;
+                    break;
+                }
+                continue;
+            }
             ok = __all_sync(0xffffffffu, mbar_wait(&acc_full[ab], (tc >> 1) & 1, abort_flag));
             if (!ok) break;
             tc_fence_after();
@@ -379,6 +538,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
     }
 
     __syncthreads();
+    // no CTA leaves while a peer may still write into its exchange slots
+    if (p.mode == kEpiResidLN) cluster_sync();
     if (threadIdx.x == 0 && *abort_flag) record_status(p.status, 0, LF_ERR_DEVICE_TIMEOUT);
     if (warp == 1) {
         tc_fence_after();
@@ -470,11 +631,23 @@ lf_status launch_t(const GemmArgs& g, int sm_count, cudaStream_t stream) {
     // when they fit in one round (R <= grid / 2): that round then takes half
     // a tile's time on up to every SM instead of a whole one on R of them.
     const int nt = p.pr[0].tiles + p.pr[1].tiles;
-    const int G = nt < sm_count ? nt : sm_count;
+    int G = nt < sm_count ? nt : sm_count;
     const int R = nt % G;
     p.n_split = (nt > G && R > 0 && 2 * R <= G) ? R : 0;
+    // kEpiResidLN: the row tile's column tiles form a cluster, whole tiles only
+    const bool ln = g.mode == kEpiResidLN;
+    const int C = ln ? p.pr[0].ntiles : 1;
+    if (ln) {
+        if (C > kMaxLnCtas || g.rows2 > 0 || !g.ln_gamma || !g.ln_beta) return LF_ERR_BAD_DIM;
+        p.n_split = 0;
+        G = G / C * C;
+    }
     p.t_full = nt - p.n_split;
     p.tiles = nt + p.n_split;
+    p.ln_gamma = g.ln_gamma;
+    p.ln_beta = g.ln_beta;
+    p.ln_eps = g.ln_eps;
+    p.ln_ctas = C;
     p.mode = g.mode;
     p.w_early = g.w_early ? 1 : 0;
     p.resid = g.resid;
@@ -492,16 +665,20 @@ lf_status launch_t(const GemmArgs& g, int sm_count, cudaStream_t stream) {
         attr[dev].store(true);
     }
     const int grid = G;
-    cudaLaunchAttribute at[1];
+    cudaLaunchAttribute at[2];
     at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     at[0].val.programmaticStreamSerializationAllowed = 1;
+    at[1].id = cudaLaunchAttributeClusterDimension;
+    at[1].val.clusterDim.x = C;
+    at[1].val.clusterDim.y = 1;
+    at[1].val.clusterDim.z = 1;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)grid);
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = kSmemBytes;
     cfg.stream = stream;
     cfg.attrs = at;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = ln ? 2 : 1;
     if (cudaLaunchKernelEx(&cfg, gemm_tc_kernel<T>, ma, mw, ma2, mw2, mwh, mw2h, p) != cudaSuccess) return LF_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? LF_OK : LF_ERR_CUDA;
 }

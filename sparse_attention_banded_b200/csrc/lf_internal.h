@@ -116,7 +116,7 @@ lf_status launch_attention_tc(const void* q, const void* k, const void* v, const
                               int32_t* gidx_out = nullptr, int32_t* gnum_out = nullptr);
 
 // ---- dense GEMM with fused epilogues (encoder layer) ----
-enum { kEpiHeads = 0, kEpiGelu = 1, kEpiResid = 2 };
+enum { kEpiHeads = 0, kEpiGelu = 1, kEpiResid = 2, kEpiResidLN = 3 };
 struct GemmArgs {
     const void* A;     // [batches][batch_stride][K], K-major
     int batches, rows, batch_stride, K;
@@ -142,6 +142,11 @@ struct GemmArgs {
     // launch (a kernel that may let it start early): their first tiles are
     // loaded before the wait for that work.
     bool w_early;
+    // kEpiResidLN: out = LayerNorm(A W^T + bias + resid) in dtype, over
+    // rows of N <= 1024 columns (population variance; gamma, beta fp32).
+    const float* ln_gamma;
+    const float* ln_beta;
+    float ln_eps;
 };
 // N % 128 == 0, K % 64 == 0; fp16 / bf16.
 lf_status launch_gemm_tc(const GemmArgs& g, lf_dtype dtype, int sm_count, cudaStream_t stream);

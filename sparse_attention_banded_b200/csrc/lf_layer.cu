@@ -7,9 +7,10 @@
 //     layout, whose few tiles run on the SMs the large one's last wave
 //     leaves free
 //   banded + global attention -> a [B, L, D]
-//   GEMM(a, W_o) + b_o + x -> z (fp32);  LayerNorm -> h
-//   GEMM(h, W_1) + b_1, GELU -> f;  GEMM(f, W_2) + b_2 + h -> z;  LayerNorm -> out
-//     (or the fused FFN kernel for the first line, which keeps f on chip)
+//   GEMM(a, W_o) + b_o + x, LayerNorm in its epilogue -> h
+//   GEMM(h, W_1) + b_1, GELU -> f;  GEMM(f, W_2) + b_2 + h, LayerNorm in its
+//     epilogue -> out  (or the fused FFN kernel, which keeps f on chip,
+//     -> z (fp32), then the LayerNorm kernel -> out)
 // With the global tokens at any position (the _any_globals entry points) the
 // partition (with its rank table) runs once per forward, the qg projection
 // multiplies only the global tokens' rows of x, gathered through global_idx,
@@ -171,18 +172,31 @@ lf_status layer_forward(const void* x, const float* local_mask, const float* glo
                                   local_mask, global_mask, B, H, L, w, attn_scale, dtype, base + ws.att,
                                   base + ws.scratch, d->status, d->sm_count, s, any ? &a : nullptr)) != LF_OK)
         return st;
-    // step 5: output projection + bias + residual, LayerNorm
+    // step 5: output projection + bias + residual with its LayerNorm in the
+    // GEMM's epilogue (the D-wide row tile's CTAs form a cluster)
     GemmArgs o{};
     o.A = base + ws.att; o.batches = B; o.rows = L; o.batch_stride = L; o.K = D;
-    o.W = wt->W_o; o.N = D; o.bias = wt->b_o; o.mode = kEpiResid; o.resid = x; o.out = base + ws.z;
+    o.W = wt->W_o; o.N = D; o.bias = wt->b_o; o.mode = kEpiResidLN; o.resid = x; o.out = base + ws.h;
+    o.ln_gamma = wt->ln1_gamma; o.ln_beta = wt->ln1_beta; o.ln_eps = ln_eps;
     o.status = d->status; o.w_early = true;
     if ((st = launch_gemm_tc(o, dtype, d->sm_count, s)) != LF_OK) return st;
-    if ((st = launch_layernorm(reinterpret_cast<float*>(base + ws.z), wt->ln1_gamma, wt->ln1_beta, B * L, D, ln_eps,
-                               dtype, base + ws.h, s)) != LF_OK)
-        return st;
     // step 6: GELU FFN + bias + residual, LayerNorm
-    if ((st = gelu_ffn(base + ws.h, wt->W_1, wt->b_1, wt->W_2, wt->b_2, B * L, D, F, dtype,
-                       ffn_path_for(B * L, D, F, g_ffn_path.load()), base + ws.f,
+    const int path = ffn_path_for(B * L, D, F, g_ffn_path.load());
+    if (path == LF_FFN_UNFUSED) {
+        // two GEMMs, the LayerNorm in the second one's epilogue
+        GemmArgs f1{};
+        f1.A = base + ws.h; f1.batches = 1; f1.rows = B * L; f1.batch_stride = B * L; f1.K = D;
+        f1.W = wt->W_1; f1.N = F; f1.bias = wt->b_1; f1.mode = kEpiGelu; f1.out = base + ws.f;
+        f1.status = d->status; f1.w_early = true;
+        if ((st = launch_gemm_tc(f1, dtype, d->sm_count, s)) != LF_OK) return st;
+        GemmArgs f2{};
+        f2.A = base + ws.f; f2.batches = 1; f2.rows = B * L; f2.batch_stride = B * L; f2.K = F;
+        f2.W = wt->W_2; f2.N = D; f2.bias = wt->b_2; f2.mode = kEpiResidLN; f2.resid = base + ws.h; f2.out = out;
+        f2.ln_gamma = wt->ln2_gamma; f2.ln_beta = wt->ln2_beta; f2.ln_eps = ln_eps;
+        f2.status = d->status; f2.w_early = true;
+        return launch_gemm_tc(f2, dtype, d->sm_count, s);
+    }
+    if ((st = gelu_ffn(base + ws.h, wt->W_1, wt->b_1, wt->W_2, wt->b_2, B * L, D, F, dtype, path, base + ws.f,
                        reinterpret_cast<float*>(base + ws.z), d, s, true)) != LF_OK)
         return st;
     return launch_layernorm(reinterpret_cast<float*>(base + ws.z), wt->ln2_gamma, wt->ln2_beta, B * L, D, ln_eps,

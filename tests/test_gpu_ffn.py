@@ -104,10 +104,12 @@ def test_ffn_workload5_full_parity():
 
 @pytest.mark.parametrize("dtype,hidden,ffn,L", [("f16", 512, 1024, 1024), ("bf16", 512, 1024, 1024),
                                                  ("f16", 1024, 4096, 4096)])
-def test_layer_ffn_paths_identical(dtype, hidden, ffn, L):
+def test_layer_ffn_paths(dtype, hidden, ffn, L):
     """The encoder layer (a 512-wide one, and workload 5's shape) with either
-    FFN path selected gives the same bits; the layer parity tests cover the
-    default path."""
+    FFN path selected matches the layer oracle; auto takes the two GEMMs at
+    these widths.  (With the two GEMMs the LayerNorm runs in the second
+    GEMM's epilogue, with the fused FFN in its own kernel, so the two paths
+    round differently.)"""
     wl, x, W, lm, gm = inputs.layer_inputs(5, hidden=hidden, ffn=ffn, B=1, L=L, dtype=dtype, g=[64], pad=[17],
                                            seed=91, bias_scale=0.1, ln_scale=0.1)
     dev = {k: v.cuda() for k, v in W.items()}
@@ -120,8 +122,16 @@ def test_layer_ffn_paths_identical(dtype, hidden, ffn, L):
     lf.lf_set_ffn_path("auto")
     torch.cuda.synchronize()
     assert lf.lf_device_status(reset=True) == 0
-    assert torch.equal(outs["unfused"], outs["fused"])
-    assert torch.equal(outs["auto"], outs["fused"])
+    assert torch.equal(outs["auto"], outs["unfused"])
+    o = {k: np.swapaxes(v.double().numpy(), -1, -2) if k in ("W_qkv_kgvg", "W_qg", "W_o", "W_1", "W_2")
+         else v.double().numpy() for k, v in W.items()}
+    ref = oracle.encoder_layer(x, lm, gm, o, hidden // 64, 256, 0.125, 1e-5,
+                               round_attention_inputs=_round_to(TDT[dtype]), round_stored=_round_to(TDT[dtype]))
+    for path in ("unfused", "fused"):
+        got = outs[path].float().cpu().numpy()
+        err = float((np.abs(got - ref) / np.maximum(1.0, np.abs(ref))).max())
+        print("layer %s ffn=%s: max scaled err %.3e" % (dtype, path, err))
+        assert err <= TOL[TDT[dtype]], (path, err)
 
 
 def test_ffn_errors():
