@@ -25,8 +25,8 @@
 //               shared memory in the 128-byte-swizzled K-major operand
 //               layout), then one thread copies the chunk into the same slot
 //               of every other CTA of the cluster (bulk shared-to-distributed
-//               -shared copies, each completing on the receiver's mbarrier;
-//               no multicast); after the last round the output epilogue
+//               -shared copies, each to one CTA and completing on its
+//               mbarrier); after the last round the output epilogue
 //               (+ b_2 + h, fp32 stores)
 // Every CTA's sums over the intermediate run over k in the order of the
 // two-GEMM path (chunk by chunk, 16 at a time), as do the sums over D.

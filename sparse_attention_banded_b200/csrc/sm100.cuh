@@ -1,5 +1,5 @@
 // Thin inline-PTX wrappers for the sm_100a features the kernels use:
-// mbarriers with bounded waits, TMA tiled loads (no multicast), and the
+// mbarriers with bounded waits, TMA tiled loads (each into this CTA only), and the
 // tcgen05 tensor-memory / MMA instructions.  Written from the public PTX ISA.
 #pragma once
 

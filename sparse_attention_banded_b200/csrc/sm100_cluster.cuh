@@ -1,5 +1,5 @@
 // Inline-PTX wrappers for thread-block clusters (distributed shared memory,
-// point to point only: no multicast) and a reducing named barrier, for the
+// point to point only: one destination CTA per access) and a reducing named barrier, for the
 // kernels whose CTAs work in clusters.  Written from the public PTX ISA.
 #pragma once
 
