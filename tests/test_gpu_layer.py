@@ -68,6 +68,8 @@ def _run_and_compare(x, W, lm, gm, H, w, dtype, rows=None, any_pos=False):
     (1, 2, 512, 64, 256, [8], [0]),
     (2, 2, 640, 128, 384, [5, 100], [0, 33]),   # ragged last M tile, padding, two samples
     (1, 4, 1024, 256, 512, [64], [17]),
+    (1, 6, 512, 64, 768, [8], [3]),             # D = 384: LayerNorm clusters of 2, the second tile half filled
+    (2, 12, 512, 128, 1536, [20, 0], [0, 40]),  # D = 768: clusters of 3
 ])
 def test_layer_small_parity(dtype, B, H, L, w, ffn, g, pad):
     wl, x, W, lm, gm = inputs.layer_inputs(5, hidden=H * 64, ffn=ffn, B=B, L=L, dtype=dtype, g=g, pad=pad,
