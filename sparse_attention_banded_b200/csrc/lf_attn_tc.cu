@@ -140,6 +140,10 @@ struct Params {
     // CTA b while the first items' scores are being computed.
     int32_t* gidx_out;  // [B][L] or NULL
     int32_t* gnum_out;  // [B]
+    // The masks are not written by the kernel before this one (inside a
+    // layer call): the planner builds its first plan and the softmax warps
+    // read their masks before waiting for that kernel.
+    int masks_early;
 };
 
 // Diagnostic builds (-DLF_TRACE=1) record per CTA and role the cycles spent
@@ -715,8 +719,16 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
     const uint32_t tmem = *tmem_slot;
     // Launched as a programmatic dependent, this grid may have started while
     // the kernel before it still runs (and may still be writing this
-    // kernel's inputs): no global memory is touched before it has completed.
-    asm volatile("griddepcontrol.wait;" ::: "memory");
+    // kernel's inputs): no global memory is touched before it has completed,
+    // except the masks when masks_early says the kernel before does not
+    // write them (the planner then waits before its first atomic; the MMA
+    // warps touch no global memory).
+    {
+        const bool early = p.masks_early != 0 && !kAny;
+        const bool reads_masks_only = warp == 2 || (warp >= kSoftmaxWarp0 && warp < kEpiWarp0);
+        const bool no_global = warp == 1 || warp == 3;
+        if (!(early && (reads_masks_only || no_global))) asm volatile("griddepcontrol.wait;" ::: "memory");
+    }
 #if LF_TRACE
     if (threadIdx.x == 0 && p.trace) {
         volatile int* d_ = p.trace + gridDim.x * 16 * 4 + (blockIdx.x * 16 + 14) * 16;
@@ -825,6 +837,7 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
                 // The first item of CTA c is item c (no atomic on the critical
                 // path of the start); later ones come from the counter, which
                 // counts past the first gridDim.x items.
+                if (k == 1 && p.masks_early && !kAny) asm volatile("griddepcontrol.wait;" ::: "memory");
                 id = k == 0 ? (int)blockIdx.x : (int)gridDim.x + atomicAdd(p.sched, 1);
                 if (id >= p.n_items) id = -1;
             }
@@ -1783,7 +1796,7 @@ lf_status launch_attention_tc(const void* q, const void* k, const void* v, const
                               const void* vg, const float* local_mask, const float* global_mask, int B, int H,
                               int L, int w, float scale, lf_dtype dtype, void* out, void* scratch, int* status,
                               int sm_count, cudaStream_t stream, const AnyGlobals* any, int32_t* gidx_out,
-                              int32_t* gnum_out) {
+                              int32_t* gnum_out, bool masks_early) {
     const Geometry geo = geometry(B, H, L, w, sm_count);
     Maps maps;
     const int BH = B * H;
@@ -1833,6 +1846,7 @@ lf_status launch_attention_tc(const void* q, const void* k, const void* v, const
     p.gcap = any ? any->gcap : 0;
     p.gidx_out = any ? nullptr : gidx_out;
     p.gnum_out = any ? nullptr : gnum_out;
+    p.masks_early = masks_early ? 1 : 0;
 #if LF_TRACE
     if (const char* a = getenv("LF_TRACE_ADDR")) p.trace = reinterpret_cast<int*>(strtoull(a, nullptr, 10));
 #endif

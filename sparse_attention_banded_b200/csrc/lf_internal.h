@@ -107,13 +107,14 @@ size_t attention_tc_scratch_zero_bytes(int B, int H, int L, int w);
 // any (may be NULL): global tokens at any position, with the compact
 // buffers filled by launch_gather_globals.  gidx_out / gnum_out (prefix
 // path, may be NULL): the kernel also writes the global-index partition
-// (as launch_global_idx with the prefix check) into them.
+// (as launch_global_idx with the prefix check) into them.  masks_early: the
+// work queued right before does not write the masks (inside a layer call).
 lf_status launch_attention_tc(const void* q, const void* k, const void* v, const void* qg,
                               const void* kg, const void* vg, const float* local_mask,
                               const float* global_mask, int B, int H, int L, int w, float scale,
                               lf_dtype dtype, void* out, void* scratch, int* status,
                               int sm_count, cudaStream_t stream, const AnyGlobals* any = nullptr,
-                              int32_t* gidx_out = nullptr, int32_t* gnum_out = nullptr);
+                              int32_t* gidx_out = nullptr, int32_t* gnum_out = nullptr, bool masks_early = false);
 
 // ---- dense GEMM with fused epilogues (encoder layer) ----
 enum { kEpiHeads = 0, kEpiGelu = 1, kEpiResid = 2, kEpiResidLN = 3 };

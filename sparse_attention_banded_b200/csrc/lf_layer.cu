@@ -170,7 +170,8 @@ lf_status layer_forward(const void* x, const float* local_mask, const float* glo
     // for them on the device; its counters are zero, see above)
     if ((st = launch_attention_tc(slot(0), slot(1), slot(2), any ? a.qg_c : base + ws.qg, slot(3), slot(4),
                                   local_mask, global_mask, B, H, L, w, attn_scale, dtype, base + ws.att,
-                                  base + ws.scratch, d->status, d->sm_count, s, any ? &a : nullptr)) != LF_OK)
+                                  base + ws.scratch, d->status, d->sm_count, s, any ? &a : nullptr, nullptr,
+                                  nullptr, true)) != LF_OK)
         return st;
     // step 5: output projection + bias + residual with its LayerNorm in the
     // GEMM's epilogue (the D-wide row tile's CTAs form a cluster)
