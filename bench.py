@@ -191,7 +191,7 @@ def traffic_from_profile(kernel_src_hash: str):
 
 def kernel_source_hash():
     h = hashlib.sha256()
-    for name in ("lf_attn_tc.cu", "lf_pair_math.cuh", "sm100.cuh"):
+    for name in ("lf_attn_tc.cu", "lf_pair_math.cuh", "lf_partition.cuh", "sm100.cuh"):
         with open(os.path.join(ROOT, "sparse_attention_banded_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -273,16 +273,16 @@ def run_ours(args):
         else:
             lf.lf_attention_forward(*ins, lm_, gm_, wl.w, out=out)
 
-    # fp16 / bf16 attention with prefix globals: the partition and the
-    # attention are one kernel launch (lf_attention_forward_idx)
-    tc_prefix = not (layer or anyg) and wl.dtype != "f32"
+    # attention with prefix globals: the partition and the attention are one
+    # kernel launch (lf_attention_forward_idx)
+    prefix_attn = not (layer or anyg)
 
     def path(ins, lm_, gm_):
         # one pass of the whole hot path: the partition and the attention
         # (the any-position calls run their partition themselves)
         if anyg or any_layer:
             compute(ins, lm_, gm_)
-        elif layer or not tc_prefix:
+        elif layer:
             lf.lf_init_global_idx(gm_, wl.w, gidx, gnum, sync=False)
             compute(ins, lm_, gm_)
         else:
@@ -293,8 +293,8 @@ def run_ours(args):
 
     def kernel_alone():
         # the dominant kernel alone: the step's one launch for the prefix
-        # tensor-core path, else the attention (or layer) call
-        if tc_prefix:
+        # attention, else the attention (or layer) call
+        if prefix_attn:
             path(args_in, lm, gm)
         else:
             compute(args_in, lm, gm)
@@ -453,10 +453,10 @@ def run_ours(args):
         # our kernels per step: any-position attention = partition-and-gather
         # + attention; any-position layer = partition + 9 per layer (8 with
         # the fused FFN); layer = partition + 7 per layer (6 with the fused
-        # FFN); prefix attention = 1 (fp16 / bf16), partition + attention (fp32)
+        # FFN); prefix attention = 1
         "gpu_launches": (2 if anyg else (1 + (8 if layer_ffn_fused else 9) * n_layers) if any_layer
                          else 1 + (6 if layer_ffn_fused else 7) * n_layers if layer
-                         else 1 if tc_prefix else 2) * K,
+                         else 1) * K,
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not layer:

@@ -147,9 +147,9 @@ size_t lf_attention_scratch_bytes(int B, int H, int L, int w, lf_dtype dtype);
 /*
  * lf_attention_forward_idx -- lf_init_global_idx (asynchronous mode) and
  * lf_attention_forward in one call: FTL §Longformer Encoder 计算流程 /
- * 预处理 followed by steps 3-5.  For fp16 / bf16 it is ONE kernel launch:
- * the attention kernel's epilogue warps of CTA b compute the partition of
- * sample b while the first scores are computed.  Arguments as
+ * 预处理 followed by steps 3-5, in ONE kernel launch: CTA b of the attention
+ * kernel also computes the partition of sample b (for fp16 / bf16 its
+ * epilogue warps, while the first scores are computed).  Arguments as
  * lf_attention_forward, plus global_idx [B, L] and global_token_nums [B]
  * (int32, device, written exactly as lf_init_global_idx writes them, with
  * its content check recorded in the device status word).  Errors: as

@@ -129,13 +129,11 @@ lf_status attention_entry(const void* q, const void* k, const void* v, const voi
     if (!d) return st;
     const float scale = 0.125f;  // 1/sqrt(64)
     cudaStream_t s = (cudaStream_t)stream;
-    if (dtype == LF_F32) {
-        if (gidx && (st = launch_global_idx(global_mask, B, L, w, gidx, gnum, d->status, s)) != LF_OK) return st;
+    if (dtype == LF_F32)
         return launch_attention_simt_f32((const float*)q, (const float*)k, (const float*)v,
                                          (const float*)qg, (const float*)kg, (const float*)vg,
                                          local_mask, global_mask, B, H, L, w, scale, (float*)out,
-                                         d->status, s);
-    }
+                                         d->status, s, nullptr, gidx, gnum);
     st = ensure_scratch(d, attention_tc_scratch_bytes(B, H, L, w));
     if (st != LF_OK) return st;
     st = prepare_scratch_counters(d, attention_tc_scratch_zero_bytes(B, H, L, w), s);

@@ -17,6 +17,7 @@
 // then its window [max(i - w, 0), min(i + w, L - 1)], where window keys that
 // are global are skipped (each key once).
 #include "lf_internal.h"
+#include "lf_partition.cuh"
 
 namespace lf {
 namespace {
@@ -114,11 +115,20 @@ attention_simt_kernel(const float* __restrict__ q, const float* __restrict__ k, 
                       const float* __restrict__ vg, const float* __restrict__ local_mask,
                       const float* __restrict__ global_mask, int B, int H, int L, int w, float scale,
                       float* __restrict__ out, int* status, const int32_t* __restrict__ gidx,
-                      const int32_t* __restrict__ gnum) {
+                      const int32_t* __restrict__ gnum, int32_t* __restrict__ gidx_out,
+                      int32_t* __restrict__ gnum_out) {
     __shared__ __align__(16) float sq[64];
     __shared__ float part_ml[kWarps][2];
     __shared__ float part_o[kWarps][64];
+    __shared__ int part_sm[5];
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    // Prefix instance, optional: the global-index partition in the same
+    // launch, sample b by the first four warps of CTA b (the other warps
+    // wait for them at the first row's barrier).
+    if (!kAny && gidx_out && wid < 4)
+        for (int b = blockIdx.x; b < B; b += gridDim.x)
+            partition_sample(global_mask + (size_t)b * L, L, w, gidx_out + (size_t)b * L, gnum_out + b, b, status,
+                             threadIdx.x, wid, lane, part_sm);
     const long long total = (long long)B * H * L;
     for (long long r = blockIdx.x; r < total; r += gridDim.x) {
         const int i = (int)(r % L);
@@ -204,17 +214,19 @@ attention_simt_kernel(const float* __restrict__ q, const float* __restrict__ k, 
 lf_status launch_attention_simt_f32(const float* q, const float* k, const float* v, const float* qg,
                                     const float* kg, const float* vg, const float* local_mask,
                                     const float* global_mask, int B, int H, int L, int w, float scale,
-                                    float* out, int* status, cudaStream_t stream, const AnyGlobals* any) {
+                                    float* out, int* status, cudaStream_t stream, const AnyGlobals* any,
+                                    int32_t* gidx_out, int32_t* gnum_out) {
     const long long rows = (long long)B * H * L;
     long long blocks = rows;
     if (blocks > 148 * 64) blocks = 148 * 64;
     if (any)
         attention_simt_kernel<true><<<(int)blocks, kWarps * 32, 0, stream>>>(
             q, k, v, qg, kg, vg, local_mask, global_mask, B, H, L, w, scale, out, status, any->global_idx,
-            any->global_token_nums);
+            any->global_token_nums, nullptr, nullptr);
     else
         attention_simt_kernel<false><<<(int)blocks, kWarps * 32, 0, stream>>>(
-            q, k, v, qg, kg, vg, local_mask, global_mask, B, H, L, w, scale, out, status, nullptr, nullptr);
+            q, k, v, qg, kg, vg, local_mask, global_mask, B, H, L, w, scale, out, status, nullptr, nullptr,
+            gidx_out, gnum_out);
     return cudaGetLastError() == cudaSuccess ? LF_OK : LF_ERR_CUDA;
 }
 

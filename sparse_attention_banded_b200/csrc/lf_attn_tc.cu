@@ -52,6 +52,7 @@
 
 #include "lf_internal.h"
 #include "lf_pair_math.cuh"
+#include "lf_partition.cuh"
 #include "sm100.cuh"
 
 namespace lf {
@@ -302,75 +303,6 @@ __device__ void band_rows2(const Params& p, int b, const int (&r0)[2], int& cach
         work[x] = __any_sync(0xffffffffu, w_);
         padded[x] = __any_sync(0xffffffffu, pd);
     }
-}
-
-// The 128 epilogue threads (te = 0..127, warp ew = 0..3 of them): the
-// global-index partition of sample b (FTL §Longformer Encoder 计算流程 /
-// 预处理): the positions with global_mask == 0.0 in ascending order, then
-// the others in descending order (the order of a stable flagged partition
-// that writes rejected items from the back), their count, and the content
-// check of the prefix rule.  sm: 5 ints of shared memory; named barrier 1.
-__device__ void partition_sample(const Params& p, int b, int te, int ew, int lane, int* sm) {
-    constexpr int kN = 128, kIt = 4;
-    const int L = p.L;
-    const float* row = p.global_mask + (size_t)b * L;
-    int32_t* idx = p.gidx_out + (size_t)b * L;
-    if (te == 0) sm[4] = L;  // first position that is not global
-    named_bar_sync(1, kN);
-    int base = 0;  // global positions before this chunk
-    for (int c0 = 0; c0 < L; c0 += kN * kIt) {
-        const int j0 = c0 + te * kIt;
-        bool f[kIt];
-        if (j0 + kIt <= L && (L & 3) == 0) {
-            const float4 m4 = *reinterpret_cast<const float4*>(row + j0);
-            f[0] = m4.x == 0.0f;
-            f[1] = m4.y == 0.0f;
-            f[2] = m4.z == 0.0f;
-            f[3] = m4.w == 0.0f;
-        } else {
-#pragma unroll
-            for (int t = 0; t < kIt; ++t) f[t] = (j0 + t < L) && row[j0 + t] == 0.0f;
-        }
-        int cnt = 0, my_first = L;
-#pragma unroll
-        for (int t = 0; t < kIt; ++t) {
-            cnt += f[t];
-            if (!f[t] && j0 + t < L && my_first == L) my_first = j0 + t;
-        }
-        if (my_first < L) atomicMin(&sm[4], my_first);
-        int incl = cnt;  // inclusive scan of the counts within the warp
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += y;
-        }
-        if (lane == 31) sm[ew] = incl;
-        named_bar_sync(1, kN);
-        int wbase = 0;
-        for (int u = 0; u < ew; ++u) wbase += sm[u];
-        const int tot = sm[0] + sm[1] + sm[2] + sm[3];
-        int sel = base + wbase + incl - cnt;  // global positions before j0
-#pragma unroll
-        for (int t = 0; t < kIt; ++t) {
-            const int j = j0 + t;
-            if (j < L) {
-                if (f[t]) {
-                    idx[sel] = j;
-                    ++sel;
-                } else {
-                    idx[L - 1 - (j - sel)] = j;  // j - sel: other positions before j
-                }
-            }
-        }
-        base += tot;
-        named_bar_sync(1, kN);  // sm[0..3] are rewritten by the next chunk
-    }
-    if (te == 0) {
-        p.gnum_out[b] = base;
-        if (sm[4] < base) record_status(p.status, b, LF_ERR_GLOBAL_NOT_PREFIX);
-        else if (base > p.w) record_status(p.status, b, LF_ERR_G_GT_W);
-    }
-    named_bar_sync(1, kN);  // sm[4] is reset for the next sample only after it was read
 }
 
 // Whole warp: the item's plan (identical in every role).
@@ -1344,7 +1276,8 @@ attention_tc_kernel(const __grid_constant__ Maps maps, const __grid_constant__ P
             if (p.gidx_out) {
                 int* sm_i = reinterpret_cast<int*>(smem + kOffMisc + 16);
                 for (int b = blockIdx.x; b < p.B; b += gridDim.x)
-                    partition_sample(p, b, r, sp, lane, sm_i);
+                    partition_sample(p.global_mask + (size_t)b * p.L, p.L, p.w, p.gidx_out + (size_t)b * p.L,
+                                     p.gnum_out + b, b, p.status, r, sp, lane, sm_i);
             }
         }
 #if LF_TRACE

@@ -95,7 +95,8 @@ lf_status launch_attention_simt_f32(const float* q, const float* k, const float*
                                     const float* kg, const float* vg, const float* local_mask,
                                     const float* global_mask, int B, int H, int L, int w,
                                     float scale, float* out, int* status, cudaStream_t stream,
-                                    const AnyGlobals* any = nullptr);
+                                    const AnyGlobals* any = nullptr, int32_t* gidx_out = nullptr,
+                                    int32_t* gnum_out = nullptr);
 
 // Tensor-core path (fp16 / bf16).  `scratch` must hold
 // attention_tc_scratch_bytes(B, H, L, w) bytes whose counter region is zero
