@@ -241,14 +241,12 @@ def run_ours(args):
                                if n.startswith("W_") else v.clone()) for n, v in wts.items()}
                          for _ in range(n_layers - 1)]
         lf.lf_set_ffn_path(args.ffn_path)
-        layer_ffn_fused = lf.lf_gelu_ffn_workspace_bytes(wl.B * wl.L, wl.H * 64, ffn, x.dtype, args.ffn_path) == 0
         ws_fn = lf.lf_encoder_any_globals_workspace_bytes if any_layer else lf.lf_encoder_workspace_bytes
         ws = torch.empty(max(256, ws_fn(n_layers, wl.B, wl.H, wl.L, wl.w, ffn, x.dtype)),
                          dtype=torch.uint8, device=dev)
         args_in = [x]
         t_cpu = None
     else:
-        layer_ffn_fused = False
         wl, t_cpu, lm_cpu, gm_cpu = inputs.workload_inputs(args.workload)
         t = {n: t_cpu[n].to(dev) for n in inputs.NAMES}
         args_in = [t[n] for n in inputs.NAMES]
@@ -451,11 +449,12 @@ def run_ours(args):
         "e2e": {"value": job_throughput(world, tokens, 1, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         # our kernels per step: any-position attention = partition-and-gather
-        # + attention; any-position layer = partition + 9 per layer (8 with
-        # the fused FFN); layer = partition + 7 per layer (6 with the fused
-        # FFN); prefix attention = 1
-        "gpu_launches": (2 if anyg else (1 + (8 if layer_ffn_fused else 9) * n_layers) if any_layer
-                         else 1 + (6 if layer_ffn_fused else 7) * n_layers if layer
+        # + attention; layer = partition + 5 per layer (projections with Qg,
+        # attention, output projection with LN1, then FFN1 and FFN2 with LN2,
+        # or the fused FFN and the LN2 kernel); any-position layer =
+        # partition + 7 per layer (the row gathers added); prefix attention = 1
+        "gpu_launches": (2 if anyg else (1 + 7 * n_layers) if any_layer
+                         else 1 + 5 * n_layers if layer
                          else 1) * K,
         "clocks": clocks,
     }
