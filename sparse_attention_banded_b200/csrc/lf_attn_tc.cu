@@ -1679,7 +1679,7 @@ lf_status launch_instance(int grid, const Maps& maps, const Params& p, cudaStrea
     // preceding work completes first, as usual.
     cudaLaunchAttribute attr_pdl[1];
     attr_pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr_pdl[0].val.programmaticStreamSerializationAllowed = kAny ? 0 : 1;
+    attr_pdl[0].val.programmaticStreamSerializationAllowed = 1;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)grid);
     cfg.blockDim = dim3(kThreads);

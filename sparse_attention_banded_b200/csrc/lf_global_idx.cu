@@ -31,9 +31,10 @@ __global__ void __launch_bounds__(kThreads)
 global_idx_kernel(const float* __restrict__ global_mask, int L, int w, int32_t* __restrict__ global_idx,
                   int32_t* __restrict__ global_token_nums, int32_t* __restrict__ rank, int require_prefix,
                   int* status) {
-    // A kernel launched after this one as a programmatic dependent may be
-    // scheduled right away (it waits for this one before touching memory).
+    // Launched as a programmatic dependent: the next kernel may be scheduled
+    // at once, and nothing is read before the kernel before has completed.
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const int b = blockIdx.x;
     const float* row = global_mask + (size_t)b * L;
     int32_t* idx = global_idx + (size_t)b * L;
@@ -117,9 +118,8 @@ global_idx_kernel(const float* __restrict__ global_mask, int L, int w, int32_t* 
 lf_status launch_global_idx(const float* global_mask, int B, int L, int w, int32_t* global_idx,
                             int32_t* global_token_nums, int* status, cudaStream_t stream, int32_t* rank,
                             bool require_prefix) {
-    global_idx_kernel<<<B, kThreads, 0, stream>>>(global_mask, L, w, global_idx, global_token_nums, rank,
-                                                  require_prefix ? 1 : 0, status);
-    return cudaGetLastError() == cudaSuccess ? LF_OK : LF_ERR_CUDA;
+    return launch_pdl(global_idx_kernel, dim3(B), dim3(kThreads), 0, stream, global_mask, L, w, global_idx,
+                      global_token_nums, rank, require_prefix ? 1 : 0, status);
 }
 
 }  // namespace lf
@@ -148,6 +148,10 @@ gather_globals_kernel(const uint4* __restrict__ qg, const uint4* __restrict__ k,
                       const float* __restrict__ local_mask, const int32_t* __restrict__ gidx,
                       const int32_t* __restrict__ gnum, int H, int L, int gcap, uint4* __restrict__ qg_c,
                       uint4* __restrict__ k_c, uint4* __restrict__ v_c, float* __restrict__ lm_c) {
+    // Launched as a programmatic dependent: the next kernel may be scheduled
+    // at once, and nothing is read before the kernel before has completed.
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const int per = gcap / 32;  // CTAs per (b, h)
     const int bh = blockIdx.x / per, b = bh / H, h = bh % H;
     const int c0 = (blockIdx.x % per) * 32;
@@ -190,6 +194,10 @@ partition_gather_kernel(const float* __restrict__ global_mask, const float* __re
                         const uint4* __restrict__ v, int32_t* __restrict__ global_idx,
                         int32_t* __restrict__ global_token_nums, int32_t* __restrict__ rank, uint4* __restrict__ qg_c,
                         uint4* __restrict__ k_c, uint4* __restrict__ v_c, float* __restrict__ lm_c, int* status) {
+    // Launched as a programmatic dependent: the next kernel may be scheduled
+    // at once, and nothing is read before the kernel before has completed.
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     extern __shared__ int slot_pos[];  // [gcap]
     const int bh = blockIdx.x, b = bh / H, h = bh % H;
     const bool lead = h == 0;  // writes the partition's outputs
@@ -288,6 +296,10 @@ partition_gather_kernel(const float* __restrict__ global_mask, const float* __re
 __global__ void __launch_bounds__(128)
 gather_rows_kernel(const uint4* __restrict__ src, const int32_t* __restrict__ gidx,
                    const int32_t* __restrict__ gnum, int L, int gcap, int parts, uint4* __restrict__ dst) {
+    // Launched as a programmatic dependent: the next kernel may be scheduled
+    // at once, and nothing is read before the kernel before has completed.
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const int b = blockIdx.x / gcap, c = blockIdx.x % gcap;
     const int g = min(gnum[b], gcap);
     uint4* d = dst + ((size_t)b * gcap + c) * parts;
@@ -305,10 +317,9 @@ lf_status launch_gather_rows(const void* src, const AnyGlobals& a, int B, int L,
                              cudaStream_t stream) {
     const long long blocks = (long long)B * a.gcap;
     if (blocks >= (1LL << 31)) return LF_ERR_TOO_LARGE;
-    gather_rows_kernel<<<(unsigned)blocks, 128, 0, stream>>>(reinterpret_cast<const uint4*>(src), a.global_idx,
-                                                             a.global_token_nums, L, a.gcap, D * 2 / 16,
-                                                             reinterpret_cast<uint4*>(dst));
-    return cudaGetLastError() == cudaSuccess ? LF_OK : LF_ERR_CUDA;
+    return launch_pdl(gather_rows_kernel, dim3((unsigned)blocks), dim3(128), 0, stream,
+                      reinterpret_cast<const uint4*>(src), a.global_idx, a.global_token_nums, L, a.gcap, D * 2 / 16,
+                      reinterpret_cast<uint4*>(dst));
 }
 
 lf_status launch_partition_gather(const float* global_mask, const float* local_mask, const void* qg, const void* k,
@@ -328,12 +339,12 @@ lf_status launch_partition_gather(const float* global_mask, const float* local_m
             attr[dev].store(true);
         }
     }
-    partition_gather_kernel<<<B * H, kThreads, smem, stream>>>(
-        global_mask, local_mask, H, L, w, a.gcap, reinterpret_cast<const uint4*>(qg),
-        reinterpret_cast<const uint4*>(k), reinterpret_cast<const uint4*>(v), const_cast<int32_t*>(a.global_idx),
-        const_cast<int32_t*>(a.global_token_nums), const_cast<int32_t*>(a.rank), reinterpret_cast<uint4*>(a.qg_c),
-        reinterpret_cast<uint4*>(a.k_c), reinterpret_cast<uint4*>(a.v_c), a.lm_c, status);
-    return cudaGetLastError() == cudaSuccess ? LF_OK : LF_ERR_CUDA;
+    return launch_pdl(partition_gather_kernel, dim3(B * H), dim3(kThreads), smem, stream, global_mask, local_mask, H,
+                      L, w, a.gcap, reinterpret_cast<const uint4*>(qg), reinterpret_cast<const uint4*>(k),
+                      reinterpret_cast<const uint4*>(v), const_cast<int32_t*>(a.global_idx),
+                      const_cast<int32_t*>(a.global_token_nums), const_cast<int32_t*>(a.rank),
+                      reinterpret_cast<uint4*>(a.qg_c), reinterpret_cast<uint4*>(a.k_c),
+                      reinterpret_cast<uint4*>(a.v_c), a.lm_c, status);
 }
 
 size_t any_globals_bytes(int B, int H, int L, int w, bool compact) {
@@ -370,12 +381,12 @@ lf_status launch_gather_globals(const void* qg, const void* k, const void* v, co
     (void)w;
     const long long blocks = (long long)B * H * (a.gcap / 32);
     if (blocks >= (1LL << 31)) return LF_ERR_TOO_LARGE;
-    gather_globals_kernel<<<(unsigned)blocks, 256, 0, stream>>>(
-        reinterpret_cast<const uint4*>(qg), reinterpret_cast<const uint4*>(k), reinterpret_cast<const uint4*>(v),
-        // (qg may be NULL: qg_c is then left to the caller)
-        local_mask, a.global_idx, a.global_token_nums, H, L, a.gcap, reinterpret_cast<uint4*>(a.qg_c),
-        reinterpret_cast<uint4*>(a.k_c), reinterpret_cast<uint4*>(a.v_c), a.lm_c);
-    return cudaGetLastError() == cudaSuccess ? LF_OK : LF_ERR_CUDA;
+    // (qg may be NULL: qg_c is then left to the caller)
+    return launch_pdl(gather_globals_kernel, dim3((unsigned)blocks), dim3(256), 0, stream,
+                      reinterpret_cast<const uint4*>(qg), reinterpret_cast<const uint4*>(k),
+                      reinterpret_cast<const uint4*>(v), local_mask, a.global_idx, a.global_token_nums, H, L,
+                      a.gcap, reinterpret_cast<uint4*>(a.qg_c), reinterpret_cast<uint4*>(a.k_c),
+                      reinterpret_cast<uint4*>(a.v_c), a.lm_c);
 }
 
 }  // namespace lf
