@@ -223,8 +223,9 @@ def test_attention_idx_small(dtype, shape):
     assert np.array_equal(nums.cpu().numpy(), e_nums)
 
 
+@pytest.mark.parametrize("dtype", ["f32", "f16"])
 @pytest.mark.parametrize("seed", range(6))
-def test_attention_idx_partition_bit_exact(seed):
+def test_attention_idx_partition_bit_exact(seed, dtype):
     """Random prefix lengths (0..w), batch sizes and window widths, among them
     L not a multiple of 4: the in-kernel partition against the oracle."""
     rng = np.random.default_rng(100 + seed)
@@ -233,7 +234,7 @@ def test_attention_idx_partition_bit_exact(seed):
     gm = np.full((B, L), -10000.0, np.float32)
     for b in range(B):
         gm[b, : int(rng.integers(0, w + 1))] = 0.0
-    t = inputs.attention_inputs(B, 1, L, "f16", seed=seed)
+    t = inputs.attention_inputs(B, 1, L, dtype, seed=seed)
     lm = torch.ones(B, L, dtype=torch.float32)
     lf.lf_device_status(reset=True)
     _, idx, nums = _run_idx(t, lm, torch.from_numpy(gm), w)
@@ -243,8 +244,9 @@ def test_attention_idx_partition_bit_exact(seed):
     assert np.array_equal(nums.cpu().numpy(), e_nums)
 
 
+@pytest.mark.parametrize("dtype", ["f32", "f16", "bf16"])
 @pytest.mark.parametrize("case", ["not_prefix", "too_many", "scatter"])
-def test_attention_idx_content_errors(case):
+def test_attention_idx_content_errors(case, dtype):
     """Masks that break the prefix rules: the combined call records the same
     status as lf_init_global_idx followed by lf_attention_forward, writes the
     oracle's partition and the same output."""
@@ -257,7 +259,7 @@ def test_attention_idx_content_errors(case):
         gm[1, :w + 1] = 0.0
     else:
         gm[2, ::7] = 0.0
-    t = inputs.attention_inputs(B, H, L, "bf16", seed=8)
+    t = inputs.attention_inputs(B, H, L, dtype, seed=8)
     lm = torch.ones(B, L, dtype=torch.float32)
     g = torch.from_numpy(gm)
     lf.lf_device_status(reset=True)
