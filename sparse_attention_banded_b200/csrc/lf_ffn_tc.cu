@@ -40,6 +40,7 @@
 
 #include <atomic>
 
+#include "lf_gelu.cuh"
 #include "lf_internal.h"
 #include "sm100_cluster.cuh"
 
@@ -119,7 +120,7 @@ __device__ __forceinline__ void tmem_ld32f(uint32_t taddr, float (&r)[32]) {
 }
 
 // The erf form of GELU, as the two-GEMM path's epilogue computes it.
-__device__ __forceinline__ float gelu_erf(float x) { return 0.5f * x * (1.0f + erff(x * 0.70710678118654752f)); }
+__device__ __forceinline__ float gelu_erf(float x) { return gelu_erf_as(x); }
 
 template <typename T, int CS>
 __global__ void __launch_bounds__(kThreads, 1)

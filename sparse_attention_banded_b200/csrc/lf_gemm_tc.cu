@@ -38,6 +38,7 @@
 #include <atomic>
 #include <mutex>
 
+#include "lf_gelu.cuh"
 #include "lf_internal.h"
 #include "sm100_cluster.cuh"
 
@@ -168,7 +169,7 @@ __device__ __forceinline__ void tmem_st32v(uint32_t taddr, const float (&r)[32])
 }
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
-__device__ __forceinline__ float gelu_erf(float x) { return 0.5f * x * (1.0f + erff(x * 0.70710678118654752f)); }
+__device__ __forceinline__ float gelu_erf(float x) { return gelu_erf_as(x); }
 
 template <typename T>
 __global__ void __launch_bounds__(kThreads, 1)
