@@ -142,6 +142,8 @@ ffn_fused_kernel(const __grid_constant__ CUtensorMap map_h, const __grid_constan
     uint64_t* drain = out_full + 1;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
+    // [CS] phases of slot_full[q] the MMA warp has taken (for the wind-down)
+    volatile uint32_t* slot_used = reinterpret_cast<volatile uint32_t*>(smem + C::kOffMisc + 16);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = CS > 1 ? cluster_ctarank() : 0;
     const int m0 = (int)(CS > 1 ? cluster_id_x() : blockIdx.x) * kTM;
@@ -163,6 +165,7 @@ ffn_fused_kernel(const __grid_constant__ CUtensorMap map_h, const __grid_constan
         for (int i = 0; i < CS; ++i) {
             mbar_init(&slot_full[i], 1);
             mbar_init(&consumed[i], 1);
+            slot_used[i] = 0;
         }
         mbar_init(slot_free, CS);
         mbar_init(out_full, 1);
@@ -278,6 +281,7 @@ ffn_fused_kernel(const __grid_constant__ CUtensorMap map_h, const __grid_constan
                     const int c = (t - 1) * CS + q;
                     ok = wait_all_cluster(&slot_full[q], (t - 1) & 1);
                     if (!ok) break;
+                    if (lane == 0) slot_used[q] = (uint32_t)t;
                     const uint32_t slot = smem_u32(smem + C::kOffSlot + q * kSlotBytes);
                     for (int a = 0; a < 2 && ok; ++a, ++kc) {
                         const uint32_t st = kc % S;
@@ -444,7 +448,24 @@ ffn_fused_kernel(const __grid_constant__ CUtensorMap map_h, const __grid_constan
 
     __syncthreads();
     // no CTA leaves while a peer may still arrive on or copy into it
-    if (CS > 1) cluster_sync();
+    if (CS > 1) {
+        cluster_sync();
+        // Every copy into this CTA has been issued by now.  A CTA that gave
+        // up may not have taken the last phase of a peer's slot: wait, with
+        // a short limit, for that phase (a copy in flight lands within
+        // microseconds; a peer that sent nothing leaves it to time out),
+        // then leave together, so that no copy's source or destination goes
+        // away while it is in flight.
+        if (warp == 1 && *abort_flag) {
+            for (int q = 0; q < CS; ++q) {
+                if (q == (int)rank) continue;
+                volatile int never = 0;
+                mbar_wait_cluster(&slot_full[q], slot_used[q] & 1u, &never, 2000000ull);
+            }
+        }
+        __syncwarp();
+        cluster_sync();
+    }
     if (threadIdx.x == 0 && *abort_flag) record_status(p.status, 0, LF_ERR_DEVICE_TIMEOUT);
     if (warp == 1) {
         tc_fence_after();
