@@ -28,9 +28,10 @@
 //                row-major out (the LayerNorm kernel reads it)
 //   kEpiResidLN: + bias + residual, then LayerNorm over the row (step 5's
 //                AddBiasResidualLayerNorm and step 6's), rounded, row-major
-//                out: the N / 256 CTAs of a row tile form a cluster and
-//                exchange per-row sums through distributed shared memory
-//                (the mean, then the centred second moment)
+//                out: the N / 256 CTAs of a row tile form a cluster; each
+//                sends its columns' sum and centred second moment of every
+//                row to the others through distributed shared memory (one
+//                exchange), and all combine them in the same order
 // Roofline: tensor-bound (2*M*N*K flops over (M*K + N*K)*2 + out bytes).
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -56,13 +57,19 @@ constexpr uint32_t kBBytes = kTN * kTK * 2;  // 32 KB
 constexpr uint32_t kOffA = 0;
 constexpr uint32_t kOffB = kOffA + kStages * kABytes;
 constexpr uint32_t kOffBias = kOffB + kStages * kBBytes;        // epilogue warps x kTN / 2 floats
-constexpr uint32_t kOffRed = kOffBias + kEpiWarps * (kTN / 2) * 4;  // kEpiResidLN: [2 halves][kTM] row sums
-constexpr int kMaxLnCtas = 4;                                          // N <= 1024
-constexpr uint32_t kOffXch = kOffRed + 2 * kTM * 4;                    // [2 sums][kMaxLnCtas][kTM] from each CTA
-constexpr uint32_t kOffBar = kOffXch + 2 * kMaxLnCtas * kTM * 4;
+// kEpiResidLN: the LayerNorm's gamma and beta of each warp's columns
+constexpr uint32_t kOffGamma = kOffBias + kEpiWarps * (kTN / 2) * 4;
+constexpr uint32_t kOffBeta = kOffGamma + kEpiWarps * (kTN / 2) * 4;
+// kEpiResidLN: [2 moments][2 halves][kTM] partial row sums of the two warps of a row
+constexpr uint32_t kOffRed = kOffBeta + kEpiWarps * (kTN / 2) * 4;
+constexpr int kMaxLnCtas = 4;  // N <= 1024
+// kEpiResidLN: [2 buffers][kMaxLnCtas][2 moments][kTM], every CTA's row moments
+constexpr uint32_t kOffXch = kOffRed + 4 * kTM * 4;
+constexpr uint32_t kOffBar = kOffXch + 2 * kMaxLnCtas * 2 * kTM * 4;
 constexpr uint32_t kNumBars = 2 * kStages + 4 + 1 + 2;
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
 constexpr uint32_t kSmemBytes = kOffMisc + 64 + 1024;
+static_assert(kSmemBytes <= 232448, "shared memory");
 constexpr uint32_t kTmemCols = 512;  // two 256-column fp32 accumulators
 
 // One GEMM problem of a launch: per batch, rows x N outputs.
@@ -185,7 +192,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
     uint64_t* acc_full = bars + 2 * kStages;
     uint64_t* acc_empty = acc_full + 2;
     uint64_t* drain = acc_empty + 2;
-    uint64_t* xbar = drain + 1;  // [2] kEpiResidLN: every CTA of the cluster has delivered its row sums
+    uint64_t* xbar = drain + 1;  // [2] kEpiResidLN: every CTA of the cluster has delivered its row moments (one per buffer)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -332,37 +339,24 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
         const int r = sp * 32 + lane;
         const uint32_t lane_off = (uint32_t)(sp * 32) << 16;
         float* bias_w = reinterpret_cast<float*>(smem + kOffBias) + (warp - 4) * (kTN / 2);
-        // kEpiResidLN: the sum over the cluster's columns of v (this
-        // thread's partial for row r): both warps' halves through shared
-        // memory, then every CTA's sum into every CTA's exchange slot, added
-        // in CTA order (so all CTAs of the cluster get the same bits).
-        // Returns false on a failure of any epilogue warp (taken together).
+        // kEpiResidLN.  Each CTA holds a row's kTN columns (column tile =
+        // cluster rank); a row's two warps each hold half of them.  red: the
+        // two halves' partial sums; xch: every CTA's (column sum, centred
+        // second moment) of each row, in two buffers used by alternate tiles.
         float* red = reinterpret_cast<float*>(smem + kOffRed);
         float* xch = reinterpret_cast<float*>(smem + kOffXch);
+        float* gam_w = reinterpret_cast<float*>(smem + kOffGamma) + (warp - 4) * (kTN / 2);
+        float* bet_w = reinterpret_cast<float*>(smem + kOffBeta) + (warp - 4) * (kTN / 2);
         const uint32_t rank = p.mode == kEpiResidLN ? cluster_ctarank() : 0;
-        auto cluster_row_sum = [&](float v, int e, uint32_t parity, bool fail, float& total) -> bool {
-            red[half * kTM + r] = v;
-            if (named_bar_any(1, kEpiWarps * 32, fail)) return false;
-            if (half == 0) {
-                const float part = red[r] + red[kTM + r];
-                const uint32_t slot = smem_u32(xch + (e * kMaxLnCtas + rank) * kTM + r);
-                for (int q = 0; q < p.ln_ctas; ++q) st_cluster_f32(mapa_shared(slot, (uint32_t)q), part);
-                fence_acq_rel_cluster();
-            }
-            named_bar_sync(1, kEpiWarps * 32);
-            if (warp == 4 && lane == 0)
-                for (int q = 0; q < p.ln_ctas; ++q) mbar_arrive_cluster(mapa_shared(smem_u32(&xbar[e]), (uint32_t)q));
-            const bool got = __all_sync(0xffffffffu, mbar_wait_cluster(&xbar[e], parity, abort_flag));
-            if (named_bar_any(1, kEpiWarps * 32, !got)) return false;
-            float t = 0.0f;
-            for (int q = 0; q < p.ln_ctas; ++q) t += xch[(e * kMaxLnCtas + q) * kTM + r];
-            total = t;
-            return true;
-        };
-        // kEpiResidLN, one tile: z = acc + bias + resid kept in TMEM, mean,
-        // centred second moment, then (z - mean) * rsqrt(var + eps) * gamma
-        // + beta rounded and stored.  False on a failure (all warps alike).
         uint32_t ln_cnt = 0;
+        // kEpiResidLN, one tile: z = acc + bias + resid kept in TMEM; this
+        // CTA's column sum S_c and, about its own mean S_c / n_c, the centred
+        // second moment M2_c; one exchange of (S_c, M2_c) over the cluster;
+        // then mean = sum S_q / N and M2 = sum (M2_q + n_q (S_q / n_q - mean)^2)
+        // (the pairwise update of Chan, Golub and LeVeque), added in CTA
+        // order so that every CTA normalises with the same bits; finally
+        // (z - mean) * rsqrt(M2 / N + eps) * gamma + beta, rounded and stored.
+        // False on a failure (all epilogue warps alike).
         auto ln_tile = [&](const TileAt& at, const GemmProb& q, uint32_t ab, uint32_t tcn, int n0, int ncols,
                            int wcols) -> bool {
             bool fail = !__all_sync(0xffffffffu, mbar_wait(&acc_full[ab], (tcn >> 1) & 1, abort_flag));
@@ -380,8 +374,15 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
                     tmem_ld32v(tz + c0, z);
                     tmem_ld_wait();
                     regs_ready<32>(z);
+                    const float4* b4 = reinterpret_cast<const float4*>(bias_w + c0);
 #pragma unroll
-                    for (int c = 0; c < 32; ++c) z[c] += bias_w[c0 + c];
+                    for (int c = 0; c < 8; ++c) {
+                        const float4 v = b4[c];
+                        z[4 * c] += v.x;
+                        z[4 * c + 1] += v.y;
+                        z[4 * c + 2] += v.z;
+                        z[4 * c + 3] += v.w;
+                    }
                     if (row_ok) {
                         const uint4* rs =
                             reinterpret_cast<const uint4*>(reinterpret_cast<const T*>(p.resid) + grow * q.N + n0 + c0);
@@ -399,11 +400,12 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
                 }
                 tmem_st_wait();
             }
-            const uint32_t parity = ln_cnt & 1;
-            ++ln_cnt;
-            float sum = 0.0f, sq = 0.0f;
-            if (!cluster_row_sum(s1, 0, parity, fail, sum)) return false;
-            const float mean = sum / (float)q.N;
+            // this CTA's columns of the row: n_c of them, sum S_c, mean m_c
+            red[half * kTM + r] = s1;
+            if (named_bar_any(1, kEpiWarps * 32, fail)) return false;
+            const int n_c = min(kTN, q.N - at.col0);
+            const float sum_c = red[r] + red[kTM + r];
+            const float mean_c = sum_c / (float)n_c;
             float s2 = 0.0f;
 #pragma unroll 1
             for (int c0 = 0; c0 < ncols; c0 += 32) {
@@ -414,12 +416,42 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
                 regs_ready<32>(z);
 #pragma unroll
                 for (int c = 0; c < 32; ++c) {
-                    const float d = z[c] - mean;
+                    const float d = z[c] - mean_c;
                     s2 = fmaf(d, d, s2);
                 }
             }
-            if (!cluster_row_sum(s2, 1, parity, false, sq)) return false;
-            const float inv = rsqrtf(sq / (float)q.N + p.ln_eps);
+            red[(2 + half) * kTM + r] = s2;
+            named_bar_sync(1, kEpiWarps * 32);
+            // (S_c, M2_c) into every CTA's slot for this CTA, then one
+            // arrival on each CTA's barrier of this buffer
+            const uint32_t e = ln_cnt & 1, parity = (ln_cnt >> 1) & 1;
+            ++ln_cnt;
+            if (half == 0) {
+                const float m2_c = red[2 * kTM + r] + red[3 * kTM + r];
+                const uint32_t slot = smem_u32(xch + ((e * kMaxLnCtas + rank) * 2) * kTM + r);
+                for (int qq = 0; qq < p.ln_ctas; ++qq) {
+                    st_cluster_f32(mapa_shared(slot, (uint32_t)qq), sum_c);
+                    st_cluster_f32(mapa_shared(slot + kTM * 4, (uint32_t)qq), m2_c);
+                }
+                fence_acq_rel_cluster();
+            }
+            named_bar_sync(1, kEpiWarps * 32);
+            if (warp == 4 && lane == 0)
+                for (int qq = 0; qq < p.ln_ctas; ++qq)
+                    mbar_arrive_cluster(mapa_shared(smem_u32(&xbar[e]), (uint32_t)qq));
+            const bool got = __all_sync(0xffffffffu, mbar_wait_cluster(&xbar[e], parity, abort_flag));
+            if (named_bar_any(1, kEpiWarps * 32, !got)) return false;
+            const float* xe = xch + (size_t)e * kMaxLnCtas * 2 * kTM + r;
+            float tot = 0.0f;
+            for (int qq = 0; qq < p.ln_ctas; ++qq) tot += xe[qq * 2 * kTM];
+            const float mean = tot / (float)q.N;
+            float m2 = 0.0f;
+            for (int qq = 0; qq < p.ln_ctas; ++qq) {
+                const float n_q = (float)min(kTN, q.N - qq * kTN);
+                const float d = xe[qq * 2 * kTM] / n_q - mean;
+                m2 += fmaf(n_q * d, d, xe[(qq * 2 + 1) * kTM]);
+            }
+            const float inv = rsqrtf(m2 / (float)q.N + p.ln_eps);
 #pragma unroll 1
             for (int c0 = 0; c0 < ncols; c0 += 32) {
                 float z[32];
@@ -430,14 +462,17 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
                 if (row_ok) {
                     const int n = n0 + c0;
                     uint4* d4 = reinterpret_cast<uint4*>(reinterpret_cast<T*>(q.out) + grow * q.N + n);
+                    const float4* g4 = reinterpret_cast<const float4*>(gam_w + c0);
+                    const float4* be4 = reinterpret_cast<const float4*>(bet_w + c0);
 #pragma unroll
                     for (int u4 = 0; u4 < 4; ++u4) {
+                        const float4 ga = g4[2 * u4], gb = g4[2 * u4 + 1];
+                        const float4 ba = be4[2 * u4], bb = be4[2 * u4 + 1];
+                        const float gm[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
+                        const float bt[8] = {ba.x, ba.y, ba.z, ba.w, bb.x, bb.y, bb.z, bb.w};
                         float y[8];
 #pragma unroll
-                        for (int j = 0; j < 8; ++j) {
-                            const int c = u4 * 8 + j;
-                            y[j] = fmaf((z[c] - mean) * inv, __ldg(p.ln_gamma + n + c), __ldg(p.ln_beta + n + c));
-                        }
+                        for (int j = 0; j < 8; ++j) y[j] = fmaf((z[u4 * 8 + j] - mean) * inv, gm[j], bt[j]);
                         uint4 u;
                         u.x = Cvt<T>::two(y[0], y[1]);
                         u.y = Cvt<T>::two(y[2], y[3]);
@@ -467,6 +502,14 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
 #pragma unroll
             for (int c = 0; c < kTN / 64; ++c)
                 if (c * 32 < ncols) bias_w[c * 32 + lane] = Cvt<T>::to_f(bias[n0 + c * 32 + lane]);
+            if (p.mode == kEpiResidLN) {  // and of its columns' gamma and beta
+#pragma unroll
+                for (int c = 0; c < kTN / 64; ++c)
+                    if (c * 32 < ncols) {
+                        gam_w[c * 32 + lane] = p.ln_gamma[n0 + c * 32 + lane];
+                        bet_w[c * 32 + lane] = p.ln_beta[n0 + c * 32 + lane];
+                    }
+            }
             __syncwarp();
             const uint32_t ab = tc & 1;
             if (p.mode == kEpiResidLN) {
@@ -500,16 +543,16 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
                 } else if (p.mode == kEpiResid) {
                     const uint4* rs = reinterpret_cast<const uint4*>(reinterpret_cast<const T*>(p.resid) + grow * q.N + n);
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        uint4 u = rs[q];
+                    for (int u4 = 0; u4 < 4; ++u4) {
+                        uint4 u = rs[u4];
                         const T* e = reinterpret_cast<const T*>(&u);
 #pragma unroll
-                        for (int j = 0; j < 8; ++j) acc[q * 8 + j] += Cvt<T>::to_f(e[j]);
+                        for (int j = 0; j < 8; ++j) acc[u4 * 8 + j] += Cvt<T>::to_f(e[j]);
                     }
                     float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(q.out) + grow * q.N + n);
 #pragma unroll
-                    for (int q = 0; q < 8; ++q)
-                        dst[q] = make_float4(acc[4 * q], acc[4 * q + 1], acc[4 * q + 2], acc[4 * q + 3]);
+                    for (int v = 0; v < 8; ++v)
+                        dst[v] = make_float4(acc[4 * v], acc[4 * v + 1], acc[4 * v + 2], acc[4 * v + 3]);
                 } else {
                     T* dst;
                     if (p.mode == kEpiHeads) {
